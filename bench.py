@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the SPIN decode step on B200.
+
+One step = the whole hot path for one batch: query quantisation, predict +
+block max-pool, budget / exploration select, paged FP8 indexer score on the
+kept blocks (with the fused EMA update) and the token top-k, for 96 requests at
+512K context (the serving-shaped workload).  Metric: decode rows/s (requests x
+query rows per second), with index-key GB/s and the fraction of the HBM
+roofline alongside.
+
+Arms:
+  default            libspin.so through its C ABI (device-resident inputs);
+                     also an end-to-end pass with host buffers, a 0% / 40% / 50%
+                     sparsity sweep, GPU-measured fidelity and the CPU oracle
+                     baseline.
+  --impl reference   the CPU oracle on this host's cores, on a bounded sample
+                     of the same workload per step.
+
+Multi-GPU (torchrun): every rank runs its own 96 requests (requests are
+independent: weak scaling, no data-path collective); the time is the max over
+ranks and the value counts every rank's rows.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "SPIN decode rows/s & index-key GB/s at 512K ctx x96 req; % of roofline"
+KEY_BYTES_PER_SLOT = 128 + 4            # E4M3 key row + fp32 scale
+SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write of V and D
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["spin", "reference"], default="spin")
+    p.add_argument("--sparsity", type=float, default=0.5)
+    p.add_argument("--requests", type=int, default=96, help="requests per GPU (96 = the serving workload)")
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# process group (one rank per GPU) and device clocks
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of this GPU while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = tempfile.mktemp(suffix=".csv")
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            ident = str(device_index)
+        self.ident = ident
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.ident}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        except Exception:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = np.array([float(r[0]) for r in rows])
+        mx = float(rows[0][1])
+        util = np.array([float(r[2]) if r[2].replace(".", "").isdigit() else 0.0 for r in rows])
+        loaded = sm[util > 0] if np.any(util > 0) else sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": int(loaded.size)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class SpinRun:
+    def __init__(self, wl, device, total_steps):
+        import indexer_sparse_attention_b200 as isa
+        self.isa = isa
+        self.wl = wl
+        self.device = device
+        self.cache = workloads.make_key_cache(wl, 0, device)
+        self.positions = total_steps + 1
+        q, w = workloads.make_queries(wl, 0, self.positions, device)
+        self.q = [q[:, t:t + 1].contiguous() for t in range(self.positions)]
+        self.w = [w[:, t:t + 1].contiguous() for t in range(self.positions)]
+        del q, w
+        ctx0 = torch.tensor(wl.ctx0, dtype=torch.int64, device=device)
+        self.ctx = [(ctx0 + t + 1).to(torch.int32) for t in range(self.positions)]
+        cfg = isa.make_config(num_layers=1, num_requests=wl.requests, max_slots=wl.max_slots, block_size=wl.b,
+                              num_heads=wl.H, head_dim=wl.d, topk=wl.topk, max_rows=1, key_fp8=True, q_bf16=True,
+                              alpha=wl.alpha, gamma=wl.gamma, target_sparsity=wl.sparsity, seed=wl.seed)
+        self.st = isa.SpinState(cfg, device=device)
+        self.mask = self.st.new_mask()
+        self.topk = torch.empty((wl.requests, 1, wl.topk), dtype=torch.int32, device=device)
+        self.scores = self.st.new_scores()
+        self.t = 0
+
+    def set_sparsity(self, s):
+        self.isa.spin_set_layer_sparsity(self.st, [s])
+
+    def step(self, defer=False, q=None, w=None, ctx=None, mask=None, topk=None):
+        t = self.t
+        c = self.cache
+        self.isa.spin_decode_step(self.st, 0, 1, t, c.keys, c.kscale, c.block_table,
+                                  self.q[t] if q is None else q, self.w[t] if w is None else w,
+                                  self.ctx[t] if ctx is None else ctx, defer,
+                                  self.mask if mask is None else mask, self.topk if topk is None else topk,
+                                  self.scores)
+        self.t += 1
+
+    def kept_slots(self):
+        """Slots scored in the last step (kept blocks, visible part)."""
+        ctx = self.ctx[self.t - 1].long()
+        nb = (ctx + self.wl.b - 1) // self.wl.b
+        m = self.mask.bool()
+        kept_blocks = m.sum(dim=1)
+        last = nb - 1
+        tail_kept = m.gather(1, last[:, None])[:, 0]
+        tail_slots = ctx - last * self.wl.b
+        slots = kept_blocks * self.wl.b - tail_kept.long() * (self.wl.b - tail_slots)
+        return int(slots.sum().item()), (kept_blocks.double() / nb.double())
+
+
+def timed_steps(run, steps, world, defer=False):
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        run.step(defer=defer)
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
+def fidelity(run, n_steps=3):
+    """Mean / p99 miss (share of the full indexer's top-k in skipped blocks)
+    and realized block sparsity, measured on the GPU with a shadow full
+    indexer on the same inputs; outside every timed region."""
+    isa, wl = run.isa, run.wl
+    full_scores = run.st.new_scores()
+    full_topk = torch.empty_like(run.topk)
+    missed = torch.zeros((wl.requests, 1), dtype=torch.int32, device=run.device)
+    total = torch.zeros_like(missed)
+    allk = torch.ones_like(run.mask)
+    miss, realized = [], []
+    c = run.cache
+    for _ in range(n_steps):
+        t = run.t
+        run.step()
+        isa.spin_indexer_score(run.st, 0, 1, c.keys, c.kscale, c.block_table, run.q[t], run.w[t], run.ctx[t],
+                               allk, full_scores)
+        isa.spin_topk(run.st, 1, full_scores, allk, run.ctx[t], full_topk)
+        isa.spin_miss_count(run.st, 1, full_topk, run.mask, missed, total)
+        miss += (missed.double() / total.double().clamp(min=1))[:, 0].tolist()
+        realized += (1 - run.kept_slots()[1]).tolist()
+    v = np.sort(np.array(miss))
+    p99 = float(v[max(int(np.ceil(0.99 * v.size)), 1) - 1])
+    return {"mean_miss": float(v.mean()), "p99_miss": p99, "realized_sparsity": float(np.mean(realized)),
+            "rows": int(v.size)}
+
+
+def e2e_pass(run, steps, world):
+    """The same decode step through the public API with host inputs: per step
+    the query, head weights and context lengths are copied in from pinned
+    host memory and the top-k indices and block mask are read back."""
+    wl = run.wl
+    t0 = run.t
+    q_h = [run.q[t0 + i].cpu().pin_memory() for i in range(steps)]
+    w_h = [run.w[t0 + i].cpu().pin_memory() for i in range(steps)]
+    c_h = [run.ctx[t0 + i].cpu().pin_memory() for i in range(steps)]
+    q_d, w_d, c_d = torch.empty_like(run.q[0]), torch.empty_like(run.w[0]), torch.empty_like(run.ctx[0])
+    topk_h = torch.empty(run.topk.shape, dtype=torch.int32).pin_memory()
+    mask_h = torch.empty(run.mask.shape, dtype=torch.uint8).pin_memory()
+    h2d = q_h[0].numel() * q_h[0].element_size() + w_h[0].numel() * 4 + c_h[0].numel() * 4
+    d2h = topk_h.numel() * 4 + mask_h.numel()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(steps):
+        q_d.copy_(q_h[i], non_blocking=True)
+        w_d.copy_(w_h[i], non_blocking=True)
+        c_d.copy_(c_h[i], non_blocking=True)
+        run.step(q=q_d, w=w_d, ctx=c_d)
+        topk_h.copy_(run.topk, non_blocking=True)
+        mask_h.copy_(run.mask, non_blocking=True)
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return ms, h2d, d2h
+
+
+def gpu_arm(args, world, rank, local):
+    import indexer_sparse_attention_b200 as isa
+    from indexer_sparse_attention_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    isa.load()
+    device = torch.device("cuda", local if world > 1 else 0)
+    W, K = args.warmup, args.steps
+    sweep = [] if args.no_sweep else [0.4, 0.0]
+    total = 1 + (W + K) * (1 + len(sweep)) + 3 + K + 2
+    base = workloads.config(2)
+    wl = workloads.config(2, seed=base.seed + 1000 * rank, steps=1, spare_slots=total + 8,
+                          requests=args.requests, ctx0=base.ctx0[:1] * args.requests)
+    run = SpinRun(wl, device, total)
+    Q = wl.requests
+    # history bootstrap: all-keep step that fills V and D
+    run.set_sparsity(0.0)
+    run.step()
+    # ---- headline: target sparsity, score kernel timed live -------------
+    run.set_sparsity(args.sparsity)
+    for _ in range(W):
+        run.step()
+    isa.spin_kernel_times(run.st)
+    isa.spin_set_kernel_timing(run.st, True)
+    with ClockSampler(device.index) as clk:
+        ms = timed_steps(run, K, world)
+    isa.spin_set_kernel_timing(run.st, False)
+    stages = isa.spin_kernel_times(run.st)
+    kept_slots, kept_frac = run.kept_slots()
+    status, word = isa.spin_get_error(run.st)
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x} during the timed region")
+    ms_step = ms / K
+    rows_s = world * Q * K / (ms / 1e3)
+    key_gbs = kept_slots * KEY_BYTES_PER_SLOT / (ms_step / 1e3) / 1e9
+    peak, peak_kind = peaks()
+    score_ms, score_n = stages["score"]
+    score_avg = score_ms / max(score_n, 1)
+    achieved = kept_slots * SCORE_BYTES_PER_SLOT / (score_avg / 1e3) / 1e9
+    launches = sum(n for _, n in stages.values())
+    out = {
+        "metric": METRIC, "value": rows_s, "unit": "rows/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3xe4m3->f32 (selection f32, exact)", "data": "synthetic",
+        "config": {"workload": wl.name, "requests_per_gpu": Q, "context_slots": wl.ctx0[0], "block_size": wl.b,
+                   "heads": wl.H, "head_dim": wl.d, "topk": wl.topk, "target_sparsity": args.sparsity,
+                   "gamma": wl.gamma, "parallelism": f"dp{world} (requests sharded, no collective)",
+                   "l2": "inputs larger than L2: 6.4 GB paged FP8 key cache and 0.4 GB EMA state per GPU"},
+        "index_key_gbs": key_gbs,
+        "key_roofline_frac": key_gbs / peak,
+        "roofline": {"bound": "hbm", "kernel": "k_score_tc (paged FP8 indexer + fused EMA)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} hbm_gbs (copy, MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s", "avg_launch_ms": score_avg,
+                     "bytes_per_launch": kept_slots * SCORE_BYTES_PER_SLOT, "traffic": None},
+        "stage_ms_per_step": {k: v[0] / K for k, v in stages.items() if v[1]},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    # ---- sparsity sweep: 40% and the 0% all-keep control ------------------
+    sw = {str(int(round(args.sparsity * 100))): ms_step}
+    for s in sweep:
+        run.set_sparsity(s)
+        for _ in range(W):
+            run.step(defer=(s == 0.0))
+        sw[str(int(round(s * 100)))] = timed_steps(run, K, world, defer=(s == 0.0)) / K
+    if sweep:
+        out["sweep_ms_per_step"] = sw
+        out["sweep_monotonic"] = bool(sw.get("0", 1e9) > sw.get("40", 0) > sw.get(str(int(round(args.sparsity * 100))), -1))
+    # ---- fidelity (outside timed regions) ---------------------------------
+    run.set_sparsity(args.sparsity)
+    out["fidelity"] = fidelity(run)
+    # ---- end to end with host buffers --------------------------------------
+    e2e_ms, h2d, d2h = e2e_pass(run, K, world)
+    out["e2e"] = {"value": world * Q * K / (e2e_ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
+    status, word = isa.spin_get_error(run.st)
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """One request of the serving workload on the host, driven by the oracle
+    (fp64 scores, OpenMP over blocks)."""
+
+    def __init__(self, request_seed_offset=0):
+        import oracle
+        self.o = oracle
+        self.o.build()
+        wl = workloads.config(2, requests=1, ctx0=(512 * 1024,), steps=64, seed=2 + request_seed_offset)
+        self.wl = wl
+        cache = workloads.make_key_cache(wl, 0, "cpu")
+        self.keys = cache.keys.numpy()
+        self.ks = cache.kscale.numpy()
+        self.bt = cache.block_table[0].numpy()
+        q, w = workloads.make_queries(wl, 0, wl.steps, "cpu")
+        self.q = q.float().numpy().astype(np.float64)
+        self.w = w.numpy()
+        nb = wl.max_blocks
+        self.V = np.full(nb * wl.b, np.inf, np.float32)
+        self.D = np.full(nb * wl.b, -np.inf, np.float32)
+        self.t = 0
+
+    def step(self, sparsity):
+        wl = self.wl
+        t = self.t % wl.steps
+        ctx = wl.ctx0[0] + t + 1
+        self.o.decode_step_request(V=self.V, D=self.D, ctx_len=ctx, rows=1, b=wl.b, sparsity=sparsity,
+                                   gamma=wl.gamma, alpha=wl.alpha, seed=wl.seed, request=0, layer=0, step=self.t,
+                                   topk=wl.topk, q=self.q[0, t:t + 1], w=self.w[0, t:t + 1], keys=self.keys,
+                                   kscale=self.ks, block_table=self.bt, key_fp8=True)
+        self.t += 1
+
+
+def threads_used():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(sparsity, seconds):
+    smp = OracleSample()
+    smp.step(0.0)                      # history bootstrap (not timed)
+    n, t0 = 0, time.perf_counter()
+    while n < 2 or time.perf_counter() - t0 < seconds:
+        smp.step(sparsity)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "rows/s", "cores": threads_used(), "kind": "oracle",
+            "sample": f"{n} decode steps of 1 of the 96 requests (512K context, {int(sparsity * 100)}% sparsity) "
+                      f"after an untimed all-keep bootstrap; fp64 scores, OpenMP over blocks; {dt:.1f} s"}
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return None
+    smp = OracleSample()
+    smp.step(0.0)
+    for _ in range(args.warmup):
+        smp.step(args.sparsity)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        smp.step(args.sparsity)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    wl = workloads.config(2)
+    return {"metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "context_slots": wl.ctx0[0], "target_sparsity": args.sparsity,
+                       "sample": "each step: one request of the 96 (the oracle on host cores)"},
+            "cpu_baseline": {"value": value, "unit": "rows/s", "cores": threads_used(), "kind": "oracle",
+                             "sample": f"{args.steps} timed steps of 1 request at 512K after "
+                                       f"{args.warmup} warm-up steps"},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        out = reference_arm(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup()
+    try:
+        out = gpu_arm(args, world, rank, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(args.sparsity, args.cpu_seconds)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

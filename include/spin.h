@@ -1,0 +1,249 @@
+/*
+ * spin.h -- C ABI of libspin.so, the SPIN (Shadow Predictive Indexer) decode
+ * step on NVIDIA B200 (sm_100a).
+ *
+ * SPIN predicts which paged-KV blocks the indexer of a DSA-style sparse
+ * attention layer will find important, scores only those blocks, takes the
+ * token top-k for core attention and keeps the predictor's history fresh.
+ * Sources, cited by page and section:
+ *   SPIN digest   -- ai4snews digest "SPIN用历史索引分数预测KV块重要性..." (核心概要,
+ *                    arXiv深度剖析, 启示与展望)
+ *   SPIN listing  -- thelatestinai listing "SaveSPIN: Shadow Predictive Indexer
+ *                    for Sparse Attention" (Abstract, Figures 1-4, Tables 1-7)
+ *   SPIN v3 record-- paperdot record of arXiv:2610.09025 v3 (摘要)
+ *   AI Radio      -- AI Radio episode "SPIN: Shadow Predictive Indexer for
+ *                    Sparse Attention" ("Title and authors", "The paper's summary")
+ * The indexer formula is the DSA lightning indexer
+ *   I_{r,s} = sigma_s * sum_h w_{r,h} * ReLU(q_{r,h} . k8_s).
+ *
+ * Conventions (every call):
+ *  - Device pointers are owned by the caller (allocate them with any CUDA
+ *    allocator, e.g. PyTorch).  Pointers documented as *_host are host memory.
+ *  - Every call is asynchronous on the given stream and never synchronises,
+ *    except spin_get_error and the export / import calls.  No call allocates
+ *    device memory: all scratch lives in the block handed to spin_state_create.
+ *  - Argument errors are reported synchronously through the return value and
+ *    launch nothing.  Errors only visible on the device (a ctx_len past the
+ *    capacity, a page id outside the cache, an accepted length outside 1..rows,
+ *    a bounded wait that gave up) set a device error word and skip the
+ *    affected work; they never trap.  spin_get_error reads and clears it.
+ *  - Results are deterministic for a given (seed, step, inputs).
+ *  - A state is not thread-safe; use it from one stream at a time.
+ *
+ * Positions: ctx_len[q] is the number of slots visible to query row 0 of
+ * request q, including that row's own key (already in the cache).  Row r
+ * (MTP verification rows, r < rows) sits at position p_r = ctx_len - 1 + r
+ * and sees slots 0..p_r.  Logical block j holds slots j*b .. j*b + b - 1.
+ */
+#ifndef SPIN_H_
+#define SPIN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPIN_API __attribute__((visibility("default")))
+#else
+#define SPIN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* spin_stream_t;
+
+typedef enum {
+  SPIN_OK = 0,
+  SPIN_EINVAL = 1,       /* bad argument; nothing was launched */
+  SPIN_ENOMEM = 2,       /* the caller's state block is smaller than spin_state_bytes() */
+  SPIN_ECUDA = 3,        /* a CUDA runtime call failed */
+  SPIN_ESTATE = 4,       /* NULL or destroyed state handle */
+  SPIN_ETIMEOUT = 5,     /* a device-side bounded wait gave up (device error word) */
+  SPIN_EDEVICE = 6,      /* a device-side argument check failed (device error word) */
+  SPIN_EUNSUPPORTED = 7  /* shape not supported by the requested kernel */
+} spin_status;
+
+typedef enum { SPIN_F32 = 0, SPIN_BF16 = 1, SPIN_FP8_E4M3 = 2 } spin_dtype;
+
+/* Score kernel choice (spin_set_score_kernel). */
+typedef enum {
+  SPIN_SCORE_AUTO = 0,   /* tcgen05 when the shape allows it, else SIMT */
+  SPIN_SCORE_SIMT = 1,   /* CUDA-core kernel: any supported shape, fp32 or FP8 keys */
+  SPIN_SCORE_TCGEN05 = 2 /* TMA + tcgen05 FP8 MMA with TMEM accumulators:
+                            FP8 keys, head_dim 128, block_size 64,
+                            rows * num_heads a multiple of 16 and <= 256 */
+} spin_score_kernel;
+
+typedef struct {
+  int32_t num_layers;      /* EMA states kept per layer */
+  int32_t num_requests;    /* Q: request slots */
+  int32_t max_slots;       /* KV capacity per request (slots) */
+  int32_t block_size;      /* b: paged-KV block size (AI Radio, "Title and authors") */
+  int32_t num_heads;       /* H: indexer heads */
+  int32_t head_dim;        /* d: indexer key / query width */
+  int32_t topk;            /* k: tokens handed to core attention */
+  int32_t max_rows;        /* 1..4 query rows per step (1 verify + drafts) */
+  int32_t key_dtype;       /* SPIN_F32 or SPIN_FP8_E4M3 (+ per-token fp32 scale) */
+  int32_t q_dtype;         /* SPIN_F32 or SPIN_BF16 (SPIN_F32 keys need SPIN_F32 queries) */
+  float alpha;             /* EMA decay: x <- alpha*x + (1-alpha)*score */
+  float gamma;             /* exploration share of the block budget (SPIN listing, Figure 4) */
+  float target_sparsity;   /* default per-layer target block sparsity, [0, 1) */
+  uint64_t seed;           /* exploration RNG seed (Philox4x32-10 key) */
+} spin_config;
+
+typedef struct spin_state_s* spin_state;
+
+/* Bytes of device memory a state needs: EMA states V and D for every layer
+ * and request, block-score / work-list / quantised-query / score scratch and
+ * the device error word.  Returns 0 for an invalid config. */
+SPIN_API size_t spin_state_bytes(const spin_config* cfg);
+
+/* Creates a state in the caller's device block dev_mem (>= spin_state_bytes,
+ * 256-byte aligned; the caller keeps ownership and must keep it alive until
+ * spin_state_destroy).  V is set to +inf and D to -inf (never observed) on
+ * `stream`.  The handle itself is host memory owned by the library. */
+SPIN_API spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t bytes,
+                              spin_stream_t stream, spin_state* out);
+
+/* Frees the host handle only; dev_mem stays the caller's. */
+SPIN_API spin_status spin_state_destroy(spin_state st);
+
+/* Per-layer target block sparsity s_l in [0, 1), from host memory
+ * [num_layers].  s_l = 0 is the all-keep control (no prediction, no
+ * exploration).  Used by the per-layer budget of the SPIN v3 record (摘要). */
+SPIN_API spin_status spin_set_layer_sparsity(spin_state st, const float* s_host);
+
+/* Selects the score kernel used by spin_indexer_score / spin_decode_step. */
+SPIN_API spin_status spin_set_score_kernel(spin_state st, int kind);
+
+/* Sets V = +inf, D = -inf for requests req_host[0..n) of one layer (layer <
+ * 0: every layer), e.g. when a slot starts a new sequence. */
+SPIN_API spin_status spin_reset_requests(spin_state st, int layer, const int32_t* req_host, int n,
+                                spin_stream_t stream);
+
+/* a1 + a2: predicted slot score z = max(V_i, D_{p_r - i}) (AI Radio, "Title
+ * and authors"; SPIN digest, arXiv深度剖析), block max-pool S_{r,j}, block
+ * budget B_r = n_r - floor(s * n_r), exploration share n_exp = floor(gamma *
+ * B_0) of uniformly random unkept blocks (SPIN digest, arXiv深度剖析; SPIN
+ * listing, Figure 4), and for rows > 1 the union of the rows' predicted sets
+ * (SPIN listing, Table 7).  Ties go to the lower block index.
+ *   ctx_len_dev [Q] int32, mask_dev [Q][max_blocks] uint8 out:
+ *   0 skipped, 1 predicted, 2 explored (blocks past the last row's range: 0).
+ *   step: decode step, part of the exploration RNG counter. */
+SPIN_API spin_status spin_predict_select(spin_state st, int layer, int rows, int64_t step,
+                                const int32_t* ctx_len_dev, uint8_t* mask_dev,
+                                spin_stream_t stream);
+
+/* a0 + a3: indexer scores on the kept blocks only (SPIN listing, Abstract;
+ * SPIN digest, arXiv深度剖析).
+ *   keys [num_pages][b][d]: uint8 E4M3 codes (key_dtype FP8) or fp32;
+ *   key_scale [num_pages][b] fp32 per-token scale (FP8 keys; NULL for fp32);
+ *   block_table [Q][bt_stride] int32 logical block -> page;
+ *   q [Q][rows][H][d] in q_dtype; w [Q][rows][H] fp32 head weights;
+ *   mask_dev as written by spin_predict_select;
+ *   scores_dev [Q][max_rows][max_slots_padded] fp32 out, with
+ *   max_slots_padded = ceil(max_slots / b) * b (spin_score_stride); only
+ *   entries of kept blocks with s <= p_r are written.
+ * FP8 keys: each (row, head) query is quantised to E4M3 with a power-of-two
+ * scale folded into its head weight; accumulation is fp32. */
+SPIN_API spin_status spin_indexer_score(spin_state st, int layer, int rows, const void* keys,
+                               const float* key_scale, int32_t num_pages,
+                               const int32_t* block_table, int32_t bt_stride, const void* q,
+                               const float* w, const int32_t* ctx_len_dev,
+                               const uint8_t* mask_dev, float* scores_dev, spin_stream_t stream);
+
+/* a4: token top-k per (request, row) over the scored slots (SPIN digest,
+ * arXiv深度剖析: the fixed top-k budget of core attention is unchanged).
+ * Higher score first, ties to the lower slot; emitted in ascending slot
+ * order; padded with -1.  topk_dev [Q][rows][k] int32 out. */
+SPIN_API spin_status spin_topk(spin_state st, int rows, const float* scores_dev, const uint8_t* mask_dev,
+                      const int32_t* ctx_len_dev, int32_t* topk_dev, spin_stream_t stream);
+
+/* a5: EMA update of V (per slot) and D (per offset p_r - s) from the scores
+ * of scored slots only (SPIN digest, 核心概要 / arXiv深度剖析; AI Radio, "The
+ * paper's summary").  x <- score if x is the never-observed sentinel, else
+ * fmaf(alpha, x, (1 - alpha) * score).  Rows 0..accepted[q]-1 are replayed in
+ * order (prefix-valid update of MTP rows, SPIN digest, arXiv深度剖析).
+ * accepted_dev [Q] int32 in 1..rows, or NULL for all rows. */
+SPIN_API spin_status spin_ema_update(spin_state st, int layer, int rows, const float* scores_dev,
+                            const uint8_t* mask_dev, const int32_t* ctx_len_dev,
+                            const int32_t* accepted_dev, spin_stream_t stream);
+
+/* a0..a5 fused on one stream: quantise q, predict + select (skipped at
+ * sparsity 0), score, top-k and -- unless defer_update -- the EMA update of
+ * all rows.  With defer_update the caller calls spin_ema_update once the
+ * accepted lengths are known.  scores_dev may be NULL (internal scratch) when
+ * defer_update is 0. */
+SPIN_API spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, const void* keys,
+                             const float* key_scale, int32_t num_pages, const int32_t* block_table,
+                             int32_t bt_stride, const void* q, const float* w,
+                             const int32_t* ctx_len_dev, int defer_update, uint8_t* mask_dev,
+                             int32_t* topk_dev, float* scores_dev, spin_stream_t stream);
+
+/* Miss count of the fidelity metric (SPIN listing, Table 5 caption): for each
+ * (request, row), the number of entries of full_topk_dev [Q][rows][k] (a
+ * full-indexer top-k, -1 padded) whose block is skipped in mask_dev.
+ *   missed_dev [Q][rows] int32 out; total_dev [Q][rows] int32 out (entries >= 0). */
+SPIN_API spin_status spin_miss_count(spin_state st, int rows, const int32_t* full_topk_dev,
+                            const uint8_t* mask_dev, int32_t* missed_dev, int32_t* total_dev,
+                            spin_stream_t stream);
+
+/* Host-side per-layer budget (SPIN v3 record, 摘要: the block budget is spread
+ * over layers by their measured miss rates).  Kept fraction
+ * f_l = clamp(c * (miss_l + 1e-3), lo_l, 1) with c such that
+ * sum f_l * blocks_l = (1 - s_glob) * sum blocks_l; if the floors alone
+ * exceed the budget, f_l = lo_l.  s_out_host[l] = 1 - f_l.  No state, no GPU. */
+SPIN_API spin_status spin_allocate_layer_sparsity(int num_layers, const double* miss_host,
+                                         const double* blocks_host, const double* lo_host,
+                                         double s_glob, float* s_out_host);
+
+/* Per-stage timing and launch counts of the library's own kernels.
+ * Stages: 0 predict + pool, 1 select, 2 query quantisation, 3 indexer score,
+ * 4 top-k, 5 EMA update (standalone), 6 mask compaction, 7 miss count.
+ * With timing enabled, every launch is bracketed by two CUDA events recorded
+ * on the launch's stream.  spin_kernel_times synchronises on the recorded
+ * events, writes the summed milliseconds and the launch counts since the last
+ * call into ms_out[n] / launches_out[n] (either may be NULL; n <= 8) and
+ * resets both.  Launches are counted whether or not timing is enabled. */
+SPIN_API spin_status spin_set_kernel_timing(spin_state st, int enable);
+SPIN_API spin_status spin_kernel_times(spin_state st, double* ms_out, int64_t* launches_out, int n);
+
+/* Test hook for the device error path.  mode 1: on its next launch, CTA 0
+ * of the tensor-core score kernel withholds the copy of its first key stage,
+ * so the matrix-issue thread's bounded wait (2 s) runs out; the kernel then
+ * raises ERR_TIMEOUT in the device error word, drains its copies, frees its
+ * tensor memory and returns, and the call's outputs are incomplete.  The
+ * mode resets to 0 after one launch.  mode 0: off. */
+SPIN_API spin_status spin_set_fault_injection(spin_state st, int mode);
+
+/* Synchronises `stream`, then reads and clears the device error word:
+ * SPIN_OK, SPIN_EDEVICE or SPIN_ETIMEOUT.  Optionally returns the raw word. */
+SPIN_API spin_status spin_get_error(spin_state st, spin_stream_t stream, uint32_t* word_out);
+
+SPIN_API const char* spin_status_string(spin_status s);
+
+/* Checkpoint of the EMA state (V and D of every layer): export_bytes() bytes,
+ * copied synchronously through host memory on `stream`. */
+SPIN_API size_t spin_state_export_bytes(spin_state st);
+SPIN_API spin_status spin_state_export(spin_state st, void* host, size_t bytes, spin_stream_t stream);
+SPIN_API spin_status spin_state_import(spin_state st, const void* host, size_t bytes, spin_stream_t stream);
+
+/* Inspection: device pointers into the state block.
+ *   spin_state_ema: V, D of `layer`, each [Q][*stride] fp32.
+ *   spin_state_block_scores: S [Q][max_rows][*stride] fp32 of the last predict.
+ *   spin_state_qquant: quantised queries [Q][max_rows][H][d] E4M3 and their
+ *   folded head weights [Q][max_rows][H] fp32 of the last FP8 score call.
+ *   spin_score_stride: slot stride of a score row (ceil(max_slots/b)*b);
+ *   spin_mask_stride: block stride of a mask row (ceil(max_slots/b)). */
+SPIN_API spin_status spin_state_ema(spin_state st, int layer, float** V, float** D, int64_t* stride);
+SPIN_API spin_status spin_state_block_scores(spin_state st, const float** S, int64_t* stride);
+SPIN_API spin_status spin_state_qquant(spin_state st, const uint8_t** q8, const float** wq);
+SPIN_API int64_t spin_score_stride(spin_state st);
+SPIN_API int64_t spin_mask_stride(spin_state st);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPIN_H_ */

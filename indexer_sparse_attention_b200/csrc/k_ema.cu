@@ -1,0 +1,188 @@
+// k_ema.cu -- a5 EMA update, state initialisation and the miss counter.
+//
+// a5: only slots that were scored update the state (SPIN digest, 核心概要 and
+//     arXiv深度剖析; AI Radio episode, "The paper's summary": skipped blocks get
+//     no update).  V_s and D_{p_r - s} move toward the observed score I_{r,s}:
+//     x <- I if x is the never-observed sentinel (V: +inf, D: -inf), else
+//     fmaf(alpha, x, beta * I), beta = fl32(1 - alpha).  For speculative rows
+//     the update waits for the accepted length a and replays rows 0..a-1 in
+//     order (SPIN digest, arXiv深度剖析: prefix-valid replay).
+//
+// Parallel layout: one warp per block j of a request.  The vertical state of
+// a slot is owned by the slot (its rows run in order inside one thread); the
+// diagonal state D_delta is owned by the block of row 0's slot
+// s_0 = p_0 - delta, and its rows r = 0..a-1 (slot s_0 + r) run in order
+// inside one thread.  Offsets delta > p_0 (only later rows see them) belong to
+// block 0.  Every (row, slot) pair is applied exactly once, in row order.
+#include <algorithm>
+
+#include "spin_internal.cuh"
+
+namespace spin {
+
+__global__ void k_fill(float* V, float* D, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    V[i] = __int_as_float(0x7f800000);
+    D[i] = __int_as_float(0xff800000);
+  }
+}
+
+cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  if (blocks < 1) blocks = 1;
+  k_fill<<<(int)blocks, 256, 0, s>>>(V, D, n);
+  return cudaGetLastError();
+}
+
+__global__ void k_reset_rows(float* V, float* D, ReqList list, int64_t stride) {
+  for (int k = blockIdx.y; k < list.n; k += gridDim.y) {
+    const int64_t base = (int64_t)list.ids[k] * stride;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < stride; i += (int64_t)gridDim.x * blockDim.x) {
+      V[base + i] = __int_as_float(0x7f800000);
+      D[base + i] = __int_as_float(0xff800000);
+    }
+  }
+}
+
+cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t stride, cudaStream_t s) {
+  dim3 grid((unsigned)std::min<int64_t>((stride + 255) / 256, 1024), (unsigned)list.n);
+  k_reset_rows<<<grid, 256, 0, s>>>(V, D, list, stride);
+  return cudaGetLastError();
+}
+
+template <int R>
+__global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
+  const Layout L = a.lay;
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wid < (int64_t)L.Q * L.max_blocks; wid += nw) {
+    const int q = (int)(wid / L.max_blocks);
+    const int64_t j = wid % L.max_blocks;
+    const int64_t ctx = a.ctx_len[q];
+    if (ctx < 1 || ctx + R - 1 > L.max_slots) continue;
+    int acc = R;
+    if (a.accepted) {
+      acc = a.accepted[q];
+      if (acc < 1 || acc > R) {
+        if (j == 0 && lane == 0) raise_error(a.err, ERR_ACCEPTED, q, (uint32_t)acc);
+        continue;
+      }
+    }
+    const int64_t p0 = ctx - 1;
+    const int64_t n_last = row_blocks(ctx, acc - 1, L.b);
+    if (j >= n_last) continue;
+    const uint8_t* mask = a.mask + (int64_t)q * L.max_blocks;
+    const bool kj = mask[j] != 0;
+    const bool kj1 = (R > 1) && (j + 1 < n_last) && mask[j + 1] != 0;
+    if (!kj && !kj1 && !(R > 1 && j == 0)) continue;
+    float* V = a.V + (int64_t)q * L.slot_stride;
+    float* D = a.D + (int64_t)q * L.slot_stride;
+    const float* sc = a.scores + (int64_t)q * L.R * L.slot_stride;
+    for (int i = lane; i < L.b; i += 32) {
+      const int64_t s = j * L.b + i;
+      // vertical state of slot s, rows in order
+      if (kj) {
+        float v = V[s];
+        bool touched = false;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (r < acc && s <= p0 + r) {
+            v = ema_v(v, sc[(int64_t)r * L.slot_stride + s], a.alpha, a.beta);
+            touched = true;
+          }
+        }
+        if (touched) V[s] = v;
+      }
+      // diagonal state delta = p0 - s (row 0's slot s), rows in order
+      if (s <= p0 && (kj || kj1)) {
+        const int64_t dlt = p0 - s;
+        float dv = D[dlt];
+        bool touched = false;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int64_t sr = s + r;
+          if (r < acc && mask[sr / L.b] != 0) {
+            dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
+            touched = true;
+          }
+        }
+        if (touched) D[dlt] = dv;
+      }
+    }
+    // offsets delta = p0 + m (m >= 1): seen only by rows r >= m at slot r - m
+    if (R > 1 && j == 0 && lane < R - 1) {
+      const int m = lane + 1;
+      const int64_t dlt = p0 + m;
+      float dv = D[dlt];
+      bool touched = false;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (r >= m && r < acc) {
+          const int64_t sr = r - m;
+          if (mask[sr / L.b] != 0) {
+            dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
+            touched = true;
+          }
+        }
+      }
+      if (touched) D[dlt] = dv;
+    }
+  }
+}
+
+cudaError_t launch_ema_update(const EmaArgs& a, cudaStream_t s) {
+  int64_t warps = (int64_t)a.lay.Q * a.lay.max_blocks;
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  switch (a.rows) {
+    case 1: k_ema_update<1><<<(int)blocks, 256, 0, s>>>(a); break;
+    case 2: k_ema_update<2><<<(int)blocks, 256, 0, s>>>(a); break;
+    case 3: k_ema_update<3><<<(int)blocks, 256, 0, s>>>(a); break;
+    default: k_ema_update<4><<<(int)blocks, 256, 0, s>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+// Miss counter of the fidelity metric: per (request, row), the entries of a
+// full-indexer top-k whose block is skipped (SPIN listing, Table 5 caption).
+__global__ void k_miss_count(Layout L, int rows, const int32_t* topk, const uint8_t* mask,
+                             int32_t* missed, int32_t* total) {
+  const int q = blockIdx.x / rows;
+  const int32_t* t = topk + (int64_t)blockIdx.x * L.k;
+  const uint8_t* m = mask + (int64_t)q * L.max_blocks;
+  int mc = 0, tc = 0;
+  for (int i = threadIdx.x; i < L.k; i += blockDim.x) {
+    const int32_t s = t[i];
+    if (s < 0) continue;
+    ++tc;
+    const int64_t j = s / L.b;
+    if (j >= L.max_blocks || m[j] == 0) ++mc;
+  }
+  __shared__ int red[2][32];
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    mc += __shfl_xor_sync(0xffffffffu, mc, o);
+    tc += __shfl_xor_sync(0xffffffffu, tc, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = mc;
+    red[1][threadIdx.x >> 5] = tc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0, b = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { a += red[0][w]; b += red[1][w]; }
+    missed[blockIdx.x] = a;
+    total[blockIdx.x] = b;
+  }
+}
+
+cudaError_t launch_miss_count(const Layout& L, int rows, const int32_t* full_topk,
+                              const uint8_t* mask, int32_t* missed, int32_t* total, cudaStream_t s) {
+  k_miss_count<<<L.Q * rows, 256, 0, s>>>(L, rows, full_topk, mask, missed, total);
+  return cudaGetLastError();
+}
+
+}  // namespace spin

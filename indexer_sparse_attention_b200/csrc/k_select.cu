@@ -1,0 +1,295 @@
+// k_select.cu -- a1 predict + block max-pool, a2 budget / predicted top /
+// exploration / row union, and mask compaction.
+//
+// a1: z_{r,i} = max(V_i, D_{p_r - i}) and S_{r,j} = max over the valid slots
+//     of block j (AI Radio episode, "Title and authors"; SPIN digest,
+//     arXiv深度剖析: per-slot and per-offset EMA states).  HBM-bound: 8 bytes
+//     per slot of context (V and D read once for all rows).
+// a2: block budget B_r = n_r - floor(s n_r); a share n_exp = floor(gamma B_0)
+//     of it goes to uniformly random unkept blocks (SPIN digest, arXiv深度剖析;
+//     SPIN listing, Figure 4); each row's top (B_r - n_exp) blocks are unioned
+//     (SPIN listing, Table 7, "Row-local union").  Ties: lower block index.
+#include "spin_internal.cuh"
+#include "block_scan.cuh"
+
+namespace spin {
+
+// ---------------------------------------------------------------------------
+// a1: one warp per pair of blocks of one request; each half-warp pools one
+// block of up to 64 slots, 4 slots per lane, float4 loads of V, scalar
+// (coalesced, reversed) loads of the D window shared by all rows.
+// Block sizes 16..256 (powers of two): larger blocks loop in 64-slot chunks.
+// ---------------------------------------------------------------------------
+template <int R>
+__global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
+  const Layout L = a.lay;
+  const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
+  const int64_t pairs = (L.max_blocks + 1) / 2;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wid < (int64_t)L.Q * pairs; wid += nwarps) {
+    const int q = (int)(wid / pairs);
+    const int64_t j = (wid % pairs) * 2 + half;
+    const int64_t ctx = a.ctx_len[q];
+    if (ctx < 1 || ctx + R - 1 > L.max_slots) continue;  // warp-uniform; select reports it
+    const int64_t n_last = row_blocks(ctx, R - 1, L.b);
+    const int64_t p0 = ctx - 1;
+    const float* V = a.V + (int64_t)q * L.slot_stride;
+    const float* D = a.D + (int64_t)q * L.slot_stride;
+    float m[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) m[r] = __int_as_float(0xff800000);
+    const bool active = j < n_last;
+    for (int c0 = 0; c0 < L.b; c0 += 64) {
+      const int64_t i0 = j * L.b + c0 + l16 * 4;
+      if (active && c0 + l16 * 4 < L.b && i0 <= p0 + R - 1) {
+        const float4 v = *reinterpret_cast<const float4*>(V + i0);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+        // D window: offsets p0 - i0 - 3 .. p0 - i0 + R - 1
+        float dw[R + 3];
+#pragma unroll
+        for (int t = 0; t < R + 3; ++t) {
+          const int64_t di = p0 - i0 - 3 + t;
+          dw[t] = (di >= 0) ? __ldg(D + di) : __int_as_float(0xff800000);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            // slot i0+k, offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + 3]
+            if (i0 + k <= p0 + r) m[r] = fmaxf(m[r], fmaxf(vv[k], dw[r - k + 3]));
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float x = m[r];
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      if (active && l16 == 0 && j < row_blocks(ctx, r, L.b))
+        a.S[((int64_t)q * L.R + r) * L.blk_stride + j] = x;
+    }
+  }
+}
+
+cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
+  const int64_t pairs = (a.lay.max_blocks + 1) / 2;
+  int64_t warps = (int64_t)a.lay.Q * pairs;
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  switch (a.rows) {
+    case 1: k_predict_pool<1><<<(int)blocks, 256, 0, s>>>(a); break;
+    case 2: k_predict_pool<2><<<(int)blocks, 256, 0, s>>>(a); break;
+    case 3: k_predict_pool<3><<<(int)blocks, 256, 0, s>>>(a); break;
+    default: k_predict_pool<4><<<(int)blocks, 256, 0, s>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// a2: one CTA (1024 threads) per request.  Keys of the candidates live in
+// shared memory; an MSB-first radix select (4 x 8-bit digits) finds the
+// threshold key T of the wanted rank and how many elements equal to T to
+// take; an ordered pass then takes every key > T and the lowest-index keys
+// == T.  Exploration reuses the same routine on ~Philox keys of the unkept
+// blocks (largest ~key = smallest key).  Finally the mask row and the
+// ascending kept-block list are written.
+// ---------------------------------------------------------------------------
+constexpr int kSelThreads = 1024;
+
+struct SelShared {
+  uint32_t hist[256];
+  uint32_t digit[2];
+  int scan[33];
+};
+
+// Radix select over keys[0..n) restricted to elements with valid(j).  `want`
+// must be in [1, #valid].  Returns T and the number of elements equal to T
+// that belong to the top `want`.
+template <class Valid>
+__device__ void radix_select_desc(const uint32_t* keys, int n, Valid valid, uint32_t want,
+                                  SelShared& sh, uint32_t* T_out, uint32_t* eq_out) {
+  uint32_t prefix = 0, pmask = 0, remaining = want;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+      if (!valid(j)) continue;
+      const uint32_t k = keys[j];
+      if ((k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) warp_find_digit_desc<256>(sh.hist, remaining, sh.digit);
+    __syncthreads();
+    prefix |= sh.digit[0] << shift;
+    pmask |= 255u << shift;
+    remaining = sh.digit[1];
+    __syncthreads();
+  }
+  *T_out = prefix;
+  *eq_out = remaining;
+}
+
+// Marks m[j] = label for the top `want` valid elements (keys > T, then the
+// lowest-index keys == T).  Each thread walks a contiguous chunk so that the
+// "lowest index" order is a block scan.
+template <class Valid>
+__device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t T, uint32_t eq_take,
+                              uint8_t* m, uint8_t label, SelShared& sh) {
+  const int chunk = (n + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * chunk, hi = min(n, lo + chunk);
+  int eq = 0;
+  for (int j = lo; j < hi; ++j)
+    if (valid(j) && keys[j] == T) ++eq;
+  int total;
+  int base = block_exclusive_scan(eq, sh.scan, &total);
+  for (int j = lo; j < hi; ++j) {
+    if (!valid(j)) continue;
+    const uint32_t k = keys[j];
+    if (k > T) {
+      m[j] = label;
+    } else if (k == T) {
+      if ((uint32_t)base < eq_take) m[j] = label;
+      ++base;
+    }
+  }
+  __syncthreads();
+}
+
+// Ordered compaction of the kept blocks of one request into its work list.
+__device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t* kept, int* scan) {
+  const int chunk = (n_last + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * chunk, hi = min(n_last, lo + chunk);
+  int c = 0;
+  for (int j = lo; j < hi; ++j) c += m[j] != 0;
+  int total;
+  int pos = block_exclusive_scan(c, scan, &total);
+  for (int j = lo; j < hi; ++j)
+    if (m[j]) work[pos++] = j;
+  if (threadIdx.x == 0) *kept = total;
+}
+
+__global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
+  const Layout L = a.lay;
+  const int q = blockIdx.x;
+  extern __shared__ __align__(16) uint8_t dyn[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);
+  uint8_t* m = dyn + 4 * L.blk_stride;
+  __shared__ SelShared sh;
+
+  const int64_t ctx = a.ctx_len[q];
+  uint8_t* mask_row = a.mask + (int64_t)q * L.max_blocks;
+  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {
+    if (threadIdx.x == 0) {
+      raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
+      a.kept[q] = 0;
+    }
+    for (int64_t j = threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = 0;
+    return;
+  }
+  const int n_last = (int)row_blocks(ctx, a.rows - 1, L.b);
+  for (int j = threadIdx.x; j < n_last; j += blockDim.x) m[j] = 0;
+  __syncthreads();
+
+  if (a.sparsity == 0.0f) {
+    for (int j = threadIdx.x; j < n_last; j += blockDim.x) m[j] = 1;
+    __syncthreads();
+  } else {
+    const int64_t n0 = row_blocks(ctx, 0, L.b);
+    const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
+    for (int r = 0; r < a.rows; ++r) {
+      const int n = (int)row_blocks(ctx, r, L.b);
+      const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
+      const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride;
+      for (int j = threadIdx.x; j < n; j += blockDim.x) keys[j] = fkey(S[j]);
+      __syncthreads();
+      auto all = [](int) { return true; };
+      if (n_pred >= n) {
+        for (int j = threadIdx.x; j < n; j += blockDim.x) m[j] = 1;
+        __syncthreads();
+      } else if (n_pred > 0) {
+        uint32_t T, eq;
+        radix_select_desc(keys, n, all, (uint32_t)n_pred, sh, &T, &eq);
+        mark_selected(keys, n, all, T, eq, m, 1, sh);
+      }
+    }
+    // exploration among the unkept blocks of the last row's range
+    auto cand = [m](int j) { return m[j] == 0; };
+    int c = 0;
+    for (int j = threadIdx.x; j < n_last; j += blockDim.x) c += (m[j] == 0);
+    int n_cand;
+    block_exclusive_scan(c, sh.scan, &n_cand);
+    const int64_t take = n_exp < n_cand ? n_exp : n_cand;
+    if (take > 0) {
+      for (int j = threadIdx.x; j < n_last; j += blockDim.x)
+        keys[j] = ~explore_key(a.seed, (uint32_t)j, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
+      __syncthreads();
+      if (take == n_cand) {
+        for (int j = threadIdx.x; j < n_last; j += blockDim.x)
+          if (m[j] == 0) m[j] = 2;
+        __syncthreads();
+      } else {
+        uint32_t T, eq;
+        radix_select_desc(keys, n_last, cand, (uint32_t)take, sh, &T, &eq);
+        // mark into a separate pass: `cand` reads m, so label after the scan
+        const int chunk = (n_last + blockDim.x - 1) / blockDim.x;
+        const int lo = threadIdx.x * chunk, hi = min(n_last, lo + chunk);
+        int e = 0;
+        for (int j = lo; j < hi; ++j)
+          if (m[j] == 0 && keys[j] == T) ++e;
+        int tot;
+        int base = block_exclusive_scan(e, sh.scan, &tot);
+        for (int j = lo; j < hi; ++j) {
+          if (m[j] != 0) continue;
+          if (keys[j] > T) {
+            m[j] = 2;
+          } else if (keys[j] == T) {
+            if ((uint32_t)base < eq) m[j] = 2;
+            ++base;
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+  for (int64_t j = threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = j < n_last ? m[j] : 0;
+  compact_row(m, n_last, a.work + (int64_t)q * L.blk_stride, a.kept + q, sh.scan);
+}
+
+cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
+  const size_t smem = (size_t)a.lay.blk_stride * 5;
+  cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_select<<<a.lay.Q, kSelThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Compaction of a caller-given mask into the work list (standalone score /
+// top-k calls).  One CTA per request.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_compact(Layout L, int rows, const int32_t* ctx_len,
+                                                  const uint8_t* mask, int32_t* work, int32_t* kept,
+                                                  ErrWord* err) {
+  __shared__ int scan[33];
+  const int q = blockIdx.x;
+  const int64_t ctx = ctx_len[q];
+  if (ctx < 1 || ctx + rows - 1 > L.max_slots) {
+    if (threadIdx.x == 0) {
+      raise_error(err, ERR_CTX_LEN, q, (uint32_t)ctx);
+      kept[q] = 0;
+    }
+    return;
+  }
+  const int n_last = (int)row_blocks(ctx, rows - 1, L.b);
+  compact_row(mask + (int64_t)q * L.max_blocks, n_last, work + (int64_t)q * L.blk_stride, kept + q, scan);
+}
+
+cudaError_t launch_compact(const Layout& L, int rows, const int32_t* ctx_len, const uint8_t* mask,
+                           int32_t* work, int32_t* kept, ErrWord* err, cudaStream_t s) {
+  k_compact<<<L.Q, 1024, 0, s>>>(L, rows, ctx_len, mask, work, kept, err);
+  return cudaGetLastError();
+}
+
+}  // namespace spin

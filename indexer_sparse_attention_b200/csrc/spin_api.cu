@@ -1,0 +1,612 @@
+// spin_api.cu -- host side of the libspin.so C ABI (include/spin.h):
+// argument validation, carving of the caller's state block, kernel launches
+// and the fused decode step.  No call allocates device memory.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "spin_internal.cuh"
+
+using namespace spin;
+
+struct spin_state_s {
+  spin_config cfg;
+  Layout lay;
+  char* base;
+  size_t bytes;
+  ErrWord* err;
+  float* V;       // [L][Q][slot_stride]
+  float* D;
+  float* S;       // [Q][R][blk_stride]
+  int32_t* work;  // [Q][blk_stride]
+  int32_t* kept;  // [Q]
+  uint8_t* q8;    // [Q][R][H][d]
+  float* wq;      // [Q][R][H]
+  float* scores;  // [Q][R][slot_stride]
+  std::vector<float> sparsity;
+  int score_kernel;
+  int inject;
+  void* encode_fn;  // cuTensorMapEncodeTiled, resolved at create
+  // per-stage timing (spin_set_kernel_timing / spin_kernel_times)
+  bool timing;
+  struct Rec { int stage; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  int64_t launches[8];
+  uint32_t magic;
+};
+
+namespace {
+
+constexpr uint32_t kMagic = 0x5350494eu;  // "SPIN"
+constexpr int64_t kMaxBlocksSelect = 40960;  // K2 keeps S and the mask of a request on chip
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool valid_config(const spin_config* c) {
+  if (!c) return false;
+  if (c->num_layers < 1 || c->num_requests < 1 || c->max_slots < 1) return false;
+  const int b = c->block_size;
+  if (b < 16 || b > 256 || (b & (b - 1))) return false;
+  if (c->num_heads < 1 || c->num_heads > 256 || c->head_dim < 1 || c->head_dim > 512) return false;
+  if (c->topk < 1 || c->topk > 65536) return false;
+  if (c->max_rows < 1 || c->max_rows > 4) return false;
+  if (c->key_dtype != SPIN_F32 && c->key_dtype != SPIN_FP8_E4M3) return false;
+  if (c->q_dtype != SPIN_F32 && c->q_dtype != SPIN_BF16) return false;
+  if (c->key_dtype == SPIN_F32 && c->q_dtype != SPIN_F32) return false;
+  if (c->key_dtype == SPIN_FP8_E4M3 && (c->head_dim % 16)) return false;
+  if (!(c->alpha >= 0.0f && c->alpha <= 1.0f)) return false;
+  if (!(c->gamma >= 0.0f && c->gamma <= 1.0f)) return false;
+  if (!(c->target_sparsity >= 0.0f && c->target_sparsity < 1.0f)) return false;
+  const int64_t max_blocks = (c->max_slots + (int64_t)b - 1) / b;
+  if (max_blocks > kMaxBlocksSelect) return false;
+  // top-k bitmap of one (request, row) lives in shared memory
+  if ((max_blocks * b + 31) / 32 * 4 > 200 * 1024) return false;
+  // SIMT score kernel keeps the queries of a request and one page on chip
+  const size_t simt = sizeof(float) * ((size_t)c->max_rows * c->num_heads * c->head_dim +
+                                       (size_t)c->max_rows * c->num_heads + (size_t)b * (c->head_dim + 1));
+  if (simt > 220 * 1024) return false;
+  return true;
+}
+
+Layout make_layout(const spin_config* c) {
+  Layout L;
+  L.L = c->num_layers;
+  L.Q = c->num_requests;
+  L.R = c->max_rows;
+  L.H = c->num_heads;
+  L.d = c->head_dim;
+  L.b = c->block_size;
+  L.k = c->topk;
+  L.max_slots = c->max_slots;
+  L.max_blocks = (c->max_slots + (int64_t)c->block_size - 1) / c->block_size;
+  L.slot_stride = L.max_blocks * c->block_size;
+  L.blk_stride = (L.max_blocks + 15) / 16 * 16;
+  return L;
+}
+
+struct Carve {
+  size_t err, V, D, S, work, kept, q8, wq, scores, total;
+};
+
+Carve carve(const Layout& L) {
+  Carve k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t at = off; off = align256(off + bytes); return at; };
+  k.err = take(sizeof(ErrWord));
+  k.V = take((size_t)L.L * L.Q * L.slot_stride * 4);
+  k.D = take((size_t)L.L * L.Q * L.slot_stride * 4);
+  k.S = take((size_t)L.Q * L.R * L.blk_stride * 4);
+  k.work = take((size_t)L.Q * L.blk_stride * 4);
+  k.kept = take((size_t)L.Q * 4);
+  k.q8 = take((size_t)L.Q * L.R * L.H * L.d);
+  k.wq = take((size_t)L.Q * L.R * L.H * 4);
+  k.scores = take((size_t)L.Q * L.R * L.slot_stride * 4);
+  k.total = off;
+  return k;
+}
+
+bool alive(spin_state st) { return st && st->magic == kMagic; }
+
+spin_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SPIN_OK;
+  fprintf(stderr, "libspin: CUDA error %s\n", cudaGetErrorString(e));
+  return SPIN_ECUDA;
+}
+
+float beta_of(float alpha) { return (float)(1.0 - (double)alpha); }
+
+StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32_t* ctx_len, uint8_t* mask) {
+  StepArgs a;
+  a.lay = st->lay;
+  a.layer = layer;
+  a.rows = rows;
+  a.step = step;
+  a.sparsity = st->sparsity[layer];
+  a.gamma = st->cfg.gamma;
+  a.alpha = st->cfg.alpha;
+  a.seed = st->cfg.seed;
+  a.ctx_len = ctx_len;
+  a.mask = mask;
+  a.S = st->S;
+  a.work = st->work;
+  a.kept = st->kept;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  a.V = st->V + per_layer * layer;
+  a.D = st->D + per_layer * layer;
+  a.err = st->err;
+  return a;
+}
+
+bool use_tc(spin_state st, int rows) {
+  const bool ok = tc_supported(st->lay, rows, st->cfg.key_dtype == SPIN_FP8_E4M3) && st->encode_fn;
+  if (st->score_kernel == SPIN_SCORE_SIMT) return false;
+  return ok;
+}
+
+enum Stage { kPredict = 0, kSelect, kQuant, kScore, kTopk, kEma, kCompact, kMiss, kNumStages };
+
+cudaEvent_t take_event(spin_state st) {
+  if (!st->pool.empty()) {
+    cudaEvent_t e = st->pool.back();
+    st->pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launches one kernel, counting it and -- with timing on -- bracketing it by
+// two events on its stream.
+template <class F>
+cudaError_t staged(spin_state st, int stage, cudaStream_t s, F launch) {
+  st->launches[stage] += 1;
+  if (!st->timing) return launch();
+  cudaEvent_t a = take_event(st), b = take_event(st);
+  if (!a || !b) return cudaErrorMemoryAllocation;
+  cudaEventRecord(a, s);
+  cudaError_t e = launch();
+  cudaEventRecord(b, s);
+  st->recs.push_back({stage, a, b});
+  return e;
+}
+
+// Quantise (FP8 keys) and score the kept blocks listed in st->work / st->kept.
+spin_status run_score(spin_state st, int layer, int rows, const void* keys, const float* key_scale,
+                      int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
+                      const float* w, const int32_t* ctx_len, const uint8_t* mask, float* scores,
+                      bool fuse_ema, cudaStream_t stream) {
+  ScoreArgs a;
+  a.lay = st->lay;
+  a.rows = rows;
+  a.key_fp8 = st->cfg.key_dtype == SPIN_FP8_E4M3;
+  a.q_bf16 = st->cfg.q_dtype == SPIN_BF16;
+  a.keys = keys;
+  a.kscale = key_scale;
+  a.num_pages = num_pages;
+  a.block_table = block_table;
+  a.bt_stride = bt_stride;
+  a.q = q;
+  a.w = w;
+  a.ctx_len = ctx_len;
+  a.mask = mask;
+  a.work = st->work;
+  a.kept = st->kept;
+  a.q8 = st->q8;
+  a.wq = st->wq;
+  a.scores = scores;
+  a.err = st->err;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  a.V = fuse_ema ? st->V + per_layer * layer : nullptr;
+  a.D = fuse_ema ? st->D + per_layer * layer : nullptr;
+  a.alpha = st->cfg.alpha;
+  a.beta = beta_of(st->cfg.alpha);
+  a.inject = 0;
+  if (a.key_fp8) {
+    spin_status s = cuda_status(staged(st, kQuant, stream, [&] { return launch_quantize_q(a, stream); }));
+    if (s != SPIN_OK) return s;
+  }
+  if (st->score_kernel == SPIN_SCORE_TCGEN05 && !use_tc(st, rows)) return SPIN_EUNSUPPORTED;
+  if (use_tc(st, rows)) {
+    a.inject = st->inject;
+    st->inject = 0;
+    return cuda_status(staged(st, kScore, stream, [&] { return launch_score_tc(a, st->encode_fn, stream); }));
+  }
+  return cuda_status(staged(st, kScore, stream, [&] { return launch_score_simt(a, stream); }));
+}
+
+spin_status check_rows(spin_state st, int rows) {
+  return (rows >= 1 && rows <= st->cfg.max_rows) ? SPIN_OK : SPIN_EINVAL;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t spin_state_bytes(const spin_config* cfg) {
+  if (!valid_config(cfg)) return 0;
+  return carve(make_layout(cfg)).total;
+}
+
+spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t bytes, spin_stream_t stream,
+                              spin_state* out) {
+  if (!out) return SPIN_EINVAL;
+  *out = nullptr;
+  if (!valid_config(cfg) || !dev_mem || ((uintptr_t)dev_mem & 255)) return SPIN_EINVAL;
+  const Layout L = make_layout(cfg);
+  const Carve k = carve(L);
+  if (bytes < k.total) return SPIN_ENOMEM;
+  spin_state st = new (std::nothrow) spin_state_s();
+  if (!st) return SPIN_EINVAL;
+  st->cfg = *cfg;
+  st->lay = L;
+  st->base = (char*)dev_mem;
+  st->bytes = bytes;
+  st->err = (ErrWord*)(st->base + k.err);
+  st->V = (float*)(st->base + k.V);
+  st->D = (float*)(st->base + k.D);
+  st->S = (float*)(st->base + k.S);
+  st->work = (int32_t*)(st->base + k.work);
+  st->kept = (int32_t*)(st->base + k.kept);
+  st->q8 = (uint8_t*)(st->base + k.q8);
+  st->wq = (float*)(st->base + k.wq);
+  st->scores = (float*)(st->base + k.scores);
+  st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
+  st->score_kernel = SPIN_SCORE_AUTO;
+  st->inject = 0;
+  st->timing = false;
+  for (int i = 0; i < 8; ++i) st->launches[i] = 0;
+  st->encode_fn = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) == cudaSuccess &&
+      qres == cudaDriverEntryPointSuccess)
+    st->encode_fn = fn;
+  cudaGetLastError();
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(st->err, 0, sizeof(ErrWord), s);
+  if (e == cudaSuccess) e = launch_init_state(st->V, st->D, (int64_t)L.L * L.Q * L.slot_stride, s);
+  if (e != cudaSuccess) {
+    delete st;
+    return cuda_status(e);
+  }
+  st->magic = kMagic;
+  *out = st;
+  return SPIN_OK;
+}
+
+spin_status spin_state_destroy(spin_state st) {
+  if (!alive(st)) return SPIN_ESTATE;
+  for (auto& r : st->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : st->pool) cudaEventDestroy(e);
+  st->magic = 0;
+  delete st;
+  return SPIN_OK;
+}
+
+spin_status spin_set_layer_sparsity(spin_state st, const float* s_host) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (!s_host) return SPIN_EINVAL;
+  for (int l = 0; l < st->cfg.num_layers; ++l)
+    if (!(s_host[l] >= 0.0f && s_host[l] < 1.0f)) return SPIN_EINVAL;
+  st->sparsity.assign(s_host, s_host + st->cfg.num_layers);
+  return SPIN_OK;
+}
+
+spin_status spin_set_score_kernel(spin_state st, int kind) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (kind < SPIN_SCORE_AUTO || kind > SPIN_SCORE_TCGEN05) return SPIN_EINVAL;
+  if (kind == SPIN_SCORE_TCGEN05 && !(tc_supported(st->lay, 1, st->cfg.key_dtype == SPIN_FP8_E4M3) &&
+                                      st->encode_fn))
+    return SPIN_EUNSUPPORTED;
+  st->score_kernel = kind;
+  return SPIN_OK;
+}
+
+spin_status spin_set_kernel_timing(spin_state st, int enable) {
+  if (!alive(st)) return SPIN_ESTATE;
+  st->timing = enable != 0;
+  return SPIN_OK;
+}
+
+spin_status spin_kernel_times(spin_state st, double* ms_out, int64_t* launches_out, int n) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (n < 0 || n > kNumStages) return SPIN_EINVAL;
+  double ms[kNumStages] = {0};
+  cudaError_t err = cudaSuccess;
+  for (auto& r : st->recs) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    ms[r.stage] += t;
+    st->pool.push_back(r.a);
+    st->pool.push_back(r.b);
+  }
+  st->recs.clear();
+  for (int i = 0; i < n; ++i) {
+    if (ms_out) ms_out[i] = ms[i];
+    if (launches_out) launches_out[i] = st->launches[i];
+  }
+  for (int i = 0; i < kNumStages; ++i) st->launches[i] = 0;
+  return cuda_status(err);
+}
+
+spin_status spin_set_fault_injection(spin_state st, int mode) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (mode < 0 || mode > 1) return SPIN_EINVAL;
+  st->inject = mode;
+  return SPIN_OK;
+}
+
+spin_status spin_reset_requests(spin_state st, int layer, const int32_t* req_host, int n,
+                                spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (n < 0 || (n > 0 && !req_host) || layer >= st->cfg.num_layers) return SPIN_EINVAL;
+  if (n == 0) return SPIN_OK;
+  for (int i = 0; i < n; ++i)
+    if (req_host[i] < 0 || req_host[i] >= st->cfg.num_requests) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  for (int i0 = 0; i0 < n; i0 += ReqList::kMax) {
+    ReqList list;
+    list.n = std::min(n - i0, ReqList::kMax);
+    for (int i = 0; i < list.n; ++i) list.ids[i] = req_host[i0 + i];
+    for (int l = 0; l < st->cfg.num_layers; ++l) {
+      if (layer >= 0 && l != layer) continue;
+      cudaError_t e = launch_reset_rows(st->V + per_layer * l, st->D + per_layer * l, list, st->lay.slot_stride, s);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+  }
+  return SPIN_OK;
+}
+
+spin_status spin_predict_select(spin_state st, int layer, int rows, int64_t step,
+                                const int32_t* ctx_len_dev, uint8_t* mask_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || !ctx_len_dev || !mask_dev || step < 0)
+    return SPIN_EINVAL;
+  StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (a.sparsity > 0.0f) {
+    spin_status r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
+    if (r != SPIN_OK) return r;
+  }
+  return cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
+}
+
+spin_status spin_indexer_score(spin_state st, int layer, int rows, const void* keys, const float* key_scale,
+                               int32_t num_pages, const int32_t* block_table, int32_t bt_stride,
+                               const void* q, const float* w, const int32_t* ctx_len_dev,
+                               const uint8_t* mask_dev, float* scores_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows)) return SPIN_EINVAL;
+  if (!keys || !block_table || !q || !w || !ctx_len_dev || !mask_dev || !scores_dev || num_pages < 1 ||
+      bt_stride < st->lay.max_blocks)
+    return SPIN_EINVAL;
+  if (st->cfg.key_dtype == SPIN_FP8_E4M3 && !key_scale) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  spin_status r = cuda_status(staged(st, kCompact, s, [&] {
+    return launch_compact(st->lay, rows, ctx_len_dev, mask_dev, st->work, st->kept, st->err, s);
+  }));
+  if (r != SPIN_OK) return r;
+  return run_score(st, layer, rows, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len_dev,
+                   mask_dev, scores_dev, false, s);
+}
+
+spin_status spin_topk(spin_state st, int rows, const float* scores_dev, const uint8_t* mask_dev,
+                      const int32_t* ctx_len_dev, int32_t* topk_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (check_rows(st, rows) || !scores_dev || !mask_dev || !ctx_len_dev || !topk_dev) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  spin_status r = cuda_status(staged(st, kCompact, s, [&] {
+    return launch_compact(st->lay, rows, ctx_len_dev, mask_dev, st->work, st->kept, st->err, s);
+  }));
+  if (r != SPIN_OK) return r;
+  TopkArgs a{st->lay, rows, scores_dev, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err};
+  return cuda_status(staged(st, kTopk, s, [&] { return launch_topk(a, s); }));
+}
+
+spin_status spin_ema_update(spin_state st, int layer, int rows, const float* scores_dev, const uint8_t* mask_dev,
+                            const int32_t* ctx_len_dev, const int32_t* accepted_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || !scores_dev || !mask_dev || !ctx_len_dev)
+    return SPIN_EINVAL;
+  EmaArgs a;
+  a.lay = st->lay;
+  a.rows = rows;
+  a.scores = scores_dev;
+  a.mask = mask_dev;
+  a.ctx_len = ctx_len_dev;
+  a.accepted = accepted_dev;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  a.V = st->V + per_layer * layer;
+  a.D = st->D + per_layer * layer;
+  a.alpha = st->cfg.alpha;
+  a.beta = beta_of(st->cfg.alpha);
+  a.err = st->err;
+  cudaStream_t s = (cudaStream_t)stream;
+  return cuda_status(staged(st, kEma, s, [&] { return launch_ema_update(a, s); }));
+}
+
+spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, const void* keys,
+                             const float* key_scale, int32_t num_pages, const int32_t* block_table,
+                             int32_t bt_stride, const void* q, const float* w, const int32_t* ctx_len_dev,
+                             int defer_update, uint8_t* mask_dev, int32_t* topk_dev, float* scores_dev,
+                             spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || step < 0) return SPIN_EINVAL;
+  if (!keys || !block_table || !q || !w || !ctx_len_dev || !mask_dev || !topk_dev || num_pages < 1 ||
+      bt_stride < st->lay.max_blocks)
+    return SPIN_EINVAL;
+  if (st->cfg.key_dtype == SPIN_FP8_E4M3 && !key_scale) return SPIN_EINVAL;
+  if (defer_update && !scores_dev) return SPIN_EINVAL;
+  float* scores = scores_dev ? scores_dev : st->scores;
+  cudaStream_t s = (cudaStream_t)stream;
+  StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
+  spin_status r;
+  if (a.sparsity > 0.0f) {
+    r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
+    if (r != SPIN_OK) return r;
+  }
+  r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
+  if (r != SPIN_OK) return r;
+  const bool fuse = !defer_update && rows == 1;
+  r = run_score(st, layer, rows, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len_dev, mask_dev,
+                scores, fuse, s);
+  if (r != SPIN_OK) return r;
+  TopkArgs t{st->lay, rows, scores, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err};
+  r = cuda_status(staged(st, kTopk, s, [&] { return launch_topk(t, s); }));
+  if (r != SPIN_OK) return r;
+  if (!defer_update && rows > 1) return spin_ema_update(st, layer, rows, scores, mask_dev, ctx_len_dev, nullptr, stream);
+  return SPIN_OK;
+}
+
+spin_status spin_miss_count(spin_state st, int rows, const int32_t* full_topk_dev, const uint8_t* mask_dev,
+                            int32_t* missed_dev, int32_t* total_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (check_rows(st, rows) || !full_topk_dev || !mask_dev || !missed_dev || !total_dev) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  return cuda_status(staged(st, kMiss, s, [&] {
+    return launch_miss_count(st->lay, rows, full_topk_dev, mask_dev, missed_dev, total_dev, s);
+  }));
+}
+
+// Exact water-filling: g(c) = sum_l clamp(c a_l, lo_l, 1) N_l is piecewise
+// linear and non-decreasing in c with breakpoints lo_l / a_l and 1 / a_l;
+// walk the sorted breakpoints to the segment that reaches the target and
+// solve the linear piece.
+spin_status spin_allocate_layer_sparsity(int n, const double* miss, const double* blocks, const double* lo,
+                                         double s_glob, float* s_out) {
+  if (n < 1 || !miss || !blocks || !lo || !s_out || !(s_glob >= 0.0 && s_glob < 1.0)) return SPIN_EINVAL;
+  std::vector<double> a(n);
+  double total = 0.0, floor_kept = 0.0;
+  for (int l = 0; l < n; ++l) {
+    if (!(miss[l] >= 0.0) || !(blocks[l] > 0.0) || !(lo[l] > 0.0 && lo[l] <= 1.0)) return SPIN_EINVAL;
+    a[l] = miss[l] + 1e-3;
+    total += blocks[l];
+    floor_kept += lo[l] * blocks[l];
+  }
+  const double target = (1.0 - s_glob) * total;
+  if (floor_kept >= target) {
+    for (int l = 0; l < n; ++l) s_out[l] = (float)(1.0 - lo[l]);
+    return SPIN_OK;
+  }
+  auto g = [&](double c) {
+    double t = 0.0;
+    for (int l = 0; l < n; ++l) t += std::min(1.0, std::max(lo[l], c * a[l])) * blocks[l];
+    return t;
+  };
+  std::vector<double> bp;
+  for (int l = 0; l < n; ++l) {
+    bp.push_back(lo[l] / a[l]);
+    bp.push_back(1.0 / a[l]);
+  }
+  std::sort(bp.begin(), bp.end());
+  double c = bp.back();
+  double prev = 0.0, g_prev = g(0.0);
+  for (double x : bp) {
+    const double gx = g(x);
+    if (gx >= target) {
+      // linear between prev and x
+      c = (gx == g_prev) ? x : prev + (target - g_prev) * (x - prev) / (gx - g_prev);
+      break;
+    }
+    prev = x;
+    g_prev = gx;
+  }
+  for (int l = 0; l < n; ++l) s_out[l] = (float)(1.0 - std::min(1.0, std::max(lo[l], c * a[l])));
+  return SPIN_OK;
+}
+
+spin_status spin_get_error(spin_state st, spin_stream_t stream, uint32_t* word_out) {
+  if (!alive(st)) return SPIN_ESTATE;
+  cudaStream_t s = (cudaStream_t)stream;
+  ErrWord h{};
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, st->err, sizeof(ErrWord), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->err, 0, sizeof(ErrWord), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (word_out) *word_out = h.flags;
+  if (h.flags & ERR_TIMEOUT) return SPIN_ETIMEOUT;
+  if (h.flags) return SPIN_EDEVICE;
+  return SPIN_OK;
+}
+
+const char* spin_status_string(spin_status s) {
+  switch (s) {
+    case SPIN_OK: return "ok";
+    case SPIN_EINVAL: return "invalid argument";
+    case SPIN_ENOMEM: return "state block too small";
+    case SPIN_ECUDA: return "CUDA runtime error";
+    case SPIN_ESTATE: return "invalid state handle";
+    case SPIN_ETIMEOUT: return "device wait timed out";
+    case SPIN_EDEVICE: return "device-side argument check failed";
+    case SPIN_EUNSUPPORTED: return "shape not supported by the requested kernel";
+  }
+  return "unknown status";
+}
+
+size_t spin_state_export_bytes(spin_state st) {
+  if (!alive(st)) return 0;
+  return (size_t)2 * st->lay.L * st->lay.Q * st->lay.slot_stride * sizeof(float);
+}
+
+spin_status spin_state_export(spin_state st, void* host, size_t bytes, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  const size_t half = spin_state_export_bytes(st) / 2;
+  if (!host || bytes < 2 * half) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(host, st->V, half, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync((char*)host + half, st->D, half, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+spin_status spin_state_import(spin_state st, const void* host, size_t bytes, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  const size_t half = spin_state_export_bytes(st) / 2;
+  if (!host || bytes < 2 * half) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(st->V, host, half, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->D, (const char*)host + half, half, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+spin_status spin_state_ema(spin_state st, int layer, float** V, float** D, int64_t* stride) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers) return SPIN_EINVAL;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  if (V) *V = st->V + per_layer * layer;
+  if (D) *D = st->D + per_layer * layer;
+  if (stride) *stride = st->lay.slot_stride;
+  return SPIN_OK;
+}
+
+spin_status spin_state_block_scores(spin_state st, const float** S, int64_t* stride) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (S) *S = st->S;
+  if (stride) *stride = st->lay.blk_stride;
+  return SPIN_OK;
+}
+
+spin_status spin_state_qquant(spin_state st, const uint8_t** q8, const float** wq) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (q8) *q8 = st->q8;
+  if (wq) *wq = st->wq;
+  return SPIN_OK;
+}
+
+int64_t spin_score_stride(spin_state st) { return alive(st) ? st->lay.slot_stride : -1; }
+int64_t spin_mask_stride(spin_state st) { return alive(st) ? st->lay.max_blocks : -1; }
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+// spin_internal.cuh -- state layout, error word and device helpers shared by
+// the SPIN kernels (sm_100a).  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/spin.h"
+
+namespace spin {
+
+// ---------------------------------------------------------------------------
+// Device error word: bits OR-ed by kernels, read by spin_get_error.
+// ---------------------------------------------------------------------------
+enum : uint32_t {
+  ERR_CTX_LEN = 1u << 0,      // ctx_len < 1 or ctx_len + rows - 1 > max_slots
+  ERR_PAGE = 1u << 1,         // block-table entry outside [0, num_pages)
+  ERR_ACCEPTED = 1u << 2,     // accepted length outside 1..rows
+  ERR_TIMEOUT = 1u << 3,      // a bounded mbarrier wait gave up
+  ERR_CAPACITY = 1u << 4,     // a shape exceeded a kernel's on-chip capacity
+};
+
+// Error word block: [0] flags, [1] first offending request, [2] first value.
+struct ErrWord {
+  uint32_t flags;
+  uint32_t request;
+  uint32_t value;
+  uint32_t pad;
+};
+
+__device__ __forceinline__ void raise_error(ErrWord* e, uint32_t bit, uint32_t req, uint32_t val) {
+  uint32_t old = atomicOr(&e->flags, bit);
+  if (old == 0) {
+    e->request = req;
+    e->value = val;
+  }
+}
+
+// Host-side view of a state; the device block is carved as documented in
+// spin_state_bytes (spin_api.cu).
+struct Layout {
+  int32_t L, Q, R, H, d, b, k;
+  int64_t max_slots;
+  int64_t max_blocks;    // ceil(max_slots / b)
+  int64_t slot_stride;   // max_blocks * b  (a score / V / D row)
+  int64_t blk_stride;    // max_blocks rounded up to 16 (mask, S, work-list rows)
+};
+
+// ---------------------------------------------------------------------------
+// Positions (see spin.h): row r sits at p_r = ctx_len - 1 + r.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t row_pos(int64_t ctx_len, int r) { return ctx_len - 1 + r; }
+__host__ __device__ __forceinline__ int64_t row_blocks(int64_t ctx_len, int r, int b) {
+  return (ctx_len + r + b - 1) / b;
+}
+
+// Budget of a row and the exploration count (computed in double from the
+// fp32 parameters, exactly as the host and the checker define them).
+__device__ __forceinline__ int64_t block_budget(int64_t n, float s) {
+  return n - (int64_t)floor((double)s * (double)n);
+}
+__device__ __forceinline__ int64_t explore_count(int64_t budget0, float g) {
+  return (int64_t)floor((double)g * (double)budget0);
+}
+
+// ---------------------------------------------------------------------------
+// Order-preserving map float -> uint32: larger float <=> larger key.  -0 is
+// folded onto +0 so that the two compare equal, as floats do.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t fkey(float x) {
+  uint32_t u = __float_as_uint(x == 0.0f ? 0.0f : x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3",
+// SC'11).  Per round: two 32x32->64 products of counter words 0 and 2 with the
+// Philox-4x32 multipliers, outputs (hi(c2*M1)^c1^k0, lo(c2*M1),
+// hi(c0*M0)^c3^k1, lo(c0*M0)); the key advances by the Weyl increments.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+  constexpr uint32_t kMulA = 0xD2511F53u, kMulB = 0xCD9E8D57u;
+  constexpr uint32_t kWeylA = 0x9E3779B9u, kWeylB = 0xBB67AE85u;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint32_t loA = kMulA * c.x, hiA = __umulhi(kMulA, c.x);
+    const uint32_t loB = kMulB * c.z, hiB = __umulhi(kMulB, c.z);
+    c = make_uint4(hiB ^ c.y ^ k.x, loB, hiA ^ c.w ^ k.y, loA);
+    k.x += kWeylA;
+    k.y += kWeylB;
+  }
+  return c;
+}
+
+// Exploration key of block j: word 0 of Philox at counter
+// (j, request, layer, step mod 2^32) under key (seed lo, seed hi).
+__device__ __forceinline__ uint32_t explore_key(uint64_t seed, uint32_t j, uint32_t req,
+                                                uint32_t layer, uint64_t step) {
+  uint4 r = philox4x32_10(make_uint4(j, req, layer, (uint32_t)step),
+                          make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
+  return r.x;
+}
+
+// EMA update with never-observed sentinels (+inf for V, -inf for D).
+__device__ __forceinline__ float ema_v(float x, float y, float alpha, float beta) {
+  return (x == __int_as_float(0x7f800000)) ? y : __fmaf_rn(alpha, x, __fmul_rn(beta, y));
+}
+__device__ __forceinline__ float ema_d(float x, float y, float alpha, float beta) {
+  return (x == __int_as_float(0xff800000)) ? y : __fmaf_rn(alpha, x, __fmul_rn(beta, y));
+}
+
+// E4M3 pair -> float2 (exact).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)v, __NV_E4M3);
+  __half2 hh;
+  memcpy(&hh, &h, sizeof(hh));
+  return __half22float2(hh);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (one per .cu file).  All return cudaGetLastError().
+// ---------------------------------------------------------------------------
+struct StepArgs {
+  Layout lay;
+  int layer, rows;
+  int64_t step;
+  float sparsity, gamma, alpha;
+  uint64_t seed;
+  const int32_t* ctx_len;
+  uint8_t* mask;
+  float* S;
+  int32_t* work;      // [Q][blk_stride] kept block ids, ascending
+  int32_t* kept;      // [Q] kept counts
+  float* V;           // layer base [Q][slot_stride]
+  float* D;
+  ErrWord* err;
+};
+
+cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s);
+struct ReqList {
+  static constexpr int kMax = 32;
+  int32_t ids[kMax];
+  int n;
+};
+cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t stride, cudaStream_t s);
+cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s);
+cudaError_t launch_select(const StepArgs& a, cudaStream_t s);
+cudaError_t launch_compact(const Layout& L, int rows, const int32_t* ctx_len, const uint8_t* mask,
+                           int32_t* work, int32_t* kept, ErrWord* err, cudaStream_t s);
+
+struct ScoreArgs {
+  Layout lay;
+  int rows;
+  int key_fp8;        // 1: E4M3 keys + scale; 0: fp32 keys
+  int q_bf16;         // 1: bf16 queries; 0: fp32
+  const void* keys;
+  const float* kscale;
+  int32_t num_pages;
+  const int32_t* block_table;
+  int32_t bt_stride;
+  const void* q;
+  const float* w;
+  const int32_t* ctx_len;
+  const uint8_t* mask;
+  const int32_t* work;
+  const int32_t* kept;
+  uint8_t* q8;        // [Q][R][H][d] quantised queries (FP8 keys)
+  float* wq;          // [Q][R][H] folded weights
+  float* scores;      // [Q][R][slot_stride]
+  ErrWord* err;
+  // fused EMA (rows == 1 only): V, D of the layer, or null
+  float* V;
+  float* D;
+  float alpha, beta;   // beta = fl32(1 - alpha), computed once on the host
+  int inject;          // test hook: withhold the first key stage of CTA 0
+};
+
+cudaError_t launch_quantize_q(const ScoreArgs& a, cudaStream_t s);
+cudaError_t launch_score_simt(const ScoreArgs& a, cudaStream_t s);
+bool tc_supported(const Layout& lay, int rows, int key_fp8);
+cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s);
+
+struct TopkArgs {
+  Layout lay;
+  int rows;
+  const float* scores;
+  const uint8_t* mask;
+  const int32_t* ctx_len;
+  const int32_t* work;
+  const int32_t* kept;
+  int32_t* topk;
+  ErrWord* err;
+};
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+struct EmaArgs {
+  Layout lay;
+  int rows;
+  const float* scores;
+  const uint8_t* mask;
+  const int32_t* ctx_len;
+  const int32_t* accepted;
+  float* V;
+  float* D;
+  float alpha, beta;
+  ErrWord* err;
+};
+cudaError_t launch_ema_update(const EmaArgs& a, cudaStream_t s);
+
+cudaError_t launch_miss_count(const Layout& lay, int rows, const int32_t* full_topk,
+                              const uint8_t* mask, int32_t* missed, int32_t* total,
+                              cudaStream_t s);
+
+}  // namespace spin

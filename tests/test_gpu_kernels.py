@@ -1,0 +1,244 @@
+"""Kernel-level parity on the GPU, through the C ABI, against the oracle.
+
+Every case uses seeded synthetic inputs at sizes the oracle finishes in
+seconds that still span several tiles and a ragged tail.  Integer and
+selection results must match bit for bit; scores within
+|gpu - ref| <= 1e-4 + 1e-3 |ref| of the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import indexer_sparse_attention_b200 as isa
+import oracle
+import workloads
+from lockstep import score_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from indexer_sparse_attention_b200 import build
+    build.build()
+    oracle.build()
+    assert torch.cuda.is_available()
+
+
+def make_state(Q=3, max_slots=8192 + 64, R=1, H=64, d=128, k=256, fp8=True, s=0.5, g=0.05, seed=7, layers=1, b=64):
+    cfg = isa.make_config(num_layers=layers, num_requests=Q, max_slots=max_slots, block_size=b, num_heads=H,
+                          head_dim=d, topk=k, max_rows=R, key_fp8=fp8, q_bf16=fp8, alpha=0.9, gamma=g,
+                          target_sparsity=s, seed=seed)
+    return isa.SpinState(cfg)
+
+
+def random_state(st, layer, rng, frac_sentinel=0.1):
+    V, D = st.ema(layer)
+    v = rng.uniform(0, 50, V.shape).astype(np.float32)
+    dd = rng.uniform(0, 50, D.shape).astype(np.float32)
+    v[rng.uniform(size=v.shape) < frac_sentinel] = np.inf
+    dd[rng.uniform(size=dd.shape) < frac_sentinel] = -np.inf
+    # coarse values create ties in the block scores
+    v = np.round(v / 4) * 4
+    V.copy_(torch.from_numpy(v))
+    D.copy_(torch.from_numpy(dd))
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("R", [1, 2, 4])
+@pytest.mark.parametrize("s,g", [(0.5, 0.05), (0.4, 0.1), (0.9, 0.3), (0.0, 0.05), (0.3, 0.0)])
+def test_predict_select_bit_exact(R, s, g):
+    rng = np.random.default_rng(int(R * 100 + s * 10 + g * 1000))
+    st = make_state(Q=5, max_slots=8192 + 64, R=R, s=s, g=g)
+    random_state(st, 0, rng)
+    ctx = np.array([1, 63, 64 * 37 + 5, 8192 - R + 1, 4096], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    for step in [0, 3, 1 << 33]:
+        isa.spin_predict_select(st, 0, R, step, ctx_t, mask)
+        assert isa.spin_get_error(st)[0] == 0
+        V, D = st.ema(0)
+        S_gpu = st.block_scores().cpu().numpy()
+        for q in range(5):
+            S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, 64, st.mask_stride)
+            if s > 0:
+                for r in range(R):
+                    n = oracle.num_blocks(int(ctx[q]), r, 64)
+                    assert np.array_equal(S_gpu[q, r, :n], S_ref[r, :n])
+            m_ref = oracle.select(S_ref, int(ctx[q]), R, 64, s, g, 7, q, 0, step)
+            assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
+
+
+def test_select_large_request_with_infinite_and_tied_scores():
+    # one 1M-slot request: 16,385 blocks, many equal block scores
+    rng = np.random.default_rng(1)
+    st = make_state(Q=2, max_slots=1024 * 1024 + 64, R=1, s=0.5, g=0.1, k=2048)
+    V, D = st.ema(0)
+    v = rng.integers(0, 3, V.shape).astype(np.float32)
+    v[:, -5000:] = np.inf
+    V.copy_(torch.from_numpy(v))
+    D.fill_(-np.inf)
+    ctx = np.array([1024 * 1024 + 1, 300000], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    isa.spin_predict_select(st, 0, 1, 11, ctx_t, mask)
+    assert isa.spin_get_error(st)[0] == 0
+    for q in range(2):
+        S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), 1, 64, st.mask_stride)
+        m_ref = oracle.select(S_ref, int(ctx[q]), 1, 64, 0.5, 0.1, 7, q, 0, 11)
+        assert np.array_equal(mask[q].cpu().numpy(), m_ref)
+
+
+def fp8_inputs(Q, R, H, d, max_slots, rng, device="cuda", permute=True):
+    wl = workloads.config(1, requests=Q, ctx0=(max_slots - 8,) * Q, steps=1, H=H, d=d, rows=R,
+                          permute_pages=permute, spare_slots=8)
+    cache = workloads.make_key_cache(wl, 0, device)
+    q = (torch.randn((Q, R, H, d), generator=torch.Generator(device).manual_seed(int(rng.integers(1 << 30))),
+                     device=device) * torch.exp(torch.randn((Q, R, H, 1), device=device) * 2)).to(torch.bfloat16)
+    q[0, 0, 3] = 0                                            # an all-zero head
+    w = torch.rand((Q, R, H), device=device)
+    return wl, cache, q.contiguous(), w.contiguous()
+
+
+def run_score(st, kind, R, cache, q, w, ctx_t, mask, fp8=True):
+    isa.spin_set_score_kernel(st, kind)
+    scores = st.new_scores()
+    scores.fill_(float("nan"))
+    isa.spin_indexer_score(st, 0, R, cache.keys, cache.kscale if fp8 else None, cache.block_table, q, w, ctx_t,
+                           mask, scores)
+    assert isa.spin_get_error(st)[0] == 0
+    return scores
+
+
+@pytest.mark.parametrize("R", [1, 2, 4])
+@pytest.mark.parametrize("kind", [isa.SPIN_SCORE_SIMT, isa.SPIN_SCORE_TCGEN05])
+def test_fp8_scores_vs_oracle(R, kind):
+    rng = np.random.default_rng(R)
+    Q, H, d, max_slots = 3, 64, 128, 64 * 41
+    st = make_state(Q=Q, max_slots=max_slots, R=R, H=H, d=d)
+    wl, cache, q, w = fp8_inputs(Q, R, H, d, max_slots, rng)
+    ctx = np.array([64 * 40 + 7 - R + 1, 130, 64 * 23], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.6).astype(np.uint8)
+    for qq in range(Q):
+        m[qq, oracle.num_blocks(int(ctx[qq]), R - 1, 64):] = 0
+        m[qq, 0] = 2                                         # odd kept counts -> half-filled tiles
+    mask = torch.from_numpy(m).cuda()
+    scores = run_score(st, kind, R, cache, q, w, ctx_t, mask)
+    q8g, wqg = st.qquant(R)
+    for qq in range(Q):
+        q8, wq, _ = oracle.quantize_q(q[qq].float().cpu().numpy().astype(np.float64), w[qq].cpu().numpy())
+        assert np.array_equal(q8g[qq].cpu().numpy(), q8)
+        assert np.array_equal(wqg[qq].cpu().numpy(), wq)
+        keys, ks, ident = workloads.request_pages(cache, qq)
+        ref = oracle.score_fp8(keys.numpy(), ks.numpy(), ident.numpy(), q8, wq, int(ctx[qq]), m[qq], st.score_stride)
+        got = scores[qq, :R].cpu().numpy()
+        sc = ~np.isnan(ref)
+        assert sc.sum() > 0
+        assert score_close(got[sc], ref[sc]).all()
+        assert np.all(np.isnan(got[~sc]))                    # nothing written outside kept, visible slots
+
+
+def test_tcgen05_agrees_with_simt_at_serving_shape():
+    rng = np.random.default_rng(5)
+    Q, R, H, d, max_slots = 8, 1, 64, 128, 64 * 300
+    st = make_state(Q=Q, max_slots=max_slots, R=R)
+    wl, cache, q, w = fp8_inputs(Q, R, H, d, max_slots, rng)
+    ctx_t = torch.full((Q,), max_slots - 3, dtype=torch.int32).cuda()
+    mask = torch.from_numpy((rng.uniform(size=(Q, st.mask_stride)) < 0.5).astype(np.uint8)).cuda()
+    a = run_score(st, isa.SPIN_SCORE_SIMT, R, cache, q, w, ctx_t, mask)
+    b = run_score(st, isa.SPIN_SCORE_TCGEN05, R, cache, q, w, ctx_t, mask)
+    fin = ~torch.isnan(a)
+    assert torch.equal(fin, ~torch.isnan(b))
+    assert score_close(b[fin].cpu().numpy(), a[fin].cpu().numpy()).all()
+
+
+def test_fp32_scores_vs_oracle():
+    rng = np.random.default_rng(9)
+    wl = workloads.config(0, ctx0=(4096,), steps=4)
+    cache = workloads.make_key_cache(wl, 0, "cuda")
+    st = make_state(Q=1, max_slots=wl.max_slots, R=1, H=8, d=64, fp8=False, k=256)
+    q = torch.randn((1, 1, 8, 64), device="cuda")
+    w = torch.rand((1, 1, 8), device="cuda")
+    ctx = 4097
+    m = (rng.uniform(size=(1, st.mask_stride)) < 0.7).astype(np.uint8)
+    scores = run_score(st, isa.SPIN_SCORE_AUTO, 1, cache, q, w, torch.tensor([ctx], dtype=torch.int32).cuda(),
+                       torch.from_numpy(m).cuda(), fp8=False)
+    ref = oracle.score_f32(cache.keys.cpu().numpy(), cache.block_table[0].cpu().numpy(), q[0].cpu().numpy(),
+                           w[0].cpu().numpy(), ctx, m[0], st.score_stride)
+    got = scores[0, :1].cpu().numpy()
+    sc = ~np.isnan(ref)
+    assert score_close(got[sc], ref[sc]).all()
+
+
+@pytest.mark.parametrize("R", [1, 4])
+@pytest.mark.parametrize("kind", ["random", "ties", "few"])
+def test_topk_bit_exact(R, kind):
+    rng = np.random.default_rng(R + len(kind))
+    Q, k = 4, 256
+    st = make_state(Q=Q, max_slots=64 * 200, R=R, k=k)
+    ctx = np.array([64 * 200 - R + 1, 64 * 37 + 11, 3, 64 * 5], np.int64)
+    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.5).astype(np.uint8)
+    if kind == "few":
+        m[:] = 0
+        m[:, 1] = 1                                         # fewer than k scored slots: padding
+    for qq in range(Q):
+        m[qq, oracle.num_blocks(int(ctx[qq]), R - 1, 64):] = 0
+    scores = st.new_scores()
+    if kind == "ties":
+        vals = rng.integers(0, 6, scores.shape).astype(np.float32)
+        vals[rng.uniform(size=vals.shape) < 0.01] = -0.0
+    else:
+        vals = rng.standard_normal(scores.shape).astype(np.float32) * 10
+    scores.copy_(torch.from_numpy(vals))
+    topk = torch.empty((Q, R, k), dtype=torch.int32, device="cuda")
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    isa.spin_topk(st, R, scores, torch.from_numpy(m).cuda(), ctx_t, topk)
+    assert isa.spin_get_error(st)[0] == 0
+    got = topk.cpu().numpy()
+    for qq in range(Q):
+        for r in range(R):
+            ref = oracle.topk_row(vals[qq, r].astype(np.float64), m[qq], int(ctx[qq]), r, 64, k)
+            assert np.array_equal(got[qq, r], ref), (qq, r)
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 4])
+def test_ema_update_prefix_valid_bit_exact(R):
+    rng = np.random.default_rng(40 + R)
+    Q = 6
+    st = make_state(Q=Q, max_slots=64 * 60, R=R)
+    random_state(st, 0, rng, frac_sentinel=0.3)
+    ctx = np.array([64 * 60 - R + 1, 64 * 10 + 1, 64 * 10, 1, 65, 64 * 33 + 17], np.int64)
+    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.5).astype(np.uint8)
+    for qq in range(Q):
+        m[qq, oracle.num_blocks(int(ctx[qq]), R - 1, 64):] = 0
+    acc = rng.integers(1, R + 1, Q).astype(np.int32)
+    scores = st.new_scores()
+    vals = rng.uniform(0, 30, scores.shape).astype(np.float32)
+    scores.copy_(torch.from_numpy(vals))
+    V, D = st.ema(0)
+    V0, D0 = V.cpu().numpy().copy(), D.cpu().numpy().copy()
+    isa.spin_ema_update(st, 0, R, scores, torch.from_numpy(m).cuda(), torch.from_numpy(ctx).to(torch.int32).cuda(),
+                        torch.from_numpy(acc).cuda())
+    assert isa.spin_get_error(st)[0] == 0
+    for qq in range(Q):
+        v, d = V0[qq].copy(), D0[qq].copy()
+        oracle.ema_update(v, d, vals[qq, :R], m[qq], int(ctx[qq]), int(acc[qq]), 64, 0.9)
+        assert np.array_equal(V[qq].cpu().numpy().view(np.uint32), v.view(np.uint32)), qq
+        assert np.array_equal(D[qq].cpu().numpy().view(np.uint32), d.view(np.uint32)), qq
+
+
+def test_miss_count():
+    rng = np.random.default_rng(3)
+    Q, R, k = 3, 2, 128
+    st = make_state(Q=Q, max_slots=64 * 50, R=R, k=k)
+    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.5).astype(np.uint8)
+    full = rng.integers(0, 64 * 50, (Q, R, k)).astype(np.int32)
+    full[:, :, -7:] = -1
+    missed = torch.zeros((Q, R), dtype=torch.int32, device="cuda")
+    total = torch.zeros((Q, R), dtype=torch.int32, device="cuda")
+    isa.spin_miss_count(st, R, torch.from_numpy(full).cuda(), torch.from_numpy(m).cuda(), missed, total)
+    for qq in range(Q):
+        for r in range(R):
+            frac = oracle.miss_fraction(full[qq, r], m[qq], 64)
+            assert total[qq, r].item() == k - 7
+            assert abs(missed[qq, r].item() / (k - 7) - frac) < 1e-12
