@@ -47,7 +47,7 @@ SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["spin", "reference"], default="spin")
     p.add_argument("--sparsity", type=float, default=0.5)
@@ -91,7 +91,7 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) of this GPU while the timed region runs."""
+    """nvidia-smi samples (every 50 ms) of this GPU while the timed region runs."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -111,7 +111,7 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.ident}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None

@@ -12,31 +12,40 @@
 // K-major, 128-byte swizzled.  The contraction is dense and small per tile;
 // the kernel is HBM-bound on the key stream (132 bytes per kept slot).
 //
-// Warp roles (192 threads, persistent, one CTA per SM):
-//   warp 0      TMA producer: query tile per request, key pages per tile
+// Warp roles (320 threads, persistent, two CTAs per SM when N <= 128):
+//   warp 0      producer: lanes gather the tile metadata one and two batches
+//               of 32 tiles ahead; lane 0 handles the query tile (per request)
+//               and the stage barriers; eight lanes issue a tile's copies in
+//               one step (key pages by TMA; the pages' scales and EMA slices
+//               by bulk copies).  One issuing warp per CTA caps the copy rate,
+//               so a second CTA per SM doubles it.
 //   warp 1      TMEM allocation; lane 0 issues the MMAs and the commits
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator quarter this warp may
-//               access (lanes 32*(warp%4) ..), ReLU, head weights, scale,
-//               store, fused EMA
-// Pipelines: kStages key stages (full/empty), 2 query buffers, 2 TMEM
-// accumulators.  Every wait is bounded (2 s of %globaltimer); on expiry the
-// CTA raises ERR_TIMEOUT, stops issuing, drains what it issued and frees TMEM.
+//   warps 2..9  two epilogue groups of four warps, taking alternate tiles; a
+//               warp reads the accumulator quarter it may access (lanes
+//               32*(warp%4) ..), applies ReLU, head weights and the scale,
+//               stores the scores and the fused EMA update
+// Pipelines: 4 stages per CTA (8 with one CTA per SM) of keys + side data,
+// 2 query buffers, 4 TMEM accumulators (2 when N > 64), so that all CTAs of
+// an SM fit the 512 TMEM columns.  Every wait is bounded (2 s of
+// %globaltimer); on expiry the CTA raises ERR_TIMEOUT, stops issuing, drains
+// what it issued and frees TMEM.
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstddef>
 
 #include "spin_internal.cuh"
 
 namespace spin {
 namespace {
 
-constexpr int kStages = 6;
 constexpr int kTileM = 128;
 constexpr int kPage = 64;          // tokens per page (block size)
 constexpr int kRowBytes = 128;     // d = 128 FP8 values
 constexpr int kPageBytes = kPage * kRowBytes;
 constexpr int kStageBytes = kTileM * kRowBytes;
-constexpr int kThreads = 192;
+constexpr int kEpiGroups = 2;                 // epilogue groups of 4 warps, alternate tiles
+constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -162,30 +171,64 @@ struct Sched {
   }
 };
 
+// Per-stage side data copied with the keys: the two pages' scales, and for
+// the fused EMA the vertical states of the two blocks and a 16-byte aligned
+// window of the diagonal states they touch, plus the tile's metadata.
+constexpr int kDWin = 68;  // floats: 64 offsets + up to 3 below for 16-byte alignment
+struct StageAux {
+  float sigma[2][kPage];
+  float v[2][kPage];
+  float d[2][kDWin];
+  int q, ctx, np, fused;
+  int j[2], valid[2], ws[2];
+  int pad[2];
+};
+static_assert(sizeof(StageAux) % 16 == 0, "aux must keep 16-byte alignment");
+
 struct SmemLayout {
-  uint32_t keys;     // kStages * kStageBytes
+  uint32_t keys;     // stages * kStageBytes
+  uint32_t aux;      // stages * sizeof(StageAux)
   uint32_t qbuf;     // 2 * N * 128
-  uint32_t wq;       // 4 * N floats: one copy per epilogue warp
+  uint32_t wq;       // 4 * kEpiGroups * N floats: one copy per epilogue warp
   uint32_t prefix;   // (Q + 1) ints
   uint32_t bars;     // barriers
   uint32_t total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int N, int Q) {
+constexpr int kMaxStages = 8;
+constexpr int kMaxAcc = 4;
+
+__host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
   SmemLayout s;
   uint32_t off = 0;
   s.keys = off;
-  off += kStages * kStageBytes;
+  off += stages * kStageBytes;
+  s.aux = off;
+  off += stages * (uint32_t)sizeof(StageAux);
+  off = (off + 1023) / 1024 * 1024;
   s.qbuf = off;
   off += 2 * N * kRowBytes;
   s.wq = off;
-  off += 4 * N * 4;
+  off += 4 * kEpiGroups * N * 4;
   s.prefix = off;
   off += ((Q + 1) * 4 + 15) / 16 * 16;
   s.bars = off;
-  off += (2 * kStages + 8) * 8 + 16;
+  off += (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) * 8 + 16;
   s.total = off + 1024;  // slack for 1024-byte alignment of the base
   return s;
+}
+
+// Launch plan: two CTAs per SM when shared memory and TMEM allow (each CTA
+// has one copy-issuing warp, and one issuer per CTA caps the copy rate), with
+// accumulators sized so that CTAs * accumulators * N <= 512 TMEM columns.
+struct TcPlan {
+  int stages, nacc, ctas;
+};
+
+__host__ __device__ inline TcPlan tc_plan(int N, int Q) {
+  if (N <= 64 && smem_layout(N, Q, 4).total * 2 <= 227 * 1024) return {4, 4, 2};
+  if (N <= 128 && smem_layout(N, Q, 4).total * 2 <= 227 * 1024) return {4, 2, 2};
+  return {kMaxStages, 2, 1};
 }
 
 struct Bars {
@@ -198,31 +241,85 @@ struct Bars {
   __device__ uint32_t ae(int i) const { return accempty + 8 * i; }
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
-    k_score_tc(ScoreArgs a, const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q) {
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"((uint64_t)src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Tile metadata, gathered by one producer lane per tile in two phases one
+// batch apart, so no load result is needed before a batch later:
+//   phase A: request, pair index, context length, kept count, block ids
+//   phase B: page ids from the block table (needs the block ids)
+struct TileMeta {
+  int q, t, ctx, kept, j0, j1, pg0, pg1;
+};
+
+__device__ __forceinline__ void meta_phase_a(TileMeta& m, const ScoreArgs& a, const Sched& sched, const int* prefix,
+                                             int g, int g1) {
+  m.q = -1;
+  if (g >= g1) return;
+  const Layout& L = a.lay;
+  const int q = sched.locate(g);
+  const int t = g - prefix[q];
+  m.q = q;
+  m.t = t;
+  m.ctx = a.ctx_len[q];
+  m.kept = a.kept[q];
+  const int32_t* work = a.work + (int64_t)q * L.blk_stride;
+  m.j0 = work[2 * t];
+  m.j1 = (2 * t + 1 < L.blk_stride) ? work[2 * t + 1] : -1;
+}
+
+__device__ __forceinline__ void meta_phase_b(TileMeta& m, const ScoreArgs& a) {
+  if (m.q < 0) return;
+  const int32_t* bt = a.block_table + (int64_t)m.q * a.bt_stride;
+  m.pg0 = bt[m.j0];
+  m.pg1 = (2 * m.t + 1 < m.kept) ? bt[m.j1] : 0;
+}
+
+__device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
+  TileMeta r;
+  r.q = __shfl_sync(0xffffffffu, m.q, src);
+  r.t = __shfl_sync(0xffffffffu, m.t, src);
+  r.ctx = __shfl_sync(0xffffffffu, m.ctx, src);
+  r.kept = __shfl_sync(0xffffffffu, m.kept, src);
+  r.j0 = __shfl_sync(0xffffffffu, m.j0, src);
+  r.j1 = __shfl_sync(0xffffffffu, m.j1, src);
+  r.pg0 = __shfl_sync(0xffffffffu, m.pg0, src);
+  r.pg1 = __shfl_sync(0xffffffffu, m.pg1, src);
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
+               const __grid_constant__ CUtensorMap tmap_q) {
   const Layout L = a.lay;
   const int N = a.rows * L.H;
+  const int stages = plan.stages, nacc = plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const SmemLayout lay = smem_layout(N, L.Q);
+  const SmemLayout lay = smem_layout(N, L.Q, stages);
   const uint32_t sbase = smem_u32(smem);
+  StageAux* aux = reinterpret_cast<StageAux*>(smem + lay.aux);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
   float* wqs = reinterpret_cast<float*>(smem + lay.wq);
   uint64_t* bar_mem = reinterpret_cast<uint64_t*>(smem + lay.bars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mem + 2 * kStages + 7);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mem + 2 * kMaxStages + 4 + 2 * kMaxAcc + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   Bars B;
   B.full = smem_u32(bar_mem);
-  B.empty = B.full + 8 * kStages;
-  B.qfull = B.empty + 8 * kStages;
+  B.empty = B.full + 8 * kMaxStages;
+  B.qfull = B.empty + 8 * kMaxStages;
   B.qempty = B.qfull + 16;
   B.accfull = B.qempty + 16;
-  B.accempty = B.accfull + 16;
-  B.done = B.accempty + 16;
+  B.accempty = B.accfull + 8 * kMaxAcc;
+  B.done = B.accempty + 8 * kMaxAcc;
   const Ctl ctl{abort_flag, a.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool fused = a.V != nullptr;
 
-  // ---- tile prefix over requests ------------------------------------------
+  // ---- tile prefix over requests, barriers ---------------------------------
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int q = 0; q < L.Q; ++q) {
@@ -233,20 +330,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     prefix[L.Q] = acc;
     *abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(B.f(s), 1);
-      mbar_init(B.e(s), 1);
+      mbar_init(B.e(s), 1 + 4);  // the MMA commit and the four epilogue warps
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(B.qf(i), 1);
       mbar_init(B.qe(i), 1);
+    }
+    for (int i = 0; i < nacc; ++i) {
       mbar_init(B.af(i), 1);
-      mbar_init(B.ae(i), 4);
+      mbar_init(B.ae(i), 4);  // the four warps of the group that owns the tile
     }
     mbar_init(B.done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const uint32_t ncols = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
+  const int acc_cols = nacc * N;
+  const uint32_t ncols = acc_cols <= 32 ? 32 : acc_cols <= 64 ? 64 : acc_cols <= 128 ? 128 : acc_cols <= 256 ? 256 : 512;
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(ncols)
@@ -264,58 +364,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Sched sched{prefix, L.Q};
 
   if (warp == 0) {
-    // ======================= TMA producer =======================
-    if (lane == 0 && g0 < g1) {
-      int q = sched.locate(g0), t = g0 - prefix[q];
-      int stage = 0;
-      uint32_t phase = 0;
-      int cur_q = -1, qiter = 0;
-      int inflight[kStages];  // parity of the last load issued into each stage, -1: none
-      for (int i = 0; i < kStages; ++i) inflight[i] = -1;
-      bool withhold = a.inject && blockIdx.x == 0;
-      for (int g = g0; g < g1; ++g, ++t) {
-        while (t >= prefix[q + 1] - prefix[q]) { ++q; t = 0; }
-        if (q != cur_q) {
-          const int nb = qiter & 1;
-          if (!wait_parity(B.qe(nb), ((qiter >> 1) & 1) ^ 1, ctl)) break;
-          mbar_expect_tx(B.qf(nb), (uint32_t)(N * kRowBytes));
-          tma_load_2d(sbase + lay.qbuf + nb * N * kRowBytes, &tmap_q, B.qf(nb), 0, q * N);
-          cur_q = q;
-          ++qiter;
-        }
-        if (!wait_parity(B.e(stage), phase ^ 1, ctl)) break;
-        const int32_t* work = a.work + (int64_t)q * L.blk_stride;
-        const int nk = a.kept[q];
-        const int i0 = 2 * t, i1 = 2 * t + 1;
-        int pages[2];
-        int np = (i1 < nk) ? 2 : 1;
-        for (int i = 0; i < np; ++i) {
-          const int j = work[i0 + i];
-          int pg = a.block_table[(int64_t)q * a.bt_stride + j];
-          if (pg < 0 || pg >= a.num_pages) {
-            raise_error(a.err, ERR_PAGE, q, (uint32_t)pg);
-            pg = 0;  // keep the pipeline in step; the epilogue skips this page
+    // ======================= producer (whole warp) =======================
+    int stage = 0;
+    uint32_t phase = 0;
+    int cur_q = -1, qiter = 0;
+    int inflight[kMaxStages];
+    for (int i = 0; i < kMaxStages; ++i) inflight[i] = -1;
+    bool withhold = a.inject && blockIdx.x == 0;
+    bool stop = false;
+    TileMeta cur, nxt, nxt2;
+    meta_phase_a(cur, a, sched, prefix, g0 + lane, g1);
+    meta_phase_b(cur, a);
+    meta_phase_a(nxt, a, sched, prefix, g0 + 32 + lane, g1);
+    // copy slot of this lane within a tile: page k = lane / 4, kind = lane % 4
+    // (0 key page, 1 scales, 2 vertical EMA slice, 3 diagonal EMA window)
+    const int ck = lane >> 2, ckind = lane & 3;
+    for (int gb = g0; gb < g1 && !stop; gb += 32) {
+      meta_phase_b(nxt, a);                                        // block ids arrived a batch ago
+      meta_phase_a(nxt2, a, sched, prefix, gb + 64 + lane, g1);    // used two batches later
+      const int nb_tiles = min(32, g1 - gb);
+      for (int i = 0; i < nb_tiles; ++i) {
+        const TileMeta m = shfl_meta(cur, i);
+        const int np = (2 * m.t + 1 < m.kept) ? 2 : 1;
+        const int pg0 = (m.pg0 >= 0 && m.pg0 < a.num_pages) ? m.pg0 : -1;
+        const int pg1 = (np == 2 && m.pg1 >= 0 && m.pg1 < a.num_pages) ? m.pg1 : -1;
+        const int p0 = m.ctx - 1;
+        int ok = 1;
+        if (lane == 0) {
+          if (m.q != cur_q) {
+            const int nb = qiter & 1;
+            ok = wait_parity(B.qe(nb), ((qiter >> 1) & 1) ^ 1, ctl);
+            if (ok) {
+              mbar_expect_tx(B.qf(nb), (uint32_t)(N * kRowBytes));
+              tma_load_2d(sbase + lay.qbuf + nb * N * kRowBytes, &tmap_q, B.qf(nb), 0, m.q * N);
+            }
           }
-          pages[i] = pg;
+          if (ok) ok = wait_parity(B.e(stage), phase ^ 1, ctl);
+          if (ok) {
+            if (pg0 < 0) raise_error(a.err, ERR_PAGE, m.q, (uint32_t)m.pg0);
+            if (np == 2 && pg1 < 0) raise_error(a.err, ERR_PAGE, m.q, (uint32_t)m.pg1);
+            StageAux* x = aux + stage;
+            x->q = m.q;
+            x->ctx = m.ctx;
+            x->np = np;
+            x->fused = fused ? 1 : 0;
+            x->valid[0] = pg0 >= 0;
+            x->valid[1] = pg1 >= 0;
+            x->j[0] = m.j0;
+            x->j[1] = m.j1;
+            uint32_t bytes = 0;
+            for (int k = 0; k < np; ++k) {
+              const int dlo = p0 - ((k ? m.j1 : m.j0) * kPage + kPage - 1);
+              x->ws[k] = (dlo > 0 ? dlo : 0) & ~3;
+              bytes += kPageBytes + kPage * 4 + (fused ? kPage * 4 + kDWin * 4 : 0);
+            }
+            if (!withhold) {
+              mbar_expect_tx(B.f(stage), bytes);
+              inflight[stage] = (int)phase;
+            }
+          }
         }
-        if (withhold) {
-          withhold = false;  // test hook: this stage never fills
-        } else {
-          mbar_expect_tx(B.f(stage), (uint32_t)(np * kPageBytes));
-          for (int i = 0; i < np; ++i)
-            tma_load_2d(sbase + lay.keys + stage * kStageBytes + i * kPageBytes, &tmap_k, B.f(stage), 0,
-                        pages[i] * kPage);
-          inflight[stage] = (int)phase;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { stop = true; break; }
+        if (m.q != cur_q) { cur_q = m.q; ++qiter; }
+        const bool issue = !__shfl_sync(0xffffffffu, withhold ? 1 : 0, 0);
+        withhold = false;  // test hook: at most the first stage is withheld
+        if (issue && ck < np && (ckind < 2 || fused)) {
+          const int j = ck ? m.j1 : m.j0;
+          const int pg = ck ? (pg1 < 0 ? 0 : pg1) : (pg0 < 0 ? 0 : pg0);  // bad pages load page 0; skipped later
+          const uint32_t bar = B.f(stage);
+          const uint32_t xdst = smem_u32(aux + stage);
+          if (ckind == 0) {
+            tma_load_2d(sbase + lay.keys + stage * kStageBytes + ck * kPageBytes, &tmap_k, bar, 0, pg * kPage);
+          } else if (ckind == 1) {
+            bulk_g2s(xdst + (uint32_t)offsetof(StageAux, sigma) + ck * kPage * 4, a.kscale + (int64_t)pg * kPage,
+                     kPage * 4, bar);
+          } else if (ckind == 2) {
+            bulk_g2s(xdst + (uint32_t)offsetof(StageAux, v) + ck * kPage * 4,
+                     a.V + (int64_t)m.q * L.slot_stride + (int64_t)j * kPage, kPage * 4, bar);
+          } else {
+            const int dlo = p0 - (j * kPage + kPage - 1);
+            const int ws = (dlo > 0 ? dlo : 0) & ~3;
+            bulk_g2s(xdst + (uint32_t)offsetof(StageAux, d) + ck * kDWin * 4,
+                     a.D + (int64_t)m.q * L.slot_stride + ws, kDWin * 4, bar);
+          }
         }
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (++stage == stages) { stage = 0; phase ^= 1; }
       }
-      // On abort, wait (bounded) until every copy this thread issued has landed.
-      if (*abort_flag) {
-        for (int s = 0; s < kStages; ++s) {
-          if (inflight[s] < 0) continue;
-          const uint64_t t0 = gtimer();
-          while (!mbar_try_wait(B.f(s), (uint32_t)inflight[s]) && gtimer() - t0 < kTimeoutNs) {}
-        }
+      cur = nxt;
+      nxt = nxt2;
+    }
+    // On abort, wait (bounded) until every copy this warp issued has landed.
+    if (lane == 0 && *abort_flag) {
+      for (int s = 0; s < stages; ++s) {
+        if (inflight[s] < 0) continue;
+        const uint64_t t0 = gtimer();
+        while (!mbar_try_wait(B.f(s), (uint32_t)inflight[s]) && gtimer() - t0 < kTimeoutNs) {}
       }
     }
   } else if (warp == 1) {
@@ -323,13 +467,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && g0 < g1) {
       const uint32_t idesc = idesc_e4m3(kTileM, N);
       int q = sched.locate(g0), t = g0 - prefix[q];
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
       int cur_q = -1, qiter = 0;
       for (int g = g0; g < g1; ++g, ++t) {
         while (t >= prefix[q + 1] - prefix[q]) { ++q; t = 0; }
+        const int i = g - g0;
+        const int stage = i % stages, acc = i % nacc;
+        const uint32_t phase = (uint32_t)(i / stages) & 1u, acc_phase = (uint32_t)(i / nacc) & 1u;
         if (q != cur_q) {
           if (cur_q >= 0) umma_commit(B.qe((qiter - 1) & 1));
           const int nb = qiter & 1;
@@ -348,8 +491,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_e4m3(d_tmem, sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
         umma_commit(B.e(stage));
         umma_commit(B.af(acc));
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
       // all MMAs issued by this thread complete before TMEM is released
       umma_commit(B.done);
@@ -357,76 +498,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!mbar_try_wait(B.done, 0) && gtimer() - t0 < kTimeoutNs) {}
     }
   } else {
-    // ======================= epilogue (warps 2..5) =======================
-    const int quarter = warp & 3;
-    const int m = quarter * 32 + lane;  // accumulator row = tile token
+    // ======================= epilogue (warps 2..9) =======================
+    const int ew = warp - 2;              // 0 .. 4*kEpiGroups-1
+    const int group = ew >> 2;
+    const int quarter = warp & 3;         // TMEM lanes this warp may access
+    const int m = quarter * 32 + lane;    // accumulator row = tile token
     const int pg_idx = m >> 6, tok = m & 63;
-    if (g0 < g1) {
-      int q = sched.locate(g0), t = g0 - prefix[q];
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      int cur_q = -1;
-      int64_t ctx = 0;
-      float* wcur = wqs + (warp - 2) * N;  // this warp's copy of the head weights
-      for (int g = g0; g < g1; ++g, ++t) {
-        while (t >= prefix[q + 1] - prefix[q]) { ++q; t = 0; }
-        if (q != cur_q) {
-          __syncwarp();
-          for (int i = lane; i < N; i += 32) wcur[i] = a.wq[(int64_t)q * N + i];
-          __syncwarp();
-          cur_q = q;
-          ctx = a.ctx_len[q];
-        }
-        // slot, page and per-slot operands (independent of the MMA: issue first)
-        const int32_t* work = a.work + (int64_t)q * L.blk_stride;
-        const int nk = a.kept[q];
-        const int li = 2 * t + pg_idx;
-        bool valid = li < nk;
-        int64_t s = 0;
-        int page = 0;
-        float sigma = 0.f, v_old = 0.f, d_old = 0.f;
-        if (valid) {
-          const int j = work[li];
-          page = a.block_table[(int64_t)q * a.bt_stride + j];
-          valid = page >= 0 && page < a.num_pages;
-          s = (int64_t)j * kPage + tok;
-          valid = valid && s <= ctx - 1 + (a.rows - 1);
-          if (valid) {
-            sigma = a.kscale[(int64_t)page * kPage + tok];
-            if (a.V && s <= ctx - 1) {
-              v_old = a.V[(int64_t)q * L.slot_stride + s];
-              d_old = a.D[(int64_t)q * L.slot_stride + (ctx - 1 - s)];
-            }
-          }
-        }
-        // every lane waits; the warp leaves together if any lane gave up, so
-        // the .sync.aligned TMEM loads below never run on a partial warp
-        if (!__all_sync(0xffffffffu, wait_parity(B.af(acc), acc_phase, ctl))) break;
-        tc_fence_after();
-        const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
-        for (int r = 0; r < a.rows; ++r) {
-          float sum = 0.f;
-          for (int c = 0; c < L.H; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(trow + (uint32_t)(r * L.H + c), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-              sum = __fmaf_rn(wcur[r * L.H + c + u], fmaxf(__uint_as_float(v[u]), 0.0f), sum);
-          }
-          if (valid && s <= ctx - 1 + r) {
-            const float score = sum * sigma;
-            a.scores[((int64_t)q * L.R + r) * L.slot_stride + s] = score;
-            if (a.V && r == 0) {
-              a.V[(int64_t)q * L.slot_stride + s] = ema_v(v_old, score, a.alpha, a.beta);
-              a.D[(int64_t)q * L.slot_stride + (ctx - 1 - s)] = ema_d(d_old, score, a.alpha, a.beta);
-            }
-          }
-        }
-        tc_fence_before();
+    int cur_q = -1;
+    float* wcur = wqs + ew * N;           // this warp's copy of the head weights
+    for (int g = g0 + group; g < g1; g += kEpiGroups) {
+      const int i = g - g0;
+      const int stage = i % stages, acc = i % nacc;
+      const uint32_t phase = (uint32_t)(i / stages) & 1u, acc_phase = (uint32_t)(i / nacc) & 1u;
+      // every lane waits; the warp leaves together if any lane gave up, so
+      // the .sync.aligned TMEM loads below never run on a partial warp
+      if (!__all_sync(0xffffffffu, wait_parity(B.f(stage), phase, ctl))) break;
+      const StageAux* x = aux + stage;
+      const int q = x->q;
+      if (q != cur_q) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(B.ae(acc));
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        for (int k = lane; k < N; k += 32) wcur[k] = a.wq[(int64_t)q * N + k];
+        __syncwarp();
+        cur_q = q;
+      }
+      const int64_t p0 = x->ctx - 1;
+      const bool present = pg_idx < x->np && x->valid[pg_idx];
+      const int64_t s = present ? (int64_t)x->j[pg_idx] * kPage + tok : 0;
+      const bool valid = present && s <= p0 + (a.rows - 1);
+      const float sigma = x->sigma[pg_idx][tok];
+      float v_old = 0.f, d_old = 0.f;
+      if (fused && valid && s <= p0) {
+        v_old = x->v[pg_idx][tok];
+        d_old = x->d[pg_idx][(p0 - s) - x->ws[pg_idx]];
+      }
+      if (!__all_sync(0xffffffffu, wait_parity(B.af(acc), acc_phase, ctl))) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
+      for (int r = 0; r < a.rows; ++r) {
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < L.H; c += 32) {
+          uint32_t v[32];
+          tmem_ld16(trow + (uint32_t)(r * L.H + c), *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          if (c + 16 < L.H) tmem_ld16(trow + (uint32_t)(r * L.H + c + 16), *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+          tmem_wait_ld();
+          const float* wr = wcur + r * L.H + c;
+          const int nu = min(32, L.H - c);
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            if (u < nu) part[u & 3] = __fmaf_rn(wr[u], fmaxf(__uint_as_float(v[u]), 0.0f), part[u & 3]);
+        }
+        const float sum = (part[0] + part[1]) + (part[2] + part[3]);
+        if (valid && s <= p0 + r) {
+          const float score = sum * sigma;
+          a.scores[((int64_t)q * L.R + r) * L.slot_stride + s] = score;
+          if (fused && r == 0) {
+            a.V[(int64_t)q * L.slot_stride + s] = ema_v(v_old, score, a.alpha, a.beta);
+            a.D[(int64_t)q * L.slot_stride + (p0 - s)] = ema_d(d_old, score, a.alpha, a.beta);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(B.ae(acc));
+        mbar_arrive(B.e(stage));
       }
     }
   }
@@ -454,8 +589,10 @@ bool encode_2d(EncodeTiledFn fn, CUtensorMap* map, const void* base, uint64_t ro
 
 bool tc_supported(const Layout& lay, int rows, int key_fp8) {
   const int N = rows * lay.H;
-  return key_fp8 && lay.d == 128 && lay.b == kPage && lay.H % 16 == 0 && N >= 16 && N <= 256 && N % 16 == 0 &&
-         smem_layout(N, lay.Q).total <= 227 * 1024;
+  if (!(key_fp8 && lay.d == 128 && lay.b == kPage && lay.H % 16 == 0 && N >= 16 && N <= 256 && N % 16 == 0))
+    return false;
+  const TcPlan plan = tc_plan(N, lay.Q);
+  return smem_layout(N, lay.Q, plan.stages).total <= 227 * 1024;
 }
 
 cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s) {
@@ -467,13 +604,14 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(encode_fn);
   if (!encode_2d(fn, &tk, a.keys, (uint64_t)a.num_pages * kPage, kPage)) return cudaErrorInvalidValue;
   if (!encode_2d(fn, &tq, a.q8, (uint64_t)L.Q * N, (uint32_t)N)) return cudaErrorInvalidValue;
-  const uint32_t smem = smem_layout(N, L.Q).total;
+  const TcPlan plan = tc_plan(N, L.Q);
+  const uint32_t smem = smem_layout(N, L.Q, plan.stages).total;
   cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  k_score_tc<<<sms, kThreads, smem, s>>>(a, tk, tq);
+  k_score_tc<<<sms * plan.ctas, kThreads, smem, s>>>(a, plan, tk, tq);
   return cudaGetLastError();
 }
 

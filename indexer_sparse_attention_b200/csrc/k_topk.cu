@@ -3,41 +3,105 @@
 // is).  Order: higher score first, ties to the lower slot; the chosen slots
 // are emitted in ascending slot order, padded with -1.
 //
-// One CTA (1024 threads) per (request, row).  Three MSB-first radix passes
-// (11 + 11 + 10 bits of the order-preserving key) over the scored slots find
-// the exact threshold key T and how many slots equal to T belong to the top
-// k.  A fourth pass marks every slot with key >= T in a shared-memory bitmap
-// indexed by position in the ascending kept-slot order; two block scans over
-// the bitmap then take the lowest-index ties and give each chosen slot its
-// output position, so the output is ascending without a sort.
+// One CTA (1024 threads) per (request, row); scores are read from HBM twice.
+//  1. A 13-bit histogram of the order-preserving score keys (sign, exponent
+//     and 4 mantissa bits) finds the bin holding the k-th largest key.
+//  2. Every scored slot whose key falls in that bin or above is collected
+//     into shared memory as (key, position in the ascending kept-slot order).
+//  3. An exact radix select over the candidates' remaining 19 key bits gives
+//     the threshold key T and how many keys equal to T belong to the top k.
+//  4. Chosen positions are set in a shared-memory bitmap; two block scans
+//     over it take the lowest-position ties and give each chosen slot its
+//     output index, so the output is ascending without a sort.
+// If the candidates do not fit on chip (a pathological score distribution)
+// step 2-3 fall back to three more full radix passes over HBM (exact).
+#include <algorithm>
+
 #include "spin_internal.cuh"
 #include "block_scan.cuh"
 
 namespace spin {
 
 constexpr int kTopkThreads = 1024;
+constexpr int kBins = 8192;           // 13-bit first digit
+constexpr int kFirstShift = 19;
+constexpr int kCandCap = 8192;        // candidates kept on chip
 
 struct TopkShared {
-  uint32_t hist[2048];
   uint32_t digit[2];
   int scan[33];
   int total;
+  int n_cand;
+  int overflow;
 };
 
+// Visits every scored slot (kept blocks, s <= p) as f(position, slot, key),
+// four float4 loads in flight per thread.
 template <class F>
-__device__ __forceinline__ void for_each_scored(const float* sc, const int32_t* work, int nk, int b,
-                                                int64_t p, F f) {
-  const int64_t n_elem = (int64_t)nk * b;
-  for (int64_t e = (int64_t)threadIdx.x * 4; e < n_elem; e += (int64_t)blockDim.x * 4) {
-    const int64_t j = work[e / b];
-    const int64_t s = j * b + (e % b);
-    if (s > p) continue;
-    const float4 v = *reinterpret_cast<const float4*>(sc + s);
-    f(e, s, fkey(v.x));
-    if (s + 1 <= p) f(e + 1, s + 1, fkey(v.y));
-    if (s + 2 <= p) f(e + 2, s + 2, fkey(v.z));
-    if (s + 3 <= p) f(e + 3, s + 3, fkey(v.w));
+__device__ __forceinline__ void for_each_scored(const float* sc, const int32_t* work, int nk, int lb, int p, F f) {
+  const int n_elem = nk << lb;
+  const int step = blockDim.x * 4;
+  for (int base = threadIdx.x * 4; base < n_elem; base += 4 * step) {
+    float4 v[4];
+    int s0[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = base + u * step;
+      s0[u] = -1;
+      if (e < n_elem) {
+        const int s = (work[e >> lb] << lb) + (e & ((1 << lb) - 1));
+        if (s <= p) {
+          s0[u] = s;
+          v[u] = *reinterpret_cast<const float4*>(sc + s);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0[u];
+      if (s < 0) continue;
+      const int e = base + u * step;
+      f(e, s, fkey(v[u].x));
+      if (s + 1 <= p) f(e + 1, s + 1, fkey(v[u].y));
+      if (s + 2 <= p) f(e + 2, s + 2, fkey(v[u].z));
+      if (s + 3 <= p) f(e + 3, s + 3, fkey(v[u].w));
+    }
   }
+}
+
+// Histogram add with the lanes of a warp that hit the same bin combined.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t mask = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(mask, bin);
+  const int leader = __ffs(peers) - 1;
+  if ((int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
+// Block-wide search of the bin holding the `want`-th largest element of a
+// histogram with nb bins (nb a positive multiple of blockDim.x): writes the
+// bin and the rank left inside it to digit[0..1].
+__device__ void block_find_bin_desc(const uint32_t* hist, int nb, uint32_t want, TopkShared& sh) {
+  const int per = nb / blockDim.x;
+  // thread t covers bins nb-1-t*per .. nb-per-t*per (from the top)
+  const int hi = nb - 1 - threadIdx.x * per;
+  uint32_t s = 0;
+  for (int i = 0; i < per; ++i) s += hist[hi - i];
+  int tot;
+  const uint32_t exc = (uint32_t)block_exclusive_scan((int)s, sh.scan, &tot);
+  if (exc < want && want <= exc + s) {
+    uint32_t cum = exc;
+    for (int i = 0; i < per; ++i) {
+      const uint32_t c = hist[hi - i];
+      if (cum + c >= want) {
+        sh.digit[0] = (uint32_t)(hi - i);
+        sh.digit[1] = want - cum;
+        break;
+      }
+      cum += c;
+    }
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
@@ -45,51 +109,71 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   const int q = blockIdx.x / a.rows, r = blockIdx.x % a.rows;
   int32_t* out = a.topk + ((int64_t)q * a.rows + r) * L.k;
   __shared__ TopkShared sh;
-  extern __shared__ uint32_t bits[];
+  extern __shared__ __align__(16) uint8_t dyn[];
   const int64_t ctx = a.ctx_len[q];
   if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {
     for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
   }
-  const int64_t p = ctx - 1 + r;
+  const int p = (int)(ctx - 1 + r);
   const int nk = a.kept[q];
   const int32_t* work = a.work + (int64_t)q * L.blk_stride;
   const float* sc = a.scores + ((int64_t)q * L.R + r) * L.slot_stride;
+  const int lb = __ffs(L.b) - 1;  // block size is a power of two
+  const int bmask = L.b - 1;
+  const int n_elem = nk << lb;
+  const int nwords = (n_elem + 31) / 32;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(dyn);
+  uint8_t* work_area = dyn + (((size_t)(L.slot_stride + 31) / 32) * 4 + 15) / 16 * 16;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(work_area);          // kBins (pass 1)
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(work_area);          // kCandCap (after pass 1)
+  uint32_t* cpos = ckey + kCandCap;
+  uint32_t* hist2 = cpos + kCandCap;                                // 256 bins (candidate passes)
 
-  // ---- radix passes -------------------------------------------------------
-  uint32_t prefix = 0, remaining = 0;
-  int shift_hi = 32;
-  const int shifts[3] = {21, 10, 0};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int sh_lo = shifts[pass];
-    const int width = shift_hi - sh_lo;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sh.hist[i] = 0;
-    __syncthreads();
-    for_each_scored(sc, work, nk, L.b, p, [&](int64_t, int64_t, uint32_t key) {
-      const bool match = (shift_hi == 32) || ((key >> shift_hi) == prefix);
-      if (match) atomicAdd(&sh.hist[(key >> sh_lo) & dmask], 1u);
-    });
-    __syncthreads();
-    if (pass == 0) {
-      // total scored and the rank wanted
-      int c = 0;
-      for (int i = threadIdx.x; i < 2048; i += blockDim.x) c += sh.hist[i];
-      int tot;
-      block_exclusive_scan(c, sh.scan, &tot);
-      if (threadIdx.x == 0) sh.total = tot;
-      __syncthreads();
-      remaining = (uint32_t)min(sh.total, L.k);
-      if (remaining == 0) break;
+  // ---- pass 1: 13-bit histogram ------------------------------------------
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+  if (threadIdx.x == 0) {
+    sh.n_cand = 0;
+    sh.overflow = 0;
+  }
+  __syncthreads();
+  {
+    const int step = blockDim.x * 4;
+    for (int it = 0; it < n_elem; it += 4 * step) {
+      const int base = it + threadIdx.x * 4;
+      float4 v[4];
+      int s0[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = base + u * step;
+        s0[u] = -1;
+        if (e < n_elem) {
+          const int s = (work[e >> lb] << lb) + (e & bmask);
+          if (s <= p) {
+            s0[u] = s;
+            v[u] = *reinterpret_cast<const float4*>(sc + s);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = s0[u];
+        const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool act = s >= 0 && s + c <= p;
+          hist_add(hist, act ? fkey(vals[c]) >> kFirstShift : 0u, act);
+        }
+      }
     }
-    if (threadIdx.x < 32) {
-      if (width == 11) warp_find_digit_desc<2048>(sh.hist, remaining, sh.digit);
-      else warp_find_digit_desc<1024>(sh.hist, remaining, sh.digit);
-    }
-    __syncthreads();
-    prefix = (prefix << width) | sh.digit[0];
-    remaining = sh.digit[1];
-    shift_hi = sh_lo;
+  }
+  __syncthreads();
+  {
+    int c = 0;
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) c += hist[i];
+    int tot;
+    block_exclusive_scan(c, sh.scan, &tot);
+    if (threadIdx.x == 0) sh.total = tot;
     __syncthreads();
   }
   const int want = min(sh.total, L.k);
@@ -97,18 +181,84 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
   }
-  const uint32_t T = prefix;
-  const uint32_t eq_take = remaining;
-
-  // ---- bitmap of keys >= T in kept-slot order -----------------------------
-  const int64_t n_elem = (int64_t)nk * L.b;
-  const int nwords = (int)((n_elem + 31) / 32);
-  for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+  block_find_bin_desc(hist, kBins, (uint32_t)want, sh);
+  const uint32_t d1 = sh.digit[0];
+  uint32_t remaining = sh.digit[1];
   __syncthreads();
-  for_each_scored(sc, work, nk, L.b, p, [&](int64_t e, int64_t, uint32_t key) {
-    if (key >= T) atomicOr(&bits[e >> 5], 1u << (e & 31));
+
+  // ---- pass 2: collect keys in bin d1 and above ------------------------------
+  // (the histogram area becomes the candidate list)
+  for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
+    if ((key >> kFirstShift) >= d1) {
+      const int slot = atomicAdd(&sh.n_cand, 1);
+      if (slot < kCandCap) {
+        ckey[slot] = key;
+        cpos[slot] = (uint32_t)e;
+      }
+    }
   });
   __syncthreads();
+  uint32_t T;
+  const int n_cand = sh.n_cand;
+  if (n_cand <= kCandCap) {
+    // ---- exact select among the candidates (rank counted from the top) -------
+    // elements above bin d1 are all chosen; `remaining` is the rank inside d1
+    uint32_t prefix = d1, pbits = 32 - kFirstShift;
+    const int shifts[3] = {11, 3, 0};
+    const int widths[3] = {8, 8, 3};
+    for (int ps = 0; ps < 3; ++ps) {
+      const int shf = shifts[ps], w = widths[ps];
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
+        const uint32_t k = ckey[i];
+        if ((k >> (32 - pbits)) == prefix) atomicAdd(&hist2[(k >> shf) & ((1u << w) - 1u)], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);  // bins >= 2^w are empty
+      __syncthreads();
+      prefix = (prefix << w) | sh.digit[0];
+      pbits += w;
+      remaining = sh.digit[1];
+      __syncthreads();
+    }
+    T = prefix;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
+      if (ckey[i] >= T) atomicOr(&bits[cpos[i] >> 5], 1u << (cpos[i] & 31));
+    __syncthreads();
+  } else {
+    // ---- fallback: three more full passes over HBM --------------------------
+    uint32_t prefix = d1;
+    int shift_hi = kFirstShift;
+    const int shifts[3] = {11, 3, 0};
+    for (int ps = 0; ps < 3; ++ps) {
+      const int sh_lo = shifts[ps];
+      const int width = shift_hi - sh_lo;
+      const uint32_t dmask = (1u << width) - 1u;
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+      __syncthreads();
+      for_each_scored(sc, work, nk, lb, p, [&](int, int, uint32_t key) {
+        if ((key >> shift_hi) == prefix) atomicAdd(&hist2[(key >> sh_lo) & dmask], 1u);
+      });
+      __syncthreads();
+      if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);
+      __syncthreads();
+      prefix = (prefix << width) | sh.digit[0];
+      remaining = sh.digit[1];
+      shift_hi = sh_lo;
+      __syncthreads();
+    }
+    T = prefix;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+    __syncthreads();
+    for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
+      if (key >= T) atomicOr(&bits[e >> 5], 1u << (e & 31));
+    });
+    __syncthreads();
+  }
+  const uint32_t eq_take = remaining;
 
   // ---- ordered tie handling and emission -----------------------------------
   const int chunk = (nwords + blockDim.x - 1) / blockDim.x;
@@ -119,8 +269,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     while (m) {
       const int bit = __ffs(m) - 1;
       m &= m - 1;
-      const int64_t e = (int64_t)w * 32 + bit;
-      const int64_t s = (int64_t)work[e / L.b] * L.b + (e % L.b);
+      const int e = w * 32 + bit;
+      const int s = (work[e >> lb] << lb) + (e & bmask);
       if (fkey(sc[s]) > T) ++n_gt; else ++n_eq;
     }
   }
@@ -134,8 +284,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     while (m) {
       const int bit = __ffs(m) - 1;
       m &= m - 1;
-      const int64_t e = (int64_t)w * 32 + bit;
-      const int64_t s = (int64_t)work[e / L.b] * L.b + (e % L.b);
+      const int e = w * 32 + bit;
+      const int s = (work[e >> lb] << lb) + (e & bmask);
       if (fkey(sc[s]) > T) {
         out[pos++] = (int32_t)s;
       } else {
@@ -147,8 +297,14 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   for (int t = want + threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
 }
 
+size_t topk_smem_bytes(const Layout& L) {
+  const size_t bitmap = ((size_t)(L.slot_stride + 31) / 32) * 4;
+  const size_t area = std::max<size_t>((size_t)kBins * 4, (size_t)kCandCap * 8 + 256 * 4);
+  return (bitmap + 15) / 16 * 16 + area;
+}
+
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)((a.lay.slot_stride + 31) / 32) * 4;
+  const size_t smem = topk_smem_bytes(a.lay);
   cudaError_t e = cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_topk<<<a.lay.Q * a.rows, kTopkThreads, smem, s>>>(a);

@@ -63,8 +63,8 @@ bool valid_config(const spin_config* c) {
   if (!(c->target_sparsity >= 0.0f && c->target_sparsity < 1.0f)) return false;
   const int64_t max_blocks = (c->max_slots + (int64_t)b - 1) / b;
   if (max_blocks > kMaxBlocksSelect) return false;
-  // top-k bitmap of one (request, row) lives in shared memory
-  if ((max_blocks * b + 31) / 32 * 4 > 200 * 1024) return false;
+  // top-k: bitmap of one (request, row) plus the candidate area on chip
+  if ((max_blocks * b + 31) / 32 * 4 > 160 * 1024) return false;
   // SIMT score kernel keeps the queries of a request and one page on chip
   const size_t simt = sizeof(float) * ((size_t)c->max_rows * c->num_heads * c->head_dim +
                                        (size_t)c->max_rows * c->num_heads + (size_t)b * (c->head_dim + 1));

@@ -173,24 +173,28 @@ def make_queries(wl: Workload, layer: int, positions: int, device="cpu"):
     starting at each request's ctx0: q [requests, positions, H, d] (bf16 or
     fp32), w [requests, positions, H] fp32."""
     Q, H, d = wl.requests, wl.H, wl.d
-    qs = torch.empty((Q, positions, H, d), dtype=torch.float32, device=device)
+    eps = torch.empty((Q, positions, H, d), dtype=torch.float32, device=device)
     ws = torch.empty((Q, positions, H), dtype=torch.float32, device=device)
+    plant = torch.empty((Q, positions, d), dtype=torch.float32, device=device)
     W = wl.per_layer(wl.diag_window, layer)
     omega = math.pi / (2 * W)
     rho = 0.95
     for q in range(Q):
         g = _gen(wl.seed, 5, layer, q, device)
-        eps = torch.randn((positions, H, d), generator=g, device=device, dtype=torch.float32)
+        eps[q] = torch.randn((positions, H, d), generator=g, device=device, dtype=torch.float32)
         ws[q] = torch.rand((positions, H), generator=g, device=device, dtype=torch.float32)
         u, e1, e2 = _planted_dirs(wl, layer, q, device)
-        x = eps[0]
-        P = wl.ctx0[q]
-        for t in range(positions):
-            if t > 0:
-                x = rho * x + math.sqrt(1 - rho * rho) * eps[t]
-            p = P + t
-            plant = math.sqrt(d) * (u + math.cos(omega * p) * e1 + math.sin(omega * p) * e2)
-            qs[q, t] = x + plant
+        p = wl.ctx0[q] + torch.arange(positions, device=device, dtype=torch.float64)
+        plant[q] = math.sqrt(d) * (u[None, :] + torch.cos(omega * p).float()[:, None] * e1[None, :]
+                                   + torch.sin(omega * p).float()[:, None] * e2[None, :])
+    qs = torch.empty((Q, positions, H, d), dtype=torch.float32, device=device)
+    x = eps[:, 0]
+    c = math.sqrt(1 - rho * rho)
+    for t in range(positions):
+        if t > 0:
+            x = rho * x + c * eps[:, t]
+        qs[:, t] = x + plant[:, t, None, :]
+    del eps
     if wl.q_bf16:
         return qs.to(torch.bfloat16), ws
     return qs, ws
