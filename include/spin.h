@@ -161,6 +161,31 @@ SPIN_API spin_status spin_indexer_score(spin_state st, int layer, int rows, cons
 SPIN_API spin_status spin_topk(spin_state st, int rows, const float* scores_dev, const uint8_t* mask_dev,
                       const int32_t* ctx_len_dev, int32_t* topk_dev, spin_stream_t stream);
 
+/* Token top-k for callers that cannot allocate device memory (no SPIN page
+ * has a counterpart to this call; it is a deployment convenience).  Code that
+ * runs during CUDA graph capture cannot call cudaMalloc, and some host
+ * applications or plug-in hosts own all device memory and give a library
+ * none, so they cannot hand spin_state_create a block.  This call needs no
+ * state: it computes exactly what spin_topk computes for the same scores,
+ * mask and context lengths, with its scratch (kept-block lists, counts and an
+ * error word) in a fixed 4 MiB array that the library reserves on every GPU
+ * that loads it, for the life of the process.  It allocates nothing.
+ *   scores_dev [num_requests][max_rows][ceil(max_slots/b)*b] fp32,
+ *   mask_dev [num_requests][ceil(max_slots/b)] uint8, ctx_len_dev [Q] int32,
+ *   topk_dev [num_requests][rows][topk] int32 out (same order and -1 padding
+ *   as spin_topk; rows whose ctx_len is out of range come back all -1).
+ * Limit: 4 + ceil(Q/64)*64 + Q * ceil(ceil(max_slots/b)/16)*16 must not
+ * exceed 2^20 (e.g. 96 requests at 512K slots with b = 64); larger problems
+ * return SPIN_EINVAL.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress), so make that first call before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU (on
+ * different streams, or from several host threads) race and must be
+ * serialised by the caller. */
+SPIN_API spin_status spin_topk_noalloc(int num_requests, int rows, int max_rows, int32_t max_slots,
+                                       int block_size, int topk, const float* scores_dev,
+                                       const uint8_t* mask_dev, const int32_t* ctx_len_dev,
+                                       int32_t* topk_dev, spin_stream_t stream);
+
 /* a5: EMA update of V (per slot) and D (per offset p_r - s) from the scores
  * of scored slots only (SPIN digest, 核心概要 / arXiv深度剖析; AI Radio, "The
  * paper's summary").  x <- score if x is the never-observed sentinel, else

@@ -23,7 +23,7 @@ __all__ = [
     "spin_decode_step", "spin_miss_count", "spin_allocate_layer_sparsity", "spin_get_error",
     "spin_set_layer_sparsity", "spin_set_score_kernel", "spin_reset_requests", "spin_set_fault_injection",
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
-    "spin_kernel_times", "STAGES",
+    "spin_kernel_times", "STAGES", "spin_topk_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,8 @@ def load():
         "spin_indexer_score": (S, [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp,
                                    _vp, _vp, _vp]),
         "spin_topk": (S, [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
+        "spin_topk_noalloc": (S, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32, ctypes.c_int, ctypes.c_int, _vp,
+                                  _vp, _vp, _vp, _vp]),
         "spin_ema_update": (S, [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
         "spin_decode_step": (S, [_vp, ctypes.c_int, ctypes.c_int, _i64, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp,
                                  ctypes.c_int, _vp, _vp, _vp, _vp]),
@@ -271,6 +273,16 @@ def spin_topk(st: SpinState, rows: int, scores, mask, ctx_len, topk, stream=None
     _check(load().spin_topk(st.handle, rows, _dev(scores, "scores", torch.float32), _dev(mask, "mask", torch.uint8),
                             _dev(ctx_len, "ctx_len", torch.int32), _dev(topk, "topk", torch.int32),
                             _stream(stream)), "spin_topk")
+
+
+def spin_topk_noalloc(num_requests: int, rows: int, max_rows: int, max_slots: int, block_size: int, k: int,
+                      scores, mask, ctx_len, topk, stream=None) -> None:
+    """Stateless top-k with the library's fixed scratch (no device allocation
+    anywhere); see include/spin.h for its size limit and sharing rules."""
+    _check(load().spin_topk_noalloc(num_requests, rows, max_rows, max_slots, block_size, k,
+                                    _dev(scores, "scores", torch.float32), _dev(mask, "mask", torch.uint8),
+                                    _dev(ctx_len, "ctx_len", torch.int32), _dev(topk, "topk", torch.int32),
+                                    _stream(stream)), "spin_topk_noalloc")
 
 
 def spin_ema_update(st: SpinState, layer: int, rows: int, scores, mask, ctx_len, accepted=None,
