@@ -3,18 +3,23 @@
 // is).  Order: higher score first, ties to the lower slot; the chosen slots
 // are emitted in ascending slot order, padded with -1.
 //
-// One CTA (1024 threads) per (request, row); scores are read from HBM twice.
+// One CTA (1024 threads) per (request, row).
 //  1. A 13-bit histogram of the order-preserving score keys (sign, exponent
-//     and 4 mantissa bits) finds the bin holding the k-th largest key.
-//  2. Every scored slot whose key falls in that bin or above is collected
-//     into shared memory as (key, position in the ascending kept-slot order).
-//  3. An exact radix select over the candidates' remaining 19 key bits gives
-//     the threshold key T and how many keys equal to T belong to the top k.
-//  4. Chosen positions are set in a shared-memory bitmap; two block scans
+//     and 4 mantissa bits) over a fixed 1/16 sample of the scored slots gives
+//     a lower threshold whose expected count is about 1.3 k.
+//  2. One pass over all scored slots appends every key at or above it to a
+//     shared-memory candidate list (key, position in the ascending kept-slot
+//     order), one atomic per warp.  If the list holds at least k keys it holds
+//     the whole top k, so the rest is exact:
+//  3. a radix select over the candidates (4 x 8-bit digits) gives the
+//     threshold key T and how many keys equal to T belong to the top k;
+//  4. chosen positions are set in a shared-memory bitmap; two block scans
 //     over it take the lowest-position ties and give each chosen slot its
 //     output index, so the output is ascending without a sort.
-// If the candidates do not fit on chip (a pathological score distribution)
-// step 2-3 fall back to three more full radix passes over HBM (exact).
+// When the estimate misses (fewer than k candidates, or more than fit), the
+// kernel falls back to an exact histogram of all keys, then a collection of
+// the keys in its threshold bin, then -- if even those do not fit -- three
+// more full radix passes.
 #include <algorithm>
 
 #include "spin_internal.cuh"
@@ -130,133 +135,252 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   uint32_t* cpos = ckey + kCandCap;
   uint32_t* hist2 = cpos + kCandCap;                                // 256 bins (candidate passes)
 
-  // ---- pass 1: 13-bit histogram ------------------------------------------
-  for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
-  if (threadIdx.x == 0) {
-    sh.n_cand = 0;
-    sh.overflow = 0;
-  }
-  __syncthreads();
+  // ---- number of scored slots -------------------------------------------
   {
-    const int step = blockDim.x * 4;
-    for (int it = 0; it < n_elem; it += 4 * step) {
-      const int base = it + threadIdx.x * 4;
-      float4 v[4];
-      int s0[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = base + u * step;
-        s0[u] = -1;
-        if (e < n_elem) {
-          const int s = (work[e >> lb] << lb) + (e & bmask);
-          if (s <= p) {
-            s0[u] = s;
-            v[u] = *reinterpret_cast<const float4*>(sc + s);
-          }
+    int c = 0;
+    for (int t = threadIdx.x; t < nk; t += blockDim.x) c += min(max(p - (work[t] << lb) + 1, 0), L.b);
+    int tot;
+    block_exclusive_scan(c, sh.scan, &tot);
+    if (threadIdx.x == 0) {
+      sh.total = tot;
+      sh.n_cand = 0;
+    }
+    __syncthreads();
+  }
+  const int total = sh.total;
+  const int want = min(total, L.k);
+  if (want == 0) {
+    for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
+    return;
+  }
+  uint32_t T = 0, remaining = 0;
+  bool done = false;
+
+  // ---- sampled threshold, one collecting pass, exact select on chip ---------
+  {
+    uint32_t t_lo = 0;  // keep everything when all scored slots fit
+    bool est_ok = true;
+    if (total > kCandCap) {
+      for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      const int n_smp = n_elem >> 6;  // one float4 out of every 64 scored positions
+      for (int it = 0; it < n_smp; it += blockDim.x) {
+        const int i = it + threadIdx.x;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        int s = -1;
+        if (i < n_smp) {
+          const int e = i << 6;
+          s = (work[e >> lb] << lb) + (e & bmask);
+          if (s <= p) v = *reinterpret_cast<const float4*>(sc + s);
         }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int s = s0[u];
-        const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        const float vals[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const bool act = s >= 0 && s + c <= p;
           hist_add(hist, act ? fkey(vals[c]) >> kFirstShift : 0u, act);
         }
       }
+      __syncthreads();
+      int c = 0;
+      for (int i = threadIdx.x; i < kBins; i += blockDim.x) c += hist[i];
+      int n_s;
+      block_exclusive_scan(c, sh.scan, &n_s);
+      const int ks = min(n_s, (int)ceilf(1.3f * (float)want * (float)n_s / (float)total) + 16);
+      if (ks >= 1) {
+        block_find_bin_desc(hist, kBins, (uint32_t)ks, sh);
+        t_lo = sh.digit[0] << kFirstShift;
+      } else {
+        est_ok = false;
+      }
+      __syncthreads();
     }
-  }
-  __syncthreads();
-  {
-    int c = 0;
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x) c += hist[i];
-    int tot;
-    block_exclusive_scan(c, sh.scan, &tot);
-    if (threadIdx.x == 0) sh.total = tot;
+    if (est_ok) {
+      // warp-uniform pass: a warp appends its takers with one atomic
+      const int step = blockDim.x * 4;
+      const int lane = threadIdx.x & 31;
+      for (int it = 0; it < n_elem; it += 4 * step) {
+        const int base = it + threadIdx.x * 4;
+        float4 v[4];
+        int s0[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = base + u * step;
+          s0[u] = -1;
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (e < n_elem) {
+            const int s = (work[e >> lb] << lb) + (e & bmask);
+            if (s <= p) {
+              s0[u] = s;
+              v[u] = *reinterpret_cast<const float4*>(sc + s);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t key = fkey(vals[c]);
+            const bool take = s0[u] >= 0 && s0[u] + c <= p && key >= t_lo;
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            if (bal) {
+              const int leader = __ffs(bal) - 1;
+              int at = 0;
+              if (lane == leader) at = atomicAdd(&sh.n_cand, __popc(bal));
+              at = __shfl_sync(0xffffffffu, at, leader) + __popc(bal & ((1u << lane) - 1u));
+              if (take && at < kCandCap) {
+                ckey[at] = key;
+                cpos[at] = (uint32_t)(base + u * step + c);
+              }
+            }
+          }
+        }
+      }
+      __syncthreads();
+      const int n_cand = sh.n_cand;
+      if (n_cand >= want && n_cand <= kCandCap) {
+        uint32_t prefix = 0, rem = (uint32_t)want;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+          for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+          __syncthreads();
+          const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+          for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
+            const uint32_t k = ckey[i];
+            if ((k & pmask) == prefix) atomicAdd(&hist2[(k >> shift) & 255u], 1u);
+          }
+          __syncthreads();
+          if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, rem, sh.digit);
+          __syncthreads();
+          prefix |= sh.digit[0] << shift;
+          rem = sh.digit[1];
+          __syncthreads();
+        }
+        T = prefix;
+        remaining = rem;
+        for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
+          if (ckey[i] >= T) atomicOr(&bits[cpos[i] >> 5], 1u << (cpos[i] & 31));
+        __syncthreads();
+        done = true;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) sh.n_cand = 0;
     __syncthreads();
   }
-  const int want = min(sh.total, L.k);
-  if (want == 0) {
-    for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
-    return;
-  }
-  block_find_bin_desc(hist, kBins, (uint32_t)want, sh);
-  const uint32_t d1 = sh.digit[0];
-  uint32_t remaining = sh.digit[1];
-  __syncthreads();
 
-  // ---- pass 2: collect keys in bin d1 and above ------------------------------
-  // (the histogram area becomes the candidate list)
-  for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
-    if ((key >> kFirstShift) >= d1) {
-      const int slot = atomicAdd(&sh.n_cand, 1);
-      if (slot < kCandCap) {
-        ckey[slot] = key;
-        cpos[slot] = (uint32_t)e;
+  if (!done) {
+    // ---- pass 1: 13-bit histogram ------------------------------------------
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    {
+      const int step = blockDim.x * 4;
+      for (int it = 0; it < n_elem; it += 4 * step) {
+        const int base = it + threadIdx.x * 4;
+        float4 v[4];
+        int s0[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = base + u * step;
+          s0[u] = -1;
+          if (e < n_elem) {
+            const int s = (work[e >> lb] << lb) + (e & bmask);
+            if (s <= p) {
+              s0[u] = s;
+              v[u] = *reinterpret_cast<const float4*>(sc + s);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int s = s0[u];
+          const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const bool act = s >= 0 && s + c <= p;
+            hist_add(hist, act ? fkey(vals[c]) >> kFirstShift : 0u, act);
+          }
+        }
       }
     }
-  });
-  __syncthreads();
-  uint32_t T;
-  const int n_cand = sh.n_cand;
-  if (n_cand <= kCandCap) {
-    // ---- exact select among the candidates (rank counted from the top) -------
-    // elements above bin d1 are all chosen; `remaining` is the rank inside d1
-    uint32_t prefix = d1, pbits = 32 - kFirstShift;
-    const int shifts[3] = {11, 3, 0};
-    const int widths[3] = {8, 8, 3};
-    for (int ps = 0; ps < 3; ++ps) {
-      const int shf = shifts[ps], w = widths[ps];
-      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
-      __syncthreads();
-      for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
-        const uint32_t k = ckey[i];
-        if ((k >> (32 - pbits)) == prefix) atomicAdd(&hist2[(k >> shf) & ((1u << w) - 1u)], 1u);
-      }
-      __syncthreads();
-      if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);  // bins >= 2^w are empty
-      __syncthreads();
-      prefix = (prefix << w) | sh.digit[0];
-      pbits += w;
-      remaining = sh.digit[1];
-      __syncthreads();
-    }
-    T = prefix;
-    for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
-      if (ckey[i] >= T) atomicOr(&bits[cpos[i] >> 5], 1u << (cpos[i] & 31));
+    block_find_bin_desc(hist, kBins, (uint32_t)want, sh);
+    const uint32_t d1 = sh.digit[0];
+    remaining = sh.digit[1];
     __syncthreads();
-  } else {
-    // ---- fallback: three more full passes over HBM --------------------------
-    uint32_t prefix = d1;
-    int shift_hi = kFirstShift;
-    const int shifts[3] = {11, 3, 0};
-    for (int ps = 0; ps < 3; ++ps) {
-      const int sh_lo = shifts[ps];
-      const int width = shift_hi - sh_lo;
-      const uint32_t dmask = (1u << width) - 1u;
-      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
-      __syncthreads();
-      for_each_scored(sc, work, nk, lb, p, [&](int, int, uint32_t key) {
-        if ((key >> shift_hi) == prefix) atomicAdd(&hist2[(key >> sh_lo) & dmask], 1u);
-      });
-      __syncthreads();
-      if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);
-      __syncthreads();
-      prefix = (prefix << width) | sh.digit[0];
-      remaining = sh.digit[1];
-      shift_hi = sh_lo;
-      __syncthreads();
-    }
-    T = prefix;
-    for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
-    __syncthreads();
+
+    // ---- pass 2: collect keys in bin d1 and above ------------------------------
+    // (the histogram area becomes the candidate list)
     for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
-      if (key >= T) atomicOr(&bits[e >> 5], 1u << (e & 31));
+      if ((key >> kFirstShift) >= d1) {
+        const int slot = atomicAdd(&sh.n_cand, 1);
+        if (slot < kCandCap) {
+          ckey[slot] = key;
+          cpos[slot] = (uint32_t)e;
+        }
+      }
     });
     __syncthreads();
+    const int n_cand = sh.n_cand;
+    if (n_cand <= kCandCap) {
+      // ---- exact select among the candidates (rank counted from the top) -------
+      // elements above bin d1 are all chosen; `remaining` is the rank inside d1
+      uint32_t prefix = d1, pbits = 32 - kFirstShift;
+      const int shifts[3] = {11, 3, 0};
+      const int widths[3] = {8, 8, 3};
+      for (int ps = 0; ps < 3; ++ps) {
+        const int shf = shifts[ps], w = widths[ps];
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
+          const uint32_t k = ckey[i];
+          if ((k >> (32 - pbits)) == prefix) atomicAdd(&hist2[(k >> shf) & ((1u << w) - 1u)], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);  // bins >= 2^w are empty
+        __syncthreads();
+        prefix = (prefix << w) | sh.digit[0];
+        pbits += w;
+        remaining = sh.digit[1];
+        __syncthreads();
+      }
+      T = prefix;
+      for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
+        if (ckey[i] >= T) atomicOr(&bits[cpos[i] >> 5], 1u << (cpos[i] & 31));
+      __syncthreads();
+    } else {
+      // ---- fallback: three more full passes over HBM --------------------------
+      uint32_t prefix = d1;
+      int shift_hi = kFirstShift;
+      const int shifts[3] = {11, 3, 0};
+      for (int ps = 0; ps < 3; ++ps) {
+        const int sh_lo = shifts[ps];
+        const int width = shift_hi - sh_lo;
+        const uint32_t dmask = (1u << width) - 1u;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+        __syncthreads();
+        for_each_scored(sc, work, nk, lb, p, [&](int, int, uint32_t key) {
+          if ((key >> shift_hi) == prefix) atomicAdd(&hist2[(key >> sh_lo) & dmask], 1u);
+        });
+        __syncthreads();
+        if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);
+        __syncthreads();
+        prefix = (prefix << width) | sh.digit[0];
+        remaining = sh.digit[1];
+        shift_hi = sh_lo;
+        __syncthreads();
+      }
+      T = prefix;
+      for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+      __syncthreads();
+      for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
+        if (key >= T) atomicOr(&bits[e >> 5], 1u << (e & 31));
+      });
+      __syncthreads();
+    }
   }
   const uint32_t eq_take = remaining;
 

@@ -242,3 +242,42 @@ def test_miss_count():
             frac = oracle.miss_fraction(full[qq, r], m[qq], 64)
             assert total[qq, r].item() == k - 7
             assert abs(missed[qq, r].item() / (k - 7) - frac) < 1e-12
+
+
+@pytest.mark.parametrize("pattern", ["hidden_from_sample", "only_in_sample", "all_equal", "heavy_ties"])
+def test_topk_fallback_paths_bit_exact(pattern):
+    """Score patterns that defeat the sampled threshold estimate (the sample
+    reads 4 of every 64 kept-slot positions) or overflow the on-chip
+    candidate list, so each exact fallback of the top-k kernel runs."""
+    rng = np.random.default_rng(len(pattern))
+    Q, R, k = 2, 1, 2048
+    st = make_state(Q=Q, max_slots=64 * 600, R=R, k=k)
+    ctx = np.array([64 * 600, 64 * 431 + 9], np.int64)
+    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.8).astype(np.uint8)
+    for qq in range(Q):
+        m[qq, oracle.num_blocks(int(ctx[qq]), R - 1, 64):] = 0
+    scores = st.new_scores()
+    vals = rng.uniform(0, 1, scores.shape).astype(np.float32)
+    pos = np.zeros(scores.shape, np.int64)
+    for qq in range(Q):       # position of each slot in the ascending kept-slot order
+        kept = np.nonzero(m[qq])[0]
+        slots = (kept[:, None] * 64 + np.arange(64)[None, :]).ravel()
+        pos[qq, 0, slots[slots < st.score_stride]] = np.arange(slots.size)[slots < st.score_stride]
+    sampled = (pos % 64) < 4
+    if pattern == "hidden_from_sample":
+        vals[~sampled] += 100.0
+    elif pattern == "only_in_sample":
+        vals[sampled] += 100.0
+    elif pattern == "all_equal":
+        vals[:] = 3.0
+    else:
+        vals = rng.integers(0, 3, scores.shape).astype(np.float32)
+    scores.copy_(torch.from_numpy(vals))
+    topk = torch.empty((Q, R, k), dtype=torch.int32, device="cuda")
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    isa.spin_topk(st, R, scores, torch.from_numpy(m).cuda(), ctx_t, topk)
+    assert isa.spin_get_error(st)[0] == 0
+    got = topk.cpu().numpy()
+    for qq in range(Q):
+        ref = oracle.topk_row(vals[qq, 0].astype(np.float64), m[qq], int(ctx[qq]), 0, 64, k)
+        assert np.array_equal(got[qq, 0], ref), (pattern, qq)
