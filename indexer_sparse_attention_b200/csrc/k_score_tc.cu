@@ -14,25 +14,27 @@
 //
 // Warp roles (320 threads, persistent, two CTAs per SM when N <= 128):
 //   warp 0      producer: lanes gather the tile metadata one and two batches
-//               of 32 tiles ahead; lane 0 handles the query tile (per request)
-//               and the stage barriers; eight lanes issue a tile's copies in
-//               one step (key pages by TMA; the pages' scales and EMA slices
-//               by bulk copies).  One issuing warp per CTA caps the copy rate,
-//               so a second CTA per SM doubles it.
+//               of 32 tiles ahead; lane 0 handles the query tile (per request),
+//               the stage barriers and the tile-info ring; two lanes issue the
+//               tile's two key-page TMA loads.  The copy engine's cost is per
+//               request, so it moves only key pages; a second CTA per SM adds
+//               a second issuer.
 //   warp 1      TMEM allocation; lane 0 issues the MMAs and the commits
 //   warps 2..9  two epilogue groups of four warps, taking alternate tiles; a
-//               warp reads the accumulator quarter it may access (lanes
-//               32*(warp%4) ..), applies ReLU, head weights and the scale,
-//               stores the scores and the fused EMA update
-// Pipelines: 4 stages per CTA (8 with one CTA per SM) of keys + side data,
-// 2 query buffers, 4 TMEM accumulators (2 when N > 64), so that all CTAs of
-// an SM fit the 512 TMEM columns.  Every wait is bounded (2 s of
+//               thread owns one token: it loads the token's scale and EMA
+//               values one tile ahead, reads its accumulator row from the TMEM
+//               quarter its warp may access (lanes 32*(warp%4) ..), applies
+//               ReLU, head weights and the scale, and stores the score and the
+//               fused EMA update
+// Pipelines: key stages freed as soon as the MMAs have read them (5 per CTA
+// at N = 64, 8 with one CTA per SM); a 16-slot ring of tile info freed by the
+// epilogue; 2 query buffers; 4 TMEM accumulators (2 when N > 64), so that all
+// CTAs of an SM fit the 512 TMEM columns.  Every wait is bounded (2 s of
 // %globaltimer); on expiry the CTA raises ERR_TIMEOUT, stops issuing, drains
 // what it issued and frees TMEM.
 #include <cuda.h>
 
 #include <algorithm>
-#include <cstddef>
 
 #include "spin_internal.cuh"
 
@@ -171,23 +173,17 @@ struct Sched {
   }
 };
 
-// Per-stage side data copied with the keys: the two pages' scales, and for
-// the fused EMA the vertical states of the two blocks and a 16-byte aligned
-// window of the diagonal states they touch, plus the tile's metadata.
-constexpr int kDWin = 68;  // floats: 64 offsets + up to 3 below for 16-byte alignment
-struct StageAux {
-  float sigma[2][kPage];
-  float v[2][kPage];
-  float d[2][kDWin];
-  int q, ctx, np, fused;
-  int j[2], valid[2], ws[2];
-  int pad[2];
+// Tile metadata the producer hands to the epilogue through a small ring in
+// shared memory (the copy engine moves only key pages: its cost is per request,
+// so the per-token scales and EMA values are read by the epilogue threads).
+struct TileInfo {
+  int q, ctx, np, pad;
+  int j[2], pg[2];  // block ids and pages; pg < 0 marks a page outside the cache
 };
-static_assert(sizeof(StageAux) % 16 == 0, "aux must keep 16-byte alignment");
 
 struct SmemLayout {
   uint32_t keys;     // stages * kStageBytes
-  uint32_t aux;      // stages * sizeof(StageAux)
+  uint32_t aux;      // kAuxSlots * sizeof(TileInfo)
   uint32_t qbuf;     // 2 * N * 128
   uint32_t wq;       // 4 * kEpiGroups * N floats: one copy per epilogue warp
   uint32_t prefix;   // (Q + 1) ints
@@ -197,6 +193,7 @@ struct SmemLayout {
 
 constexpr int kMaxStages = 8;
 constexpr int kMaxAcc = 4;
+constexpr int kAuxSlots = 16;  // tile-info ring: freed by the epilogue, not by the MMA
 
 __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
   SmemLayout s;
@@ -204,7 +201,7 @@ __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
   s.keys = off;
   off += stages * kStageBytes;
   s.aux = off;
-  off += stages * (uint32_t)sizeof(StageAux);
+  off += kAuxSlots * (uint32_t)sizeof(TileInfo);
   off = (off + 1023) / 1024 * 1024;
   s.qbuf = off;
   off += 2 * N * kRowBytes;
@@ -213,7 +210,7 @@ __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
   s.prefix = off;
   off += ((Q + 1) * 4 + 15) / 16 * 16;
   s.bars = off;
-  off += (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) * 8 + 16;
+  off += (2 * kMaxStages + 2 * kAuxSlots + 4 + 2 * kMaxAcc + 1) * 8 + 16;
   s.total = off + 1024;  // slack for 1024-byte alignment of the base
   return s;
 }
@@ -226,26 +223,26 @@ struct TcPlan {
 };
 
 __host__ __device__ inline TcPlan tc_plan(int N, int Q) {
-  if (N <= 64 && smem_layout(N, Q, 4).total * 2 <= 227 * 1024) return {4, 4, 2};
-  if (N <= 128 && smem_layout(N, Q, 4).total * 2 <= 227 * 1024) return {4, 2, 2};
+  // two CTAs share an SM's 228 KB when each takes <= 113 KB (1 KB per CTA is reserved)
+  constexpr uint32_t kTwoPerSm = 115712;
+  if (N <= 128)
+    for (int st = kMaxStages; st >= 3; --st)
+      if (smem_layout(N, Q, st).total <= kTwoPerSm) return {st, N <= 64 ? 4 : 2, 2};
   return {kMaxStages, 2, 1};
 }
 
 struct Bars {
-  uint32_t full, empty, qfull, qempty, accfull, accempty, done;
+  uint32_t full, empty, afull, aempty, qfull, qempty, accfull, accempty, done;
   __device__ uint32_t f(int s) const { return full + 8 * s; }
   __device__ uint32_t e(int s) const { return empty + 8 * s; }
+  __device__ uint32_t xf(int s) const { return afull + 8 * s; }
+  __device__ uint32_t xe(int s) const { return aempty + 8 * s; }
   __device__ uint32_t qf(int i) const { return qfull + 8 * i; }
   __device__ uint32_t qe(int i) const { return qempty + 8 * i; }
   __device__ uint32_t af(int i) const { return accfull + 8 * i; }
   __device__ uint32_t ae(int i) const { return accempty + 8 * i; }
 };
 
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"((uint64_t)src), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // Tile metadata, gathered by one producer lane per tile in two phases one
 // batch apart, so no load result is needed before a batch later:
@@ -301,16 +298,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const SmemLayout lay = smem_layout(N, L.Q, stages);
   const uint32_t sbase = smem_u32(smem);
-  StageAux* aux = reinterpret_cast<StageAux*>(smem + lay.aux);
+  TileInfo* aux = reinterpret_cast<TileInfo*>(smem + lay.aux);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
   float* wqs = reinterpret_cast<float*>(smem + lay.wq);
   uint64_t* bar_mem = reinterpret_cast<uint64_t*>(smem + lay.bars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mem + 2 * kMaxStages + 4 + 2 * kMaxAcc + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mem + 2 * kMaxStages + 2 * kAuxSlots + 4 + 2 * kMaxAcc + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   Bars B;
   B.full = smem_u32(bar_mem);
   B.empty = B.full + 8 * kMaxStages;
-  B.qfull = B.empty + 8 * kMaxStages;
+  B.afull = B.empty + 8 * kMaxStages;
+  B.aempty = B.afull + 8 * kAuxSlots;
+  B.qfull = B.aempty + 8 * kAuxSlots;
   B.qempty = B.qfull + 16;
   B.accfull = B.qempty + 16;
   B.accempty = B.accfull + 8 * kMaxAcc;
@@ -332,7 +331,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     *abort_flag = 0;
     for (int s = 0; s < stages; ++s) {
       mbar_init(B.f(s), 1);
-      mbar_init(B.e(s), 1 + 4);  // the MMA commit and the four epilogue warps
+      mbar_init(B.e(s), 1);  // the MMA commit: keys are free once the MMAs read them
+    }
+    for (int s = 0; s < kAuxSlots; ++s) {
+      mbar_init(B.xf(s), 1);  // the producer's arrive after writing the tile info
+      mbar_init(B.xe(s), 4);  // the four epilogue warps of the group that owns the tile
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(B.qf(i), 1);
@@ -368,6 +371,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     int stage = 0;
     uint32_t phase = 0;
     int cur_q = -1, qiter = 0;
+    int xslot = 0;
+    uint32_t xphase = 0;
     int inflight[kMaxStages];
     for (int i = 0; i < kMaxStages; ++i) inflight[i] = -1;
     bool withhold = a.inject && blockIdx.x == 0;
@@ -376,9 +381,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     meta_phase_a(cur, a, sched, prefix, g0 + lane, g1);
     meta_phase_b(cur, a);
     meta_phase_a(nxt, a, sched, prefix, g0 + 32 + lane, g1);
-    // copy slot of this lane within a tile: page k = lane / 4, kind = lane % 4
-    // (0 key page, 1 scales, 2 vertical EMA slice, 3 diagonal EMA window)
-    const int ck = lane >> 2, ckind = lane & 3;
     for (int gb = g0; gb < g1 && !stop; gb += 32) {
       meta_phase_b(nxt, a);                                        // block ids arrived a batch ago
       meta_phase_a(nxt2, a, sched, prefix, gb + 64 + lane, g1);    // used two batches later
@@ -388,7 +390,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int np = (2 * m.t + 1 < m.kept) ? 2 : 1;
         const int pg0 = (m.pg0 >= 0 && m.pg0 < a.num_pages) ? m.pg0 : -1;
         const int pg1 = (np == 2 && m.pg1 >= 0 && m.pg1 < a.num_pages) ? m.pg1 : -1;
-        const int p0 = m.ctx - 1;
         int ok = 1;
         if (lane == 0) {
           if (m.q != cur_q) {
@@ -400,26 +401,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
           if (ok) ok = wait_parity(B.e(stage), phase ^ 1, ctl);
+          if (ok) ok = wait_parity(B.xe(xslot), xphase ^ 1, ctl);
           if (ok) {
             if (pg0 < 0) raise_error(a.err, ERR_PAGE, m.q, (uint32_t)m.pg0);
             if (np == 2 && pg1 < 0) raise_error(a.err, ERR_PAGE, m.q, (uint32_t)m.pg1);
-            StageAux* x = aux + stage;
+            TileInfo* x = aux + xslot;
             x->q = m.q;
             x->ctx = m.ctx;
             x->np = np;
-            x->fused = fused ? 1 : 0;
-            x->valid[0] = pg0 >= 0;
-            x->valid[1] = pg1 >= 0;
             x->j[0] = m.j0;
             x->j[1] = m.j1;
-            uint32_t bytes = 0;
-            for (int k = 0; k < np; ++k) {
-              const int dlo = p0 - ((k ? m.j1 : m.j0) * kPage + kPage - 1);
-              x->ws[k] = (dlo > 0 ? dlo : 0) & ~3;
-              bytes += kPageBytes + kPage * 4 + (fused ? kPage * 4 + kDWin * 4 : 0);
-            }
+            x->pg[0] = pg0;
+            x->pg[1] = pg1;
+            mbar_arrive(B.xf(xslot));  // release: the epilogue's wait sees the info
             if (!withhold) {
-              mbar_expect_tx(B.f(stage), bytes);
+              mbar_expect_tx(B.f(stage), (uint32_t)(np * kPageBytes));
               inflight[stage] = (int)phase;
             }
           }
@@ -429,27 +425,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (m.q != cur_q) { cur_q = m.q; ++qiter; }
         const bool issue = !__shfl_sync(0xffffffffu, withhold ? 1 : 0, 0);
         withhold = false;  // test hook: at most the first stage is withheld
-        if (issue && ck < np && (ckind < 2 || fused)) {
-          const int j = ck ? m.j1 : m.j0;
-          const int pg = ck ? (pg1 < 0 ? 0 : pg1) : (pg0 < 0 ? 0 : pg0);  // bad pages load page 0; skipped later
-          const uint32_t bar = B.f(stage);
-          const uint32_t xdst = smem_u32(aux + stage);
-          if (ckind == 0) {
-            tma_load_2d(sbase + lay.keys + stage * kStageBytes + ck * kPageBytes, &tmap_k, bar, 0, pg * kPage);
-          } else if (ckind == 1) {
-            bulk_g2s(xdst + (uint32_t)offsetof(StageAux, sigma) + ck * kPage * 4, a.kscale + (int64_t)pg * kPage,
-                     kPage * 4, bar);
-          } else if (ckind == 2) {
-            bulk_g2s(xdst + (uint32_t)offsetof(StageAux, v) + ck * kPage * 4,
-                     a.V + (int64_t)m.q * L.slot_stride + (int64_t)j * kPage, kPage * 4, bar);
-          } else {
-            const int dlo = p0 - (j * kPage + kPage - 1);
-            const int ws = (dlo > 0 ? dlo : 0) & ~3;
-            bulk_g2s(xdst + (uint32_t)offsetof(StageAux, d) + ck * kDWin * 4,
-                     a.D + (int64_t)m.q * L.slot_stride + ws, kDWin * 4, bar);
-          }
+        if (issue && lane < np) {
+          const int pg = lane ? (pg1 < 0 ? 0 : pg1) : (pg0 < 0 ? 0 : pg0);  // bad pages load page 0; skipped later
+          tma_load_2d(sbase + lay.keys + stage * kStageBytes + lane * kPageBytes, &tmap_k, B.f(stage), 0, pg * kPage);
         }
         if (++stage == stages) { stage = 0; phase ^= 1; }
+        if (++xslot == kAuxSlots) { xslot = 0; xphase ^= 1; }
       }
       cur = nxt;
       nxt = nxt2;
@@ -506,31 +487,45 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int pg_idx = m >> 6, tok = m & 63;
     int cur_q = -1;
     float* wcur = wqs + ew * N;           // this warp's copy of the head weights
-    for (int g = g0 + group; g < g1; g += kEpiGroups) {
-      const int i = g - g0;
-      const int stage = i % stages, acc = i % nacc;
-      const uint32_t phase = (uint32_t)(i / stages) & 1u, acc_phase = (uint32_t)(i / nacc) & 1u;
+    const int n_local = g1 - g0;
+    // Per-token operands of a tile, loaded one tile (of this group) ahead.
+    struct Pre {
+      int q, s, valid, upd;
+      int64_t p0;
+      float sigma, v, d;
+    };
+    auto prefetch = [&](int i, Pre& r) -> bool {
+      const int xs = i % kAuxSlots;
+      const uint32_t xph = (uint32_t)(i / kAuxSlots) & 1u;
+      if (!__all_sync(0xffffffffu, wait_parity(B.xf(xs), xph, ctl))) return false;
+      const TileInfo* x = aux + xs;
+      r.q = x->q;
+      r.p0 = x->ctx - 1;
+      const int pg = x->pg[pg_idx];
+      const bool present = pg_idx < x->np && pg >= 0;
+      r.s = present ? x->j[pg_idx] * kPage + tok : 0;
+      r.valid = present && r.s <= r.p0 + (a.rows - 1);
+      r.upd = fused && r.valid && r.s <= r.p0;
+      r.sigma = r.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
+      r.v = r.upd ? a.V[(int64_t)r.q * L.slot_stride + r.s] : 0.f;
+      r.d = r.upd ? a.D[(int64_t)r.q * L.slot_stride + (r.p0 - r.s)] : 0.f;
+      return true;
+    };
+    Pre nx;
+    bool alive_ = group < n_local && prefetch(group, nx);
+    for (int i = group; alive_ && i < n_local; i += kEpiGroups) {
+      const Pre cur = nx;
+      if (i + kEpiGroups < n_local && !prefetch(i + kEpiGroups, nx)) break;
+      const int xs = i % kAuxSlots, acc = i % nacc;
+      const uint32_t acc_phase = (uint32_t)(i / nacc) & 1u;
+      if (cur.q != cur_q) {
+        __syncwarp();
+        for (int k = lane; k < N; k += 32) wcur[k] = a.wq[(int64_t)cur.q * N + k];
+        __syncwarp();
+        cur_q = cur.q;
+      }
       // every lane waits; the warp leaves together if any lane gave up, so
       // the .sync.aligned TMEM loads below never run on a partial warp
-      if (!__all_sync(0xffffffffu, wait_parity(B.f(stage), phase, ctl))) break;
-      const StageAux* x = aux + stage;
-      const int q = x->q;
-      if (q != cur_q) {
-        __syncwarp();
-        for (int k = lane; k < N; k += 32) wcur[k] = a.wq[(int64_t)q * N + k];
-        __syncwarp();
-        cur_q = q;
-      }
-      const int64_t p0 = x->ctx - 1;
-      const bool present = pg_idx < x->np && x->valid[pg_idx];
-      const int64_t s = present ? (int64_t)x->j[pg_idx] * kPage + tok : 0;
-      const bool valid = present && s <= p0 + (a.rows - 1);
-      const float sigma = x->sigma[pg_idx][tok];
-      float v_old = 0.f, d_old = 0.f;
-      if (fused && valid && s <= p0) {
-        v_old = x->v[pg_idx][tok];
-        d_old = x->d[pg_idx][(p0 - s) - x->ws[pg_idx]];
-      }
       if (!__all_sync(0xffffffffu, wait_parity(B.af(acc), acc_phase, ctl))) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
@@ -548,12 +543,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (u < nu) part[u & 3] = __fmaf_rn(wr[u], fmaxf(__uint_as_float(v[u]), 0.0f), part[u & 3]);
         }
         const float sum = (part[0] + part[1]) + (part[2] + part[3]);
-        if (valid && s <= p0 + r) {
-          const float score = sum * sigma;
-          a.scores[((int64_t)q * L.R + r) * L.slot_stride + s] = score;
-          if (fused && r == 0) {
-            a.V[(int64_t)q * L.slot_stride + s] = ema_v(v_old, score, a.alpha, a.beta);
-            a.D[(int64_t)q * L.slot_stride + (p0 - s)] = ema_d(d_old, score, a.alpha, a.beta);
+        if (cur.valid && cur.s <= cur.p0 + r) {
+          const float score = sum * cur.sigma;
+          a.scores[((int64_t)cur.q * L.R + r) * L.slot_stride + cur.s] = score;
+          if (cur.upd && r == 0) {
+            a.V[(int64_t)cur.q * L.slot_stride + cur.s] = ema_v(cur.v, score, a.alpha, a.beta);
+            a.D[(int64_t)cur.q * L.slot_stride + (cur.p0 - cur.s)] = ema_d(cur.d, score, a.alpha, a.beta);
           }
         }
       }
@@ -561,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(B.ae(acc));
-        mbar_arrive(B.e(stage));
+        mbar_arrive(B.xe(xs));
       }
     }
   }
