@@ -82,12 +82,27 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: every rank takes the same collective step."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(rank: int, requests: int, spare_slots: int):
+    """The serving workload a rank runs: the same shape on every rank, its
+    own seeded data (requests are independent, so ranks share nothing)."""
+    base = workloads.config(2)
+    return workloads.config(2, seed=base.seed + 1000 * rank, steps=1, spare_slots=spare_slots,
+                            requests=requests, ctx0=base.ctx0[:1] * requests)
+
+
+def job_rows_per_s(rows_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's rows over the slowest rank's time."""
+    return world * rows_per_rank / (max_ms / 1e3)
 
 
 class ClockSampler:
@@ -292,9 +307,7 @@ def gpu_arm(args, world, rank, local):
     W, K = args.warmup, args.steps
     sweep = [] if args.no_sweep else [0.4, 0.0]
     total = 1 + (W + K) * (1 + len(sweep)) + 3 + K + 2
-    base = workloads.config(2)
-    wl = workloads.config(2, seed=base.seed + 1000 * rank, steps=1, spare_slots=total + 8,
-                          requests=args.requests, ctx0=base.ctx0[:1] * args.requests)
+    wl = rank_workload(rank, args.requests, total + 8)
     run = SpinRun(wl, device, total)
     Q = wl.requests
     # history bootstrap: all-keep step that fills V and D
@@ -315,7 +328,7 @@ def gpu_arm(args, world, rank, local):
     if status != 0:
         raise RuntimeError(f"device error word {word:#x} during the timed region")
     ms_step = ms / K
-    rows_s = world * Q * K / (ms / 1e3)
+    rows_s = job_rows_per_s(Q * K, world, ms)
     key_gbs = kept_slots * KEY_BYTES_PER_SLOT / (ms_step / 1e3) / 1e9
     peak, peak_kind = peaks()
     score_ms, score_n = stages["score"]
@@ -356,7 +369,7 @@ def gpu_arm(args, world, rank, local):
     out["fidelity"] = fidelity(run)
     # ---- end to end with host buffers --------------------------------------
     e2e_ms, h2d, d2h = e2e_pass(run, K, world)
-    out["e2e"] = {"value": world * Q * K / (e2e_ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": h2d,
+    out["e2e"] = {"value": job_rows_per_s(Q * K, world, e2e_ms), "unit": "rows/s", "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
     status, word = isa.spin_get_error(run.st)
     if status != 0:

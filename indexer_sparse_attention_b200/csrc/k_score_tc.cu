@@ -26,10 +26,11 @@
 //               quarter its warp may access (lanes 32*(warp%4) ..), applies
 //               ReLU, head weights and the scale, and stores the score and the
 //               fused EMA update
-// Pipelines: key stages freed as soon as the MMAs have read them (5 per CTA
+// Pipelines: key stages freed as soon as the MMAs have read them (6 per CTA
 // at N = 64, 8 with one CTA per SM); a 16-slot ring of tile info freed by the
-// epilogue; 2 query buffers; 4 TMEM accumulators (2 when N > 64), so that all
-// CTAs of an SM fit the 512 TMEM columns.  Every wait is bounded (2 s of
+// epilogue; 1 query buffer with two CTAs per SM (2 with one); 4 TMEM
+// accumulators (2 when N > 64), so that all CTAs of an SM fit the 512 TMEM
+// columns.  Every wait is bounded (2 s of
 // %globaltimer); on expiry the CTA raises ERR_TIMEOUT, stops issuing, drains
 // what it issued and frees TMEM.
 #include <cuda.h>
@@ -177,8 +178,8 @@ struct Sched {
 // shared memory (the copy engine moves only key pages: its cost is per request,
 // so the per-token scales and EMA values are read by the epilogue threads).
 struct TileInfo {
-  int q, ctx, np, pad;
-  int j[2], pg[2];  // block ids and pages; pg < 0 marks a page outside the cache
+  int q, ctx, np, t;  // t: pair index of the tile within its request
+  int j[2], pg[2];    // block ids and pages; pg < 0 marks a page outside the cache
 };
 
 struct SmemLayout {
@@ -195,7 +196,7 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxAcc = 4;
 constexpr int kAuxSlots = 16;  // tile-info ring: freed by the epilogue, not by the MMA
 
-__host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
+__host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages, int nq) {
   SmemLayout s;
   uint32_t off = 0;
   s.keys = off;
@@ -204,7 +205,7 @@ __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
   off += kAuxSlots * (uint32_t)sizeof(TileInfo);
   off = (off + 1023) / 1024 * 1024;
   s.qbuf = off;
-  off += 2 * N * kRowBytes;
+  off += nq * N * kRowBytes;
   s.wq = off;
   off += 4 * kEpiGroups * N * 4;
   s.prefix = off;
@@ -219,16 +220,18 @@ __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages) {
 // has one copy-issuing warp, and one issuer per CTA caps the copy rate), with
 // accumulators sized so that CTAs * accumulators * N <= 512 TMEM columns.
 struct TcPlan {
-  int stages, nacc, ctas;
+  int stages, nacc, ctas, nq;  // key stages, TMEM accumulators, CTAs per SM, query buffers
 };
 
 __host__ __device__ inline TcPlan tc_plan(int N, int Q) {
-  // two CTAs share an SM's 228 KB when each takes <= 113 KB (1 KB per CTA is reserved)
+  // two CTAs share an SM's 228 KB when each takes <= 113 KB (1 KB per CTA is
+  // reserved); one query buffer (a request change drains the MMAs first, a
+  // CTA meets one or two) leaves room for more key stages
   constexpr uint32_t kTwoPerSm = 115712;
   if (N <= 128)
     for (int st = kMaxStages; st >= 3; --st)
-      if (smem_layout(N, Q, st).total <= kTwoPerSm) return {st, N <= 64 ? 4 : 2, 2};
-  return {kMaxStages, 2, 1};
+      if (smem_layout(N, Q, st, 1).total <= kTwoPerSm) return {st, N <= 64 ? 4 : 2, 2, 1};
+  return {kMaxStages, 2, 1, 2};
 }
 
 struct Bars {
@@ -296,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int stages = plan.stages, nacc = plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const SmemLayout lay = smem_layout(N, L.Q, stages);
+  const SmemLayout lay = smem_layout(N, L.Q, stages, plan.nq);
+  const int nq = plan.nq;
   const uint32_t sbase = smem_u32(smem);
   TileInfo* aux = reinterpret_cast<TileInfo*>(smem + lay.aux);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
@@ -393,8 +397,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         int ok = 1;
         if (lane == 0) {
           if (m.q != cur_q) {
-            const int nb = qiter & 1;
-            ok = wait_parity(B.qe(nb), ((qiter >> 1) & 1) ^ 1, ctl);
+            const int nb = qiter % nq;
+            ok = wait_parity(B.qe(nb), ((qiter / nq) & 1) ^ 1, ctl);
             if (ok) {
               mbar_expect_tx(B.qf(nb), (uint32_t)(N * kRowBytes));
               tma_load_2d(sbase + lay.qbuf + nb * N * kRowBytes, &tmap_q, B.qf(nb), 0, m.q * N);
@@ -409,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             x->q = m.q;
             x->ctx = m.ctx;
             x->np = np;
+            x->t = m.t;
             x->j[0] = m.j0;
             x->j[1] = m.j1;
             x->pg[0] = pg0;
@@ -455,9 +460,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int stage = i % stages, acc = i % nacc;
         const uint32_t phase = (uint32_t)(i / stages) & 1u, acc_phase = (uint32_t)(i / nacc) & 1u;
         if (q != cur_q) {
-          if (cur_q >= 0) umma_commit(B.qe((qiter - 1) & 1));
-          const int nb = qiter & 1;
-          if (!wait_parity(B.qf(nb), (qiter >> 1) & 1, ctl)) break;
+          if (cur_q >= 0) umma_commit(B.qe((qiter - 1) % nq));
+          const int nb = qiter % nq;
+          if (!wait_parity(B.qf(nb), (qiter / nq) & 1, ctl)) break;
           cur_q = q;
           ++qiter;
         }
@@ -465,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!wait_parity(B.f(stage), phase, ctl)) break;
         tc_fence_after();
         const uint32_t a_addr = sbase + lay.keys + stage * kStageBytes;
-        const uint32_t b_addr = sbase + lay.qbuf + ((qiter - 1) & 1) * N * kRowBytes;
+        const uint32_t b_addr = sbase + lay.qbuf + ((qiter - 1) % nq) * N * kRowBytes;
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
 #pragma unroll
         for (int kk = 0; kk < kRowBytes / 32; ++kk)
@@ -490,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int n_local = g1 - g0;
     // Per-token operands of a tile, loaded one tile (of this group) ahead.
     struct Pre {
-      int q, s, valid, upd;
+      int q, s, valid, upd, t;
       int64_t p0;
       float sigma, v, d;
     };
@@ -500,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!__all_sync(0xffffffffu, wait_parity(B.xf(xs), xph, ctl))) return false;
       const TileInfo* x = aux + xs;
       r.q = x->q;
+      r.t = x->t;
       r.p0 = x->ctx - 1;
       const int pg = x->pg[pg_idx];
       const bool present = pg_idx < x->np && pg >= 0;
@@ -543,7 +549,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (u < nu) part[u & 3] = __fmaf_rn(wr[u], fmaxf(__uint_as_float(v[u]), 0.0f), part[u & 3]);
         }
         const float sum = (part[0] + part[1]) + (part[2] + part[3]);
-        if (cur.valid && cur.s <= cur.p0 + r) {
+        const bool scored = cur.valid && cur.s <= cur.p0 + r;
+        if (a.gmax) {
+          // max over this warp's 32 slots = group 4t + quarter of the kept-slot order
+          float g = scored ? sum * cur.sigma : __int_as_float(0xff800000);
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
+          if (lane == 0) a.gmax[((int64_t)cur.q * L.R + r) * a.gstride + 4 * cur.t + quarter] = g;
+        }
+        if (scored) {
           const float score = sum * cur.sigma;
           a.scores[((int64_t)cur.q * L.R + r) * L.slot_stride + cur.s] = score;
           if (cur.upd && r == 0) {
@@ -587,7 +601,7 @@ bool tc_supported(const Layout& lay, int rows, int key_fp8) {
   if (!(key_fp8 && lay.d == 128 && lay.b == kPage && lay.H % 16 == 0 && N >= 16 && N <= 256 && N % 16 == 0))
     return false;
   const TcPlan plan = tc_plan(N, lay.Q);
-  return smem_layout(N, lay.Q, plan.stages).total <= 227 * 1024;
+  return smem_layout(N, lay.Q, plan.stages, plan.nq).total <= 227 * 1024;
 }
 
 cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s) {
@@ -600,7 +614,7 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   if (!encode_2d(fn, &tk, a.keys, (uint64_t)a.num_pages * kPage, kPage)) return cudaErrorInvalidValue;
   if (!encode_2d(fn, &tq, a.q8, (uint64_t)L.Q * N, (uint32_t)N)) return cudaErrorInvalidValue;
   const TcPlan plan = tc_plan(N, L.Q);
-  const uint32_t smem = smem_layout(N, L.Q, plan.stages).total;
+  const uint32_t smem = smem_layout(N, L.Q, plan.stages, plan.nq).total;
   cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;

@@ -15,69 +15,74 @@
 namespace spin {
 
 // ---------------------------------------------------------------------------
-// a1: one warp per pair of blocks of one request; each half-warp pools one
-// block of up to 64 slots, 4 slots per lane, float4 loads of V, scalar
-// (coalesced, reversed) loads of the D window shared by all rows.
-// Block sizes 16..256 (powers of two): larger blocks loop in 64-slot chunks.
+// a1: one warp per 256-slot chunk of one request; a lane takes 8 consecutive
+// slots (two float4 loads of V and the D window its rows need, all issued
+// before any use), and the b/8 lanes of a block reduce with shuffles.
+// Block sizes 16..256 (powers of two).
 // ---------------------------------------------------------------------------
 template <int R>
 __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
   const Layout L = a.lay;
-  const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
-  const int64_t pairs = (L.max_blocks + 1) / 2;
+  const int lane = threadIdx.x & 31;
+  const int lb = __ffs(L.b) - 1;
+  const int lpb = L.b >> 3;  // lanes per block
+  const int64_t chunks = (L.slot_stride + 255) / 256;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       wid < (int64_t)L.Q * pairs; wid += nwarps) {
-    const int q = (int)(wid / pairs);
-    const int64_t j = (wid % pairs) * 2 + half;
+  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wid < (int64_t)L.Q * chunks;
+       wid += nwarps) {
+    const int q = (int)(wid / chunks);
+    const int64_t c = wid % chunks;
     const int64_t ctx = a.ctx_len[q];
     if (ctx < 1 || ctx + R - 1 > L.max_slots) continue;  // warp-uniform; select reports it
     const int64_t n_last = row_blocks(ctx, R - 1, L.b);
+    if (c * 256 >= n_last * L.b) continue;                 // warp-uniform
     const int64_t p0 = ctx - 1;
+    const int64_t i0 = c * 256 + lane * 8;
+    const int64_t j = i0 >> lb;
+    const bool active = j < n_last && i0 <= p0 + R - 1;
     const float* V = a.V + (int64_t)q * L.slot_stride;
     const float* D = a.D + (int64_t)q * L.slot_stride;
+    float vv[8];
+    float dw[R + 7];  // D at offsets p0 - i0 - 7 .. p0 - i0 + R - 1
+#pragma unroll
+    for (int k = 0; k < 8; ++k) vv[k] = __int_as_float(0xff800000);
+#pragma unroll
+    for (int t = 0; t < R + 7; ++t) dw[t] = __int_as_float(0xff800000);
+    if (active) {
+      const float4 v0 = __ldg(reinterpret_cast<const float4*>(V + i0));
+      const float4 v1 = __ldg(reinterpret_cast<const float4*>(V + i0 + 4));
+      vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
+      vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+#pragma unroll
+      for (int t = 0; t < R + 7; ++t) {
+        const int64_t di = p0 - i0 - 7 + t;
+        if (di >= 0) dw[t] = __ldg(D + di);
+      }
+    }
     float m[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) m[r] = __int_as_float(0xff800000);
-    const bool active = j < n_last;
-    for (int c0 = 0; c0 < L.b; c0 += 64) {
-      const int64_t i0 = j * L.b + c0 + l16 * 4;
-      if (active && c0 + l16 * 4 < L.b && i0 <= p0 + R - 1) {
-        const float4 v = *reinterpret_cast<const float4*>(V + i0);
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-        // D window: offsets p0 - i0 - 3 .. p0 - i0 + R - 1
-        float dw[R + 3];
+    for (int r = 0; r < R; ++r) {
+      m[r] = __int_as_float(0xff800000);
 #pragma unroll
-        for (int t = 0; t < R + 3; ++t) {
-          const int64_t di = p0 - i0 - 3 + t;
-          dw[t] = (di >= 0) ? __ldg(D + di) : __int_as_float(0xff800000);
-        }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            // slot i0+k, offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + 3]
-            if (i0 + k <= p0 + r) m[r] = fmaxf(m[r], fmaxf(vv[k], dw[r - k + 3]));
-          }
-        }
-      }
+      for (int k = 0; k < 8; ++k)
+        // slot i0+k at offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + 7]
+        if (active && i0 + k <= p0 + r) m[r] = fmaxf(m[r], fmaxf(vv[k], dw[r - k + 7]));
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float x = m[r];
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-      if (active && l16 == 0 && j < row_blocks(ctx, r, L.b))
+      for (int o = lpb >> 1; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      if (active && (lane & (lpb - 1)) == 0 && j < row_blocks(ctx, r, L.b))
         a.S[((int64_t)q * L.R + r) * L.blk_stride + j] = x;
     }
   }
 }
 
 cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
-  const int64_t pairs = (a.lay.max_blocks + 1) / 2;
-  int64_t warps = (int64_t)a.lay.Q * pairs;
+  const int64_t chunks = (a.lay.slot_stride + 255) / 256;
+  const int64_t warps = (int64_t)a.lay.Q * chunks;
   int64_t blocks = (warps + 7) / 8;
-  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks > 148 * 32) blocks = 148 * 32;
   switch (a.rows) {
     case 1: k_predict_pool<1><<<(int)blocks, 256, 0, s>>>(a); break;
     case 2: k_predict_pool<2><<<(int)blocks, 256, 0, s>>>(a); break;

@@ -3,23 +3,29 @@
 // is).  Order: higher score first, ties to the lower slot; the chosen slots
 // are emitted in ascending slot order, padded with -1.
 //
-// One CTA (1024 threads) per (request, row).
-//  1. A 13-bit histogram of the order-preserving score keys (sign, exponent
-//     and 4 mantissa bits) over a fixed 1/16 sample of the scored slots gives
-//     a lower threshold whose expected count is about 1.3 k.
-//  2. One pass over all scored slots appends every key at or above it to a
-//     shared-memory candidate list (key, position in the ascending kept-slot
-//     order), one atomic per warp.  If the list holds at least k keys it holds
-//     the whole top k, so the rest is exact:
+// One CTA (1024 threads) per (request, row).  Scores are compared through
+// their order-preserving 32-bit keys.
+//  1. Candidates.  When the score kernel left the maximum of every 32 slots
+//     (the fused decode step), M = the k-th largest group maximum bounds the
+//     k-th score from below; only the groups whose maximum is >= M are read
+//     and their scores >= M kept.  Otherwise a lower threshold comes from the
+//     13-bit histogram of a fixed 1/16 sample (about 1.3 k keys expected
+//     above it) and one pass over all scored slots keeps the keys above it.
+//     Candidates are (key, position in the ascending kept-slot order) in
+//     shared memory, appended with one shared atomic per warp.  If the list
+//     holds at least k keys it holds the whole top k, so the rest is exact:
 //  3. a radix select over the candidates (4 x 8-bit digits) gives the
-//     threshold key T and how many keys equal to T belong to the top k;
-//  4. chosen positions are set in a shared-memory bitmap; two block scans
-//     over it take the lowest-position ties and give each chosen slot its
-//     output index, so the output is ascending without a sort.
-// When the estimate misses (fewer than k candidates, or more than fit), the
-// kernel falls back to an exact histogram of all keys, then a collection of
-// the keys in its threshold bin, then -- if even those do not fit -- three
-// more full radix passes.
+//     threshold key T and how many keys equal to T belong to the top k; the
+//     keys equal to T are ranked by position (lowest first) with a second
+//     radix select;
+//  4. the chosen positions are set in a shared-memory bitmap, and one block
+//     scan over it gives every chosen slot its output index, so the output is
+//     ascending without a sort.
+// A sample that misses (too few or too many candidates) falls back to an
+// exact histogram of all keys, a collection of the keys in its threshold bin
+// and -- if even those do not fit -- three more full radix passes, after
+// which ties are resolved by re-reading the scores.  Every path gives the
+// same result; the sample only decides the speed.
 #include <algorithm>
 
 #include "spin_internal.cuh"
@@ -37,39 +43,55 @@ struct TopkShared {
   int scan[33];
   int total;
   int n_cand;
-  int overflow;
+  int n_eq;
 };
 
-// Visits every scored slot (kept blocks, s <= p) as f(position, slot, key),
-// four float4 loads in flight per thread.
+struct TopkCtx {
+  const float* sc;
+  const int32_t* work;
+  int nk, lb, bmask, p, n_elem, nwords;
+  uint32_t* bits;
+  uint32_t* hist;   // kBins
+  uint32_t* ckey;   // kCandCap (aliases hist)
+  uint32_t* cpos;   // kCandCap
+  uint32_t* hist2;  // 256
+};
+
+
+// Visits every scored slot (kept blocks, s <= p) as f(position, key), with
+// the work-list loads of eight float4s issued before their score loads.
 template <class F>
-__device__ __forceinline__ void for_each_scored(const float* sc, const int32_t* work, int nk, int lb, int p, F f) {
-  const int n_elem = nk << lb;
+__device__ __forceinline__ void for_each_scored(const TopkCtx& c, F f) {
   const int step = blockDim.x * 4;
-  for (int base = threadIdx.x * 4; base < n_elem; base += 4 * step) {
-    float4 v[4];
-    int s0[4];
+  for (int it = 0; it < c.n_elem; it += 8 * step) {
+    int blk[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int e = base + u * step;
+    for (int u = 0; u < 8; ++u) {
+      const int e = it + threadIdx.x * 4 + u * step;
+      blk[u] = e < c.n_elem ? c.work[e >> c.lb] : -1;
+    }
+    float4 v[8];
+    int s0[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = it + threadIdx.x * 4 + u * step;
       s0[u] = -1;
-      if (e < n_elem) {
-        const int s = (work[e >> lb] << lb) + (e & ((1 << lb) - 1));
-        if (s <= p) {
+      if (blk[u] >= 0) {
+        const int s = (blk[u] << c.lb) + (e & c.bmask);
+        if (s <= c.p) {
           s0[u] = s;
-          v[u] = *reinterpret_cast<const float4*>(sc + s);
+          v[u] = *reinterpret_cast<const float4*>(c.sc + s);
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int s = s0[u];
-      if (s < 0) continue;
-      const int e = base + u * step;
-      f(e, s, fkey(v[u].x));
-      if (s + 1 <= p) f(e + 1, s + 1, fkey(v[u].y));
-      if (s + 2 <= p) f(e + 2, s + 2, fkey(v[u].z));
-      if (s + 3 <= p) f(e + 3, s + 3, fkey(v[u].w));
+    for (int u = 0; u < 8; ++u) {
+      if (s0[u] < 0) continue;
+      const int e = it + threadIdx.x * 4 + u * step;
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (s0[u] + k <= c.p) f(e + k, fkey(vals[k]));
     }
   }
 }
@@ -88,8 +110,7 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
 // bin and the rank left inside it to digit[0..1].
 __device__ void block_find_bin_desc(const uint32_t* hist, int nb, uint32_t want, TopkShared& sh) {
   const int per = nb / blockDim.x;
-  // thread t covers bins nb-1-t*per .. nb-per-t*per (from the top)
-  const int hi = nb - 1 - threadIdx.x * per;
+  const int hi = nb - 1 - threadIdx.x * per;  // this thread's bins, from the top
   uint32_t s = 0;
   for (int i = 0; i < per; ++i) s += hist[hi - i];
   int tot;
@@ -109,6 +130,294 @@ __device__ void block_find_bin_desc(const uint32_t* hist, int nb, uint32_t want,
   __syncthreads();
 }
 
+// Lower threshold from the 13-bit histogram of a fixed 1/16 sample (one
+// float4 out of every 64 scored positions) where about 1.3 `want` keys of
+// the `total` are expected above it.
+__device__ uint32_t sample_threshold(const TopkCtx& c, int want, int total, TopkShared& sh) {
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) c.hist[i] = 0;
+  __syncthreads();
+  const int n_smp = c.n_elem >> 6;
+  for (int it = 0; it < n_smp; it += 4 * blockDim.x) {
+    float4 v[4];
+    int s0[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = it + u * blockDim.x + threadIdx.x;
+      s0[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < n_smp) {
+        const int e = i << 6;
+        const int s = (c.work[e >> c.lb] << c.lb) + (e & c.bmask);
+        if (s <= c.p) {
+          s0[u] = s;
+          v[u] = *reinterpret_cast<const float4*>(c.sc + s);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const bool act = s0[u] >= 0 && s0[u] + k <= c.p;
+        hist_add(c.hist, act ? fkey(vals[k]) >> kFirstShift : 0u, act);
+      }
+    }
+  }
+  __syncthreads();
+  int cnt = 0;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) cnt += c.hist[i];
+  int n_s;
+  block_exclusive_scan(cnt, sh.scan, &n_s);
+  const int ks = min(n_s, (int)ceilf(1.3f * (float)want * (float)n_s / (float)total) + 16);
+  uint32_t t_lo = 0;
+  if (ks >= 1) {
+    block_find_bin_desc(c.hist, kBins, (uint32_t)ks, sh);
+    t_lo = sh.digit[0] << kFirstShift;
+  }
+  __syncthreads();
+  return t_lo;
+}
+
+// Appends every scored key >= t_lo; returns how many there are (the list
+// keeps the first kCandCap).  The loop is uniform across a warp, so takers
+// are counted with a ballot and reserved with one atomic per warp.
+__device__ int collect_ge(const TopkCtx& c, uint32_t t_lo, TopkShared& sh) {
+  if (threadIdx.x == 0) sh.n_cand = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int step = blockDim.x * 4;
+  for (int it = 0; it < c.n_elem; it += 8 * step) {
+    int blk[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = it + threadIdx.x * 4 + u * step;
+      blk[u] = e < c.n_elem ? c.work[e >> c.lb] : -1;
+    }
+    float4 v[8];
+    int s0[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = it + threadIdx.x * 4 + u * step;
+      s0[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (blk[u] >= 0) {
+        const int s = (blk[u] << c.lb) + (e & c.bmask);
+        if (s <= c.p) {
+          s0[u] = s;
+          v[u] = *reinterpret_cast<const float4*>(c.sc + s);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t takes = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= t_lo) takes |= 1u << k;
+      const int n_my = __popc(takes);
+      if (!__any_sync(0xffffffffu, n_my != 0)) continue;  // the common case
+      int incl = n_my;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int base = 0;
+      if (lane == 31) base = atomicAdd(&sh.n_cand, incl);
+      base = __shfl_sync(0xffffffffu, base, 31) + incl - n_my;
+      const int e0 = it + threadIdx.x * 4 + u * step;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (takes & (1u << k)) {
+          if (base < kCandCap) {
+            c.ckey[base] = fkey(vals[k]);
+            c.cpos[base] = (uint32_t)(e0 + k);
+          }
+          ++base;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  return sh.n_cand;
+}
+
+// Radix select over the first n entries of `keys` (largest first when desc,
+// else smallest first): the key of rank `want` and how many keys equal to it
+// are taken.
+__device__ void radix_select_list(const uint32_t* keys, int n, uint32_t want, bool desc, uint32_t* hist2,
+                                  TopkShared& sh, uint32_t* key_out, uint32_t* eq_out) {
+  uint32_t prefix = 0, rem = want;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+    __syncthreads();
+    const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t k = desc ? keys[i] : ~keys[i];
+      if ((k & pmask) == prefix) atomicAdd(&hist2[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, rem, sh.digit);
+    __syncthreads();
+    prefix |= sh.digit[0] << shift;
+    rem = sh.digit[1];
+    __syncthreads();
+  }
+  *key_out = desc ? prefix : ~prefix;
+  *eq_out = rem;
+}
+
+// Exact top `want` among n_cand (>= want) candidates: sets exactly the chosen
+// positions in the bitmap.  Returns the threshold key T.
+__device__ uint32_t select_candidates(const TopkCtx& c, int n_cand, int want, TopkShared& sh) {
+  uint32_t T, eq_take;
+  radix_select_list(c.ckey, n_cand, (uint32_t)want, true, c.hist2, sh, &T, &eq_take);
+  for (int i = threadIdx.x; i < c.nwords; i += blockDim.x) c.bits[i] = 0;
+  if (threadIdx.x == 0) sh.n_eq = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
+    if (c.ckey[i] > T) atomicOr(&c.bits[c.cpos[i] >> 5], 1u << (c.cpos[i] & 31));
+  // Keys equal to T: their positions are compacted to the front of the key
+  // array (the keys are no longer needed; a round reads before it writes,
+  // and writes only reach indices already read), then the eq_take lowest
+  // positions are chosen.
+  uint32_t* epos = c.ckey;
+  for (int base = 0; base < n_cand; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const bool eq = i < n_cand && c.ckey[i] == T;
+    const uint32_t pos = i < n_cand ? c.cpos[i] : 0u;
+    __syncthreads();
+    if (eq) epos[atomicAdd(&sh.n_eq, 1)] = pos;
+    __syncthreads();
+  }
+  const int n_eq = sh.n_eq;
+  if ((uint32_t)n_eq <= eq_take) {
+    for (int i = threadIdx.x; i < n_eq; i += blockDim.x) atomicOr(&c.bits[epos[i] >> 5], 1u << (epos[i] & 31));
+  } else {
+    uint32_t P, unused;
+    radix_select_list(epos, n_eq, eq_take, false, c.hist2, sh, &P, &unused);
+    for (int i = threadIdx.x; i < n_eq; i += blockDim.x)
+      if (epos[i] <= P) atomicOr(&c.bits[epos[i] >> 5], 1u << (epos[i] & 31));
+  }
+  __syncthreads();
+  return T;
+}
+
+// Key of rank `want` (largest first) among keys[0..n), with warp-combined
+// histogram adds (group maxima share their leading key bits).
+__device__ uint32_t radix_select_agg(const uint32_t* keys, int n, uint32_t want, uint32_t* hist2, TopkShared& sh) {
+  uint32_t prefix = 0, rem = want;
+  const int lane = threadIdx.x & 31;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+    __syncthreads();
+    const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int base = 0; base < n; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      const uint32_t k = i < n ? keys[i] : 0u;
+      const bool act = i < n && (k & pmask) == prefix;
+      const uint32_t bin = (k >> shift) & 255u;
+      const uint32_t m = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t peers = __match_any_sync(m, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist2[bin], (uint32_t)__popc(peers));
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, rem, sh.digit);
+    __syncthreads();
+    prefix |= sh.digit[0] << shift;
+    rem = sh.digit[1];
+    __syncthreads();
+  }
+  return prefix;
+}
+
+// Candidates from group maxima (the score kernel's max of every 32 slots of
+// the kept-slot order).  M = the want-th largest group maximum; at least
+// `want` scores are >= M (each of the want best groups holds one), and every
+// score >= M lies in a group whose maximum is >= M, so gathering those groups'
+// scores >= M yields a candidate list that holds the whole top `want`.
+// The group keys and then the compacted group list live in the bitmap area.
+__device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want, TopkShared& sh) {
+  const int n_groups = (c.n_elem + 31) / 32;  // == c.nwords
+  uint32_t* gk = c.bits;
+  for (int g = threadIdx.x; g < n_groups; g += blockDim.x) gk[g] = fkey(gmax[g]);
+  __syncthreads();
+  const uint32_t M = radix_select_agg(gk, n_groups, (uint32_t)want, c.hist2, sh);
+  // compact the qualifying group ids to the front, in place (a round reads
+  // before it writes, and writes only reach indices already read)
+  if (threadIdx.x == 0) sh.n_eq = 0;
+  __syncthreads();
+  for (int base = 0; base < n_groups; base += blockDim.x) {
+    const int g = base + threadIdx.x;
+    const bool take = g < n_groups && gk[g] >= M;
+    __syncthreads();
+    if (take) gk[atomicAdd(&sh.n_eq, 1)] = (uint32_t)g;
+    __syncthreads();
+  }
+  const int n_q = sh.n_eq;
+  if (threadIdx.x == 0) sh.n_cand = 0;
+  __syncthreads();
+  // gather: a warp takes 32 groups at a time, 8 lanes x float4 per group
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int base = warp * 32; base < n_q; base += nw * 32) {
+    int e0[8];
+    float4 v[8];
+    int s0[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int gi = base + u * 4 + (lane >> 3);
+      e0[u] = gi < n_q ? (int)gk[gi] * 32 + (lane & 7) * 4 : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      s0[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0[u] >= 0 && e0[u] < c.n_elem) {
+        const int s = (c.work[e0[u] >> c.lb] << c.lb) + (e0[u] & c.bmask);
+        if (s <= c.p) {
+          s0[u] = s;
+          v[u] = *reinterpret_cast<const float4*>(c.sc + s);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t takes = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << k;
+      const int n_my = __popc(takes);
+      if (!__any_sync(0xffffffffu, n_my != 0)) continue;
+      int incl = n_my;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int at = 0;
+      if (lane == 31) at = atomicAdd(&sh.n_cand, incl);
+      at = __shfl_sync(0xffffffffu, at, 31) + incl - n_my;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (takes & (1u << k)) {
+          if (at < kCandCap) {
+            c.ckey[at] = fkey(vals[k]);
+            c.cpos[at] = (uint32_t)(e0[u] + k);
+          }
+          ++at;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  return sh.n_cand;
+}
+
 __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   const Layout L = a.lay;
   const int q = blockIdx.x / a.rows, r = blockIdx.x % a.rows;
@@ -120,31 +429,29 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
   }
-  const int p = (int)(ctx - 1 + r);
-  const int nk = a.kept[q];
-  const int32_t* work = a.work + (int64_t)q * L.blk_stride;
-  const float* sc = a.scores + ((int64_t)q * L.R + r) * L.slot_stride;
-  const int lb = __ffs(L.b) - 1;  // block size is a power of two
-  const int bmask = L.b - 1;
-  const int n_elem = nk << lb;
-  const int nwords = (n_elem + 31) / 32;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(dyn);
-  uint8_t* work_area = dyn + (((size_t)(L.slot_stride + 31) / 32) * 4 + 15) / 16 * 16;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(work_area);          // kBins (pass 1)
-  uint32_t* ckey = reinterpret_cast<uint32_t*>(work_area);          // kCandCap (after pass 1)
-  uint32_t* cpos = ckey + kCandCap;
-  uint32_t* hist2 = cpos + kCandCap;                                // 256 bins (candidate passes)
+  TopkCtx c;
+  c.p = (int)(ctx - 1 + r);
+  c.nk = a.kept[q];
+  c.work = a.work + (int64_t)q * L.blk_stride;
+  c.sc = a.scores + ((int64_t)q * L.R + r) * L.slot_stride;
+  c.lb = __ffs(L.b) - 1;  // block size is a power of two
+  c.bmask = L.b - 1;
+  c.n_elem = c.nk << c.lb;
+  c.nwords = (c.n_elem + 31) / 32;
+  c.bits = reinterpret_cast<uint32_t*>(dyn);
+  uint8_t* area = dyn + (((size_t)(L.slot_stride + 31) / 32) * 4 + 15) / 16 * 16;
+  c.hist = reinterpret_cast<uint32_t*>(area);
+  c.ckey = reinterpret_cast<uint32_t*>(area);
+  c.cpos = c.ckey + kCandCap;
+  c.hist2 = c.cpos + kCandCap;
 
   // ---- number of scored slots -------------------------------------------
   {
-    int c = 0;
-    for (int t = threadIdx.x; t < nk; t += blockDim.x) c += min(max(p - (work[t] << lb) + 1, 0), L.b);
+    int cnt = 0;
+    for (int t = threadIdx.x; t < c.nk; t += blockDim.x) cnt += min(max(c.p - (c.work[t] << c.lb) + 1, 0), L.b);
     int tot;
-    block_exclusive_scan(c, sh.scan, &tot);
-    if (threadIdx.x == 0) {
-      sh.total = tot;
-      sh.n_cand = 0;
-    }
+    block_exclusive_scan(cnt, sh.scan, &tot);
+    if (threadIdx.x == 0) sh.total = tot;
     __syncthreads();
   }
   const int total = sh.total;
@@ -153,192 +460,78 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
   }
-  uint32_t T = 0, remaining = 0;
-  bool done = false;
 
-  // ---- sampled threshold, one collecting pass, exact select on chip ---------
+  // ---- fast path: threshold, one collecting pass, exact select on chip ----
+  bool exact_bits = false;
+  uint32_t T = 0, eq_take = 0;
   {
-    uint32_t t_lo = 0;  // keep everything when all scored slots fit
-    bool est_ok = true;
-    if (total > kCandCap) {
-      for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
-      __syncthreads();
-      const int n_smp = n_elem >> 6;  // one float4 out of every 64 scored positions
-      for (int it = 0; it < n_smp; it += blockDim.x) {
-        const int i = it + threadIdx.x;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        int s = -1;
-        if (i < n_smp) {
-          const int e = i << 6;
-          s = (work[e >> lb] << lb) + (e & bmask);
-          if (s <= p) v = *reinterpret_cast<const float4*>(sc + s);
-        }
-        const float vals[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const bool act = s >= 0 && s + c <= p;
-          hist_add(hist, act ? fkey(vals[c]) >> kFirstShift : 0u, act);
-        }
-      }
-      __syncthreads();
-      int c = 0;
-      for (int i = threadIdx.x; i < kBins; i += blockDim.x) c += hist[i];
-      int n_s;
-      block_exclusive_scan(c, sh.scan, &n_s);
-      const int ks = min(n_s, (int)ceilf(1.3f * (float)want * (float)n_s / (float)total) + 16);
-      if (ks >= 1) {
-        block_find_bin_desc(hist, kBins, (uint32_t)ks, sh);
-        t_lo = sh.digit[0] << kFirstShift;
-      } else {
-        est_ok = false;
-      }
-      __syncthreads();
+    int n_cand = -1;
+    if (total <= kCandCap) {
+      n_cand = collect_ge(c, 0u, sh);  // everything fits
+    } else {
+      if (a.gmax) n_cand = collect_from_groups(c, a.gmax + ((int64_t)q * L.R + r) * a.gstride, want, sh);
+      if (n_cand < want || n_cand > kCandCap) n_cand = collect_ge(c, sample_threshold(c, want, total, sh), sh);
     }
-    if (est_ok) {
-      // warp-uniform pass: a warp appends its takers with one atomic
-      const int step = blockDim.x * 4;
-      const int lane = threadIdx.x & 31;
-      for (int it = 0; it < n_elem; it += 4 * step) {
-        const int base = it + threadIdx.x * 4;
-        float4 v[4];
-        int s0[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = base + u * step;
-          s0[u] = -1;
-          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (e < n_elem) {
-            const int s = (work[e >> lb] << lb) + (e & bmask);
-            if (s <= p) {
-              s0[u] = s;
-              v[u] = *reinterpret_cast<const float4*>(sc + s);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t key = fkey(vals[c]);
-            const bool take = s0[u] >= 0 && s0[u] + c <= p && key >= t_lo;
-            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            if (bal) {
-              const int leader = __ffs(bal) - 1;
-              int at = 0;
-              if (lane == leader) at = atomicAdd(&sh.n_cand, __popc(bal));
-              at = __shfl_sync(0xffffffffu, at, leader) + __popc(bal & ((1u << lane) - 1u));
-              if (take && at < kCandCap) {
-                ckey[at] = key;
-                cpos[at] = (uint32_t)(base + u * step + c);
-              }
-            }
-          }
-        }
-      }
-      __syncthreads();
-      const int n_cand = sh.n_cand;
-      if (n_cand >= want && n_cand <= kCandCap) {
-        uint32_t prefix = 0, rem = (uint32_t)want;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-          for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
-          __syncthreads();
-          const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
-          for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
-            const uint32_t k = ckey[i];
-            if ((k & pmask) == prefix) atomicAdd(&hist2[(k >> shift) & 255u], 1u);
-          }
-          __syncthreads();
-          if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, rem, sh.digit);
-          __syncthreads();
-          prefix |= sh.digit[0] << shift;
-          rem = sh.digit[1];
-          __syncthreads();
-        }
-        T = prefix;
-        remaining = rem;
-        for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
-          if (ckey[i] >= T) atomicOr(&bits[cpos[i] >> 5], 1u << (cpos[i] & 31));
-        __syncthreads();
-        done = true;
-      }
+    if (n_cand >= want && n_cand <= kCandCap) {
+      T = select_candidates(c, n_cand, want, sh);
+      exact_bits = true;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) sh.n_cand = 0;
-    __syncthreads();
   }
 
-  if (!done) {
-    // ---- pass 1: 13-bit histogram ------------------------------------------
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+  if (!exact_bits) {
+    // ---- exact fallback: 13-bit histogram of all keys ---------------------
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) c.hist[i] = 0;
     __syncthreads();
     {
       const int step = blockDim.x * 4;
-      for (int it = 0; it < n_elem; it += 4 * step) {
-        const int base = it + threadIdx.x * 4;
+      for (int it = 0; it < c.n_elem; it += 4 * step) {
         float4 v[4];
         int s0[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int e = base + u * step;
+          const int e = it + threadIdx.x * 4 + u * step;
           s0[u] = -1;
-          if (e < n_elem) {
-            const int s = (work[e >> lb] << lb) + (e & bmask);
-            if (s <= p) {
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (e < c.n_elem) {
+            const int s = (c.work[e >> c.lb] << c.lb) + (e & c.bmask);
+            if (s <= c.p) {
               s0[u] = s;
-              v[u] = *reinterpret_cast<const float4*>(sc + s);
+              v[u] = *reinterpret_cast<const float4*>(c.sc + s);
             }
           }
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int s = s0[u];
           const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const bool act = s >= 0 && s + c <= p;
-            hist_add(hist, act ? fkey(vals[c]) >> kFirstShift : 0u, act);
+          for (int k = 0; k < 4; ++k) {
+            const bool act = s0[u] >= 0 && s0[u] + k <= c.p;
+            hist_add(c.hist, act ? fkey(vals[k]) >> kFirstShift : 0u, act);
           }
         }
       }
     }
     __syncthreads();
-    block_find_bin_desc(hist, kBins, (uint32_t)want, sh);
+    block_find_bin_desc(c.hist, kBins, (uint32_t)want, sh);
     const uint32_t d1 = sh.digit[0];
-    remaining = sh.digit[1];
+    uint32_t remaining = sh.digit[1];
     __syncthreads();
-
-    // ---- pass 2: collect keys in bin d1 and above ------------------------------
-    // (the histogram area becomes the candidate list)
-    for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
-      if ((key >> kFirstShift) >= d1) {
-        const int slot = atomicAdd(&sh.n_cand, 1);
-        if (slot < kCandCap) {
-          ckey[slot] = key;
-          cpos[slot] = (uint32_t)e;
-        }
-      }
-    });
-    __syncthreads();
-    const int n_cand = sh.n_cand;
+    const int n_cand = collect_ge(c, d1 << kFirstShift, sh);
     if (n_cand <= kCandCap) {
-      // ---- exact select among the candidates (rank counted from the top) -------
-      // elements above bin d1 are all chosen; `remaining` is the rank inside d1
+      // exact select among the keys of bin d1 (rank `remaining` inside it)
       uint32_t prefix = d1, pbits = 32 - kFirstShift;
       const int shifts[3] = {11, 3, 0};
       const int widths[3] = {8, 8, 3};
       for (int ps = 0; ps < 3; ++ps) {
         const int shf = shifts[ps], w = widths[ps];
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) c.hist2[i] = 0;
         __syncthreads();
         for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
-          const uint32_t k = ckey[i];
-          if ((k >> (32 - pbits)) == prefix) atomicAdd(&hist2[(k >> shf) & ((1u << w) - 1u)], 1u);
+          const uint32_t k = c.ckey[i];
+          if ((k >> (32 - pbits)) == prefix) atomicAdd(&c.hist2[(k >> shf) & ((1u << w) - 1u)], 1u);
         }
         __syncthreads();
-        if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);  // bins >= 2^w are empty
+        if (threadIdx.x < 32) warp_find_digit_desc<256>(c.hist2, remaining, sh.digit);  // bins >= 2^w are empty
         __syncthreads();
         prefix = (prefix << w) | sh.digit[0];
         pbits += w;
@@ -346,13 +539,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
         __syncthreads();
       }
       T = prefix;
-      for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+      for (int i = threadIdx.x; i < c.nwords; i += blockDim.x) c.bits[i] = 0;
       __syncthreads();
       for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
-        if (ckey[i] >= T) atomicOr(&bits[cpos[i] >> 5], 1u << (cpos[i] & 31));
+        if (c.ckey[i] >= T) atomicOr(&c.bits[c.cpos[i] >> 5], 1u << (c.cpos[i] & 31));
       __syncthreads();
     } else {
-      // ---- fallback: three more full passes over HBM --------------------------
+      // three more full passes over the scores
       uint32_t prefix = d1;
       int shift_hi = kFirstShift;
       const int shifts[3] = {11, 3, 0};
@@ -360,13 +553,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
         const int sh_lo = shifts[ps];
         const int width = shift_hi - sh_lo;
         const uint32_t dmask = (1u << width) - 1u;
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) c.hist2[i] = 0;
         __syncthreads();
-        for_each_scored(sc, work, nk, lb, p, [&](int, int, uint32_t key) {
-          if ((key >> shift_hi) == prefix) atomicAdd(&hist2[(key >> sh_lo) & dmask], 1u);
+        for_each_scored(c, [&](int, uint32_t key) {
+          if ((key >> shift_hi) == prefix) atomicAdd(&c.hist2[(key >> sh_lo) & dmask], 1u);
         });
         __syncthreads();
-        if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, remaining, sh.digit);
+        if (threadIdx.x < 32) warp_find_digit_desc<256>(c.hist2, remaining, sh.digit);
         __syncthreads();
         prefix = (prefix << width) | sh.digit[0];
         remaining = sh.digit[1];
@@ -374,28 +567,34 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
         __syncthreads();
       }
       T = prefix;
-      for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0;
+      for (int i = threadIdx.x; i < c.nwords; i += blockDim.x) c.bits[i] = 0;
       __syncthreads();
-      for_each_scored(sc, work, nk, lb, p, [&](int e, int, uint32_t key) {
-        if (key >= T) atomicOr(&bits[e >> 5], 1u << (e & 31));
+      for_each_scored(c, [&](int e, uint32_t key) {
+        if (key >= T) atomicOr(&c.bits[e >> 5], 1u << (e & 31));
       });
       __syncthreads();
     }
+    eq_take = remaining;
   }
-  const uint32_t eq_take = remaining;
 
-  // ---- ordered tie handling and emission -----------------------------------
-  const int chunk = (nwords + blockDim.x - 1) / blockDim.x;
-  const int w0 = threadIdx.x * chunk, w1 = min(nwords, w0 + chunk);
+  // ---- emission in ascending slot order --------------------------------------
+  // Exact bitmaps need no score; the fallback's bitmap holds every key >= T
+  // and takes the lowest-position eq_take of the keys equal to T.
+  const int chunk = (c.nwords + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * chunk, w1 = min(c.nwords, w0 + chunk);
   int n_gt = 0, n_eq = 0;
   for (int w = w0; w < w1; ++w) {
-    uint32_t m = bits[w];
+    uint32_t m = c.bits[w];
+    if (exact_bits) {
+      n_gt += __popc(m);
+      continue;
+    }
     while (m) {
       const int bit = __ffs(m) - 1;
       m &= m - 1;
       const int e = w * 32 + bit;
-      const int s = (work[e >> lb] << lb) + (e & bmask);
-      if (fkey(sc[s]) > T) ++n_gt; else ++n_eq;
+      const int s = (c.work[e >> c.lb] << c.lb) + (e & c.bmask);
+      if (fkey(c.sc[s]) > T) ++n_gt; else ++n_eq;
     }
   }
   int tot;
@@ -404,13 +603,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   int pos = block_exclusive_scan(n_gt + take, sh.scan, &tot);
   int eq_rank = eq_base;
   for (int w = w0; w < w1; ++w) {
-    uint32_t m = bits[w];
+    uint32_t m = c.bits[w];
     while (m) {
       const int bit = __ffs(m) - 1;
       m &= m - 1;
       const int e = w * 32 + bit;
-      const int s = (work[e >> lb] << lb) + (e & bmask);
-      if (fkey(sc[s]) > T) {
+      const int s = (c.work[e >> c.lb] << c.lb) + (e & c.bmask);
+      if (exact_bits || fkey(c.sc[s]) > T) {
         out[pos++] = (int32_t)s;
       } else {
         if ((uint32_t)eq_rank < eq_take) out[pos++] = (int32_t)s;

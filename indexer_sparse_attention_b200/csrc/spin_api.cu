@@ -26,6 +26,8 @@ struct spin_state_s {
   uint8_t* q8;    // [Q][R][H][d]
   float* wq;      // [Q][R][H]
   float* scores;  // [Q][R][slot_stride]
+  float* gmax;    // [Q][R][gstride] group maxima of the last tensor-core score
+  int64_t gstride;
   std::vector<float> sparsity;
   int score_kernel;
   int inject;
@@ -88,8 +90,11 @@ Layout make_layout(const spin_config* c) {
   return L;
 }
 
+// Group maxima: one per 32 slots of the kept-slot order.
+int64_t gmax_stride(const Layout& L) { return L.blk_stride * std::max(1, L.b / 32); }
+
 struct Carve {
-  size_t err, V, D, S, work, kept, q8, wq, scores, total;
+  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, total;
 };
 
 Carve carve(const Layout& L) {
@@ -105,6 +110,7 @@ Carve carve(const Layout& L) {
   k.q8 = take((size_t)L.Q * L.R * L.H * L.d);
   k.wq = take((size_t)L.Q * L.R * L.H * 4);
   k.scores = take((size_t)L.Q * L.R * L.slot_stride * 4);
+  k.gmax = take((size_t)L.Q * L.R * gmax_stride(L) * 4);
   k.total = off;
   return k;
 }
@@ -179,7 +185,7 @@ cudaError_t staged(spin_state st, int stage, cudaStream_t s, F launch) {
 spin_status run_score(spin_state st, int layer, int rows, const void* keys, const float* key_scale,
                       int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
                       const float* w, const int32_t* ctx_len, const uint8_t* mask, float* scores,
-                      bool fuse_ema, cudaStream_t stream) {
+                      bool fuse_ema, cudaStream_t stream, bool* wrote_gmax = nullptr) {
   ScoreArgs a;
   a.lay = st->lay;
   a.rows = rows;
@@ -206,6 +212,9 @@ spin_status run_score(spin_state st, int layer, int rows, const void* keys, cons
   a.alpha = st->cfg.alpha;
   a.beta = beta_of(st->cfg.alpha);
   a.inject = 0;
+  a.gmax = nullptr;
+  a.gstride = st->gstride;
+  if (wrote_gmax) *wrote_gmax = false;
   if (a.key_fp8) {
     spin_status s = cuda_status(staged(st, kQuant, stream, [&] { return launch_quantize_q(a, stream); }));
     if (s != SPIN_OK) return s;
@@ -214,6 +223,10 @@ spin_status run_score(spin_state st, int layer, int rows, const void* keys, cons
   if (use_tc(st, rows)) {
     a.inject = st->inject;
     st->inject = 0;
+    if (wrote_gmax) {
+      a.gmax = st->gmax;
+      *wrote_gmax = true;
+    }
     return cuda_status(staged(st, kScore, stream, [&] { return launch_score_tc(a, st->encode_fn, stream); }));
   }
   return cuda_status(staged(st, kScore, stream, [&] { return launch_score_simt(a, stream); }));
@@ -255,6 +268,8 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->q8 = (uint8_t*)(st->base + k.q8);
   st->wq = (float*)(st->base + k.wq);
   st->scores = (float*)(st->base + k.scores);
+  st->gmax = (float*)(st->base + k.gmax);
+  st->gstride = gmax_stride(L);
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
   st->inject = 0;
@@ -410,7 +425,7 @@ spin_status spin_topk(spin_state st, int rows, const float* scores_dev, const ui
     return launch_compact(st->lay, rows, ctx_len_dev, mask_dev, st->work, st->kept, st->err, s);
   }));
   if (r != SPIN_OK) return r;
-  TopkArgs a{st->lay, rows, scores_dev, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err};
+  TopkArgs a{st->lay, rows, scores_dev, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err, nullptr, 0};
   return cuda_status(staged(st, kTopk, s, [&] { return launch_topk(a, s); }));
 }
 
@@ -459,10 +474,12 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
   if (r != SPIN_OK) return r;
   const bool fuse = !defer_update && rows == 1;
+  bool gm = false;
   r = run_score(st, layer, rows, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len_dev, mask_dev,
-                scores, fuse, s);
+                scores, fuse, s, &gm);
   if (r != SPIN_OK) return r;
-  TopkArgs t{st->lay, rows, scores, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err};
+  TopkArgs t{st->lay, rows, scores, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err,
+             gm ? st->gmax : nullptr, st->gstride};
   r = cuda_status(staged(st, kTopk, s, [&] { return launch_topk(t, s); }));
   if (r != SPIN_OK) return r;
   if (!defer_update && rows > 1) return spin_ema_update(st, layer, rows, scores, mask_dev, ctx_len_dev, nullptr, stream);

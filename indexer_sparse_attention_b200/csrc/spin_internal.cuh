@@ -175,6 +175,8 @@ struct ScoreArgs {
   float* D;
   float alpha, beta;   // beta = fl32(1 - alpha), computed once on the host
   int inject;          // test hook: withhold the first key stage of CTA 0
+  float* gmax;         // [Q][R][gstride] max score of each 32-slot group of the
+  int64_t gstride;     // kept-slot order (tensor-core kernel only), or null
 };
 
 cudaError_t launch_quantize_q(const ScoreArgs& a, cudaStream_t s);
@@ -192,6 +194,8 @@ struct TopkArgs {
   const int32_t* kept;
   int32_t* topk;
   ErrWord* err;
+  const float* gmax;  // group maxima written by the score kernel, or null
+  int64_t gstride;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 

@@ -93,7 +93,7 @@ extern "C" SPIN_API spin_status spin_topk_noalloc(int num_requests, int rows, in
   e = cudaMemsetAsync(err, 0, sizeof(ErrWord), s);
   if (e == cudaSuccess) e = launch_compact(L, rows, ctx_len_dev, mask_dev, work, kept, err, s);
   if (e == cudaSuccess) {
-    TopkArgs a{L, rows, scores_dev, mask_dev, ctx_len_dev, work, kept, topk_dev, err};
+    TopkArgs a{L, rows, scores_dev, mask_dev, ctx_len_dev, work, kept, topk_dev, err, nullptr, 0};
     e = launch_topk(a, s);
   }
   if (e != cudaSuccess) {
