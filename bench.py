@@ -40,8 +40,16 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "SPIN decode rows/s & index-key GB/s at 512K ctx x96 req; % of roofline"
+WORKLOADS = {"serve-96x512K": 2, "mtp-32x128K-r4": 3, "ragged-8Lx8-256K-1M": 4, "dsa-1x64K": 1, "tiny-fp32-4K": 0}
 KEY_BYTES_PER_SLOT = 128 + 4            # E4M3 key row + fp32 scale
 SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write of V and D
+# DRAM traffic of one k_score_tc launch (dram__bytes_read.sum + dram__bytes_write.sum)
+# per kept slot, from one ncu capture of the kernel on 16 requests at 512K, 50% sparsity,
+# fused EMA (traffic grows with kept slots: each is read once), valid for the kernel
+# source with this hash prefix
+SCORE_TRAFFIC = {"src_sha256_16": "0f18bc853bfdb0f1", "bytes_per_kept_slot": 151.36,
+                 "sources": ("indexer_sparse_attention_b200/csrc/k_score_tc.cu",
+                             "indexer_sparse_attention_b200/csrc/spin_internal.cuh")}
 
 
 def parse():
@@ -55,6 +63,8 @@ def parse():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--workload", choices=list(WORKLOADS), default="serve-96x512K",
+                   help="serve-96x512K is the headline; the others print their own line")
     return p.parse_args()
 
 
@@ -165,6 +175,17 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def score_traffic_per_slot():
+    """The captured DRAM bytes per kept slot, or None once the kernel source
+    differs from the one the counters were taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in SCORE_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return SCORE_TRAFFIC["bytes_per_kept_slot"] if h.hexdigest()[:16] == SCORE_TRAFFIC["src_sha256_16"] else None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -334,6 +355,7 @@ def gpu_arm(args, world, rank, local):
     score_ms, score_n = stages["score"]
     score_avg = score_ms / max(score_n, 1)
     achieved = kept_slots * SCORE_BYTES_PER_SLOT / (score_avg / 1e3) / 1e9
+    traffic_slot = score_traffic_per_slot()
     launches = sum(n for _, n in stages.values())
     out = {
         "metric": METRIC, "value": rows_s, "unit": "rows/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -349,7 +371,10 @@ def gpu_arm(args, world, rank, local):
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs (copy, MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s", "avg_launch_ms": score_avg,
-                     "bytes_per_launch": kept_slots * SCORE_BYTES_PER_SLOT, "traffic": None},
+                     "bytes_per_launch": kept_slots * SCORE_BYTES_PER_SLOT,
+                     "traffic": (None if traffic_slot is None else traffic_slot * kept_slots),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
+                                       "(16-request capture, scaled by kept slots)"},
         "stage_ms_per_step": {k: v[0] / K for k, v in stages.items() if v[1]},
         "gpu_launches": launches,
         "clocks": clk.summary(),
@@ -371,6 +396,242 @@ def gpu_arm(args, world, rank, local):
     e2e_ms, h2d, d2h = e2e_pass(run, K, world)
     out["e2e"] = {"value": job_rows_per_s(Q * K, world, e2e_ms), "unit": "rows/s", "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
+    status, word = isa.spin_get_error(run.st)
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# The other workloads (MTP rows, multi-layer ragged contexts, single request,
+# tiny fp32): one JSON line each, same keys as the headline where they apply
+# ---------------------------------------------------------------------------
+L2_BYTES = 126 * 1024 * 1024
+
+
+def score_bytes_per_slot(rows: int, fused: bool, key_fp8: bool, d: int) -> int:
+    """Algorithmic bytes of the score kernel per kept slot: the key row and
+    its scale, one score per row, and (fused, one row) the EMA read/write of
+    V and D."""
+    key = (d + 4) if key_fp8 else 4 * d
+    return key + 4 * rows + (16 if fused else 0)
+
+
+class WorkloadRun:
+    """A workload through the C ABI with every layer's key cache and queries
+    resident on the device.  The per-step inputs (each request's query rows
+    at its committed position, context lengths, accepted lengths) are built
+    before any timed region."""
+
+    def __init__(self, wl, device, total_steps):
+        import indexer_sparse_attention_b200 as isa
+        self.isa, self.wl, self.device = isa, wl, device
+        Q, R, Ly = wl.requests, wl.rows, wl.layers
+        self.caches = [workloads.make_key_cache(wl, l, device) for l in range(Ly)]
+        acc = workloads.accepted_lengths(wl, total_steps).numpy()
+        committed = np.array(wl.ctx0, np.int64)
+        ctx0 = committed.copy()
+        plans = []
+        for t in range(total_steps):
+            plans.append((committed - ctx0, committed + 1, acc[t]))
+            committed = committed + acc[t]
+        self.ctx = [torch.from_numpy(c.astype(np.int32)).to(device) for _, c, _ in plans]
+        self.acc = [torch.from_numpy(a.astype(np.int32)).to(device) for _, _, a in plans]
+        self.qw = [[None] * Ly for _ in range(total_steps)]
+        rows_idx = torch.arange(R)
+        for l in range(Ly):
+            q_all, w_all = workloads.make_queries(wl, l, total_steps * R + R, device)
+            for t, (pos0, _, _) in enumerate(plans):
+                idx = (torch.from_numpy(pos0)[:, None] + rows_idx[None, :]).to(device)
+                ar = torch.arange(Q, device=device)[:, None]
+                self.qw[t][l] = (q_all[ar, idx].contiguous(), w_all[ar, idx].contiguous())
+            del q_all, w_all
+        cfg = isa.make_config(num_layers=Ly, num_requests=Q, max_slots=wl.max_slots, block_size=wl.b,
+                              num_heads=wl.H, head_dim=wl.d, topk=wl.topk, max_rows=R, key_fp8=wl.key_fp8,
+                              q_bf16=wl.q_bf16, alpha=wl.alpha, gamma=wl.gamma, target_sparsity=wl.sparsity,
+                              seed=wl.seed)
+        self.st = isa.SpinState(cfg, device=device)
+        self.masks = [self.st.new_mask() for _ in range(Ly)]
+        self.topks = [torch.empty((Q, R, wl.topk), dtype=torch.int32, device=device) for _ in range(Ly)]
+        self.scores = self.st.new_scores()
+        self.t = 0
+
+    def set_sparsity(self, per_layer):
+        self.isa.spin_set_layer_sparsity(self.st, list(per_layer))
+
+    def step(self, layers=None):
+        """One decode step of every layer: a0..a5, and for MTP rows the
+        prefix-valid EMA replay once the accepted lengths are known."""
+        isa, wl, t = self.isa, self.wl, self.t
+        R = wl.rows
+        for l in (range(wl.layers) if layers is None else layers):
+            c = self.caches[l]
+            q, w = self.qw[t][l]
+            isa.spin_decode_step(self.st, l, R, t, c.keys, c.kscale if wl.key_fp8 else None, c.block_table, q, w,
+                                 self.ctx[t], R > 1, self.masks[l], self.topks[l], self.scores)
+            if R > 1:
+                isa.spin_ema_update(self.st, l, R, self.scores, self.masks[l], self.ctx[t], self.acc[t])
+        self.t += 1
+
+    def kept_slots(self, t):
+        """Visible slots of the kept blocks at step t (row R-1 sees the most),
+        summed over layers, and the realized sparsity per (layer, request)."""
+        wl = self.wl
+        ctx = self.ctx[t].long() + wl.rows - 1
+        nb = (ctx + wl.b - 1) // wl.b
+        total, realized = 0, []
+        for m8 in self.masks:
+            m = m8[:, : int(nb.max())].bool()
+            kept = m.sum(dim=1)
+            last = nb - 1
+            tail_kept = m.gather(1, last[:, None])[:, 0]
+            slots = kept * wl.b - tail_kept.long() * (wl.b - (ctx - last * wl.b))
+            total += int(slots.sum().item())
+            realized += (1 - kept.double() / nb.double()).tolist()
+        return total, realized
+
+    def miss(self):
+        """Share of the full indexer's top-k in skipped blocks, per layer and
+        (request, row), for the step just run (shadow all-keep indexer)."""
+        isa, wl, t = self.isa, self.wl, self.t - 1
+        R, Q = wl.rows, wl.requests
+        full_scores = self.st.new_scores()
+        full_topk = torch.empty((Q, R, wl.topk), dtype=torch.int32, device=self.device)
+        missed = torch.zeros((Q, R), dtype=torch.int32, device=self.device)
+        total = torch.zeros_like(missed)
+        out = []
+        for l in range(wl.layers):
+            c = self.caches[l]
+            q, w = self.qw[t][l]
+            allk = torch.ones_like(self.masks[l])
+            isa.spin_indexer_score(self.st, l, R, c.keys, c.kscale if wl.key_fp8 else None, c.block_table, q, w,
+                                   self.ctx[t], allk, full_scores)
+            isa.spin_topk(self.st, R, full_scores, allk, self.ctx[t], full_topk)
+            isa.spin_miss_count(self.st, R, full_topk, self.masks[l], missed, total)
+            out.append((missed.double() / total.double().clamp(min=1)).flatten().tolist())
+        return out
+
+
+def workload_arm(args, world, rank, local):
+    """One of the non-headline workloads: history bootstrap, the workload's
+    own warm-up protocol, then K timed steps (every layer, every row)."""
+    import indexer_sparse_attention_b200 as isa
+    from indexer_sparse_attention_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    isa.load()
+    device = torch.device("cuda", local if world > 1 else 0)
+    base = workloads.config(WORKLOADS[args.workload])
+    W, K = max(args.warmup, 3), args.steps
+    fid_steps = 3
+    total = 1 + base.warmup_steps + W + K + fid_steps
+    wl = workloads.config(WORKLOADS[args.workload], seed=base.seed + 1000 * rank, steps=total,
+                          spare_slots=base.rows * 4)
+    run = WorkloadRun(wl, device, total)
+    Ly, Q, R = wl.layers, wl.requests, wl.rows
+    # history bootstrap (all-keep), then the workload's warm-up protocol
+    run.set_sparsity([0.0] * Ly)
+    run.step()
+    sparsity = [wl.sparsity] * Ly
+    run.set_sparsity(sparsity)
+    alloc = None
+    if wl.warmup_steps:
+        # uniform target with a shadow full indexer measuring each layer's miss,
+        # then budgets in proportion to the measured miss (per-layer budget)
+        miss = np.zeros(Ly)
+        for _ in range(wl.warmup_steps):
+            run.step()
+            miss += np.array([np.mean(m) for m in run.miss()])
+        miss /= wl.warmup_steps
+        nblk = (np.array(wl.ctx0, np.float64) + wl.b - 1) // wl.b
+        blocks = np.full(Ly, nblk.sum())
+        lo = np.full(Ly, max(0.05, float(np.ceil(wl.topk / wl.b) / nblk.min())))
+        sparsity = isa.spin_allocate_layer_sparsity(miss.tolist(), blocks.tolist(), lo.tolist(), wl.sparsity)
+        run.set_sparsity(sparsity)
+        alloc = {"warmup_miss": miss.tolist(), "layer_sparsity": sparsity}
+    for _ in range(W):
+        run.step()
+    # L2-resident workloads are timed step by step with L2 flushed in between
+    input_bytes = sum(c.keys.numel() * c.keys.element_size() for c in run.caches)
+    flush = input_bytes < 2 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device) if flush else None
+    isa.spin_kernel_times(run.st)
+    isa.spin_set_kernel_timing(run.st, True)
+    s = torch.cuda.current_stream()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        if flush:
+            ms = 0.0
+            for _ in range(K):
+                scratch.fill_(1.0)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                run.step()
+                e1.record(s)
+                e1.synchronize()
+                ms += e0.elapsed_time(e1)
+        else:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(K):
+                run.step()
+            e1.record(s)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+    barrier(world)
+    ms = max_over_ranks(ms, world)
+    isa.spin_set_kernel_timing(run.st, False)
+    stages = isa.spin_kernel_times(run.st)
+    status, word = isa.spin_get_error(run.st)
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x} during the timed region")
+    kept, _ = run.kept_slots(run.t - 1)
+    ms_step = ms / K
+    rows_step = Q * R
+    peak, peak_kind = peaks()
+    fused = R == 1
+    per_slot = score_bytes_per_slot(R, fused, wl.key_fp8, wl.d)
+    key_slot = (wl.d + 4) if wl.key_fp8 else 4 * wl.d
+    score_ms, score_n = stages["score"]
+    score_avg = score_ms / max(score_n, 1)
+    per_launch = kept / Ly * per_slot
+    achieved = per_launch / (score_avg / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": job_rows_per_s(rows_step * K, world, ms),
+        "unit": "rows/s" if Ly == 1 else f"rows/s (a row passes all {Ly} layers)",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3xe4m3->f32 (selection f32, exact)" if wl.key_fp8 else "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "requests_per_gpu": Q, "layers": Ly, "rows": R,
+                   "context_slots": [min(wl.ctx0), max(wl.ctx0)], "block_size": wl.b, "heads": wl.H,
+                   "head_dim": wl.d, "topk": wl.topk, "target_sparsity": wl.sparsity, "gamma": wl.gamma,
+                   "parallelism": f"dp{world} (requests sharded, no collective)",
+                   "l2": "flushed before every timed step (inputs L2-resident)" if flush
+                   else f"inputs larger than L2: {input_bytes / 1e9:.2f} GB of keys"},
+        "index_key_gbs": kept * key_slot / (ms_step / 1e3) / 1e9,
+        "key_roofline_frac": kept * key_slot / (ms_step / 1e3) / 1e9 / peak,
+        "roofline": {"bound": "hbm", "kernel": ("k_score_tc" if wl.key_fp8 else "k_score_simt"),
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} hbm_gbs", "avg_launch_ms": score_avg,
+                     "bytes_per_launch": per_launch, "bytes_per_kept_slot": per_slot, "traffic": None},
+        "stage_ms_per_step": {k: v[0] / K for k, v in stages.items() if v[1]},
+        "gpu_launches": sum(n for _, n in stages.values()),
+        "clocks": clk.summary(),
+    }
+    if alloc:
+        out["config"]["per_layer_budget"] = alloc
+    miss_all, realized = [], []
+    for _ in range(fid_steps):
+        run.step()
+        miss_all += [x for m in run.miss() for x in m]
+        realized += run.kept_slots(run.t - 1)[1]
+    v = np.sort(np.array(miss_all))
+    out["fidelity"] = {"mean_miss": float(v.mean()),
+                       "p99_miss": float(v[max(int(np.ceil(0.99 * v.size)), 1) - 1]),
+                       "realized_sparsity": float(np.mean(realized)), "rows": int(v.size)}
     status, word = isa.spin_get_error(run.st)
     if status != 0:
         raise RuntimeError(f"device error word {word:#x}")
@@ -465,6 +726,11 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
+        if args.workload != "serve-96x512K":
+            out = workload_arm(args, world, rank, local)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+            return
         out = gpu_arm(args, world, rank, local)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
