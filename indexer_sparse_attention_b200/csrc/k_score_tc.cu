@@ -19,13 +19,16 @@
 //               tile's two key-page TMA loads.  The copy engine's cost is per
 //               request, so it moves only key pages; a second CTA per SM adds
 //               a second issuer.
-//   warp 1      TMEM allocation; lane 0 issues the MMAs and the commits
+//   warp 1      TMEM allocation; lane 0 issues the MMAs and one commit per
+//               tile, which frees the key stage for the producer and marks
+//               the accumulator full for the epilogue
 //   warps 2..9  two epilogue groups of four warps, taking alternate tiles; a
 //               thread owns one token: it loads the token's scale and EMA
 //               values one tile ahead, reads its accumulator row from the TMEM
-//               quarter its warp may access (lanes 32*(warp%4) ..), applies
-//               ReLU, head weights and the scale, and stores the score and the
-//               fused EMA update
+//               quarter its warp may access (lanes 32*(warp%4) ..), hands
+//               the accumulator back as soon as its last columns are in
+//               registers, applies ReLU, head weights and the scale, and
+//               stores the score and the fused EMA update
 // Pipelines: key stages freed as soon as the MMAs have read them (6 per CTA
 // at N = 64, 8 with one CTA per SM); a 16-slot ring of tile info freed by the
 // epilogue; 1 query buffer with two CTAs per SM (2 with one); 4 TMEM
@@ -235,14 +238,13 @@ __host__ __device__ inline TcPlan tc_plan(int N, int Q) {
 }
 
 struct Bars {
-  uint32_t full, empty, afull, aempty, qfull, qempty, accfull, accempty, done;
+  uint32_t full, empty, afull, aempty, qfull, qempty, accempty, done;
   __device__ uint32_t f(int s) const { return full + 8 * s; }
   __device__ uint32_t e(int s) const { return empty + 8 * s; }
   __device__ uint32_t xf(int s) const { return afull + 8 * s; }
   __device__ uint32_t xe(int s) const { return aempty + 8 * s; }
   __device__ uint32_t qf(int i) const { return qfull + 8 * i; }
   __device__ uint32_t qe(int i) const { return qempty + 8 * i; }
-  __device__ uint32_t af(int i) const { return accfull + 8 * i; }
   __device__ uint32_t ae(int i) const { return accempty + 8 * i; }
 };
 
@@ -315,8 +317,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   B.aempty = B.afull + 8 * kAuxSlots;
   B.qfull = B.aempty + 8 * kAuxSlots;
   B.qempty = B.qfull + 16;
-  B.accfull = B.qempty + 16;
-  B.accempty = B.accfull + 8 * kMaxAcc;
+  B.accempty = B.qempty + 16;
   B.done = B.accempty + 8 * kMaxAcc;
   const Ctl ctl{abort_flag, a.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -345,10 +346,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(B.qf(i), 1);
       mbar_init(B.qe(i), 1);
     }
-    for (int i = 0; i < nacc; ++i) {
-      mbar_init(B.af(i), 1);
-      mbar_init(B.ae(i), 4);  // the four warps of the group that owns the tile
-    }
+    for (int i = 0; i < nacc; ++i) mbar_init(B.ae(i), 4);  // the four warps of the group that owns the tile
     mbar_init(B.done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -451,32 +449,42 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (lane == 0 && g0 < g1) {
+      // The loop is the serial path of the CTA: counters advance without
+      // divisions, the request is re-resolved only at its last tile, and one
+      // commit per tile signals both the producer (stage free) and the
+      // epilogue (accumulator full).
       const uint32_t idesc = idesc_e4m3(kTileM, N);
-      int q = sched.locate(g0), t = g0 - prefix[q];
-      int cur_q = -1, qiter = 0;
-      for (int g = g0; g < g1; ++g, ++t) {
-        while (t >= prefix[q + 1] - prefix[q]) { ++q; t = 0; }
-        const int i = g - g0;
-        const int stage = i % stages, acc = i % nacc;
-        const uint32_t phase = (uint32_t)(i / stages) & 1u, acc_phase = (uint32_t)(i / nacc) & 1u;
-        if (q != cur_q) {
-          if (cur_q >= 0) umma_commit(B.qe((qiter - 1) % nq));
-          const int nb = qiter % nq;
-          if (!wait_parity(B.qf(nb), (qiter / nq) & 1, ctl)) break;
-          cur_q = q;
+      int q = sched.locate(g0);
+      int q_end = prefix[q + 1];  // first global tile of the next request
+      int qiter = 0, qbuf = 0;
+      uint32_t qphase = 0;
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = wait_parity(B.qf(0), 0, ctl);
+      for (int g = g0; ok && g < g1; ++g) {
+        if (g >= q_end) {
+          do { ++q; } while (prefix[q + 1] <= g);
+          q_end = prefix[q + 1];
+          umma_commit(B.qe(qbuf));  // the previous query tile is free once its MMAs complete
           ++qiter;
+          qbuf = qiter % nq;
+          qphase = (uint32_t)(qiter / nq) & 1u;
+          if (!wait_parity(B.qf(qbuf), qphase, ctl)) break;
         }
         if (!wait_parity(B.ae(acc), acc_phase ^ 1, ctl)) break;
         if (!wait_parity(B.f(stage), phase, ctl)) break;
         tc_fence_after();
-        const uint32_t a_addr = sbase + lay.keys + stage * kStageBytes;
-        const uint32_t b_addr = sbase + lay.qbuf + ((qiter - 1) % nq) * N * kRowBytes;
+        const uint64_t a_desc = sw128_desc(sbase + lay.keys + stage * kStageBytes);
+        const uint64_t b_desc = sw128_desc(sbase + lay.qbuf + qbuf * N * kRowBytes);
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
+        // K = 128 bytes as four K = 32 steps; a 32-byte step inside the
+        // swizzled atom advances the descriptor's start address by 2 (16-byte units)
 #pragma unroll
         for (int kk = 0; kk < kRowBytes / 32; ++kk)
-          umma_e4m3(d_tmem, sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
+          umma_e4m3(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
         umma_commit(B.e(stage));
-        umma_commit(B.af(acc));
+        if (++stage == stages) { stage = 0; phase ^= 1u; }
+        if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
       }
       // all MMAs issued by this thread complete before TMEM is released
       umma_commit(B.done);
@@ -522,17 +530,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = group; alive_ && i < n_local; i += kEpiGroups) {
       const Pre cur = nx;
       if (i + kEpiGroups < n_local && !prefetch(i + kEpiGroups, nx)) break;
-      const int xs = i % kAuxSlots, acc = i % nacc;
-      const uint32_t acc_phase = (uint32_t)(i / nacc) & 1u;
+      const int xs = i % kAuxSlots, acc = i % nacc, stage = i % stages;
+      const uint32_t phase = (uint32_t)(i / stages) & 1u;
       if (cur.q != cur_q) {
         __syncwarp();
         for (int k = lane; k < N; k += 32) wcur[k] = a.wq[(int64_t)cur.q * N + k];
         __syncwarp();
         cur_q = cur.q;
       }
-      // every lane waits; the warp leaves together if any lane gave up, so
-      // the .sync.aligned TMEM loads below never run on a partial warp
-      if (!__all_sync(0xffffffffu, wait_parity(B.af(acc), acc_phase, ctl))) break;
+      // The MMA's commit on the key stage also marks the accumulator full.
+      // Every lane waits; the warp leaves together if any lane gave up, so
+      // the .sync.aligned TMEM loads below never run on a partial warp.
+      if (!__all_sync(0xffffffffu, wait_parity(B.e(stage), phase, ctl))) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
       for (int r = 0; r < a.rows; ++r) {
@@ -542,11 +551,28 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld16(trow + (uint32_t)(r * L.H + c), *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           if (c + 16 < L.H) tmem_ld16(trow + (uint32_t)(r * L.H + c + 16), *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
           tmem_wait_ld();
-          const float* wr = wcur + r * L.H + c;
-          const int nu = min(32, L.H - c);
+          if (r == a.rows - 1 && c + 32 >= L.H) {
+            // last accumulator columns are in registers: hand the accumulator
+            // (and the tile-info slot, read a tile ago) back before the math
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(B.ae(acc));
+              mbar_arrive(B.xe(xs));
+            }
+          }
+          const float4* wr = reinterpret_cast<const float4*>(wcur + r * L.H + c);
+          const int nu = min(32, L.H - c);  // 16 or 32: H is a multiple of 16
 #pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (u < nu) part[u & 3] = __fmaf_rn(wr[u], fmaxf(__uint_as_float(v[u]), 0.0f), part[u & 3]);
+          for (int u = 0; u < 32; u += 4) {
+            if (u < nu) {
+              const float4 w4 = wr[u >> 2];
+              part[0] = __fmaf_rn(w4.x, fmaxf(__uint_as_float(v[u + 0]), 0.0f), part[0]);
+              part[1] = __fmaf_rn(w4.y, fmaxf(__uint_as_float(v[u + 1]), 0.0f), part[1]);
+              part[2] = __fmaf_rn(w4.z, fmaxf(__uint_as_float(v[u + 2]), 0.0f), part[2]);
+              part[3] = __fmaf_rn(w4.w, fmaxf(__uint_as_float(v[u + 3]), 0.0f), part[3]);
+            }
+          }
         }
         const float sum = (part[0] + part[1]) + (part[2] + part[3]);
         const bool scored = cur.valid && cur.s <= cur.p0 + r;
@@ -565,12 +591,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             a.D[(int64_t)cur.q * L.slot_stride + (cur.p0 - cur.s)] = ema_d(cur.d, score, a.alpha, a.beta);
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(B.ae(acc));
-        mbar_arrive(B.xe(xs));
       }
     }
   }
