@@ -40,6 +40,7 @@
 
 #include <algorithm>
 
+#include "block_scan.cuh"
 #include "spin_internal.cuh"
 
 namespace spin {
@@ -156,6 +157,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+// Two independent fp32 fused multiply-adds (round to nearest) in one packed
+// instruction: (a0, a1) += (w0 * x0, w1 * x1), each rounded once as fmaf.
+__device__ __forceinline__ void fma2_rn(float& a0, float& a1, float w0, float w1, float x0, float x1) {
+  asm("{\n\t.reg .b64 acc, w, x;\n\tmov.b64 acc, {%0, %1};\n\tmov.b64 w, {%2, %3};\n\t"
+      "mov.b64 x, {%4, %5};\n\tfma.rn.f32x2 acc, w, x, acc;\n\tmov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -323,16 +332,27 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool fused = a.V != nullptr;
 
-  // ---- tile prefix over requests, barriers ---------------------------------
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int q = 0; q < L.Q; ++q) {
-      prefix[q] = acc;
-      const int64_t ctx = a.ctx_len[q];
-      const bool ok = ctx >= 1 && ctx + a.rows - 1 <= L.max_slots;
-      acc += ok ? (a.kept[q] + 1) / 2 : 0;
+  // ---- tile prefix over requests (all threads: one load pair each, block
+  // scan), barriers ------------------------------------------------------
+  {
+    int* scan_tmp = reinterpret_cast<int*>(wqs);  // 33 ints; the epilogue fills wqs later
+    int carry = 0;
+    for (int base = 0; base < L.Q; base += kThreads) {
+      const int q = base + (int)threadIdx.x;
+      int v = 0;
+      if (q < L.Q) {
+        const int64_t ctx = a.ctx_len[q];
+        const bool ok = ctx >= 1 && ctx + a.rows - 1 <= L.max_slots;
+        v = ok ? (a.kept[q] + 1) / 2 : 0;
+      }
+      int tot;
+      const int ex = block_exclusive_scan(v, scan_tmp, &tot);
+      if (q < L.Q) prefix[q] = carry + ex;
+      carry += tot;
     }
-    prefix[L.Q] = acc;
+    if (threadIdx.x == 0) prefix[L.Q] = carry;
+  }
+  if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < stages; ++s) {
       mbar_init(B.f(s), 1);
@@ -567,10 +587,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int u = 0; u < 32; u += 4) {
             if (u < nu) {
               const float4 w4 = wr[u >> 2];
-              part[0] = __fmaf_rn(w4.x, fmaxf(__uint_as_float(v[u + 0]), 0.0f), part[0]);
-              part[1] = __fmaf_rn(w4.y, fmaxf(__uint_as_float(v[u + 1]), 0.0f), part[1]);
-              part[2] = __fmaf_rn(w4.z, fmaxf(__uint_as_float(v[u + 2]), 0.0f), part[2]);
-              part[3] = __fmaf_rn(w4.w, fmaxf(__uint_as_float(v[u + 3]), 0.0f), part[3]);
+              fma2_rn(part[0], part[1], w4.x, w4.y, fmaxf(__uint_as_float(v[u + 0]), 0.0f),
+                      fmaxf(__uint_as_float(v[u + 1]), 0.0f));
+              fma2_rn(part[2], part[3], w4.z, w4.w, fmaxf(__uint_as_float(v[u + 2]), 0.0f),
+                      fmaxf(__uint_as_float(v[u + 3]), 0.0f));
             }
           }
         }

@@ -162,6 +162,66 @@ __device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t
   __syncthreads();
 }
 
+// Exploration draw by a short list: the Philox keys are uniform, so the
+// `take` smallest of n_cand lie below t = (1.25 take + 64) / n_cand * 2^32
+// with overwhelming probability.  Candidates under t are appended to a
+// shared list (one atomic per warp), the list is sorted by (key, block
+// index), and its first `take` blocks are explored.  Returns false -- nothing marked -- when the list holds fewer
+// than `take` entries or overflows, and the caller runs the radix select.
+constexpr int kExpCap = 2048;
+
+__device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last, int take, int n_cand,
+                                uint2* list, SelShared& sh) {
+  const double frac = (1.25 * take + 64.0) / (double)n_cand;
+  const uint64_t t = frac >= 1.0 ? (1ull << 32) : (uint64_t)(frac * 4294967296.0);
+  if (threadIdx.x == 0) sh.digit[0] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  for (int j0 = 0; j0 < n_last; j0 += blockDim.x) {  // warp-uniform trip count
+    const int j = j0 + (int)threadIdx.x;
+    uint32_t u = 0;
+    bool in = false;
+    if (j < n_last && m[j] == 0) {
+      u = explore_key(a.seed, (uint32_t)j, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
+      in = (uint64_t)u < t;
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    if (!bal) continue;
+    uint32_t at = 0;
+    if (lane == 0) at = atomicAdd(&sh.digit[0], (uint32_t)__popc(bal));
+    at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+    if (in && at < (uint32_t)kExpCap) list[at] = make_uint2(u, (uint32_t)j);
+  }
+  __syncthreads();
+  const int cnt = (int)sh.digit[0];
+  if (cnt < take || cnt > kExpCap) return false;  // uniform: every thread reads the same count
+  // bitonic sort of the list by (key, block), padded to a power of two with
+  // entries that sort last; the first `take` entries are the draw
+  int n2 = 1;
+  while (n2 < cnt) n2 <<= 1;
+  for (int i = cnt + (int)threadIdx.x; i < n2; i += blockDim.x) list[i] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const uint2 x = list[i], y = list[ixj];
+          const bool gt = x.x > y.x || (x.x == y.x && x.y > y.y);
+          if (gt == ((i & k) == 0)) {
+            list[i] = y;
+            list[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < take; i += blockDim.x) m[list[i].y] = 2;
+  __syncthreads();
+  return true;
+}
+
 // Ordered compaction of the kept blocks of one request into its work list.
 __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t* kept, int* scan) {
   const int chunk = (n_last + blockDim.x - 1) / blockDim.x;
@@ -181,6 +241,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
   extern __shared__ __align__(16) uint8_t dyn[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);
   uint8_t* m = dyn + 4 * L.blk_stride;
+  uint2* list = reinterpret_cast<uint2*>(dyn + 5 * L.blk_stride);  // kExpCap (key, block) pairs
   __shared__ SelShared sh;
 
   const int64_t ctx = a.ctx_len[q];
@@ -207,7 +268,19 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
       const int n = (int)row_blocks(ctx, r, L.b);
       const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
       const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride;
-      for (int j = threadIdx.x; j < n; j += blockDim.x) keys[j] = fkey(S[j]);
+      for (int j0 = 0; j0 < n; j0 += 4 * kSelThreads) {  // four loads in flight per thread
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + u * kSelThreads + (int)threadIdx.x;
+          v[u] = j < n ? S[j] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + u * kSelThreads + (int)threadIdx.x;
+          if (j < n) keys[j] = fkey(v[u]);
+        }
+      }
       __syncthreads();
       auto all = [](int) { return true; };
       if (n_pred >= n) {
@@ -226,15 +299,17 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
     int n_cand;
     block_exclusive_scan(c, sh.scan, &n_cand);
     const int64_t take = n_exp < n_cand ? n_exp : n_cand;
-    if (take > 0) {
+    if (take == n_cand) {
+      for (int j = threadIdx.x; j < n_last; j += blockDim.x)
+        if (m[j] == 0) m[j] = 2;
+      __syncthreads();
+    } else if (take > 0 && explore_by_list(a, q, m, n_last, (int)take, n_cand, list, sh)) {
+      // done: the `take` smallest keys came from the short list
+    } else if (take > 0) {
       for (int j = threadIdx.x; j < n_last; j += blockDim.x)
         keys[j] = ~explore_key(a.seed, (uint32_t)j, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
       __syncthreads();
-      if (take == n_cand) {
-        for (int j = threadIdx.x; j < n_last; j += blockDim.x)
-          if (m[j] == 0) m[j] = 2;
-        __syncthreads();
-      } else {
+      {
         uint32_t T, eq;
         radix_select_desc(keys, n_last, cand, (uint32_t)take, sh, &T, &eq);
         // mark into a separate pass: `cand` reads m, so label after the scan
@@ -263,7 +338,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
 }
 
 cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)a.lay.blk_stride * 5;
+  const size_t smem = (size_t)a.lay.blk_stride * 5 + (size_t)kExpCap * sizeof(uint2);
   cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_select<<<a.lay.Q, kSelThreads, smem, s>>>(a);

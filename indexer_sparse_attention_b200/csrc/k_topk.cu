@@ -37,8 +37,10 @@ constexpr int kTopkThreads = 1024;
 constexpr int kBins = 8192;           // 13-bit first digit
 constexpr int kFirstShift = 19;
 constexpr int kCandCap = 8192;        // candidates kept on chip
+constexpr uint32_t kEmptyGroup = 0x007FFFFFu;  // key of -inf: a group with no scored slot
 
 struct TopkShared {
+  uint32_t k_and, k_or;
   uint32_t digit[2];
   int scan[33];
   int total;
@@ -305,48 +307,76 @@ __device__ uint32_t select_candidates(const TopkCtx& c, int n_cand, int want, To
   return T;
 }
 
-// Key of rank `want` (largest first) among keys[0..n), with warp-combined
-// histogram adds (group maxima share their leading key bits).
-__device__ uint32_t radix_select_agg(const uint32_t* keys, int n, uint32_t want, uint32_t* hist2, TopkShared& sh) {
-  uint32_t prefix = 0, rem = want;
-  const int lane = threadIdx.x & 31;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist2[i] = 0;
-    __syncthreads();
-    const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int base = 0; base < n; base += blockDim.x) {
-      const int i = base + threadIdx.x;
-      const uint32_t k = i < n ? keys[i] : 0u;
-      const bool act = i < n && (k & pmask) == prefix;
-      const uint32_t bin = (k >> shift) & 255u;
-      const uint32_t m = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const uint32_t peers = __match_any_sync(m, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist2[bin], (uint32_t)__popc(peers));
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) warp_find_digit_desc<256>(hist2, rem, sh.digit);
-    __syncthreads();
-    prefix |= sh.digit[0] << shift;
-    rem = sh.digit[1];
-    __syncthreads();
-  }
-  return prefix;
-}
-
 // Candidates from group maxima (the score kernel's max of every 32 slots of
-// the kept-slot order).  M = the want-th largest group maximum; at least
-// `want` scores are >= M (each of the want best groups holds one), and every
-// score >= M lies in a group whose maximum is >= M, so gathering those groups'
-// scores >= M yields a candidate list that holds the whole top `want`.
-// The group keys and then the compacted group list live in the bitmap area.
+// the kept-slot order), for n_groups > want.  Any M no larger than the
+// want-th largest group maximum works: at least `want` scores are >= M (each
+// of the want best groups holds one), and every score >= M lies in a group
+// whose maximum is >= M, so gathering those groups' scores >= M yields a
+// candidate list that holds the whole top `want`.  M is the lower edge of the
+// 13-bit histogram bin that holds the want-th largest group key, with the bin
+// window placed just below the leading bits all group keys share.  The group
+// keys and then the compacted group list live in the bitmap area.
 __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want, TopkShared& sh) {
   const int n_groups = (c.n_elem + 31) / 32;  // == c.nwords
   uint32_t* gk = c.bits;
-  for (int g = threadIdx.x; g < n_groups; g += blockDim.x) gk[g] = fkey(gmax[g]);
+  if (threadIdx.x == 0) {
+    sh.k_and = 0xFFFFFFFFu;
+    sh.k_or = 0u;
+  }
   __syncthreads();
-  const uint32_t M = radix_select_agg(gk, n_groups, (uint32_t)want, c.hist2, sh);
+  uint32_t k_and = 0xFFFFFFFFu, k_or = 0u;
+  for (int g0 = 0; g0 < n_groups; g0 += 4 * blockDim.x) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int g = g0 + u * blockDim.x + threadIdx.x;
+      v[u] = g < n_groups ? gmax[g] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int g = g0 + u * blockDim.x + threadIdx.x;
+      if (g < n_groups) {
+        const uint32_t k = fkey(v[u]);
+        gk[g] = k;
+        if (k != kEmptyGroup) {  // a group with no scored slot never qualifies
+          k_and &= k;
+          k_or |= k;
+        }
+      }
+    }
+  }
+  k_and = __reduce_and_sync(0xffffffffu, k_and);
+  k_or = __reduce_or_sync(0xffffffffu, k_or);
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) c.hist[i] = 0;
+  if ((threadIdx.x & 31) == 0) {
+    atomicAnd(&sh.k_and, k_and);
+    atomicOr(&sh.k_or, k_or);
+  }
+  __syncthreads();
+  const uint32_t diff = sh.k_and ^ sh.k_or;
+  uint32_t M = sh.k_and;  // every scored group's key is equal (or none is scored)
+  if (sh.k_or == 0u) M = kEmptyGroup;
+  if (diff) {
+    const int hb = 31 - __clz(diff);                 // highest bit where keys differ
+    const int shift = hb >= 12 ? hb - 12 : 0;        // 13-bit window [shift, shift + 12]
+    for (int g0 = 0; g0 < n_groups; g0 += blockDim.x) {  // warp-uniform trip count
+      const int g = g0 + threadIdx.x;
+      const bool act = g < n_groups && gk[g] != kEmptyGroup;
+      hist_add(c.hist, act ? (gk[g] >> shift) & (kBins - 1) : 0u, act);
+    }
+    __syncthreads();
+    int cnt = 0;
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) cnt += c.hist[i];
+    int n_scored_groups;
+    block_exclusive_scan(cnt, sh.scan, &n_scored_groups);
+    if (n_scored_groups >= want) {
+      block_find_bin_desc(c.hist, kBins, (uint32_t)want, sh);
+      const uint32_t high = shift + 13 >= 32 ? 0u : (sh.k_and & ~((1u << (shift + 13)) - 1u));
+      M = high | (sh.digit[0] << shift);
+    } else {
+      M = sh.k_and;  // fewer scored groups than wanted: every scored group qualifies
+    }
+  }
   // compact the qualifying group ids to the front, in place (a round reads
   // before it writes, and writes only reach indices already read)
   if (threadIdx.x == 0) sh.n_eq = 0;
@@ -469,7 +499,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     if (total <= kCandCap) {
       n_cand = collect_ge(c, 0u, sh);  // everything fits
     } else {
-      if (a.gmax) n_cand = collect_from_groups(c, a.gmax + ((int64_t)q * L.R + r) * a.gstride, want, sh);
+      if (a.gmax && c.nwords > want)
+        n_cand = collect_from_groups(c, a.gmax + ((int64_t)q * L.R + r) * a.gstride, want, sh);
       if (n_cand < want || n_cand > kCandCap) n_cand = collect_ge(c, sample_threshold(c, want, total, sh), sh);
     }
     if (n_cand >= want && n_cand <= kCandCap) {
