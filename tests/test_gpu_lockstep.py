@@ -182,3 +182,18 @@ def test_device_argument_errors_set_error_word():
         isa.spin_decode_step(h.st, 0, 2, 0, cache.keys, cache.kscale, cache.block_table, qstep, wstep, ctx,
                              False, h.mask, topk, None)     # rows > max_rows: SPIN_EINVAL
     assert isa.spin_get_error(h.st)[0] == 0
+
+
+def test_scores_jumping_between_steps():
+    """Head weights scaled by 4 and then by 1/16 between steps move every
+    score (and so the top-k threshold and the EMA state) far from the last
+    step's values; every step still matches the oracle bit for bit."""
+    wl = workloads.config(2, requests=3, ctx0=(200_000, 150_000, 90_011), steps=8)
+    h = Harness(wl)
+    bootstrap(h, sample_blocks=48)
+    _, wall = h.queries[0]
+    for factor in (1.0, 1.0, 4.0, 4.0, 0.25, 1.0, 1.0):
+        pos = h.committed - np.array(wl.ctx0, np.int64)    # each request's next query position
+        for qi in range(wl.requests):
+            wall[qi, int(pos[qi])] *= factor               # head weights scale every score
+        h.run_step(0, check=range(wl.requests), sample_blocks=48)
