@@ -102,8 +102,8 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
         bool touched = false;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const int64_t sr = s + r;
-          if (r < acc && mask[sr / L.b] != 0) {
+          const int64_t sr = s + r;  // in block j, or past its end in block j + 1
+          if (r < acc && ((sr / L.b == j) ? kj : kj1)) {
             dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
             touched = true;
           }
@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         if (r >= m && r < acc) {
-          const int64_t sr = r - m;
-          if (mask[sr / L.b] != 0) {
+          const int64_t sr = r - m;  // in block 0 (r < R <= 4 < b)
+          if (kj) {
             dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
             touched = true;
           }

@@ -51,8 +51,10 @@ constexpr int kPage = 64;          // tokens per page (block size)
 constexpr int kRowBytes = 128;     // d = 128 FP8 values
 constexpr int kPageBytes = kPage * kRowBytes;
 constexpr int kStageBytes = kTileM * kRowBytes;
-constexpr int kEpiGroups = 2;                 // epilogue groups of 4 warps, alternate tiles
-constexpr int kThreads = 64 + kEpiGroups * 128;
+// Epilogue groups of 4 warps take tiles round robin: 2 groups with two CTAs
+// per SM (N <= 128), 4 groups with one CTA per SM (the MTP rows' N = 256, whose
+// epilogue reduces four rows of heads per token).
+__host__ __device__ constexpr int threads_for(int groups) { return 64 + groups * 128; }
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -198,7 +200,7 @@ struct SmemLayout {
   uint32_t keys;     // stages * kStageBytes
   uint32_t aux;      // kAuxSlots * sizeof(TileInfo)
   uint32_t qbuf;     // 2 * N * 128
-  uint32_t wq;       // 4 * kEpiGroups * N floats: one copy per epilogue warp
+  uint32_t wq;       // 4 * groups * N floats: one copy per epilogue warp
   uint32_t prefix;   // (Q + 1) ints
   uint32_t bars;     // barriers
   uint32_t total;
@@ -208,7 +210,7 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxAcc = 4;
 constexpr int kAuxSlots = 16;  // tile-info ring: freed by the epilogue, not by the MMA
 
-__host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages, int nq) {
+__host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages, int nq, int groups) {
   SmemLayout s;
   uint32_t off = 0;
   s.keys = off;
@@ -219,7 +221,7 @@ __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages, int 
   s.qbuf = off;
   off += nq * N * kRowBytes;
   s.wq = off;
-  off += 4 * kEpiGroups * N * 4;
+  off += 4 * groups * N * 4;
   s.prefix = off;
   off += ((Q + 1) * 4 + 15) / 16 * 16;
   s.bars = off;
@@ -233,6 +235,7 @@ __host__ __device__ inline SmemLayout smem_layout(int N, int Q, int stages, int 
 // accumulators sized so that CTAs * accumulators * N <= 512 TMEM columns.
 struct TcPlan {
   int stages, nacc, ctas, nq;  // key stages, TMEM accumulators, CTAs per SM, query buffers
+  int groups;                  // epilogue groups of four warps
 };
 
 __host__ __device__ inline TcPlan tc_plan(int N, int Q) {
@@ -242,8 +245,8 @@ __host__ __device__ inline TcPlan tc_plan(int N, int Q) {
   constexpr uint32_t kTwoPerSm = 115712;
   if (N <= 128)
     for (int st = kMaxStages; st >= 3; --st)
-      if (smem_layout(N, Q, st, 1).total <= kTwoPerSm) return {st, N <= 64 ? 4 : 2, 2, 1};
-  return {kMaxStages, 2, 1, 2};
+      if (smem_layout(N, Q, st, 1, 2).total <= kTwoPerSm) return {st, N <= 64 ? 4 : 2, 2, 1, 2};
+  return {kMaxStages, 2, 1, 2, 4};
 }
 
 struct Bars {
@@ -302,15 +305,18 @@ __device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
   return r;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int G>
+__global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
+  constexpr int kThreads = threads_for(G);
+  constexpr int kEpiGroups = G;
   const Layout L = a.lay;
   const int N = a.rows * L.H;
   const int stages = plan.stages, nacc = plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const SmemLayout lay = smem_layout(N, L.Q, stages, plan.nq);
+  const SmemLayout lay = smem_layout(N, L.Q, stages, plan.nq, G);
   const int nq = plan.nq;
   const uint32_t sbase = smem_u32(smem);
   TileInfo* aux = reinterpret_cast<TileInfo*>(smem + lay.aux);
@@ -641,7 +647,7 @@ bool tc_supported(const Layout& lay, int rows, int key_fp8) {
   if (!(key_fp8 && lay.d == 128 && lay.b == kPage && lay.H % 16 == 0 && N >= 16 && N <= 256 && N % 16 == 0))
     return false;
   const TcPlan plan = tc_plan(N, lay.Q);
-  return smem_layout(N, lay.Q, plan.stages, plan.nq).total <= 227 * 1024;
+  return smem_layout(N, lay.Q, plan.stages, plan.nq, plan.groups).total <= 227 * 1024;
 }
 
 cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s) {
@@ -654,13 +660,14 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   if (!encode_2d(fn, &tk, a.keys, (uint64_t)a.num_pages * kPage, kPage)) return cudaErrorInvalidValue;
   if (!encode_2d(fn, &tq, a.q8, (uint64_t)L.Q * N, (uint32_t)N)) return cudaErrorInvalidValue;
   const TcPlan plan = tc_plan(N, L.Q);
-  const uint32_t smem = smem_layout(N, L.Q, plan.stages, plan.nq).total;
-  cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const uint32_t smem = smem_layout(N, L.Q, plan.stages, plan.nq, plan.groups).total;
+  auto kernel = plan.groups == 2 ? k_score_tc<2> : k_score_tc<4>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  k_score_tc<<<sms * plan.ctas, kThreads, smem, s>>>(a, plan, tk, tq);
+  kernel<<<sms * plan.ctas, threads_for(plan.groups), smem, s>>>(a, plan, tk, tq);
   return cudaGetLastError();
 }
 

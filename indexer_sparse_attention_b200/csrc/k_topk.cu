@@ -39,6 +39,18 @@ constexpr int kFirstShift = 19;
 constexpr int kCandCap = 8192;        // candidates kept on chip
 constexpr uint32_t kEmptyGroup = 0x007FFFFFu;  // key of -inf: a group with no scored slot
 
+// Dynamic shared memory: the slot bitmap, the histogram / candidate area and,
+// when it fits, a copy of the request's kept-block list.
+__host__ __device__ inline size_t topk_bitmap_bytes(const Layout& L) {
+  return (((size_t)(L.slot_stride + 31) / 32) * 4 + 15) / 16 * 16;
+}
+__host__ __device__ constexpr size_t topk_area_bytes() {
+  return (size_t)kBins * 4 > (size_t)kCandCap * 8 + 256 * 4 ? (size_t)kBins * 4 : (size_t)kCandCap * 8 + 256 * 4;
+}
+__host__ __device__ inline bool topk_stages_work(const Layout& L) {
+  return topk_bitmap_bytes(L) + topk_area_bytes() + (size_t)L.blk_stride * 4 <= 220 * 1024;
+}
+
 struct TopkShared {
   uint32_t k_and, k_or;
   uint32_t digit[2];
@@ -362,7 +374,7 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
     for (int g0 = 0; g0 < n_groups; g0 += blockDim.x) {  // warp-uniform trip count
       const int g = g0 + threadIdx.x;
       const bool act = g < n_groups && gk[g] != kEmptyGroup;
-      hist_add(c.hist, act ? (gk[g] >> shift) & (kBins - 1) : 0u, act);
+      if (act) atomicAdd(&c.hist[(gk[g] >> shift) & (kBins - 1)], 1u);  // spread keys: little contention
     }
     __syncthreads();
     int cnt = 0;
@@ -469,16 +481,34 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   c.n_elem = c.nk << c.lb;
   c.nwords = (c.n_elem + 31) / 32;
   c.bits = reinterpret_cast<uint32_t*>(dyn);
-  uint8_t* area = dyn + (((size_t)(L.slot_stride + 31) / 32) * 4 + 15) / 16 * 16;
+  uint8_t* area = dyn + topk_bitmap_bytes(L);
   c.hist = reinterpret_cast<uint32_t*>(area);
   c.ckey = reinterpret_cast<uint32_t*>(area);
   c.cpos = c.ckey + kCandCap;
   c.hist2 = c.cpos + kCandCap;
 
-  // ---- number of scored slots -------------------------------------------
+  // ---- number of scored slots; the kept-block list is staged on chip when
+  // the launch reserved room for it (every later pass reads it) ------------
   {
+    int32_t* staged = topk_stages_work(L) ? reinterpret_cast<int32_t*>(area + topk_area_bytes()) : nullptr;
     int cnt = 0;
-    for (int t = threadIdx.x; t < c.nk; t += blockDim.x) cnt += min(max(c.p - (c.work[t] << c.lb) + 1, 0), L.b);
+    for (int t0 = 0; t0 < c.nk; t0 += 4 * blockDim.x) {  // four loads in flight per thread
+      int w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * blockDim.x + threadIdx.x;
+        w[u] = t < c.nk ? c.work[t] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * blockDim.x + threadIdx.x;
+        if (t < c.nk) {
+          cnt += min(max(c.p - (w[u] << c.lb) + 1, 0), L.b);
+          if (staged) staged[t] = w[u];
+        }
+      }
+    }
+    if (staged) c.work = staged;  // visible to every thread after the scan's barriers
     int tot;
     block_exclusive_scan(cnt, sh.scan, &tot);
     if (threadIdx.x == 0) sh.total = tot;
@@ -652,9 +682,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
 }
 
 size_t topk_smem_bytes(const Layout& L) {
-  const size_t bitmap = ((size_t)(L.slot_stride + 31) / 32) * 4;
-  const size_t area = std::max<size_t>((size_t)kBins * 4, (size_t)kCandCap * 8 + 256 * 4);
-  return (bitmap + 15) / 16 * 16 + area;
+  return topk_bitmap_bytes(L) + topk_area_bytes() + (topk_stages_work(L) ? (size_t)L.blk_stride * 4 : 0);
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
