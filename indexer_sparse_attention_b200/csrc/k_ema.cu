@@ -80,35 +80,46 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
     float* V = a.V + (int64_t)q * L.slot_stride;
     float* D = a.D + (int64_t)q * L.slot_stride;
     const float* sc = a.scores + (int64_t)q * L.R * L.slot_stride;
-    for (int i = lane; i < L.b; i += 32) {
-      const int64_t s = j * L.b + i;
-      // vertical state of slot s, rows in order
-      if (kj) {
-        float v = V[s];
-        bool touched = false;
+    // Two slots per lane per pass (i, i + 32): every load of the pass is
+    // issued before the first store, so the pass costs one memory latency.
+    for (int i0 = lane; i0 < L.b; i0 += 64) {
+      float v[2], dv[2], sv[2][R], sd[2][R];
+      bool do_v[2], do_d[2], use_v[2][R], use_d[2][R];
+      int64_t sl[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = i0 + 32 * h;
+        sl[h] = j * L.b + i;
+        const int64_t s = sl[h];
+        do_v[h] = i < L.b && kj;                         // vertical state of slot s
+        do_d[h] = i < L.b && s <= p0 && (kj || kj1);     // diagonal state delta = p0 - s
+        v[h] = do_v[h] ? V[s] : 0.f;
+        dv[h] = do_d[h] ? D[p0 - s] : 0.f;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          if (r < acc && s <= p0 + r) {
-            v = ema_v(v, sc[(int64_t)r * L.slot_stride + s], a.alpha, a.beta);
-            touched = true;
-          }
+          use_v[h][r] = do_v[h] && r < acc && s <= p0 + r;
+          const int64_t sr = s + r;  // row r's slot for delta: in block j, or past its end in block j + 1
+          use_d[h][r] = do_d[h] && r < acc && ((sr / L.b == j) ? kj : kj1);
+          sv[h][r] = use_v[h][r] ? sc[(int64_t)r * L.slot_stride + s] : 0.f;
+          sd[h][r] = use_d[h][r] ? sc[(int64_t)r * L.slot_stride + sr] : 0.f;
         }
-        if (touched) V[s] = v;
       }
-      // diagonal state delta = p0 - s (row 0's slot s), rows in order
-      if (s <= p0 && (kj || kj1)) {
-        const int64_t dlt = p0 - s;
-        float dv = D[dlt];
-        bool touched = false;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const int64_t sr = s + r;  // in block j, or past its end in block j + 1
-          if (r < acc && ((sr / L.b == j) ? kj : kj1)) {
-            dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
-            touched = true;
+      for (int h = 0; h < 2; ++h) {
+        bool tv = false, td = false;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {  // rows in order
+          if (use_v[h][r]) {
+            v[h] = ema_v(v[h], sv[h][r], a.alpha, a.beta);
+            tv = true;
+          }
+          if (use_d[h][r]) {
+            dv[h] = ema_d(dv[h], sd[h][r], a.alpha, a.beta);
+            td = true;
           }
         }
-        if (touched) D[dlt] = dv;
+        if (tv) V[sl[h]] = v[h];
+        if (td) D[p0 - sl[h]] = dv[h];
       }
     }
     // offsets delta = p0 + m (m >= 1): seen only by rows r >= m at slot r - m

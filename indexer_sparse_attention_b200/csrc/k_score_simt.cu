@@ -1,10 +1,8 @@
 // k_score_simt.cu -- a0 query quantisation and the CUDA-core indexer score.
 //
 // a0: each (row, head) query vector is quantised to E4M3 with a power-of-two
-//     scale 2^e, e = smallest integer with amax <= 448 * 2^e, and the scale is
-//     folded into the head weight (ReLU(c x) = c ReLU(x) for c > 0), so the
-//     FP8 indexer computes the same score.  The pages give no precision; this
-//     is the reading used throughout.
+//     scale folded into the head weight (quantize_vec); the decode step does
+//     this inside its select kernel, the standalone score call here.
 // a3: I_{r,s} = sigma_s * sum_h w'_{r,h} * ReLU(q8_{r,h} . k8_s) over the slots
 //     of kept blocks with s <= p_r (SPIN listing, Abstract; SPIN digest,
 //     arXiv深度剖析: the indexer input is pruned to the kept blocks).  fp32 keys:
@@ -17,58 +15,13 @@
 
 namespace spin {
 
-// 2^k as a float for k in [-126, 127].
-__device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
-
-// Smallest e with amax <= 448 * 2^e from the exponent and mantissa bits:
-// amax = (1 + f) 2^E -> e = E - 8 if 1 + f <= 1.75 else E - 7.
-__device__ __forceinline__ int q_exponent(float amax) {
-  if (!(amax > 0.0f)) return 0;
-  uint32_t u = __float_as_uint(amax);
-  int E = (int)((u >> 23) & 0xFF);
-  uint32_t frac = u & 0x7FFFFFu;
-  if (E == 0) {  // subnormal: normalise the fraction
-    int msb = 31 - __clz(frac);
-    E = msb - 149 + 127;
-    frac = (frac << (23 - msb)) & 0x7FFFFFu;
-  }
-  return (E - 127) - 8 + (frac > 0x600000u ? 1 : 0);
-}
-
-__device__ __forceinline__ float load_q(const void* q, int64_t i, int bf16) {
-  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[i]);
-  return reinterpret_cast<const float*>(q)[i];
-}
-
 // One warp per (request, row, head).
 __global__ void __launch_bounds__(256) k_quantize_q(ScoreArgs a) {
   const Layout L = a.lay;
   const int64_t nvec = (int64_t)L.Q * a.rows * L.H;
-  const int lane = threadIdx.x & 31;
   const int64_t v = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (v >= nvec) return;
-  const int64_t base = v * L.d;
-  float amax = 0.0f;
-  for (int i = lane; i < L.d; i += 32) amax = fmaxf(amax, fabsf(load_q(a.q, base + i, a.q_bf16)));
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const int e = q_exponent(amax);
-  // x * 2^-e, split in two exact steps when 2^-e is not a normal float.
-  const int ne = -e;
-  const int s1 = ne > 127 ? 127 : ne;
-  const int s2 = ne - s1;
-  const float f1 = pow2f(s1), f2 = pow2f(s2);
-  for (int i = 2 * lane; i < L.d; i += 64) {
-    float x0 = load_q(a.q, base + i, a.q_bf16) * f1 * f2;
-    float x1 = (i + 1 < L.d) ? load_q(a.q, base + i + 1, a.q_bf16) * f1 * f2 : 0.0f;
-    __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
-    a.q8[base + i] = (uint8_t)(p & 0xFF);
-    if (i + 1 < L.d) a.q8[base + i + 1] = (uint8_t)(p >> 8);
-  }
-  if (lane == 0) {
-    // w * 2^e rounded once (double holds the exact product).
-    a.wq[v] = __double2float_rn((double)a.w[v] * ldexp(1.0, e));
-  }
+  quantize_vec(a.q, a.w, a.q_bf16, L.d, v, a.q8, a.wq);
 }
 
 cudaError_t launch_quantize_q(const ScoreArgs& a, cudaStream_t s) {

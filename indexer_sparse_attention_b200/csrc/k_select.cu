@@ -244,6 +244,13 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
   uint2* list = reinterpret_cast<uint2*>(dyn + 5 * L.blk_stride);  // kExpCap (key, block) pairs
   __shared__ SelShared sh;
 
+  if (a.q8) {
+    // a0 for this request's (row, head) vectors, one warp each; the score
+    // kernel reads them after this kernel
+    const int nv = a.rows * L.H, warp = threadIdx.x >> 5;
+    for (int i = warp; i < nv; i += kSelThreads / 32)
+      quantize_vec(a.q, a.w, a.q_bf16, L.d, (int64_t)q * nv + i, a.q8, a.wq);
+  }
   const int64_t ctx = a.ctx_len[q];
   uint8_t* mask_row = a.mask + (int64_t)q * L.max_blocks;
   if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {

@@ -144,6 +144,11 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   a.V = st->V + per_layer * layer;
   a.D = st->D + per_layer * layer;
   a.err = st->err;
+  a.q = nullptr;
+  a.w = nullptr;
+  a.q_bf16 = st->cfg.q_dtype == SPIN_BF16;
+  a.q8 = nullptr;
+  a.wq = nullptr;
   return a;
 }
 
@@ -185,7 +190,7 @@ cudaError_t staged(spin_state st, int stage, cudaStream_t s, F launch) {
 spin_status run_score(spin_state st, int layer, int rows, const void* keys, const float* key_scale,
                       int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
                       const float* w, const int32_t* ctx_len, const uint8_t* mask, float* scores,
-                      bool fuse_ema, cudaStream_t stream, bool* wrote_gmax = nullptr) {
+                      bool fuse_ema, cudaStream_t stream, bool* wrote_gmax = nullptr, bool quantized = false) {
   ScoreArgs a;
   a.lay = st->lay;
   a.rows = rows;
@@ -215,7 +220,7 @@ spin_status run_score(spin_state st, int layer, int rows, const void* keys, cons
   a.gmax = nullptr;
   a.gstride = st->gstride;
   if (wrote_gmax) *wrote_gmax = false;
-  if (a.key_fp8) {
+  if (a.key_fp8 && !quantized) {
     spin_status s = cuda_status(staged(st, kQuant, stream, [&] { return launch_quantize_q(a, stream); }));
     if (s != SPIN_OK) return s;
   }
@@ -466,6 +471,13 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   float* scores = scores_dev ? scores_dev : st->scores;
   cudaStream_t s = (cudaStream_t)stream;
   StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
+  const bool fp8 = st->cfg.key_dtype == SPIN_FP8_E4M3;
+  if (fp8) {  // a0 runs inside the select kernel
+    a.q = q;
+    a.w = w;
+    a.q8 = st->q8;
+    a.wq = st->wq;
+  }
   spin_status r;
   if (a.sparsity > 0.0f) {
     r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
@@ -476,7 +488,7 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   const bool fuse = !defer_update && rows == 1;
   bool gm = false;
   r = run_score(st, layer, rows, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len_dev, mask_dev,
-                scores, fuse, s, &gm);
+                scores, fuse, s, &gm, fp8);
   if (r != SPIN_OK) return r;
   TopkArgs t{st->lay, rows, scores, mask_dev, ctx_len_dev, st->work, st->kept, topk_dev, st->err,
              gm ? st->gmax : nullptr, st->gstride};

@@ -120,6 +120,62 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
 }
 
 // ---------------------------------------------------------------------------
+// a0: query quantisation of one (request, row, head) vector by one warp.  The
+// vector is scaled by 2^-e, e = smallest integer with amax <= 448 * 2^e, and
+// rounded to E4M3 (nearest, saturating); the head weight absorbs 2^e, since
+// ReLU(c x) = c ReLU(x) for c > 0.  The pages give no precision; this is the
+// reading used throughout.
+// ---------------------------------------------------------------------------
+// 2^k as a float for k in [-126, 127].
+__device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+
+// Smallest e with amax <= 448 * 2^e from the exponent and mantissa bits:
+// amax = (1 + f) 2^E -> e = E - 8 if 1 + f <= 1.75 else E - 7.
+__device__ __forceinline__ int q_exponent(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  uint32_t u = __float_as_uint(amax);
+  int E = (int)((u >> 23) & 0xFF);
+  uint32_t frac = u & 0x7FFFFFu;
+  if (E == 0) {  // subnormal: normalise the fraction
+    int msb = 31 - __clz(frac);
+    E = msb - 149 + 127;
+    frac = (frac << (23 - msb)) & 0x7FFFFFu;
+  }
+  return (E - 127) - 8 + (frac > 0x600000u ? 1 : 0);
+}
+
+__device__ __forceinline__ float load_q(const void* q, int64_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[i]);
+  return reinterpret_cast<const float*>(q)[i];
+}
+
+// Vector v (elements v*d .. v*d + d - 1 of q, weight w[v]) -> q8, wq[v].
+// Called by all 32 lanes of a warp.
+__device__ __forceinline__ void quantize_vec(const void* q, const float* w, int q_bf16, int d, int64_t v,
+                                             uint8_t* q8, float* wq) {
+  const int lane = threadIdx.x & 31;
+  const int64_t base = v * d;
+  float amax = 0.0f;
+  for (int i = lane; i < d; i += 32) amax = fmaxf(amax, fabsf(load_q(q, base + i, q_bf16)));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int e = q_exponent(amax);
+  // x * 2^-e, split in two exact steps when 2^-e is not a normal float.
+  const int ne = -e;
+  const int s1 = ne > 127 ? 127 : ne;
+  const int s2 = ne - s1;
+  const float f1 = pow2f(s1), f2 = pow2f(s2);
+  for (int i = 2 * lane; i < d; i += 64) {
+    float x0 = load_q(q, base + i, q_bf16) * f1 * f2;
+    float x1 = (i + 1 < d) ? load_q(q, base + i + 1, q_bf16) * f1 * f2 : 0.0f;
+    __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+    q8[base + i] = (uint8_t)(p & 0xFF);
+    if (i + 1 < d) q8[base + i + 1] = (uint8_t)(p >> 8);
+  }
+  if (lane == 0) wq[v] = __double2float_rn((double)w[v] * ldexp(1.0, e));  // w * 2^e rounded once
+}
+
+// ---------------------------------------------------------------------------
 // Kernel launchers (one per .cu file).  All return cudaGetLastError().
 // ---------------------------------------------------------------------------
 struct StepArgs {
@@ -136,6 +192,12 @@ struct StepArgs {
   float* V;           // layer base [Q][slot_stride]
   float* D;
   ErrWord* err;
+  // a0 folded into the select kernel (decode step with FP8 keys), or q8 null
+  const void* q;      // [Q][rows][H][d]
+  const float* w;     // [Q][rows][H]
+  int q_bf16;
+  uint8_t* q8;
+  float* wq;
 };
 
 cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s);
