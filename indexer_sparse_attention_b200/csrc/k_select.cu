@@ -28,8 +28,17 @@ __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
   const int lpb = L.b >> 3;  // lanes per block
   const int64_t chunks = (L.slot_stride + 255) / 256;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wid < (int64_t)L.Q * chunks;
-       wid += nwarps) {
+  // a0 rides along when asked: the first nvec warp tasks quantise the
+  // (request, row, head) query vectors; this kernel is bound by HBM, so they
+  // cost next to nothing and the select kernel that follows is spared them
+  const int64_t nvec = a.q8 ? (int64_t)L.Q * R * L.H : 0;
+  for (int64_t wid0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wid0 < nvec + (int64_t)L.Q * chunks; wid0 += nwarps) {
+    if (wid0 < nvec) {
+      quantize_vec(a.q, a.w, a.q_bf16, L.d, wid0, a.q8, a.wq);
+      continue;
+    }
+    const int64_t wid = wid0 - nvec;
     const int q = (int)(wid / chunks);
     const int64_t c = wid % chunks;
     const int64_t ctx = a.ctx_len[q];
@@ -80,7 +89,7 @@ __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
 
 cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   const int64_t chunks = (a.lay.slot_stride + 255) / 256;
-  const int64_t warps = (int64_t)a.lay.Q * chunks;
+  const int64_t warps = (int64_t)a.lay.Q * chunks + (a.q8 ? (int64_t)a.lay.Q * a.rows * a.lay.H : 0);
   int64_t blocks = (warps + 7) / 8;
   if (blocks > 148 * 32) blocks = 148 * 32;
   switch (a.rows) {
@@ -165,13 +174,15 @@ __device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t
 // Exploration draw by a short list: the Philox keys are uniform, so the
 // `take` smallest of n_cand lie below t = (1.25 take + 64) / n_cand * 2^32
 // with overwhelming probability.  Candidates under t are appended to a
-// shared list (one atomic per warp), the list is sorted by (key, block
-// index), and its first `take` blocks are explored.  Returns false -- nothing marked -- when the list holds fewer
+// shared list (one atomic per warp), each entry is ranked by (key, block
+// index) -- by counting for short lists, by a bitonic sort for long ones --
+// and the first `take` blocks are explored.  Returns false -- nothing marked -- when the list holds fewer
 // than `take` entries or overflows, and the caller runs the radix select.
 constexpr int kExpCap = 2048;
+constexpr int kRankMax = 512;  // longest list ranked by counting
 
 __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last, int take, int n_cand,
-                                uint2* list, SelShared& sh) {
+                                uint2* list, int* rank, SelShared& sh) {
   const double frac = (1.25 * take + 64.0) / (double)n_cand;
   const uint64_t t = frac >= 1.0 ? (1ull << 32) : (uint64_t)(frac * 4294967296.0);
   if (threadIdx.x == 0) sh.digit[0] = 0;
@@ -195,7 +206,32 @@ __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last
   __syncthreads();
   const int cnt = (int)sh.digit[0];
   if (cnt < take || cnt > kExpCap) return false;  // uniform: every thread reads the same count
-  // bitonic sort of the list by (key, block), padded to a power of two with
+  if (cnt <= kRankMax) {
+    // exact rank of every entry by (key, block): `parts` threads per entry
+    // each count a slice of the list; the `take` lowest ranks are drawn
+    // (cnt^2 comparisons: cheaper than a sort's barriers for short lists)
+    int parts = 1;
+    while (parts * 2 * cnt <= (int)blockDim.x) parts *= 2;
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) rank[i] = 0;
+    __syncthreads();
+    const int i = (int)threadIdx.x / parts, part = (int)threadIdx.x % parts;
+    if (i < cnt) {
+      const uint2 me = list[i];
+      const int k0 = (int)((int64_t)cnt * part / parts), k1 = (int)((int64_t)cnt * (part + 1) / parts);
+      int below = 0;
+      for (int k = k0; k < k1; ++k) {
+        const uint2 o = list[k];
+        below += (o.x < me.x) || (o.x == me.x && o.y < me.y);
+      }
+      if (below) atomicAdd(&rank[i], below);
+    }
+    __syncthreads();
+    for (int i2 = threadIdx.x; i2 < cnt; i2 += blockDim.x)
+      if (rank[i2] < take) m[list[i2].y] = 2;
+    __syncthreads();
+    return true;
+  }
+  // longer lists: bitonic sort by (key, block), padded to a power of two with
   // entries that sort last; the first `take` entries are the draw
   int n2 = 1;
   while (n2 < cnt) n2 <<= 1;
@@ -310,7 +346,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
       for (int j = threadIdx.x; j < n_last; j += blockDim.x)
         if (m[j] == 0) m[j] = 2;
       __syncthreads();
-    } else if (take > 0 && explore_by_list(a, q, m, n_last, (int)take, n_cand, list, sh)) {
+    } else if (take > 0 && explore_by_list(a, q, m, n_last, (int)take, n_cand, list,
+                                           reinterpret_cast<int*>(keys), sh)) {  // block keys are spent
       // done: the `take` smallest keys came from the short list
     } else if (take > 0) {
       for (int j = threadIdx.x; j < n_last; j += blockDim.x)

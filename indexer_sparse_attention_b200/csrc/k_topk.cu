@@ -426,27 +426,33 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
         }
       }
     }
+    // every take of this pass in one 32-bit mask per lane (4 bits per step),
+    // then one warp scan and one shared atomic for the whole pass
+    uint32_t takes = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      uint32_t takes = 0;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << k;
-      const int n_my = __popc(takes);
-      if (!__any_sync(0xffffffffu, n_my != 0)) continue;
-      int incl = n_my;
+        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << (4 * u + k);
+    }
+    const int n_my = __popc(takes);
+    if (!__any_sync(0xffffffffu, n_my != 0)) continue;
+    int incl = n_my;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      int at = 0;
-      if (lane == 31) at = atomicAdd(&sh.n_cand, incl);
-      at = __shfl_sync(0xffffffffu, at, 31) + incl - n_my;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int at = 0;
+    if (lane == 31) at = atomicAdd(&sh.n_cand, incl);
+    at = __shfl_sync(0xffffffffu, at, 31) + incl - n_my;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        if (takes & (1u << k)) {
+        if (takes & (1u << (4 * u + k))) {
           if (at < kCandCap) {
             c.ckey[at] = fkey(vals[k]);
             c.cpos[at] = (uint32_t)(e0[u] + k);
@@ -659,7 +665,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     }
   }
   int tot;
-  const int eq_base = block_exclusive_scan(n_eq, sh.scan, &tot);
+  const int eq_base = exact_bits ? 0 : block_exclusive_scan(n_eq, sh.scan, &tot);  // exact: no ties left
   const int take = max(0, min(n_eq, (int)eq_take - eq_base));
   int pos = block_exclusive_scan(n_gt + take, sh.scan, &tot);
   int eq_rank = eq_base;

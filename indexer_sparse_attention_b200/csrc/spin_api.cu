@@ -472,7 +472,7 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   cudaStream_t s = (cudaStream_t)stream;
   StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
   const bool fp8 = st->cfg.key_dtype == SPIN_FP8_E4M3;
-  if (fp8) {  // a0 runs inside the select kernel
+  if (fp8) {  // a0 rides in the predict kernel, or in select when there is no prediction
     a.q = q;
     a.w = w;
     a.q8 = st->q8;
@@ -482,6 +482,7 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   if (a.sparsity > 0.0f) {
     r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
     if (r != SPIN_OK) return r;
+    a.q8 = nullptr;  // done
   }
   r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
   if (r != SPIN_OK) return r;
