@@ -26,6 +26,8 @@
 // and -- if even those do not fit -- three more full radix passes, after
 // which ties are resolved by re-reading the scores.  Every path gives the
 // same result; the sample only decides the speed.
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "spin_internal.cuh"
@@ -52,7 +54,7 @@ __host__ __device__ inline bool topk_stages_work(const Layout& L) {
 }
 
 struct TopkShared {
-  uint32_t k_and, k_or;
+  uint32_t k_and, k_or, M;
   uint32_t digit[2];
   int scan[33];
   int total;
@@ -466,15 +468,183 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
   return sh.n_cand;
 }
 
+// The group path spread over a cluster of CTAs (few requests, many idle SMs):
+// rank c takes the c-th share of the groups, the ranks' key bits and
+// histograms meet in rank 0 through distributed shared memory, rank 0 finds
+// M and sends it back, and every rank gathers its share's candidates
+// straight into rank 0's list.  Returns the candidate count in rank 0 and -2
+// in the other ranks, which are done.
+__device__ __forceinline__ int collect_from_groups_cluster(const TopkCtx& c, const float* gmax, int want, TopkShared& sh) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
+  const int n_groups = (c.n_elem + 31) / 32;
+  const int gs0 = (int)((int64_t)n_groups * cr / C), gs1 = (int)((int64_t)n_groups * (cr + 1) / C);
+  const int n_my = gs1 - gs0;
+  uint32_t* gk = c.bits;  // this share's group keys, then its qualifying group ids
+  TopkShared* sh0 = cl.map_shared_rank(&sh, 0);
+  if (threadIdx.x == 0) {
+    sh.k_and = 0xFFFFFFFFu;
+    sh.k_or = 0u;
+    sh.n_cand = 0;
+    sh.n_eq = 0;
+  }
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) c.hist[i] = 0;
+  cl.sync();
+  uint32_t k_and = 0xFFFFFFFFu, k_or = 0u;
+  for (int g0 = 0; g0 < n_my; g0 += 4 * blockDim.x) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int g = g0 + u * blockDim.x + threadIdx.x;
+      v[u] = g < n_my ? gmax[gs0 + g] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int g = g0 + u * blockDim.x + threadIdx.x;
+      if (g < n_my) {
+        const uint32_t k = fkey(v[u]);
+        gk[g] = k;
+        if (k != kEmptyGroup) {
+          k_and &= k;
+          k_or |= k;
+        }
+      }
+    }
+  }
+  k_and = __reduce_and_sync(0xffffffffu, k_and);
+  k_or = __reduce_or_sync(0xffffffffu, k_or);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAnd(&sh0->k_and, k_and);
+    atomicOr(&sh0->k_or, k_or);
+  }
+  cl.sync();
+  const uint32_t all_and = sh0->k_and, all_or = sh0->k_or;
+  const uint32_t diff = all_and ^ all_or;
+  const int hb = diff ? 31 - __clz(diff) : 0;
+  const int shift = hb >= 12 ? hb - 12 : 0;
+  if (diff) {
+    for (int g0 = 0; g0 < n_my; g0 += blockDim.x) {
+      const int g = g0 + threadIdx.x;
+      if (g < n_my && gk[g] != kEmptyGroup) atomicAdd(&c.hist[(gk[g] >> shift) & (kBins - 1)], 1u);
+    }
+  }
+  cl.sync();
+  if (cr == 0) {
+    uint32_t M = all_or == 0u ? kEmptyGroup : all_and;
+    if (diff) {
+      // the cluster's histogram, bin by bin, into rank 0's
+      int cnt = 0;
+      for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
+        uint32_t t = c.hist[i];
+        for (int k = 1; k < C; ++k) t += cl.map_shared_rank(c.hist, k)[i];
+        c.hist[i] = t;
+        cnt += (int)t;
+      }
+      int n_scored_groups;
+      block_exclusive_scan(cnt, sh.scan, &n_scored_groups);
+      if (n_scored_groups >= want) {
+        block_find_bin_desc(c.hist, kBins, (uint32_t)want, sh);
+        const uint32_t high = shift + 13 >= 32 ? 0u : (all_and & ~((1u << (shift + 13)) - 1u));
+        M = high | (sh.digit[0] << shift);
+      } else {
+        M = all_and;  // fewer scored groups than wanted: every scored group qualifies
+      }
+    }
+    if ((int)threadIdx.x < C) cl.map_shared_rank(&sh, (int)threadIdx.x)->M = M;
+  }
+  cl.sync();
+  const uint32_t M = sh.M;
+  // this share's qualifying groups to the front of gk, in place (a round
+  // reads before it writes, and writes only reach indices already read)
+  for (int base = 0; base < n_my; base += blockDim.x) {
+    const int g = base + threadIdx.x;
+    const bool take = g < n_my && gk[g] >= M;
+    __syncthreads();
+    if (take) gk[atomicAdd(&sh.n_eq, 1)] = (uint32_t)(gs0 + g);
+    __syncthreads();
+  }
+  const int n_q = sh.n_eq;
+  uint32_t* ckey0 = cl.map_shared_rank(c.ckey, 0);
+  uint32_t* cpos0 = cl.map_shared_rank(c.cpos, 0);
+  // gather: a warp takes 32 groups at a time, 8 lanes x float4 per group
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int base = warp * 32; base < n_q; base += nw * 32) {
+    int e0[8];
+    float4 v[8];
+    int s0[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int gi = base + u * 4 + (lane >> 3);
+      e0[u] = gi < n_q ? (int)gk[gi] * 32 + (lane & 7) * 4 : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      s0[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0[u] >= 0 && e0[u] < c.n_elem) {
+        const int s = (c.work[e0[u] >> c.lb] << c.lb) + (e0[u] & c.bmask);
+        if (s <= c.p) {
+          s0[u] = s;
+          v[u] = *reinterpret_cast<const float4*>(c.sc + s);
+        }
+      }
+    }
+    uint32_t takes = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << (4 * u + k);
+    }
+    const int n_t = __popc(takes);
+    if (!__any_sync(0xffffffffu, n_t != 0)) continue;
+    int incl = n_t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int at = 0;
+    if (lane == 31) at = atomicAdd(&sh0->n_cand, incl);
+    at = __shfl_sync(0xffffffffu, at, 31) + incl - n_t;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (takes & (1u << (4 * u + k))) {
+          if (at < kCandCap) {
+            ckey0[at] = fkey(vals[k]);
+            cpos0[at] = (uint32_t)(e0[u] + k);
+          }
+          ++at;
+        }
+      }
+    }
+  }
+  cl.sync();  // every rank's candidates are in rank 0 before it goes on
+  return cr == 0 ? sh.n_cand : -2;
+}
+
+// kCluster: launched with a cluster of C CTAs per (request, row), which share
+// the group path; otherwise one CTA per pair.
+template <bool kCluster>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   const Layout L = a.lay;
-  const int q = blockIdx.x / a.rows, r = blockIdx.x % a.rows;
+  namespace cg = cooperative_groups;
+  const int C = kCluster ? (int)cg::this_cluster().num_blocks() : 1;
+  const int cr = kCluster ? (int)cg::this_cluster().block_rank() : 0;
+  const unsigned rid = blockIdx.x / (unsigned)C;
+  const int q = rid / a.rows, r = rid % a.rows;
   int32_t* out = a.topk + ((int64_t)q * a.rows + r) * L.k;
   __shared__ TopkShared sh;
   extern __shared__ __align__(16) uint8_t dyn[];
   const int64_t ctx = a.ctx_len[q];
   if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {
-    for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
+    if (cr == 0)
+      for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
   }
   TopkCtx c;
@@ -522,6 +692,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   }
   const int total = sh.total;
   const int want = min(total, L.k);
+  // every rank computed the same count; only the group path uses the cluster
+  if (kCluster && cr != 0 && !(total > kCandCap && a.gmax && c.nwords > want)) return;
   if (want == 0) {
     for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
@@ -535,8 +707,15 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     if (total <= kCandCap) {
       n_cand = collect_ge(c, 0u, sh);  // everything fits
     } else {
-      if (a.gmax && c.nwords > want)
-        n_cand = collect_from_groups(c, a.gmax + ((int64_t)q * L.R + r) * a.gstride, want, sh);
+      if (a.gmax && c.nwords > want) {
+        const float* gm = a.gmax + ((int64_t)q * L.R + r) * a.gstride;
+        if constexpr (kCluster) {
+          n_cand = collect_from_groups_cluster(c, gm, want, sh);
+          if (n_cand == -2) return;  // a helper rank of the cluster: its part is done
+        } else {
+          n_cand = collect_from_groups(c, gm, want, sh);
+        }
+      }
       if (n_cand < want || n_cand > kCandCap) n_cand = collect_ge(c, sample_threshold(c, want, total, sh), sh);
     }
     if (n_cand >= want && n_cand <= kCandCap) {
@@ -693,9 +872,38 @@ size_t topk_smem_bytes(const Layout& L) {
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const size_t smem = topk_smem_bytes(a.lay);
-  cudaError_t e = cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_topk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_topk<<<a.lay.Q * a.rows, kTopkThreads, smem, s>>>(a);
+  // Few (request, row) pairs leave most SMs idle: give each a cluster of up to
+  // 8 CTAs for the group path.  A cluster shape the device cannot place falls
+  // back to one CTA per pair.
+  const int pairs = a.lay.Q * a.rows;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int C = 1;
+  if (a.gmax)
+    while (C < 8 && pairs * C * 2 <= sms) C *= 2;
+  if (C > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(pairs * C));
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, k_topk<true>, &cfg);
+    if (e == cudaSuccess && clusters >= 1) return cudaLaunchKernelEx(&cfg, k_topk<true>, a);
+    cudaGetLastError();  // this shape cannot be placed: one CTA per pair
+  }
+  k_topk<false><<<pairs, kTopkThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -68,10 +68,14 @@ def test_predict_select_bit_exact(R, s, g):
             assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
 
 
-def test_select_large_request_with_infinite_and_tied_scores():
-    # one 1M-slot request: 16,385 blocks, many equal block scores
+@pytest.mark.parametrize("g", [0.1, 0.3])
+def test_select_large_request_with_infinite_and_tied_scores(g):
+    # one 1M-slot request: 16,385 blocks, many equal block scores.  The
+    # exploration draw of ~820 blocks (g = 0.1) goes through the sorted short
+    # list, ~2,460 (g = 0.3) overflow it and take the radix select; the
+    # 300K-slot request's draw is ranked by counting.
     rng = np.random.default_rng(1)
-    st = make_state(Q=2, max_slots=1024 * 1024 + 64, R=1, s=0.5, g=0.1, k=2048)
+    st = make_state(Q=2, max_slots=1024 * 1024 + 64, R=1, s=0.5, g=g, k=2048)
     V, D = st.ema(0)
     v = rng.integers(0, 3, V.shape).astype(np.float32)
     v[:, -5000:] = np.inf
@@ -84,7 +88,7 @@ def test_select_large_request_with_infinite_and_tied_scores():
     assert isa.spin_get_error(st)[0] == 0
     for q in range(2):
         S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), 1, 64, st.mask_stride)
-        m_ref = oracle.select(S_ref, int(ctx[q]), 1, 64, 0.5, 0.1, 7, q, 0, 11)
+        m_ref = oracle.select(S_ref, int(ctx[q]), 1, 64, 0.5, g, 7, q, 0, 11)
         assert np.array_equal(mask[q].cpu().numpy(), m_ref)
 
 
