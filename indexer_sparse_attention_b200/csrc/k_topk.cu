@@ -628,6 +628,84 @@ __device__ __forceinline__ int collect_from_groups_cluster(const TopkCtx& c, con
   return cr == 0 ? sh.n_cand : -2;
 }
 
+// The sampled-threshold path spread over a cluster (contexts with fewer
+// 32-slot groups than k): rank 0 takes the threshold from its sample and
+// sends it to every rank; each rank then collects its share of the kept
+// slots (whole blocks) straight into rank 0's candidate list.  Returns the
+// candidate count in rank 0 and -2 in the other ranks, which are done.
+__device__ __forceinline__ int collect_sampled_cluster(const TopkCtx& c, int want, int total, TopkShared& sh) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
+  if (cr == 0) {
+    const uint32_t t_lo = sample_threshold(c, want, total, sh);
+    if (threadIdx.x == 0) sh.n_cand = 0;
+    if ((int)threadIdx.x < C) cl.map_shared_rank(&sh, (int)threadIdx.x)->M = t_lo;
+  }
+  cl.sync();
+  const uint32_t t_lo = sh.M;
+  TopkShared* sh0 = cl.map_shared_rank(&sh, 0);
+  uint32_t* ckey0 = cl.map_shared_rank(c.ckey, 0);
+  uint32_t* cpos0 = cl.map_shared_rank(c.cpos, 0);
+  const int b0 = (int)((int64_t)c.nk * cr / C), b1 = (int)((int64_t)c.nk * (cr + 1) / C);
+  const int E0 = b0 << c.lb, E1 = b1 << c.lb;  // this rank's kept-slot positions
+  const int lane = threadIdx.x & 31;
+  const int step = blockDim.x * 4;
+  for (int it = E0; it < E1; it += 4 * step) {
+    float4 v[4];
+    int s0[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = it + threadIdx.x * 4 + u * step;
+      s0[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E1) {
+        const int s = (c.work[e >> c.lb] << c.lb) + (e & c.bmask);
+        if (s <= c.p) {
+          s0[u] = s;
+          v[u] = *reinterpret_cast<const float4*>(c.sc + s);
+        }
+      }
+    }
+    uint32_t takes = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= t_lo) takes |= 1u << (4 * u + k);
+    }
+    const int n_t = __popc(takes);
+    if (!__any_sync(0xffffffffu, n_t != 0)) continue;
+    int incl = n_t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int at = 0;
+    if (lane == 31) at = atomicAdd(&sh0->n_cand, incl);
+    at = __shfl_sync(0xffffffffu, at, 31) + incl - n_t;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      const int e0 = it + threadIdx.x * 4 + u * step;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (takes & (1u << (4 * u + k))) {
+          if (at < kCandCap) {
+            ckey0[at] = fkey(vals[k]);
+            cpos0[at] = (uint32_t)(e0 + k);
+          }
+          ++at;
+        }
+      }
+    }
+  }
+  cl.sync();  // every rank's candidates are in rank 0 before it goes on
+  return cr == 0 ? sh.n_cand : -2;
+}
+
 // kCluster: launched with a cluster of C CTAs per (request, row), which share
 // the group path; otherwise one CTA per pair.
 template <bool kCluster>
@@ -692,8 +770,9 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   }
   const int total = sh.total;
   const int want = min(total, L.k);
-  // every rank computed the same count; only the group path uses the cluster
-  if (kCluster && cr != 0 && !(total > kCandCap && a.gmax && c.nwords > want)) return;
+  // every rank computed the same count; the cluster shares the candidate
+  // search when not everything fits on chip
+  if (kCluster && cr != 0 && total <= kCandCap) return;
   if (want == 0) {
     for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
@@ -714,6 +793,12 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
           if (n_cand == -2) return;  // a helper rank of the cluster: its part is done
         } else {
           n_cand = collect_from_groups(c, gm, want, sh);
+        }
+      }
+      if constexpr (kCluster) {
+        if (!(a.gmax && c.nwords > want)) {  // every rank takes this branch alike
+          n_cand = collect_sampled_cluster(c, want, total, sh);
+          if (n_cand == -2) return;
         }
       }
       if (n_cand < want || n_cand > kCandCap) n_cand = collect_ge(c, sample_threshold(c, want, total, sh), sh);
@@ -876,15 +961,14 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Few (request, row) pairs leave most SMs idle: give each a cluster of up to
-  // 8 CTAs for the group path.  A cluster shape the device cannot place falls
+  // 8 CTAs for the candidate search.  A cluster shape the device cannot place falls
   // back to one CTA per pair.
   const int pairs = a.lay.Q * a.rows;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int C = 1;
-  if (a.gmax)
-    while (C < 8 && pairs * C * 2 <= sms) C *= 2;
+  while (C < 8 && pairs * C * 2 <= sms) C *= 2;
   if (C > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(pairs * C));
