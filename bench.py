@@ -285,35 +285,69 @@ def fidelity(run, n_steps=3):
 
 
 def e2e_pass(run, steps, world):
-    """The same decode step through the public API with host inputs: per step
-    the query, head weights and context lengths are copied in from pinned
-    host memory and the top-k indices and block mask are read back."""
+    """The same decode step through the public API with host buffers, run the
+    way a server overlaps transfers: while step i computes, a copy stream
+    brings step i+1's query, head weights and context lengths in from pinned
+    host memory and reads step i-1's top-k indices and block mask back (two
+    device buffers of each alternate).  Every step's copies lie inside the
+    timed region, which ends when the last read-back has landed."""
     wl = run.wl
     t0 = run.t
     q_h = [run.q[t0 + i].cpu().pin_memory() for i in range(steps)]
     w_h = [run.w[t0 + i].cpu().pin_memory() for i in range(steps)]
     c_h = [run.ctx[t0 + i].cpu().pin_memory() for i in range(steps)]
-    q_d, w_d, c_d = torch.empty_like(run.q[0]), torch.empty_like(run.w[0]), torch.empty_like(run.ctx[0])
-    topk_h = torch.empty(run.topk.shape, dtype=torch.int32).pin_memory()
-    mask_h = torch.empty(run.mask.shape, dtype=torch.uint8).pin_memory()
+    q_d = [torch.empty_like(run.q[0]) for _ in range(2)]
+    w_d = [torch.empty_like(run.w[0]) for _ in range(2)]
+    c_d = [torch.empty_like(run.ctx[0]) for _ in range(2)]
+    topk_d = [torch.empty_like(run.topk) for _ in range(2)]
+    mask_d = [torch.empty_like(run.mask) for _ in range(2)]
+    topk_h = [torch.empty(run.topk.shape, dtype=torch.int32).pin_memory() for _ in range(2)]
+    mask_h = [torch.empty(run.mask.shape, dtype=torch.uint8).pin_memory() for _ in range(2)]
     h2d = q_h[0].numel() * q_h[0].element_size() + w_h[0].numel() * 4 + c_h[0].numel() * 4
-    d2h = topk_h.numel() * 4 + mask_h.numel()
+    d2h = topk_h[0].numel() * 4 + mask_h[0].numel()
+    compute = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready, done, out_read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     barrier(world)
     torch.cuda.synchronize()
-    s = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
+    e0.record(compute)
+    copy.wait_stream(compute)
+
+    def bring_in(i, b):
+        with torch.cuda.stream(copy):
+            q_d[b].copy_(q_h[i], non_blocking=True)
+            w_d[b].copy_(w_h[i], non_blocking=True)
+            c_d[b].copy_(c_h[i], non_blocking=True)
+            in_ready[b].record(copy)
+
+    bring_in(0, 0)
     for i in range(steps):
-        q_d.copy_(q_h[i], non_blocking=True)
-        w_d.copy_(w_h[i], non_blocking=True)
-        c_d.copy_(c_h[i], non_blocking=True)
-        run.step(q=q_d, w=w_d, ctx=c_d)
-        topk_h.copy_(run.topk, non_blocking=True)
-        mask_h.copy_(run.mask, non_blocking=True)
-    e1.record(s)
+        b = i % 2
+        if i + 1 < steps:
+            if i >= 1:
+                copy.wait_event(done[1 - b])   # step i-1 no longer reads buffer 1-b
+            bring_in(i + 1, 1 - b)
+        compute.wait_event(in_ready[b])
+        if i >= 2:
+            compute.wait_event(out_read[b])    # step i-2's results are out of buffer b
+        run.step(q=q_d[b], w=w_d[b], ctx=c_d[b], mask=mask_d[b], topk=topk_d[b])
+        done[b].record(compute)
+        copy.wait_event(done[b])
+        with torch.cuda.stream(copy):
+            topk_h[b].copy_(topk_d[b], non_blocking=True)
+            mask_h[b].copy_(mask_d[b], non_blocking=True)
+            out_read[b].record(copy)
+    compute.wait_stream(copy)
+    e1.record(compute)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # the last step's results as read back equal the device copy
+    if not (torch.equal(topk_h[(steps - 1) % 2], topk_d[(steps - 1) % 2].cpu())
+            and torch.equal(mask_h[(steps - 1) % 2], mask_d[(steps - 1) % 2].cpu())):
+        raise RuntimeError("end-to-end read-back does not match the device results")
     return ms, h2d, d2h
 
 
