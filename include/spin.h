@@ -233,6 +233,10 @@ SPIN_API spin_status spin_allocate_layer_sparsity(int num_layers, const double* 
  * call into ms_out[n] / launches_out[n] (either may be NULL; n <= 8) and
  * resets both.  Launches are counted whether or not timing is enabled. */
 SPIN_API spin_status spin_set_kernel_timing(spin_state st, int enable);
+/* Times only the stages in stage_mask (bit n = stage n, as listed above);
+ * the other launches get no events, so they keep running back to back.
+ * 0 turns timing off.  SPIN_EINVAL for bits past the last stage. */
+SPIN_API spin_status spin_set_kernel_timing_mask(spin_state st, uint32_t stage_mask);
 SPIN_API spin_status spin_kernel_times(spin_state st, double* ms_out, int64_t* launches_out, int n);
 
 /* Test hook for the device error path.  mode 1: on its next launch, CTA 0

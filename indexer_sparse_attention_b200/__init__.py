@@ -23,7 +23,7 @@ __all__ = [
     "spin_decode_step", "spin_miss_count", "spin_allocate_layer_sparsity", "spin_get_error",
     "spin_set_layer_sparsity", "spin_set_score_kernel", "spin_reset_requests", "spin_set_fault_injection",
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
-    "spin_kernel_times", "STAGES", "spin_topk_noalloc",
+    "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_set_kernel_timing_mask",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +80,7 @@ def load():
         "spin_set_score_kernel": (S, [_vp, ctypes.c_int]),
         "spin_set_fault_injection": (S, [_vp, ctypes.c_int]),
         "spin_set_kernel_timing": (S, [_vp, ctypes.c_int]),
+        "spin_set_kernel_timing_mask": (S, [_vp, _u32]),
         "spin_kernel_times": (S, [_vp, _vp, _vp, ctypes.c_int]),
         "spin_reset_requests": (S, [_vp, ctypes.c_int, _vp, ctypes.c_int, _vp]),
         "spin_predict_select": (S, [_vp, ctypes.c_int, ctypes.c_int, _i64, _vp, _vp, _vp]),
@@ -236,6 +237,16 @@ STAGES = ["predict", "select", "quantize", "score", "topk", "ema", "compact", "m
 
 def spin_set_kernel_timing(st: SpinState, enable: bool) -> None:
     _check(load().spin_set_kernel_timing(st.handle, int(bool(enable))), "spin_set_kernel_timing")
+
+
+def spin_set_kernel_timing_mask(st: SpinState, stages) -> None:
+    """Time only the named stages (see STAGES); the others run without events."""
+    mask = 0
+    for name in stages:
+        if name not in STAGES:
+            raise ValueError(f"unknown stage {name!r}; stages are {STAGES}")
+        mask |= 1 << STAGES.index(name)
+    _check(load().spin_set_kernel_timing_mask(st.handle, mask), "spin_set_kernel_timing_mask")
 
 
 def spin_kernel_times(st: SpinState):

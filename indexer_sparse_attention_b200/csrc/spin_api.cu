@@ -33,7 +33,7 @@ struct spin_state_s {
   int inject;
   void* encode_fn;  // cuTensorMapEncodeTiled, resolved at create
   // per-stage timing (spin_set_kernel_timing / spin_kernel_times)
-  bool timing;
+  uint32_t timing;  // stages whose launches are bracketed by events (bit n = stage n)
   struct Rec { int stage; cudaEvent_t a, b; };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
@@ -176,7 +176,7 @@ cudaEvent_t take_event(spin_state st) {
 template <class F>
 cudaError_t staged(spin_state st, int stage, cudaStream_t s, F launch) {
   st->launches[stage] += 1;
-  if (!st->timing) return launch();
+  if (!((st->timing >> stage) & 1u)) return launch();
   cudaEvent_t a = take_event(st), b = take_event(st);
   if (!a || !b) return cudaErrorMemoryAllocation;
   cudaEventRecord(a, s);
@@ -278,7 +278,7 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
   st->inject = 0;
-  st->timing = false;
+  st->timing = 0;
   for (int i = 0; i < 8; ++i) st->launches[i] = 0;
   st->encode_fn = nullptr;
   cudaDriverEntryPointQueryResult qres;
@@ -332,7 +332,14 @@ spin_status spin_set_score_kernel(spin_state st, int kind) {
 
 spin_status spin_set_kernel_timing(spin_state st, int enable) {
   if (!alive(st)) return SPIN_ESTATE;
-  st->timing = enable != 0;
+  st->timing = enable != 0 ? 0xFFu : 0u;
+  return SPIN_OK;
+}
+
+spin_status spin_set_kernel_timing_mask(spin_state st, uint32_t stage_mask) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (stage_mask >> kNumStages) return SPIN_EINVAL;
+  st->timing = stage_mask;
   return SPIN_OK;
 }
 

@@ -285,3 +285,28 @@ def test_topk_fallback_paths_bit_exact(pattern):
     for qq in range(Q):
         ref = oracle.topk_row(vals[qq, 0].astype(np.float64), m[qq], int(ctx[qq]), 0, 64, k)
         assert np.array_equal(got[qq, 0], ref), (pattern, qq)
+
+
+def test_kernel_timing_mask_times_only_named_stages():
+    """spin_set_kernel_timing_mask brackets only the named stages with events;
+    every launch is still counted."""
+    wl = workloads.config(1, requests=2, ctx0=(9000, 20000), steps=2, spare_slots=8)
+    cache = workloads.make_key_cache(wl, 0, "cuda")
+    q, w = workloads.make_queries(wl, 0, 1, "cuda")
+    st = make_state(Q=2, max_slots=wl.max_slots, k=wl.topk, s=0.4)
+    ctx = torch.tensor([9001, 20001], dtype=torch.int32, device="cuda")
+    mask = st.new_mask()
+    topk = torch.empty((2, 1, wl.topk), dtype=torch.int32, device="cuda")
+    isa.spin_kernel_times(st)
+    isa.spin_set_kernel_timing_mask(st, ["score"])
+    for step in range(2):
+        isa.spin_decode_step(st, 0, 1, step, cache.keys, cache.kscale, cache.block_table, q[:, :1].contiguous(),
+                             w[:, :1].contiguous(), ctx, False, mask, topk)
+    isa.spin_set_kernel_timing(st, False)
+    times = isa.spin_kernel_times(st)
+    assert times["score"][1] == 2 and times["score"][0] > 0
+    for stage in ("predict", "select", "topk"):
+        assert times[stage][1] == 2 and times[stage][0] == 0
+    assert isa.spin_get_error(st)[0] == 0
+    with pytest.raises(ValueError):
+        isa.spin_set_kernel_timing_mask(st, ["no such stage"])
