@@ -197,3 +197,27 @@ def test_scores_jumping_between_steps():
         for qi in range(wl.requests):
             wall[qi, int(pos[qi])] *= factor               # head weights scale every score
         h.run_step(0, check=range(wl.requests), sample_blocks=48)
+
+
+@pytest.mark.parametrize("b", [16, 32, 128, 256])
+def test_block_sizes_other_than_64(b):
+    """Paged blocks of 16..256 slots (the CUDA-core indexer takes them; the
+    tensor-core tile is built for 64): predict, select, score, top-k and EMA
+    in lock step."""
+    wl = workloads.config(1, b=b, steps=4, ctx0=(12_000 + 37,), sparsity=0.5)
+    h = Harness(wl)
+    bootstrap(h)
+    for _ in range(wl.steps - 1):
+        h.run_step(0, check=[0], sample_blocks=max(8, 3072 // b))
+
+
+def test_maximum_context():
+    """One request at the largest context a state accepts (the top-k keeps a
+    1.31M-slot bitmap on chip): 20,480 blocks, sampled lock-step checks."""
+    limit = 160 * 1024 * 8                                  # slots the on-chip top-k bitmap holds
+    wl = workloads.config(2, requests=1, ctx0=(limit - 8,), steps=3, spare_slots=0)
+    assert wl.max_slots <= limit
+    h = Harness(wl)
+    bootstrap(h, sample_blocks=32)
+    for _ in range(wl.steps - 1):
+        h.run_step(0, check=[0], sample_blocks=32)
