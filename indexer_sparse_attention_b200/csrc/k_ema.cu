@@ -53,6 +53,7 @@ cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t s
 
 template <int R>
 __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
+  pdl_enter();
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -147,13 +148,13 @@ cudaError_t launch_ema_update(const EmaArgs& a, cudaStream_t s) {
   int64_t warps = (int64_t)a.lay.Q * a.lay.max_blocks;
   int64_t blocks = (warps + 7) / 8;
   if (blocks > 148 * 64) blocks = 148 * 64;
+  PdlLaunch l(dim3((unsigned)blocks), dim3(256), 0, s);
   switch (a.rows) {
-    case 1: k_ema_update<1><<<(int)blocks, 256, 0, s>>>(a); break;
-    case 2: k_ema_update<2><<<(int)blocks, 256, 0, s>>>(a); break;
-    case 3: k_ema_update<3><<<(int)blocks, 256, 0, s>>>(a); break;
-    default: k_ema_update<4><<<(int)blocks, 256, 0, s>>>(a); break;
+    case 1: return cudaLaunchKernelEx(&l.cfg, k_ema_update<1>, a);
+    case 2: return cudaLaunchKernelEx(&l.cfg, k_ema_update<2>, a);
+    case 3: return cudaLaunchKernelEx(&l.cfg, k_ema_update<3>, a);
+    default: return cudaLaunchKernelEx(&l.cfg, k_ema_update<4>, a);
   }
-  return cudaGetLastError();
 }
 
 // Miss counter of the fidelity metric: per (request, row), the entries of a

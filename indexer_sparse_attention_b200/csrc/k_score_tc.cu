@@ -309,6 +309,7 @@ template <int G>
 __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
+  pdl_enter();
   constexpr int kThreads = threads_for(G);
   constexpr int kEpiGroups = G;
   const Layout L = a.lay;
@@ -667,8 +668,8 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  kernel<<<sms * plan.ctas, threads_for(plan.groups), smem, s>>>(a, plan, tk, tq);
-  return cudaGetLastError();
+  PdlLaunch l(dim3(sms * plan.ctas), dim3(threads_for(plan.groups)), smem, s);
+  return cudaLaunchKernelEx(&l.cfg, kernel, a, plan, tk, tq);
 }
 
 }  // namespace spin

@@ -22,6 +22,7 @@ namespace spin {
 // ---------------------------------------------------------------------------
 template <int R>
 __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
+  pdl_enter();
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
   const int lb = __ffs(L.b) - 1;
@@ -92,13 +93,13 @@ cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   const int64_t warps = (int64_t)a.lay.Q * chunks + (a.q8 ? (int64_t)a.lay.Q * a.rows * a.lay.H : 0);
   int64_t blocks = (warps + 7) / 8;
   if (blocks > 148 * 32) blocks = 148 * 32;
+  PdlLaunch l(dim3((unsigned)blocks), dim3(256), 0, s);
   switch (a.rows) {
-    case 1: k_predict_pool<1><<<(int)blocks, 256, 0, s>>>(a); break;
-    case 2: k_predict_pool<2><<<(int)blocks, 256, 0, s>>>(a); break;
-    case 3: k_predict_pool<3><<<(int)blocks, 256, 0, s>>>(a); break;
-    default: k_predict_pool<4><<<(int)blocks, 256, 0, s>>>(a); break;
+    case 1: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<1>, a);
+    case 2: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<2>, a);
+    case 3: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<3>, a);
+    default: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<4>, a);
   }
-  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -272,6 +273,7 @@ __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t
 }
 
 __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
+  pdl_enter();
   const Layout L = a.lay;
   const int q = blockIdx.x;
   extern __shared__ __align__(16) uint8_t dyn[];
@@ -385,8 +387,8 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)a.lay.blk_stride * 5 + (size_t)kExpCap * sizeof(uint2);
   cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_select<<<a.lay.Q, kSelThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  PdlLaunch l(dim3(a.lay.Q), dim3(kSelThreads), smem, s);
+  return cudaLaunchKernelEx(&l.cfg, k_select, a);
 }
 
 // ---------------------------------------------------------------------------

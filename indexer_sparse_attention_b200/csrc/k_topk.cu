@@ -710,6 +710,7 @@ __device__ __forceinline__ int collect_sampled_cluster(const TopkCtx& c, int wan
 // the group path; otherwise one CTA per pair.
 template <bool kCluster>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
+  pdl_enter();
   const Layout L = a.lay;
   namespace cg = cooperative_groups;
   const int C = kCluster ? (int)cg::this_cluster().num_blocks() : 1;
@@ -975,20 +976,22 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     cfg.blockDim = dim3(kTopkThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     int clusters = 0;
     e = cudaOccupancyMaxActiveClusters(&clusters, k_topk<true>, &cfg);
     if (e == cudaSuccess && clusters >= 1) return cudaLaunchKernelEx(&cfg, k_topk<true>, a);
     cudaGetLastError();  // this shape cannot be placed: one CTA per pair
   }
-  k_topk<false><<<pairs, kTopkThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  PdlLaunch l(dim3(pairs), dim3(kTopkThreads), smem, s);
+  return cudaLaunchKernelEx(&l.cfg, k_topk<false>, a);
 }
 
 }  // namespace spin

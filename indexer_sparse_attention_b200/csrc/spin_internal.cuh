@@ -176,6 +176,37 @@ __device__ __forceinline__ void quantize_vec(const void* q, const float* w, int 
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  The decode step's kernels are launched so
+// that each may be scheduled while its predecessor in the stream finishes,
+// which hides the launch gap.  Each of them starts by waiting until every
+// earlier grid has completed and its memory is visible (a no-op for an
+// ordinary launch), and only then lets its own successor be scheduled, so
+// the stream's ordering is kept for every byte either kernel touches.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch configuration with programmatic stream serialization; use in place.
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t s) : cfg(), attr() {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  PdlLaunch(const PdlLaunch&) = delete;
+  PdlLaunch& operator=(const PdlLaunch&) = delete;
+};
+
+// ---------------------------------------------------------------------------
 // Kernel launchers (one per .cu file).  All return cudaGetLastError().
 // ---------------------------------------------------------------------------
 struct StepArgs {
