@@ -439,7 +439,9 @@ def gpu_arm(args, world, rank, local):
     # ---- end to end with host buffers --------------------------------------
     e2e_ms, h2d, d2h = e2e_pass(run, K, world)
     out["e2e"] = {"value": job_rows_per_s(Q * K, world, e2e_ms), "unit": "rows/s", "h2d_bytes_per_step": h2d,
-                  "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
+                  "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
+                  "transfers": "pinned host buffers; step i+1's inputs in and step i-1's results out on a copy "
+                               "stream while step i computes (double-buffered), all inside the timed region"}
     status, word = isa.spin_get_error(run.st)
     if status != 0:
         raise RuntimeError(f"device error word {word:#x}")
