@@ -9,6 +9,8 @@
 //     of it goes to uniformly random unkept blocks (SPIN digest, arXiv深度剖析;
 //     SPIN listing, Figure 4); each row's top (B_r - n_exp) blocks are unioned
 //     (SPIN listing, Table 7, "Row-local union").  Ties: lower block index.
+#include <cooperative_groups.h>
+
 #include "spin_internal.cuh"
 #include "block_scan.cuh"
 
@@ -172,6 +174,66 @@ __device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t
   __syncthreads();
 }
 
+constexpr int kExpCap = 2048;
+constexpr int kRankMax = 512;  // longest list ranked by counting
+
+// The `take` entries of list[0 .. cnt) first by (key, block index) go to
+// mark(block): ranked by counting for up to kRankMax entries, by a bitonic
+// sort for longer lists.  `rank` holds cnt ints of scratch.  All threads of
+// the CTA call it.
+template <class Mark>
+__device__ void draw_from_list(uint2* list, int cnt, int take, int* rank, Mark mark) {
+  if (cnt <= kRankMax) {
+    // exact rank of every entry: `parts` threads per entry each count a
+    // slice of the list (cnt^2 comparisons: cheaper than a sort's barriers
+    // for short lists)
+    int parts = 1;
+    while (parts * 2 * cnt <= (int)blockDim.x) parts *= 2;
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) rank[i] = 0;
+    __syncthreads();
+    const int i = (int)threadIdx.x / parts, part = (int)threadIdx.x % parts;
+    if (i < cnt) {
+      const uint2 me = list[i];
+      const int k0 = (int)((int64_t)cnt * part / parts), k1 = (int)((int64_t)cnt * (part + 1) / parts);
+      int below = 0;
+      for (int k = k0; k < k1; ++k) {
+        const uint2 o = list[k];
+        below += (o.x < me.x) || (o.x == me.x && o.y < me.y);
+      }
+      if (below) atomicAdd(&rank[i], below);
+    }
+    __syncthreads();
+    for (int i2 = threadIdx.x; i2 < cnt; i2 += blockDim.x)
+      if (rank[i2] < take) mark((int)list[i2].y);
+    __syncthreads();
+    return;
+  }
+  // longer lists: bitonic sort by (key, block), padded to a power of two with
+  // entries that sort last; the first `take` entries are the draw
+  int n2 = 1;
+  while (n2 < cnt) n2 <<= 1;
+  for (int i = cnt + (int)threadIdx.x; i < n2; i += blockDim.x) list[i] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const uint2 x = list[i], y = list[ixj];
+          const bool gt = x.x > y.x || (x.x == y.x && x.y > y.y);
+          if (gt == ((i & k) == 0)) {
+            list[i] = y;
+            list[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < take; i += blockDim.x) mark((int)list[i].y);
+  __syncthreads();
+}
+
 // Exploration draw by a short list: the Philox keys are uniform, so the
 // `take` smallest of n_cand lie below t = (1.25 take + 64) / n_cand * 2^32
 // with overwhelming probability.  Candidates under t are appended to a
@@ -179,8 +241,6 @@ __device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t
 // index) -- by counting for short lists, by a bitonic sort for long ones --
 // and the first `take` blocks are explored.  Returns false -- nothing marked -- when the list holds fewer
 // than `take` entries or overflows, and the caller runs the radix select.
-constexpr int kExpCap = 2048;
-constexpr int kRankMax = 512;  // longest list ranked by counting
 
 __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last, int take, int n_cand,
                                 uint2* list, int* rank, SelShared& sh) {
@@ -207,55 +267,7 @@ __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last
   __syncthreads();
   const int cnt = (int)sh.digit[0];
   if (cnt < take || cnt > kExpCap) return false;  // uniform: every thread reads the same count
-  if (cnt <= kRankMax) {
-    // exact rank of every entry by (key, block): `parts` threads per entry
-    // each count a slice of the list; the `take` lowest ranks are drawn
-    // (cnt^2 comparisons: cheaper than a sort's barriers for short lists)
-    int parts = 1;
-    while (parts * 2 * cnt <= (int)blockDim.x) parts *= 2;
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) rank[i] = 0;
-    __syncthreads();
-    const int i = (int)threadIdx.x / parts, part = (int)threadIdx.x % parts;
-    if (i < cnt) {
-      const uint2 me = list[i];
-      const int k0 = (int)((int64_t)cnt * part / parts), k1 = (int)((int64_t)cnt * (part + 1) / parts);
-      int below = 0;
-      for (int k = k0; k < k1; ++k) {
-        const uint2 o = list[k];
-        below += (o.x < me.x) || (o.x == me.x && o.y < me.y);
-      }
-      if (below) atomicAdd(&rank[i], below);
-    }
-    __syncthreads();
-    for (int i2 = threadIdx.x; i2 < cnt; i2 += blockDim.x)
-      if (rank[i2] < take) m[list[i2].y] = 2;
-    __syncthreads();
-    return true;
-  }
-  // longer lists: bitonic sort by (key, block), padded to a power of two with
-  // entries that sort last; the first `take` entries are the draw
-  int n2 = 1;
-  while (n2 < cnt) n2 <<= 1;
-  for (int i = cnt + (int)threadIdx.x; i < n2; i += blockDim.x) list[i] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-  __syncthreads();
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const uint2 x = list[i], y = list[ixj];
-          const bool gt = x.x > y.x || (x.x == y.x && x.y > y.y);
-          if (gt == ((i & k) == 0)) {
-            list[i] = y;
-            list[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int i = threadIdx.x; i < take; i += blockDim.x) m[list[i].y] = 2;
-  __syncthreads();
+  draw_from_list(list, cnt, take, rank, [m](int j) { m[j] = 2; });
   return true;
 }
 
@@ -383,10 +395,302 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
   compact_row(m, n_last, a.work + (int64_t)q * L.blk_stride, a.kept + q, sh.scan);
 }
 
+// ---------------------------------------------------------------------------
+// a2 spread over a cluster of C CTAs per request (few requests, many idle
+// SMs).  Rank c owns the contiguous block range [j0_c, j1_c) of the request:
+// its block keys, its part of the mask and of the kept list.  The radix
+// passes merge the ranks' 256-bin histograms through distributed shared
+// memory (every rank finds the same digit); keys equal to the threshold are
+// taken in block order across ranks through a prefix of the ranks' counts;
+// the exploration list gathers in rank 0, which marks the drawn blocks in
+// their owners' masks.  Results equal the one-CTA kernel's.
+// ---------------------------------------------------------------------------
+struct SelCluster {
+  uint32_t hist[2][256];  // this rank's histogram, double-buffered by pass
+  int cnt[4];             // per-phase counts read by the other ranks
+  uint32_t list_n;        // rank 0: entries of the exploration list
+};
+
+__device__ __forceinline__ int range_lo(int n, int c, int C) { return (int)((int64_t)n * c / C); }
+
+// Radix select over the cluster's keys: this rank's keys[0 .. hi) (block
+// j0 + i) with valid(i); want in [1, #valid cluster-wide].  Every rank
+// returns the same T and eq.
+template <class Valid>
+__device__ void cl_radix_select_desc(const uint32_t* keys, int hi, Valid valid, uint32_t want, SelShared& sh,
+                                     SelCluster& sc, uint32_t* T_out, uint32_t* eq_out) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks();
+  uint32_t prefix = 0, pmask = 0, remaining = want;
+  int pass = 0;
+  for (int shift = 24; shift >= 0; shift -= 8, ++pass) {
+    uint32_t* h = sc.hist[pass & 1];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < hi; i += blockDim.x) {
+      if (!valid(i)) continue;
+      const uint32_t k = keys[i];
+      if ((k & pmask) == prefix) atomicAdd(&h[(k >> shift) & 255u], 1u);
+    }
+    cl.sync();  // every rank's histogram of this pass is complete
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+      uint32_t t = 0;
+      for (int r = 0; r < C; ++r) t += cl.map_shared_rank(h, r)[b];
+      sh.hist[b] = t;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) warp_find_digit_desc<256>(sh.hist, remaining, sh.digit);
+    __syncthreads();
+    prefix |= sh.digit[0] << shift;
+    pmask |= 255u << shift;
+    remaining = sh.digit[1];
+    __syncthreads();
+  }
+  *T_out = prefix;
+  *eq_out = remaining;
+}
+
+// Sum of `v` over the ranks below this one, and over all ranks, through
+// counter slot `slot` (each slot is used once per kernel).
+__device__ __forceinline__ int cl_rank_prefix(int v, int slot, SelCluster& sc, int* total) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
+  if (threadIdx.x == 0) sc.cnt[slot] = v;
+  cl.sync();
+  int below = 0, all = 0;
+  for (int r = 0; r < C; ++r) {
+    const int x = cl.map_shared_rank(sc.cnt, r)[slot];
+    all += x;
+    if (r < cr) below += x;
+  }
+  *total = all;
+  return below;
+}
+
+// Marks m[i] = label for this rank's share of the cluster's top `want`:
+// keys > T, then keys == T in block order across ranks (eq_take of them).
+template <class Valid>
+__device__ void cl_mark_selected(const uint32_t* keys, int hi, Valid valid, uint32_t T, uint32_t eq_take,
+                                 uint8_t* m, uint8_t label, SelShared& sh, SelCluster& sc, int slot) {
+  const int chunk = (hi + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * chunk, up = min(hi, lo + chunk);
+  int eq = 0;
+  for (int i = lo; i < up; ++i)
+    if (valid(i) && keys[i] == T) ++eq;
+  int local_total, all;
+  int base = block_exclusive_scan(eq, sh.scan, &local_total);
+  base += cl_rank_prefix(local_total, slot, sc, &all);
+  for (int i = lo; i < up; ++i) {
+    if (!valid(i)) continue;
+    const uint32_t k = keys[i];
+    if (k > T) {
+      m[i] = label;
+    } else if (k == T) {
+      if ((uint32_t)base < eq_take) m[i] = label;
+      ++base;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a) {
+  pdl_enter();
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
+  const Layout L = a.lay;
+  const int q = (int)(blockIdx.x / (unsigned)C);
+  extern __shared__ __align__(16) uint8_t dyn[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);  // this rank's range
+  uint8_t* m = dyn + 4 * L.blk_stride;
+  uint2* list = reinterpret_cast<uint2*>(dyn + 5 * L.blk_stride);  // rank 0: kExpCap entries
+  __shared__ SelShared sh;
+  __shared__ SelCluster sc;
+
+  if (a.q8) {  // a0 on all-keep steps, the request's vectors split over the ranks
+    const int nv = a.rows * L.H, warp = threadIdx.x >> 5;
+    for (int i = cr * (kSelThreads / 32) + warp; i < nv; i += C * (kSelThreads / 32))
+      quantize_vec(a.q, a.w, a.q_bf16, L.d, (int64_t)q * nv + i, a.q8, a.wq);
+  }
+  const int64_t ctx = a.ctx_len[q];
+  uint8_t* mask_row = a.mask + (int64_t)q * L.max_blocks;
+  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {  // alike in every rank
+    if (cr == 0 && threadIdx.x == 0) {
+      raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
+      a.kept[q] = 0;
+    }
+    const int z0 = range_lo((int)L.max_blocks, cr, C), z1 = range_lo((int)L.max_blocks, cr + 1, C);
+    for (int j = z0 + threadIdx.x; j < z1; j += blockDim.x) mask_row[j] = 0;
+    return;
+  }
+  const int n_last = (int)row_blocks(ctx, a.rows - 1, L.b);
+  const int j0 = range_lo(n_last, cr, C), j1 = range_lo(n_last, cr + 1, C);
+  const int nl = j1 - j0;  // this rank's blocks: j = j0 + i
+  for (int i = threadIdx.x; i < nl; i += blockDim.x) m[i] = 0;
+  if (threadIdx.x == 0) sc.list_n = 0;
+  __syncthreads();
+
+  if (a.sparsity == 0.0f) {
+    for (int i = threadIdx.x; i < nl; i += blockDim.x) m[i] = 1;
+    __syncthreads();
+  } else {
+    const int64_t n0 = row_blocks(ctx, 0, L.b);
+    const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
+    auto all = [](int) { return true; };
+    for (int r = 0; r < a.rows; ++r) {
+      const int n = (int)row_blocks(ctx, r, L.b);
+      const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
+      const int hi = max(0, min(j1, n) - j0);  // this rank's blocks visible to row r
+      const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride + j0;
+      for (int i0 = 0; i0 < hi; i0 += 4 * kSelThreads) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * kSelThreads + (int)threadIdx.x;
+          v[u] = i < hi ? S[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * kSelThreads + (int)threadIdx.x;
+          if (i < hi) keys[i] = fkey(v[u]);
+        }
+      }
+      __syncthreads();
+      if (n_pred >= n) {
+        for (int i = threadIdx.x; i < hi; i += blockDim.x) m[i] = 1;
+        __syncthreads();
+      } else if (n_pred > 0) {
+        uint32_t T, eq;
+        cl_radix_select_desc(keys, hi, all, (uint32_t)n_pred, sh, sc, &T, &eq);
+        cl_mark_selected(keys, hi, all, T, eq, m, 1, sh, sc, r);  // slots 0..3: one per row
+      }
+    }
+    // exploration among the unkept blocks of the last row's range
+    int c = 0;
+    for (int i = threadIdx.x; i < nl; i += blockDim.x) c += (m[i] == 0);
+    int local_cand, n_cand;
+    block_exclusive_scan(c, sh.scan, &local_cand);
+    cl.sync();  // every rank's row marks are final before the counts are shared
+    if (threadIdx.x == 0) sc.cnt[0] = local_cand;  // slot 0 is free again: its last reader passed the barrier
+    cl.sync();
+    n_cand = 0;
+    for (int rr = 0; rr < C; ++rr) n_cand += cl.map_shared_rank(sc.cnt, rr)[0];
+    const int64_t take = n_exp < n_cand ? n_exp : n_cand;
+    if (take == n_cand) {
+      for (int i = threadIdx.x; i < nl; i += blockDim.x)
+        if (m[i] == 0) m[i] = 2;
+      __syncthreads();
+    } else if (take > 0) {
+      // candidates under the Philox-key threshold go to rank 0's list
+      const double frac = (1.25 * take + 64.0) / (double)n_cand;
+      const uint64_t t = frac >= 1.0 ? (1ull << 32) : (uint64_t)(frac * 4294967296.0);
+      uint32_t* list_n0 = &cl.map_shared_rank(&sc, 0)->list_n;
+      uint2* list0 = cl.map_shared_rank(list, 0);
+      const int lane = threadIdx.x & 31;
+      for (int i0 = 0; i0 < nl; i0 += blockDim.x) {  // warp-uniform trip count
+        const int i = i0 + (int)threadIdx.x;
+        uint32_t u = 0;
+        bool in = false;
+        if (i < nl && m[i] == 0) {
+          u = explore_key(a.seed, (uint32_t)(j0 + i), (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
+          in = (uint64_t)u < t;
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        if (!bal) continue;
+        uint32_t at = 0;
+        if (lane == 0) at = atomicAdd(list_n0, (uint32_t)__popc(bal));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+        if (in && at < (uint32_t)kExpCap) list0[at] = make_uint2(u, (uint32_t)(j0 + i));
+      }
+      cl.sync();
+      const int cnt = (int)*list_n0;  // alike in every rank
+      if (cnt >= take && cnt <= kExpCap) {
+        if (cr == 0) {
+          // the first `take` entries by (key, block), marked in their owners' masks
+          draw_from_list(list, cnt, (int)take, reinterpret_cast<int*>(keys), [&](int j) {
+            int owner = C - 1;
+            while (owner > 0 && range_lo(n_last, owner, C) > j) --owner;
+            cl.map_shared_rank(m, owner)[j - range_lo(n_last, owner, C)] = 2;
+          });
+        }
+        cl.sync();  // the drawn blocks are marked in every owner's mask
+      } else {
+        // radix select over all candidates' ~keys (largest ~key = smallest key)
+        for (int i = threadIdx.x; i < nl; i += blockDim.x)
+          keys[i] = ~explore_key(a.seed, (uint32_t)(j0 + i), (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
+        __syncthreads();
+        auto cand = [m](int i) { return m[i] == 0; };
+        uint32_t T, eq;
+        cl_radix_select_desc(keys, nl, cand, (uint32_t)take, sh, sc, &T, &eq);
+        // count ties first (cand reads m), then label
+        const int chunk = (nl + blockDim.x - 1) / blockDim.x;
+        const int lo = threadIdx.x * chunk, up = min(nl, lo + chunk);
+        int e = 0;
+        for (int i = lo; i < up; ++i)
+          if (m[i] == 0 && keys[i] == T) ++e;
+        int local_e, all_e;
+        int base = block_exclusive_scan(e, sh.scan, &local_e);
+        base += cl_rank_prefix(local_e, 1, sc, &all_e);  // slot 1: its row-1 use is behind two barriers
+        for (int i = lo; i < up; ++i) {
+          if (m[i] != 0) continue;
+          if (keys[i] > T) {
+            m[i] = 2;
+          } else if (keys[i] == T) {
+            if ((uint32_t)base < eq) m[i] = 2;
+            ++base;
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+  // mask row and the ascending kept list, each rank its own range
+  for (int i = threadIdx.x; i < nl; i += blockDim.x) mask_row[j0 + i] = m[i];
+  if (cr == C - 1)
+    for (int64_t j = n_last + threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = 0;
+  const int chunk = (nl + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * chunk, up = min(nl, lo + chunk);
+  int kc = 0;
+  for (int i = lo; i < up; ++i) kc += m[i] != 0;
+  int local_kept, total_kept;
+  int pos = block_exclusive_scan(kc, sh.scan, &local_kept);
+  cl.sync();  // slot 2 / 3 readers of earlier phases are done
+  pos += cl_rank_prefix(local_kept, 2, sc, &total_kept);
+  int32_t* work = a.work + (int64_t)q * L.blk_stride;
+  for (int i = lo; i < up; ++i)
+    if (m[i]) work[pos++] = j0 + i;
+  if (cr == 0 && threadIdx.x == 0) a.kept[q] = total_kept;
+  cl.sync();  // no rank leaves while another may still read its counters
+}
+
 cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)a.lay.blk_stride * 5 + (size_t)kExpCap * sizeof(uint2);
   cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // Few requests with long contexts leave most SMs idle: a cluster of up to 8
+  // CTAs per request, each keeping >= 2048 blocks (below that the cluster
+  // barriers cost more than the split saves).  A cluster shape the device
+  // cannot place falls back to one CTA each.
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int C = 1;
+  while (C < 8 && a.lay.Q * C * 2 <= sms && a.lay.max_blocks >= (int64_t)C * 2 * 2048) C *= 2;
+  if (C > 1) {
+    PdlLaunch l(dim3(a.lay.Q * C), dim3(kSelThreads), smem, s);
+    l.attr[1].id = cudaLaunchAttributeClusterDimension;
+    l.attr[1].val.clusterDim.x = (unsigned)C;
+    l.attr[1].val.clusterDim.y = 1;
+    l.attr[1].val.clusterDim.z = 1;
+    l.cfg.numAttrs = 2;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, k_select_cluster, &l.cfg);
+    if (e == cudaSuccess && clusters >= 1) return cudaLaunchKernelEx(&l.cfg, k_select_cluster, a);
+    cudaGetLastError();  // this shape cannot be placed
+  }
   PdlLaunch l(dim3(a.lay.Q), dim3(kSelThreads), smem, s);
   return cudaLaunchKernelEx(&l.cfg, k_select, a);
 }

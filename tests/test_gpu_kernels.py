@@ -310,3 +310,30 @@ def test_kernel_timing_mask_times_only_named_stages():
     assert isa.spin_get_error(st)[0] == 0
     with pytest.raises(ValueError):
         isa.spin_set_kernel_timing_mask(st, ["no such stage"])
+
+
+@pytest.mark.parametrize("R", [1, 2, 4])
+@pytest.mark.parametrize("s,g", [(0.5, 0.05), (0.4, 0.3), (0.0, 0.05), (0.3, 0.0), (0.999, 0.5)])
+def test_select_cluster_paths_bit_exact(R, s, g):
+    """Long contexts take the cluster select (8 CTAs per request): the rows'
+    radix selects across ranks, ties in block order across ranks, the
+    exploration draw by list and by radix, all-keep, and empty requests."""
+    rng = np.random.default_rng(int(R * 1000 + s * 100 + g * 10))
+    st = make_state(Q=4, max_slots=1024 * 1024 + 64, R=R, s=s, g=g, k=2048)
+    V, D = st.ema(0)
+    v = rng.integers(0, 4, V.shape).astype(np.float32)    # many equal block scores
+    v[:, -3000:] = np.inf
+    V.copy_(torch.from_numpy(v))
+    d = rng.standard_normal(D.shape).astype(np.float32)
+    d[rng.random(D.shape) < 0.5] = -np.inf
+    D.copy_(torch.from_numpy(d))
+    ctx = np.array([1, 1024 * 1024 - R + 1, 300_000 + 37, 64 * 5000], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    for step in [0, 5]:
+        isa.spin_predict_select(st, 0, R, step, ctx_t, mask)
+        assert isa.spin_get_error(st)[0] == 0
+        for q in range(4):
+            S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, 64, st.mask_stride)
+            m_ref = oracle.select(S_ref, int(ctx[q]), R, 64, s, g, 7, q, 0, step)
+            assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
