@@ -123,6 +123,16 @@ SPIN_API spin_status spin_set_score_kernel(spin_state st, int kind);
 SPIN_API spin_status spin_reset_requests(spin_state st, int layer, const int32_t* req_host, int n,
                                 spin_stream_t stream);
 
+/* Decode step numbers.  Every call that takes `step` accepts either an
+ * explicit step >= 0 or SPIN_STEP_DEVICE, which reads the state's device step
+ * counter when the kernels run.  spin_set_step / spin_advance_step change the
+ * counter in stream order and launch nothing else, so a decode step (all its
+ * layers) followed by spin_advance_step can be captured once in a CUDA graph
+ * and replayed every step with the right exploration draw. */
+#define SPIN_STEP_DEVICE (-1)
+SPIN_API spin_status spin_set_step(spin_state st, int64_t step, spin_stream_t stream);
+SPIN_API spin_status spin_advance_step(spin_state st, spin_stream_t stream);
+
 /* a1 + a2: predicted slot score z = max(V_i, D_{p_r - i}) (AI Radio, "Title
  * and authors"; SPIN digest, arXiv深度剖析), block max-pool S_{r,j}, block
  * budget B_r = n_r - floor(s * n_r), exploration share n_exp = floor(gamma *
@@ -131,7 +141,8 @@ SPIN_API spin_status spin_reset_requests(spin_state st, int layer, const int32_t
  * (SPIN listing, Table 7).  Ties go to the lower block index.
  *   ctx_len_dev [Q] int32, mask_dev [Q][max_blocks] uint8 out:
  *   0 skipped, 1 predicted, 2 explored (blocks past the last row's range: 0).
- *   step: decode step, part of the exploration RNG counter. */
+ *   step: decode step (>= 0, or SPIN_STEP_DEVICE), part of the exploration
+ *   RNG counter. */
 SPIN_API spin_status spin_predict_select(spin_state st, int layer, int rows, int64_t step,
                                 const int32_t* ctx_len_dev, uint8_t* mask_dev,
                                 spin_stream_t stream);

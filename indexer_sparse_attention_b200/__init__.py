@@ -24,6 +24,7 @@ __all__ = [
     "spin_set_layer_sparsity", "spin_set_score_kernel", "spin_reset_requests", "spin_set_fault_injection",
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
     "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_set_kernel_timing_mask",
+    "SPIN_STEP_DEVICE", "spin_set_step", "spin_advance_step",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +32,7 @@ LIB_PATH = os.path.join(_HERE, "libspin.so")
 
 SPIN_F32, SPIN_BF16, SPIN_FP8_E4M3 = 0, 1, 2
 SPIN_SCORE_AUTO, SPIN_SCORE_SIMT, SPIN_SCORE_TCGEN05 = 0, 1, 2
+SPIN_STEP_DEVICE = -1  # step argument: read the state's device step counter
 STATUS_NAMES = {0: "SPIN_OK", 1: "SPIN_EINVAL", 2: "SPIN_ENOMEM", 3: "SPIN_ECUDA", 4: "SPIN_ESTATE",
                 5: "SPIN_ETIMEOUT", 6: "SPIN_EDEVICE", 7: "SPIN_EUNSUPPORTED"}
 
@@ -81,6 +83,8 @@ def load():
         "spin_set_fault_injection": (S, [_vp, ctypes.c_int]),
         "spin_set_kernel_timing": (S, [_vp, ctypes.c_int]),
         "spin_set_kernel_timing_mask": (S, [_vp, _u32]),
+        "spin_set_step": (S, [_vp, _i64, _vp]),
+        "spin_advance_step": (S, [_vp, _vp]),
         "spin_kernel_times": (S, [_vp, _vp, _vp, ctypes.c_int]),
         "spin_reset_requests": (S, [_vp, ctypes.c_int, _vp, ctypes.c_int, _vp]),
         "spin_predict_select": (S, [_vp, ctypes.c_int, ctypes.c_int, _i64, _vp, _vp, _vp]),
@@ -237,6 +241,14 @@ STAGES = ["predict", "select", "quantize", "score", "topk", "ema", "compact", "m
 
 def spin_set_kernel_timing(st: SpinState, enable: bool) -> None:
     _check(load().spin_set_kernel_timing(st.handle, int(bool(enable))), "spin_set_kernel_timing")
+
+
+def spin_set_step(st: SpinState, step: int, stream=None) -> None:
+    _check(load().spin_set_step(st.handle, int(step), _stream(stream)), "spin_set_step")
+
+
+def spin_advance_step(st: SpinState, stream=None) -> None:
+    _check(load().spin_advance_step(st.handle, _stream(stream)), "spin_advance_step")
 
 
 def spin_set_kernel_timing_mask(st: SpinState, stages) -> None:

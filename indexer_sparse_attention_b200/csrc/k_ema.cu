@@ -35,6 +35,13 @@ cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+__global__ void k_step_op(int64_t* p, int set, int64_t value) { *p = set ? value : *p + 1; }
+
+cudaError_t launch_step_op(int64_t* p, bool set, int64_t value, cudaStream_t s) {
+  k_step_op<<<1, 1, 0, s>>>(p, set ? 1 : 0, value);
+  return cudaGetLastError();
+}
+
 __global__ void k_reset_rows(float* V, float* D, ReqList list, int64_t stride) {
   for (int k = blockIdx.y; k < list.n; k += gridDim.y) {
     const int64_t base = (int64_t)list.ids[k] * stride;

@@ -284,8 +284,10 @@ __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t
   if (threadIdx.x == 0) *kept = total;
 }
 
-__global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a) {
+__global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   pdl_enter();
+  StepArgs a = a_in;
+  if (a.step_dev) a.step = *a.step_dev;  // the state's counter (read after the predecessors finished)
   const Layout L = a.lay;
   const int q = blockIdx.x;
   extern __shared__ __align__(16) uint8_t dyn[];
@@ -495,8 +497,10 @@ __device__ void cl_mark_selected(const uint32_t* keys, int hi, Valid valid, uint
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a) {
+__global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
   pdl_enter();
+  StepArgs a = a_in;
+  if (a.step_dev) a.step = *a.step_dev;  // the state's counter (read after the predecessors finished)
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();

@@ -28,6 +28,7 @@ struct spin_state_s {
   float* scores;  // [Q][R][slot_stride]
   float* gmax;    // [Q][R][gstride] group maxima of the last tensor-core score
   int64_t gstride;
+  int64_t* step_dev;  // device step counter (SPIN_STEP_DEVICE)
   std::vector<float> sparsity;
   int score_kernel;
   int inject;
@@ -94,7 +95,7 @@ Layout make_layout(const spin_config* c) {
 int64_t gmax_stride(const Layout& L) { return L.blk_stride * std::max(1, L.b / 32); }
 
 struct Carve {
-  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, total;
+  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, step, total;
 };
 
 Carve carve(const Layout& L) {
@@ -111,6 +112,7 @@ Carve carve(const Layout& L) {
   k.wq = take((size_t)L.Q * L.R * L.H * 4);
   k.scores = take((size_t)L.Q * L.R * L.slot_stride * 4);
   k.gmax = take((size_t)L.Q * L.R * gmax_stride(L) * 4);
+  k.step = take(sizeof(int64_t));
   k.total = off;
   return k;
 }
@@ -130,7 +132,8 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   a.lay = st->lay;
   a.layer = layer;
   a.rows = rows;
-  a.step = step;
+  a.step = step < 0 ? 0 : step;
+  a.step_dev = step == SPIN_STEP_DEVICE ? st->step_dev : nullptr;
   a.sparsity = st->sparsity[layer];
   a.gamma = st->cfg.gamma;
   a.alpha = st->cfg.alpha;
@@ -275,6 +278,7 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->scores = (float*)(st->base + k.scores);
   st->gmax = (float*)(st->base + k.gmax);
   st->gstride = gmax_stride(L);
+  st->step_dev = (int64_t*)(st->base + k.step);
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
   st->inject = 0;
@@ -290,6 +294,7 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(st->err, 0, sizeof(ErrWord), s);
   if (e == cudaSuccess) e = launch_init_state(st->V, st->D, (int64_t)L.L * L.Q * L.slot_stride, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->step_dev, 0, sizeof(int64_t), s);
   if (e != cudaSuccess) {
     delete st;
     return cuda_status(e);
@@ -328,6 +333,17 @@ spin_status spin_set_score_kernel(spin_state st, int kind) {
     return SPIN_EUNSUPPORTED;
   st->score_kernel = kind;
   return SPIN_OK;
+}
+
+spin_status spin_set_step(spin_state st, int64_t step, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (step < 0) return SPIN_EINVAL;
+  return cuda_status(launch_step_op(st->step_dev, true, step, (cudaStream_t)stream));
+}
+
+spin_status spin_advance_step(spin_state st, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  return cuda_status(launch_step_op(st->step_dev, false, 0, (cudaStream_t)stream));
 }
 
 spin_status spin_set_kernel_timing(spin_state st, int enable) {
@@ -398,7 +414,8 @@ spin_status spin_reset_requests(spin_state st, int layer, const int32_t* req_hos
 spin_status spin_predict_select(spin_state st, int layer, int rows, int64_t step,
                                 const int32_t* ctx_len_dev, uint8_t* mask_dev, spin_stream_t stream) {
   if (!alive(st)) return SPIN_ESTATE;
-  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || !ctx_len_dev || !mask_dev || step < 0)
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || !ctx_len_dev || !mask_dev ||
+      step < SPIN_STEP_DEVICE)
     return SPIN_EINVAL;
   StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
   cudaStream_t s = (cudaStream_t)stream;
@@ -469,7 +486,8 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
                              int defer_update, uint8_t* mask_dev, int32_t* topk_dev, float* scores_dev,
                              spin_stream_t stream) {
   if (!alive(st)) return SPIN_ESTATE;
-  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || step < 0) return SPIN_EINVAL;
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || step < SPIN_STEP_DEVICE)
+    return SPIN_EINVAL;
   if (!keys || !block_table || !q || !w || !ctx_len_dev || !mask_dev || !topk_dev || num_pages < 1 ||
       bt_stride < st->lay.max_blocks)
     return SPIN_EINVAL;

@@ -213,6 +213,7 @@ struct StepArgs {
   Layout lay;
   int layer, rows;
   int64_t step;
+  const int64_t* step_dev;  // non-null: the step is read from the state's counter
   float sparsity, gamma, alpha;
   uint64_t seed;
   const int32_t* ctx_len;
@@ -232,6 +233,8 @@ struct StepArgs {
 };
 
 cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s);
+// Sets (*p = value) or advances (*p += 1) the device step counter.
+cudaError_t launch_step_op(int64_t* p, bool set, int64_t value, cudaStream_t s);
 struct ReqList {
   static constexpr int kMax = 32;
   int32_t ids[kMax];

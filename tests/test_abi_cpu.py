@@ -54,7 +54,7 @@ def _expected_bytes(L, Q, R, H, d, b, max_slots):
     slot = mb * b
     blk = -(-mb // 16) * 16
     parts = [16, L * Q * slot * 4, L * Q * slot * 4, Q * R * blk * 4, Q * blk * 4, Q * 4, Q * R * H * d,
-             Q * R * H * 4, Q * R * slot * 4, Q * R * blk * max(1, b // 32) * 4]
+             Q * R * H * 4, Q * R * slot * 4, Q * R * blk * max(1, b // 32) * 4, 8]
     return sum(a(p) for p in parts)
 
 
