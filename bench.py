@@ -442,10 +442,45 @@ def gpu_arm(args, world, rank, local):
                   "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                   "transfers": "pinned host buffers; step i+1's inputs in and step i-1's results out on a copy "
                                "stream while step i computes (double-buffered), all inside the timed region"}
+    # ---- the same step replayed from one captured CUDA graph ---------------
+    out["graph_replay"] = graph_pass(run, W, K, world)
     status, word = isa.spin_get_error(run.st)
     if status != 0:
         raise RuntimeError(f"device error word {word:#x}")
     return out
+
+
+def graph_pass(run, warmup, steps, world):
+    """The decode step captured once in a CUDA graph -- the step number from
+    the state's device counter, advanced inside the graph -- and replayed;
+    every replay uses the same query rows and context lengths."""
+    isa, wl = run.isa, run.wl
+    t = run.t
+    q_buf, w_buf, c_buf = run.q[t].clone(), run.w[t].clone(), run.ctx[t].clone()
+    isa.spin_set_step(run.st, t)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    c = run.cache
+    with torch.cuda.graph(graph):
+        isa.spin_decode_step(run.st, 0, 1, isa.SPIN_STEP_DEVICE, c.keys, c.kscale, c.block_table, q_buf, w_buf,
+                             c_buf, False, run.mask, run.topk, run.scores)
+        isa.spin_advance_step(run.st)
+    for _ in range(warmup):
+        graph.replay()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        graph.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    del graph
+    return {"value": job_rows_per_s(wl.requests * steps, world, ms), "unit": "rows/s", "ms_per_step": ms / steps,
+            "note": "one captured graph per step (device step counter), same inputs every replay"}
 
 
 # ---------------------------------------------------------------------------
