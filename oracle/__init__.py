@@ -64,6 +64,8 @@ def _load():
             lib.orc_num_blocks.argtypes = [_i64, ctypes.c_int, ctypes.c_int]
             lib.orc_num_blocks.restype = _i64
             lib.orc_predict_pool.argtypes = [_f32p, _f32p, _i64, ctypes.c_int, ctypes.c_int, _i64, _f32p]
+            lib.orc_predict_pool_mode.argtypes = [_f32p, _f32p, _i64, ctypes.c_int, ctypes.c_int, _i64, ctypes.c_int,
+                                                  _f32p]
             lib.orc_budget.argtypes = [_i64, ctypes.c_double]
             lib.orc_budget.restype = _i64
             lib.orc_explore_count.argtypes = [_i64, ctypes.c_double]
@@ -154,13 +156,17 @@ def quantize_q(q: np.ndarray, w: np.ndarray):
     return q8, wq, e
 
 
-def predict_pool(V: np.ndarray, D: np.ndarray, ctx_len: int, rows: int, b: int, n_stride: int):
-    """Block scores S [rows, n_stride] (entries past each row's block count are NaN)."""
+POOL_MAX, POOL_MEAN, POOL_TOP4 = 0, 1, 2
+
+
+def predict_pool(V: np.ndarray, D: np.ndarray, ctx_len: int, rows: int, b: int, n_stride: int, pooling: int = 0):
+    """Block scores S [rows, n_stride] (entries past each row's block count are
+    NaN); pooling: POOL_MAX (the method's), POOL_MEAN or POOL_TOP4."""
     lib = _load()
     V = _c(V, np.float32)
     D = _c(D, np.float32)
     S = np.full((rows, n_stride), np.nan, np.float32)
-    lib.orc_predict_pool(_p(V, _f32p), _p(D, _f32p), ctx_len, rows, b, n_stride, _p(S, _f32p))
+    lib.orc_predict_pool_mode(_p(V, _f32p), _p(D, _f32p), ctx_len, rows, b, n_stride, int(pooling), _p(S, _f32p))
     return S
 
 

@@ -183,6 +183,64 @@ ORC_API void orc_predict_pool(const float* V, const float* D, int64_t ctx_len, i
   }
 }
 
+/* Block-reduction variants of the pool ([listing] Figure 3: "Mean and Top-4
+ * compared with Max pooling"; the pages do not define them, so these are the
+ * plainest readings).  Over the block's visible slots of row r:
+ *   Mean  = (sum of z) / count,
+ *   Top-4 = (sum of the min(4, count) largest z) / min(4, count),
+ * each computed in double in a fixed order and rounded once to float: the
+ * Mean sums every run of 8 consecutive slots in slot order, then adds the
+ * runs' sums pairwise (runs 2k and 2k+1, then pairs of pairs, ...); the
+ * Top-4 adds its values from the largest down.  +inf (a never-observed slot)
+ * makes either +inf.  mode 0 is the max-pool above. */
+static double orc_tree_sum(double* c, int n) {  /* n a power of two */
+  for (int w = 1; w < n; w *= 2)
+    for (int u = 0; u + w < n; u += 2 * w) c[u] = c[u] + c[u + w];
+  return c[0];
+}
+
+ORC_API void orc_predict_pool_mode(const float* V, const float* D, int64_t ctx_len, int rows, int b,
+                                   int64_t n_stride, int mode, float* S) {
+  if (mode == 0) {
+    orc_predict_pool(V, D, ctx_len, rows, b, n_stride, S);
+    return;
+  }
+  double runs[32];  /* b <= 256: at most 32 runs of 8 slots */
+  for (int r = 0; r < rows; ++r) {
+    int64_t p = pos_of_row(ctx_len, r);
+    int64_t n = nblocks_of_row(ctx_len, r, b);
+    for (int64_t j = 0; j < n; ++j) {
+      int count = 0;
+      float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      int nr = b / 8;
+      for (int u = 0; u < nr; ++u) runs[u] = 0.0;
+      for (int64_t i = j * b; i < (j + 1) * b && i <= p; ++i) {
+        float z = fmaxf(V[i], D[p - i]);
+        ++count;
+        runs[(i - j * b) / 8] += (double)z;
+        /* insert into the descending top-4 */
+        for (int k = 0; k < 4; ++k) {
+          if (z > top[k]) {
+            for (int m = 3; m > k; --m) top[m] = top[m - 1];
+            top[k] = z;
+            break;
+          }
+        }
+      }
+      double v;
+      if (mode == 1) {
+        v = orc_tree_sum(runs, nr) / (double)count;
+      } else {
+        int m = count < 4 ? count : 4;
+        double t = 0.0;
+        for (int k = 0; k < m; ++k) t += (double)top[k];
+        v = t / (double)m;
+      }
+      S[(int64_t)r * n_stride + j] = (float)v;
+    }
+  }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Block selection.                                                          */
 /* Budget: B = n - floor(s n) blocks for target block sparsity s ([listing]  */

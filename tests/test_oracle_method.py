@@ -451,3 +451,68 @@ def test_p99_nearest_rank(oracle_lib):
     assert oracle_lib.p99(np.arange(1, 101)) == 99
     assert oracle_lib.p99(np.arange(1, 1001)) == 990
     assert oracle_lib.p99([3.0]) == 3.0
+
+
+# --------------------------------------------------------------------------
+# Block-reduction variants (SPIN listing, Figure 3: Mean and Top-4 against
+# Max pooling; the pages define neither, the oracle takes the plain readings)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("b", [16, 64, 256])
+def test_pool_mean_and_top4_on_exact_integers(oracle_lib, b):
+    """Integer-valued z: every partial sum is exact, so the mean and the top-4
+    mean must equal the brute-force values whatever the summation order."""
+    rng = np.random.default_rng(b)
+    n_slots = 5 * b + 7                                   # a ragged last block
+    V = rng.integers(0, 1000, n_slots + 8).astype(np.float32)
+    D = np.where(rng.random(n_slots + 8) < 0.5, -np.inf, rng.integers(0, 1000, n_slots + 8)).astype(np.float32)
+    ctx = n_slots
+    for rows in (1, 3):
+        S_mean = oracle_lib.predict_pool(V, D, ctx, rows, b, 8, oracle_lib.POOL_MEAN)
+        S_top4 = oracle_lib.predict_pool(V, D, ctx, rows, b, 8, oracle_lib.POOL_TOP4)
+        S_max = oracle_lib.predict_pool(V, D, ctx, rows, b, 8, oracle_lib.POOL_MAX)
+        for r in range(rows):
+            p = ctx - 1 + r
+            for j in range(oracle_lib.num_blocks(ctx, r, b)):
+                i = np.arange(j * b, min((j + 1) * b, p + 1))
+                z = np.maximum(V[i], D[p - i]).astype(np.float64)
+                assert S_mean[r, j] == np.float32(z.mean())
+                top = np.sort(z)[::-1][:4]
+                assert S_top4[r, j] == np.float32(top.mean())
+                assert S_max[r, j] == np.float32(z.max())
+
+
+def test_pool_variants_order_and_sentinels(oracle_lib):
+    """Mean <= Top-4 <= Max on real-valued z; a never-observed slot (V = +inf)
+    makes every variant +inf; a block with fewer than 4 visible slots averages
+    them all."""
+    rng = np.random.default_rng(3)
+    n = 64 * 40 + 3
+    V = rng.standard_normal(n + 4).astype(np.float32) * 10
+    D = rng.standard_normal(n + 4).astype(np.float32) * 10
+    V[64 * 7 + 5] = np.inf
+    S = {m: oracle_lib.predict_pool(V, D, n, 1, 64, 48, m)[0] for m in (0, 1, 2)}
+    nb = oracle_lib.num_blocks(n, 0, 64)
+    assert np.all(S[1][:nb] <= S[2][:nb]) and np.all(S[2][:nb] <= S[0][:nb])
+    assert all(np.isinf(S[m][7]) for m in (0, 1, 2))
+    # the last block holds 3 visible slots
+    p = n - 1
+    i = np.arange(64 * (nb - 1), n)
+    z = np.maximum(V[i], D[p - i]).astype(np.float64)
+    assert len(i) == 3 and S[2][nb - 1] == np.float32(z.mean())
+
+
+def test_pool_mean_sums_runs_of_eight_then_pairwise(oracle_lib):
+    """The Mean's fixed order: each run of 8 slots is summed in slot order,
+    then the runs are added pairwise.  With z spanning 2^60 the order shows:
+    a 1.0 in the run of 2^60 is absorbed (the double ulp there is 2^8), so
+    runs (2^60 + 1) and (-2^60 + 1) sum to 0, where a single left-to-right sum
+    over the block would give 1."""
+    b = 16
+    D = np.full(b, -np.inf, np.float32)
+    V = np.zeros(b, np.float32)
+    V[0], V[1], V[8], V[9] = 2.0 ** 60, 1.0, -(2.0 ** 60), 1.0
+    assert oracle_lib.predict_pool(V, D, b, 1, b, 1, oracle_lib.POOL_MEAN)[0, 0] == np.float32(0.0)
+    # a value of one ulp survives its run: (2^60 + 256) + (-2^60) = 256
+    V2 = np.zeros(b, np.float32)
+    V2[0], V2[1], V2[8] = 2.0 ** 60, 256.0, -(2.0 ** 60)
+    assert oracle_lib.predict_pool(V2, D, b, 1, b, 1, oracle_lib.POOL_MEAN)[0, 0] == np.float32(256.0 / b)
