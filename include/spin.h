@@ -91,7 +91,20 @@ typedef struct {
   float gamma;             /* exploration share of the block budget (SPIN listing, Figure 4) */
   float target_sparsity;   /* default per-layer target block sparsity, [0, 1) */
   uint64_t seed;           /* exploration RNG seed (Philox4x32-10 key) */
+  int32_t pooling;         /* block reduction of the predicted slot scores: spin_pooling */
 } spin_config;
+
+/* Block reduction of the predicted slot scores z into a block score (SPIN
+ * listing, Figure 3 compares Max, the method's, with Mean and Top-4 pooling;
+ * the pages do not define the latter two).  Over a block's visible slots:
+ *   SPIN_POOL_MAX   the largest z;
+ *   SPIN_POOL_MEAN  the mean of z;
+ *   SPIN_POOL_TOP4  the mean of the min(4, count) largest z.
+ * Mean and Top-4 are computed in double and rounded once to float, in a
+ * fixed order (runs of 8 consecutive slots summed in slot order, then the
+ * runs added pairwise; the Top-4 values from the largest down), so the
+ * result does not depend on the launch. */
+typedef enum { SPIN_POOL_MAX = 0, SPIN_POOL_MEAN = 1, SPIN_POOL_TOP4 = 2 } spin_pooling;
 
 typedef struct spin_state_s* spin_state;
 

@@ -22,7 +22,7 @@ namespace spin {
 // before any use), and the b/8 lanes of a block reduce with shuffles.
 // Block sizes 16..256 (powers of two).
 // ---------------------------------------------------------------------------
-template <int R>
+template <int R, int P>
 __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
   pdl_enter();
   const Layout L = a.lay;
@@ -71,19 +71,74 @@ __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
         if (di >= 0) dw[t] = __ldg(D + di);
       }
     }
-    float m[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      m[r] = __int_as_float(0xff800000);
+      // this lane's slots i0 .. i0+7 visible to row r: z = max(V_i, D_{p_r - i}),
+      // slot i0+k at offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + 7]
+      float x;
+      if (P == SPIN_POOL_MAX) {
+        x = __int_as_float(0xff800000);
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        // slot i0+k at offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + 7]
-        if (active && i0 + k <= p0 + r) m[r] = fmaxf(m[r], fmaxf(vv[k], dw[r - k + 7]));
-    }
+        for (int k = 0; k < 8; ++k)
+          if (active && i0 + k <= p0 + r) x = fmaxf(x, fmaxf(vv[k], dw[r - k + 7]));
+        for (int o = lpb >> 1; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      } else if (P == SPIN_POOL_MEAN) {
+        // the run of 8 slots in slot order, then runs added pairwise (lanes
+        // l and l^1, then pairs of pairs, ...): the order the reduction fixes
+        double sum = 0.0;
+        int cnt = 0;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      float x = m[r];
-      for (int o = lpb >> 1; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+        for (int k = 0; k < 8; ++k)
+          if (active && i0 + k <= p0 + r) {
+            sum += (double)fmaxf(vv[k], dw[r - k + 7]);
+            ++cnt;
+          }
+        for (int o = 1; o < lpb; o <<= 1) {
+          sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        }
+        x = cnt ? (float)(sum / (double)cnt) : 0.f;
+      } else {
+        // the block's four largest z (a multiset: any merge order gives it),
+        // summed from the largest down
+        float t[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
+                      __int_as_float(0xff800000)};
+        int cnt = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (active && i0 + k <= p0 + r) {
+            float z = fmaxf(vv[k], dw[r - k + 7]);
+            ++cnt;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {  // insert, keeping t descending
+              const float hi = fmaxf(t[u], z), lo = fminf(t[u], z);
+              t[u] = hi;
+              z = lo;
+            }
+          }
+        for (int o = 1; o < lpb; o <<= 1) {
+          float u4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) u4[u] = __shfl_xor_sync(0xffffffffu, t[u], o);
+          cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {  // insert the partner's values
+            float z = u4[u];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float hi = fmaxf(t[w], z), lo = fminf(t[w], z);
+              t[w] = hi;
+              z = lo;
+            }
+          }
+        }
+        const int mtop = cnt < 4 ? cnt : 4;
+        double sum = 0.0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (u < mtop) sum += (double)t[u];
+        x = mtop ? (float)(sum / (double)mtop) : 0.f;
+      }
       if (active && (lane & (lpb - 1)) == 0 && j < row_blocks(ctx, r, L.b))
         a.S[((int64_t)q * L.R + r) * L.blk_stride + j] = x;
     }
@@ -96,12 +151,24 @@ cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   int64_t blocks = (warps + 7) / 8;
   if (blocks > 148 * 32) blocks = 148 * 32;
   PdlLaunch l(dim3((unsigned)blocks), dim3(256), 0, s);
+  void (*k)(StepArgs) = nullptr;
+#define SPIN_PREDICT_CASE(R)                                            \
+  case R:                                                               \
+    k = a.pooling == SPIN_POOL_MEAN   ? k_predict_pool<R, SPIN_POOL_MEAN> \
+        : a.pooling == SPIN_POOL_TOP4 ? k_predict_pool<R, SPIN_POOL_TOP4> \
+                                      : k_predict_pool<R, SPIN_POOL_MAX>; \
+    break;
   switch (a.rows) {
-    case 1: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<1>, a);
-    case 2: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<2>, a);
-    case 3: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<3>, a);
-    default: return cudaLaunchKernelEx(&l.cfg, k_predict_pool<4>, a);
+    SPIN_PREDICT_CASE(1)
+    SPIN_PREDICT_CASE(2)
+    SPIN_PREDICT_CASE(3)
+    default:
+      k = a.pooling == SPIN_POOL_MEAN   ? k_predict_pool<4, SPIN_POOL_MEAN>
+          : a.pooling == SPIN_POOL_TOP4 ? k_predict_pool<4, SPIN_POOL_TOP4>
+                                        : k_predict_pool<4, SPIN_POOL_MAX>;
   }
+#undef SPIN_PREDICT_CASE
+  return cudaLaunchKernelEx(&l.cfg, k, a);
 }
 
 // ---------------------------------------------------------------------------

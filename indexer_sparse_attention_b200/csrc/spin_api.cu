@@ -64,6 +64,7 @@ bool valid_config(const spin_config* c) {
   if (!(c->alpha >= 0.0f && c->alpha <= 1.0f)) return false;
   if (!(c->gamma >= 0.0f && c->gamma <= 1.0f)) return false;
   if (!(c->target_sparsity >= 0.0f && c->target_sparsity < 1.0f)) return false;
+  if (c->pooling < SPIN_POOL_MAX || c->pooling > SPIN_POOL_TOP4) return false;
   const int64_t max_blocks = (c->max_slots + (int64_t)b - 1) / b;
   if (max_blocks > kMaxBlocksSelect) return false;
   // top-k: bitmap of one (request, row) plus the candidate area on chip
@@ -132,6 +133,7 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   a.lay = st->lay;
   a.layer = layer;
   a.rows = rows;
+  a.pooling = st->cfg.pooling;
   a.step = step < 0 ? 0 : step;
   a.step_dev = step == SPIN_STEP_DEVICE ? st->step_dev : nullptr;
   a.sparsity = st->sparsity[layer];

@@ -214,6 +214,7 @@ struct StepArgs {
   int layer, rows;
   int64_t step;
   const int64_t* step_dev;  // non-null: the step is read from the state's counter
+  int pooling;              // spin_pooling: block reduction of the predicted scores
   float sparsity, gamma, alpha;
   uint64_t seed;
   const int32_t* ctx_len;

@@ -37,7 +37,7 @@ class Harness:
         cfg = isa.make_config(num_layers=wl.layers, num_requests=wl.requests, max_slots=wl.max_slots,
                               block_size=wl.b, num_heads=wl.H, head_dim=wl.d, topk=wl.topk, max_rows=wl.rows,
                               key_fp8=wl.key_fp8, q_bf16=wl.q_bf16, alpha=wl.alpha, gamma=wl.gamma,
-                              target_sparsity=wl.sparsity, seed=wl.seed)
+                              target_sparsity=wl.sparsity, seed=wl.seed, pooling=wl.pooling)
         self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
         isa.spin_set_score_kernel(self.st, score_kernel)
@@ -107,7 +107,7 @@ class Harness:
         wl = self.wl
         V0, D0 = snap
         nstride = self.st.mask_stride
-        S_ref = oracle.predict_pool(V0, D0, ctx_len, rows, wl.b, nstride)
+        S_ref = oracle.predict_pool(V0, D0, ctx_len, rows, wl.b, nstride, wl.pooling)
         s = float(np.float32(self.sparsity[layer]))
         if s > 0:
             S_gpu = self.st.block_scores()[q, :rows, :nstride].cpu().numpy()

@@ -337,3 +337,35 @@ def test_select_cluster_paths_bit_exact(R, s, g):
             S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, 64, st.mask_stride)
             m_ref = oracle.select(S_ref, int(ctx[q]), R, 64, s, g, 7, q, 0, step)
             assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
+
+
+@pytest.mark.parametrize("pooling", [isa.SPIN_POOL_MEAN, isa.SPIN_POOL_TOP4])
+@pytest.mark.parametrize("R,b", [(1, 64), (4, 64), (2, 16), (1, 256)])
+def test_pooling_variants_bit_exact(pooling, R, b):
+    """Mean and Top-4 block pooling: block scores and masks equal the
+    oracle's bit for bit (fixed summation order on both sides)."""
+    rng = np.random.default_rng(pooling * 100 + R * 10 + b)
+    max_slots = 200 * b + 64
+    cfg = isa.make_config(num_layers=1, num_requests=3, max_slots=max_slots, block_size=b, topk=256, max_rows=R,
+                          gamma=0.05, target_sparsity=0.5, seed=7, pooling=pooling)
+    st = isa.SpinState(cfg)
+    V, D = st.ema(0)
+    v = (rng.standard_normal(V.shape) * 10).astype(np.float32)
+    v[rng.random(V.shape) < 0.02] = np.inf                # never-observed slots
+    V.copy_(torch.from_numpy(v))
+    d = (rng.standard_normal(D.shape) * 10).astype(np.float32)
+    d[rng.random(D.shape) < 0.3] = -np.inf
+    D.copy_(torch.from_numpy(d))
+    ctx = np.array([1, 37 * b + 5, max_slots - R + 1], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    isa.spin_predict_select(st, 0, R, 3, ctx_t, mask)
+    assert isa.spin_get_error(st)[0] == 0
+    S_gpu = st.block_scores().cpu().numpy()
+    for q in range(3):
+        S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, b, st.mask_stride, pooling)
+        for r in range(R):
+            n = oracle.num_blocks(int(ctx[q]), r, b)
+            assert np.array_equal(S_gpu[q, r, :n].view(np.uint32), S_ref[r, :n].view(np.uint32)), (q, r)
+        m_ref = oracle.select(S_ref, int(ctx[q]), R, b, 0.5, 0.05, 7, q, 0, 3)
+        assert np.array_equal(mask[q].cpu().numpy(), m_ref), q

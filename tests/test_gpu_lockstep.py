@@ -221,3 +221,13 @@ def test_maximum_context():
     bootstrap(h, sample_blocks=32)
     for _ in range(wl.steps - 1):
         h.run_step(0, check=[0], sample_blocks=32)
+
+
+@pytest.mark.parametrize("pooling", [isa.SPIN_POOL_MEAN, isa.SPIN_POOL_TOP4])
+def test_decode_steps_with_pooling_variants(pooling):
+    """Serving-shaped steps with Mean and Top-4 block pooling, in lock step."""
+    wl = workloads.config(2, requests=2, ctx0=(120_000, 64 * 900 + 11), steps=4, pooling=pooling)
+    h = Harness(wl)
+    bootstrap(h, sample_blocks=32)
+    for _ in range(wl.steps - 1):
+        h.run_step(0, check=range(wl.requests), sample_blocks=32)

@@ -56,6 +56,7 @@ class Workload:
     diag_amp: Sequence[float] = (3.0,)     # per layer A
     accept_probs: Optional[Sequence[float]] = None  # P(a = 1..rows)
     warmup_steps: int = 0         # config with a per-layer budget: uniform-sparsity warm-up steps
+    pooling: int = 0              # block reduction of the predicted scores: 0 max, 1 mean, 2 top-4
     spare_slots: int = 0          # extra capacity beyond ctx0 + steps * rows
 
     @property
