@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "SPIN decode rows/s & index-key GB/s at 512K ctx x96 req; % of roofline"
+POOLINGS = {"max": 0, "mean": 1, "top4": 2}
 WORKLOADS = {"serve-96x512K": 2, "mtp-32x128K-r4": 3, "ragged-8Lx8-256K-1M": 4, "dsa-1x64K": 1, "tiny-fp32-4K": 0}
 KEY_BYTES_PER_SLOT = 128 + 4            # E4M3 key row + fp32 scale
 SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write of V and D
@@ -65,6 +66,10 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--workload", choices=list(WORKLOADS), default="serve-96x512K",
                    help="serve-96x512K is the headline; the others print their own line")
+    p.add_argument("--pooling", choices=list(POOLINGS), default="max",
+                   help="block reduction of the predicted scores (max is the method's)")
+    p.add_argument("--ablation", choices=["pooling"], default=None,
+                   help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities")
     return p.parse_args()
 
 
@@ -195,7 +200,7 @@ def peaks():
 
 
 class SpinRun:
-    def __init__(self, wl, device, total_steps):
+    def __init__(self, wl, device, total_steps, pooling=0):
         import indexer_sparse_attention_b200 as isa
         self.isa = isa
         self.wl = wl
@@ -210,7 +215,9 @@ class SpinRun:
         self.ctx = [(ctx0 + t + 1).to(torch.int32) for t in range(self.positions)]
         cfg = isa.make_config(num_layers=1, num_requests=wl.requests, max_slots=wl.max_slots, block_size=wl.b,
                               num_heads=wl.H, head_dim=wl.d, topk=wl.topk, max_rows=1, key_fp8=True, q_bf16=True,
-                              alpha=wl.alpha, gamma=wl.gamma, target_sparsity=wl.sparsity, seed=wl.seed)
+                              alpha=wl.alpha, gamma=wl.gamma, target_sparsity=wl.sparsity, seed=wl.seed,
+                              pooling=pooling)
+        self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
         self.mask = self.st.new_mask()
         self.topk = torch.empty((wl.requests, 1, wl.topk), dtype=torch.int32, device=device)
@@ -364,7 +371,7 @@ def gpu_arm(args, world, rank, local):
     KS = min(K, 40)  # steps of the per-stage timing pass
     total = 1 + (W + K) * (1 + len(sweep)) + 3 + K + KS + 2
     wl = rank_workload(rank, args.requests, total + 8)
-    run = SpinRun(wl, device, total)
+    run = SpinRun(wl, device, total, POOLINGS[args.pooling])
     Q = wl.requests
     # history bootstrap: all-keep step that fills V and D
     run.set_sparsity(0.0)
@@ -406,7 +413,8 @@ def gpu_arm(args, world, rank, local):
         "dtype": "e4m3xe4m3->f32 (selection f32, exact)", "data": "synthetic",
         "config": {"workload": wl.name, "requests_per_gpu": Q, "context_slots": wl.ctx0[0], "block_size": wl.b,
                    "heads": wl.H, "head_dim": wl.d, "topk": wl.topk, "target_sparsity": args.sparsity,
-                   "gamma": wl.gamma, "parallelism": f"dp{world} (requests sharded, no collective)",
+                   "gamma": wl.gamma, "pooling": args.pooling,
+                   "parallelism": f"dp{world} (requests sharded, no collective)",
                    "l2": "inputs larger than L2: 6.4 GB paged FP8 key cache and 0.4 GB EMA state per GPU"},
         "index_key_gbs": key_gbs,
         "key_roofline_frac": key_gbs / peak,
@@ -720,6 +728,63 @@ def workload_arm(args, world, rank, local):
 
 
 # ---------------------------------------------------------------------------
+# Block-pooling ablation (SPIN listing, Figure 3 compares Mean and Top-4 with
+# Max pooling by their P99 miss)
+# ---------------------------------------------------------------------------
+def pooling_ablation(args, world, rank, local):
+    """The serving workload (args.requests requests at 512K) run three times,
+    once per pooling, through the same target sparsities in rising order:
+    after a bootstrap and W warm-up steps at each sparsity, mean / p99 miss
+    and realized sparsity over 4 steps (shadow full indexer), then K timed
+    steps.  One JSON line."""
+    import indexer_sparse_attention_b200 as isa
+    from indexer_sparse_attention_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    isa.load()
+    device = torch.device("cuda", local if world > 1 else 0)
+    sparsities = (0.5, 0.8, 0.9)
+    W, K, F = max(args.warmup, 3), args.steps, 4
+    total = 1 + len(sparsities) * (W + F + K) + 2
+    wl = rank_workload(rank, args.requests, total + 8)
+    run = SpinRun(wl, device, total, 0)
+    results = {}
+    for name, pooling in POOLINGS.items():
+        cfg = run.cfg
+        cfg.pooling = pooling
+        run.st = isa.SpinState(cfg, device=device)
+        run.t = 0
+        run.set_sparsity(0.0)
+        run.step()
+        per = {}
+        for s in sparsities:
+            run.set_sparsity(s)
+            for _ in range(W):
+                run.step()
+            fid = fidelity(run, n_steps=F)
+            ms = timed_steps(run, K, world) / K
+            per[str(s)] = {"mean_miss": fid["mean_miss"], "p99_miss": fid["p99_miss"],
+                           "realized_sparsity": fid["realized_sparsity"], "ms_per_step": ms}
+        status, word = isa.spin_get_error(run.st)
+        if status != 0:
+            raise RuntimeError(f"device error word {word:#x}")
+        results[name] = per
+    rel = {}
+    for name in ("mean", "top4"):
+        rel[name] = {}
+        for s in sparsities:
+            base = results["max"][str(s)]["p99_miss"]
+            v = results[name][str(s)]["p99_miss"]
+            rel[name][str(s)] = None if base == 0 else (v - base) / base
+    return {"ablation": "block pooling: max (the method's) vs mean and top-4", "unit": "miss fraction / ms",
+            "config": {"workload": wl.name, "requests_per_gpu": wl.requests, "context_slots": wl.ctx0[0],
+                       "gamma": wl.gamma, "warmup_steps_per_sparsity": W, "fidelity_steps": F, "timed_steps": K},
+            "results": results, "p99_change_vs_max": rel,
+            "note": "relative change is null where max pooling misses nothing"}
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
 class OracleSample:
@@ -807,6 +872,11 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
+        if args.ablation == "pooling":
+            out = pooling_ablation(args, world, rank, local)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+            return
         if args.workload != "serve-96x512K":
             out = workload_arm(args, world, rank, local)
             if rank == 0:
