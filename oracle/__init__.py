@@ -71,7 +71,8 @@ def _load():
             lib.orc_explore_count.argtypes = [_i64, ctypes.c_double]
             lib.orc_explore_count.restype = _i64
             lib.orc_select.argtypes = [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_float,
-                                       ctypes.c_float, _u64, ctypes.c_uint32, ctypes.c_uint32, _u64, _u8p]
+                                       ctypes.c_float, _u64, ctypes.c_uint32, ctypes.c_uint32, _u64, ctypes.c_int,
+                                       _u8p]
             lib.orc_score_fp8.argtypes = [_u8p, _f32p, _i32p, ctypes.c_int, ctypes.c_int, _u8p, _f32p,
                                           ctypes.c_int, ctypes.c_int, _i64, _u8p, _i64, _f64p]
             lib.orc_score_f32.argtypes = [_f32p, _i32p, ctypes.c_int, ctypes.c_int, _f32p, _f32p,
@@ -170,15 +171,27 @@ def predict_pool(V: np.ndarray, D: np.ndarray, ctx_len: int, rows: int, b: int, 
     return S
 
 
+# MTP policies (SPIN listing, Table 7 and Figure 2): the method's row-local
+# union of the rows' masks with a prefix-valid EMA replay, or the baseline
+# that shares row 0's mask and updates the EMA from row 0 alone.
+MTP_UNION_PREFIX, MTP_ROW0 = 0, 1
+
+
 def select(S: np.ndarray, ctx_len: int, rows: int, b: int, sparsity: float, gamma: float,
-           seed: int, request: int, layer: int, step: int) -> np.ndarray:
+           seed: int, request: int, layer: int, step: int, mtp_policy: int = MTP_UNION_PREFIX) -> np.ndarray:
     lib = _load()
     S = _c(S, np.float32)
     n_stride = S.shape[1]
     mask = np.zeros(n_stride, np.uint8)
     lib.orc_select(_p(S, _f32p), n_stride, ctx_len, rows, b, float(sparsity), float(gamma), seed,
-                   request, layer, step, _p(mask, _u8p))
+                   request, layer, step, int(mtp_policy), _p(mask, _u8p))
     return mask
+
+
+def update_rows(mtp_policy: int, accepted: int) -> int:
+    """Rows whose scores the EMA update replays: the accepted prefix, or row 0
+    alone under the row-0 policy."""
+    return min(accepted, 1) if mtp_policy == MTP_ROW0 else accepted
 
 
 def score_fp8(keys8, kscale, block_table, q8, wq, ctx_len, mask, slot_stride):
@@ -268,7 +281,8 @@ def p99(values) -> float:
 # --------------------------------------------------------------------------
 def decode_step_request(*, V, D, ctx_len, rows, b, sparsity, gamma, alpha, seed, request, layer,
                         step, topk, q, w, keys, kscale, block_table, key_fp8: bool,
-                        accepted=None, scores_in=None, n_stride=None, update=True):
+                        accepted=None, scores_in=None, n_stride=None, update=True,
+                        pooling=POOL_MAX, mtp_policy=MTP_UNION_PREFIX):
     """Run predict -> pool -> select -> score -> top-k -> EMA update for one
     request.  V and D (fp32, [max_slots]) are updated in place when ``update``.
 
@@ -280,8 +294,8 @@ def decode_step_request(*, V, D, ctx_len, rows, b, sparsity, gamma, alpha, seed,
     if n_stride is None:
         n_stride = block_table.shape[0]
     slot_stride = n_stride * b
-    S = predict_pool(V, D, ctx_len, rows, b, n_stride)
-    mask = select(S, ctx_len, rows, b, sparsity, gamma, seed, request, layer, step)
+    S = predict_pool(V, D, ctx_len, rows, b, n_stride, pooling)
+    mask = select(S, ctx_len, rows, b, sparsity, gamma, seed, request, layer, step, mtp_policy)
     out = {"S": S, "mask": mask}
     if key_fp8:
         q8, wq, e = quantize_q(q, w)
@@ -295,5 +309,6 @@ def decode_step_request(*, V, D, ctx_len, rows, b, sparsity, gamma, alpha, seed,
     if update:
         s32 = (scores.astype(np.float32) if scores_in is None
                else np.ascontiguousarray(scores_in, np.float32))
-        ema_update(V, D, s32, mask, ctx_len, rows if accepted is None else accepted, b, alpha)
+        ema_update(V, D, s32, mask, ctx_len, update_rows(mtp_policy, rows if accepted is None else accepted),
+                   b, alpha)
     return out

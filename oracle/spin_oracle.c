@@ -254,7 +254,17 @@ ORC_API void orc_predict_pool_mode(const float* V, const float* D, int64_t ctx_l
 /* labelled predicted.  Ties go to the lower block index.                    */
 /* mask[j] = 1 predicted (in the union), 2 explored, 0 skipped, for          */
 /* j < n_stride; blocks past the last row's visible range are 0.             */
+/*                                                                          */
+/* policy ORC_MTP_ROW0 is the baseline MTP policy of [listing] Table 7 and  */
+/* Figure 2, "Row-0 sharing": row 0 alone predicts (its own budget, the    */
+/* exploration share of that budget drawn among row 0's unkept blocks) and */
+/* every row uses its mask.  Blocks past row 0's range hold only the new    */
+/* keys of this step's draft tokens, which no step has scored yet; they are */
+/* kept (labelled predicted) so that the draft rows see them.  With one row */
+/* both policies are the same selection.                                    */
 /* ------------------------------------------------------------------------ */
+#define ORC_MTP_UNION_PREFIX 0
+#define ORC_MTP_ROW0 1
 typedef struct { float s; int64_t j; } orc_sj;
 typedef struct { uint32_t key; int64_t j; } orc_kj;
 
@@ -282,7 +292,7 @@ ORC_API int64_t orc_explore_count(int64_t budget_row0, double gamma) {
 
 ORC_API void orc_select(const float* S, int64_t n_stride, int64_t ctx_len, int rows, int b,
                         float sparsity, float gamma, uint64_t seed, uint32_t request,
-                        uint32_t layer, uint64_t step, uint8_t* mask) {
+                        uint32_t layer, uint64_t step, int policy, uint8_t* mask) {
   int64_t n_last = nblocks_of_row(ctx_len, rows - 1, b);
   memset(mask, 0, (size_t)n_stride);
   if (sparsity == 0.0f) {
@@ -291,8 +301,9 @@ ORC_API void orc_select(const float* S, int64_t n_stride, int64_t ctx_len, int r
   }
   int64_t n0 = nblocks_of_row(ctx_len, 0, b);
   int64_t n_exp = orc_explore_count(orc_budget(n0, (double)sparsity), (double)gamma);
+  int predicting_rows = policy == ORC_MTP_ROW0 ? 1 : rows;
   orc_sj* order = (orc_sj*)malloc(sizeof(orc_sj) * (size_t)n_last);
-  for (int r = 0; r < rows; ++r) {
+  for (int r = 0; r < predicting_rows; ++r) {
     int64_t n = nblocks_of_row(ctx_len, r, b);
     int64_t n_pred = orc_budget(n, (double)sparsity) - n_exp;
     for (int64_t j = 0; j < n; ++j) { order[j].s = S[(int64_t)r * n_stride + j]; order[j].j = j; }
@@ -300,6 +311,8 @@ ORC_API void orc_select(const float* S, int64_t n_stride, int64_t ctx_len, int r
     for (int64_t t = 0; t < n_pred && t < n; ++t) mask[order[t].j] = 1;
   }
   free(order);
+  if (policy == ORC_MTP_ROW0)
+    for (int64_t j = n0; j < n_last; ++j) mask[j] = 1;  /* the drafts' own new keys */
   orc_kj* cand = (orc_kj*)malloc(sizeof(orc_kj) * (size_t)n_last);
   int64_t nc = 0;
   for (int64_t j = 0; j < n_last; ++j) {
