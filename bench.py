@@ -41,6 +41,7 @@ import workloads  # noqa: E402
 
 METRIC = "SPIN decode rows/s & index-key GB/s at 512K ctx x96 req; % of roofline"
 POOLINGS = {"max": 0, "mean": 1, "top4": 2}
+MTP_POLICIES = {"union-prefix": 0, "row0": 1}   # the method's policy, then the baseline it is compared with
 WORKLOADS = {"serve-96x512K": 2, "mtp-32x128K-r4": 3, "ragged-8Lx8-256K-1M": 4, "dsa-1x64K": 1, "tiny-fp32-4K": 0}
 KEY_BYTES_PER_SLOT = 128 + 4            # E4M3 key row + fp32 scale
 SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write of V and D
@@ -68,8 +69,11 @@ def parse():
                    help="serve-96x512K is the headline; the others print their own line")
     p.add_argument("--pooling", choices=list(POOLINGS), default="max",
                    help="block reduction of the predicted scores (max is the method's)")
-    p.add_argument("--ablation", choices=["pooling"], default=None,
-                   help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities")
+    p.add_argument("--mtp-policy", choices=list(MTP_POLICIES), default="union-prefix",
+                   help="several query rows: row-local union + prefix-valid update (the method's) or row 0 alone")
+    p.add_argument("--ablation", choices=["pooling", "mtp"], default=None,
+                   help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities; "
+                        "mtp: p99 miss vs realized sparsity of the two MTP policies on the 4-row workload")
     return p.parse_args()
 
 
@@ -538,7 +542,8 @@ class WorkloadRun:
         cfg = isa.make_config(num_layers=Ly, num_requests=Q, max_slots=wl.max_slots, block_size=wl.b,
                               num_heads=wl.H, head_dim=wl.d, topk=wl.topk, max_rows=R, key_fp8=wl.key_fp8,
                               q_bf16=wl.q_bf16, alpha=wl.alpha, gamma=wl.gamma, target_sparsity=wl.sparsity,
-                              seed=wl.seed)
+                              seed=wl.seed, pooling=wl.pooling, mtp_policy=wl.mtp_policy)
+        self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
         self.masks = [self.st.new_mask() for _ in range(Ly)]
         self.topks = [torch.empty((Q, R, wl.topk), dtype=torch.int32, device=device) for _ in range(Ly)]
@@ -547,6 +552,14 @@ class WorkloadRun:
 
     def set_sparsity(self, per_layer):
         self.isa.spin_set_layer_sparsity(self.st, list(per_layer))
+
+    def restart(self, **cfg_fields):
+        """A fresh state (never-observed V, D) with some config fields
+        changed; the inputs are replayed from step 0."""
+        for k, v in cfg_fields.items():
+            setattr(self.cfg, k, v)
+        self.st = self.isa.SpinState(self.cfg, device=self.device)
+        self.t = 0
 
     def step(self, layers=None):
         """One decode step of every layer: a0..a5, and for MTP rows the
@@ -616,7 +629,8 @@ def workload_arm(args, world, rank, local):
     fid_steps = 3
     total = 1 + base.warmup_steps + W + K + fid_steps
     wl = workloads.config(WORKLOADS[args.workload], seed=base.seed + 1000 * rank, steps=total,
-                          spare_slots=base.rows * 4)
+                          spare_slots=base.rows * 4, pooling=POOLINGS[args.pooling],
+                          mtp_policy=MTP_POLICIES[args.mtp_policy])
     run = WorkloadRun(wl, device, total)
     Ly, Q, R = wl.layers, wl.requests, wl.rows
     # history bootstrap (all-keep), then the workload's warm-up protocol
@@ -695,6 +709,7 @@ def workload_arm(args, world, rank, local):
         "dtype": "e4m3xe4m3->f32 (selection f32, exact)" if wl.key_fp8 else "f32",
         "data": "synthetic",
         "config": {"workload": wl.name, "requests_per_gpu": Q, "layers": Ly, "rows": R,
+                   "pooling": args.pooling, "mtp_policy": args.mtp_policy if R > 1 else None,
                    "context_slots": [min(wl.ctx0), max(wl.ctx0)], "block_size": wl.b, "heads": wl.H,
                    "head_dim": wl.d, "topk": wl.topk, "target_sparsity": wl.sparsity, "gamma": wl.gamma,
                    "parallelism": f"dp{world} (requests sharded, no collective)",
@@ -785,6 +800,88 @@ def pooling_ablation(args, world, rank, local):
 
 
 # ---------------------------------------------------------------------------
+# MTP policy ablation (SPIN listing, Figure 2: p99 miss against realized block
+# sparsity, one point per target sparsity and policy, draft length three)
+# ---------------------------------------------------------------------------
+def mtp_ablation(args, world, rank, local):
+    """The 4-row MTP workload (32 requests at 128K) run once per policy on the
+    same inputs and accepted lengths, through the same target sparsities in
+    rising order: after a bootstrap and W warm-up steps at each sparsity, the
+    miss of every (request, row) and of the accepted rows alone, and realized
+    sparsity, over F steps (shadow full indexer), then K timed steps.  One
+    JSON line."""
+    import indexer_sparse_attention_b200 as isa
+    from indexer_sparse_attention_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    isa.load()
+    device = torch.device("cuda", local if world > 1 else 0)
+    sparsities = (0.4, 0.5, 0.6, 0.7, 0.8)
+    W, K, F = max(args.warmup, 3), args.steps, 4
+    total = 1 + len(sparsities) * (W + F + K) + 2
+    base = workloads.config(WORKLOADS["mtp-32x128K-r4"])
+    wl = workloads.config(WORKLOADS["mtp-32x128K-r4"], seed=base.seed + 1000 * rank, steps=total,
+                          spare_slots=base.rows * 4)
+    run = WorkloadRun(wl, device, total)
+    Q, R = wl.requests, wl.rows
+    s_ev = torch.cuda.current_stream()
+    results = {}
+    for name, pol in MTP_POLICIES.items():
+        run.restart(mtp_policy=pol)
+        run.set_sparsity([0.0])
+        run.step()
+        per = {}
+        for sp in sparsities:
+            run.set_sparsity([sp])
+            for _ in range(W):
+                run.step()
+            miss_all, miss_acc, realized = [], [], []
+            for _ in range(F):
+                run.step()
+                m = np.array(run.miss()[0]).reshape(Q, R)
+                acc = run.acc[run.t - 1].cpu().numpy()
+                miss_all += m.flatten().tolist()
+                miss_acc += [m[q, r] for q in range(Q) for r in range(int(acc[q]))]
+                realized += run.kept_slots(run.t - 1)[1]
+            barrier(world)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s_ev)
+            for _ in range(K):
+                run.step()
+            e1.record(s_ev)
+            torch.cuda.synchronize()
+            barrier(world)
+            ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+            per[str(sp)] = {"p99_miss": p99_of(miss_all), "mean_miss": float(np.mean(miss_all)),
+                            "p99_miss_accepted_rows": p99_of(miss_acc),
+                            "realized_sparsity": float(np.mean(realized)), "ms_per_step": ms}
+        status, word = isa.spin_get_error(run.st)
+        if status != 0:
+            raise RuntimeError(f"device error word {word:#x}")
+        results[name] = per
+    rel = {}
+    for sp in sparsities:
+        base_p99 = results["row0"][str(sp)]["p99_miss"]
+        v = results["union-prefix"][str(sp)]["p99_miss"]
+        rel[str(sp)] = None if base_p99 == 0 else (v - base_p99) / base_p99
+    return {"ablation": "MTP policy: row-local union + prefix-valid update (the method's) vs row-0 sharing + "
+                        "row-0 update", "unit": "miss fraction / ms",
+            "config": {"workload": wl.name, "requests_per_gpu": Q, "rows": R, "context_slots": wl.ctx0[0],
+                       "gamma": wl.gamma, "accept_probs": list(wl.accept_probs),
+                       "warmup_steps_per_sparsity": W, "fidelity_steps": F, "timed_steps": K},
+            "results": results, "p99_change_union_vs_row0": rel,
+            "note": "miss over every (request, row) of the fidelity steps; accepted lengths drawn from the "
+                    "workload's distribution, the same for both policies"}
+
+
+def p99_of(values):
+    v = np.sort(np.asarray(values, np.float64))
+    return float(v[max(int(np.ceil(0.99 * v.size)), 1) - 1]) if v.size else 0.0
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
 class OracleSample:
@@ -872,8 +969,8 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
-        if args.ablation == "pooling":
-            out = pooling_ablation(args, world, rank, local)
+        if args.ablation in ("pooling", "mtp"):
+            out = (pooling_ablation if args.ablation == "pooling" else mtp_ablation)(args, world, rank, local)
             if rank == 0:
                 print(json.dumps(out), flush=True)
             return

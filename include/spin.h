@@ -92,6 +92,7 @@ typedef struct {
   float target_sparsity;   /* default per-layer target block sparsity, [0, 1) */
   uint64_t seed;           /* exploration RNG seed (Philox4x32-10 key) */
   int32_t pooling;         /* block reduction of the predicted slot scores: spin_pooling */
+  int32_t mtp_policy;      /* mask and EMA policy for several query rows: spin_mtp_policy */
 } spin_config;
 
 /* Block reduction of the predicted slot scores z into a block score (SPIN
@@ -105,6 +106,19 @@ typedef struct {
  * runs added pairwise; the Top-4 values from the largest down), so the
  * result does not depend on the launch. */
 typedef enum { SPIN_POOL_MAX = 0, SPIN_POOL_MEAN = 1, SPIN_POOL_TOP4 = 2 } spin_pooling;
+
+/* Policy for steps with several query rows (MTP verification; SPIN listing,
+ * Table 7 and Figure 2 compare the two).
+ *   SPIN_MTP_UNION_PREFIX  the method's: each row predicts with its own
+ *     budget, the kept mask is the union, and the EMA update replays the
+ *     accepted prefix rows 0..a-1 in order.
+ *   SPIN_MTP_ROW0  the baseline: row 0 alone predicts (its budget, and the
+ *     exploration share of it drawn among row 0's unkept blocks) and every
+ *     row uses that mask; blocks past row 0's range, which hold only the new
+ *     keys of this step's drafts, are kept (label 1).  The EMA update uses
+ *     row 0's scores alone, whatever the accepted length.
+ * With one row the two are the same. */
+typedef enum { SPIN_MTP_UNION_PREFIX = 0, SPIN_MTP_ROW0 = 1 } spin_mtp_policy;
 
 typedef struct spin_state_s* spin_state;
 
@@ -151,7 +165,8 @@ SPIN_API spin_status spin_advance_step(spin_state st, spin_stream_t stream);
  * budget B_r = n_r - floor(s * n_r), exploration share n_exp = floor(gamma *
  * B_0) of uniformly random unkept blocks (SPIN digest, arXiv深度剖析; SPIN
  * listing, Figure 4), and for rows > 1 the union of the rows' predicted sets
- * (SPIN listing, Table 7).  Ties go to the lower block index.
+ * (SPIN listing, Table 7), or row 0's set under SPIN_MTP_ROW0 (whose block
+ * scores then hold row 0 only).  Ties go to the lower block index.
  *   ctx_len_dev [Q] int32, mask_dev [Q][max_blocks] uint8 out:
  *   0 skipped, 1 predicted, 2 explored (blocks past the last row's range: 0).
  *   step: decode step (>= 0, or SPIN_STEP_DEVICE), part of the exploration
@@ -214,7 +229,8 @@ SPIN_API spin_status spin_topk_noalloc(int num_requests, int rows, int max_rows,
  * of scored slots only (SPIN digest, 核心概要 / arXiv深度剖析; AI Radio, "The
  * paper's summary").  x <- score if x is the never-observed sentinel, else
  * fmaf(alpha, x, (1 - alpha) * score).  Rows 0..accepted[q]-1 are replayed in
- * order (prefix-valid update of MTP rows, SPIN digest, arXiv深度剖析).
+ * order (prefix-valid update of MTP rows, SPIN digest, arXiv深度剖析); under
+ * SPIN_MTP_ROW0 row 0 alone is applied (accepted_dev is still checked).
  * accepted_dev [Q] int32 in 1..rows, or NULL for all rows. */
 SPIN_API spin_status spin_ema_update(spin_state st, int layer, int rows, const float* scores_dev,
                             const uint8_t* mask_dev, const int32_t* ctx_len_dev,

@@ -25,6 +25,7 @@ __all__ = [
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
     "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_set_kernel_timing_mask",
     "SPIN_STEP_DEVICE", "spin_set_step", "spin_advance_step", "SPIN_POOL_MAX", "SPIN_POOL_MEAN", "SPIN_POOL_TOP4",
+    "SPIN_MTP_UNION_PREFIX", "SPIN_MTP_ROW0",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +35,7 @@ SPIN_F32, SPIN_BF16, SPIN_FP8_E4M3 = 0, 1, 2
 SPIN_SCORE_AUTO, SPIN_SCORE_SIMT, SPIN_SCORE_TCGEN05 = 0, 1, 2
 SPIN_STEP_DEVICE = -1  # step argument: read the state's device step counter
 SPIN_POOL_MAX, SPIN_POOL_MEAN, SPIN_POOL_TOP4 = 0, 1, 2  # block reduction of the predicted scores
+SPIN_MTP_UNION_PREFIX, SPIN_MTP_ROW0 = 0, 1  # mask / EMA policy for several query rows
 STATUS_NAMES = {0: "SPIN_OK", 1: "SPIN_EINVAL", 2: "SPIN_ENOMEM", 3: "SPIN_ECUDA", 4: "SPIN_ESTATE",
                 5: "SPIN_ETIMEOUT", 6: "SPIN_EDEVICE", 7: "SPIN_EUNSUPPORTED"}
 
@@ -45,7 +47,8 @@ class SpinConfig(ctypes.Structure):
                 ("topk", ctypes.c_int32), ("max_rows", ctypes.c_int32),
                 ("key_dtype", ctypes.c_int32), ("q_dtype", ctypes.c_int32),
                 ("alpha", ctypes.c_float), ("gamma", ctypes.c_float),
-                ("target_sparsity", ctypes.c_float), ("seed", ctypes.c_uint64), ("pooling", ctypes.c_int32)]
+                ("target_sparsity", ctypes.c_float), ("seed", ctypes.c_uint64), ("pooling", ctypes.c_int32),
+                ("mtp_policy", ctypes.c_int32)]
 
 
 class SpinError(RuntimeError):
@@ -143,10 +146,10 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None) -> _vp:
 
 def make_config(*, num_layers, num_requests, max_slots, block_size=64, num_heads=64, head_dim=128, topk=2048,
                 max_rows=1, key_fp8=True, q_bf16=True, alpha=0.9, gamma=0.05, target_sparsity=0.5,
-                seed=0, pooling=SPIN_POOL_MAX) -> SpinConfig:
+                seed=0, pooling=SPIN_POOL_MAX, mtp_policy=SPIN_MTP_UNION_PREFIX) -> SpinConfig:
     return SpinConfig(num_layers, num_requests, max_slots, block_size, num_heads, head_dim, topk, max_rows,
                       SPIN_FP8_E4M3 if key_fp8 else SPIN_F32, SPIN_BF16 if q_bf16 else SPIN_F32,
-                      alpha, gamma, target_sparsity, seed, pooling)
+                      alpha, gamma, target_sparsity, seed, pooling, mtp_policy)
 
 
 def spin_state_bytes(cfg: SpinConfig) -> int:

@@ -6,7 +6,8 @@
 //     x <- I if x is the never-observed sentinel (V: +inf, D: -inf), else
 //     fmaf(alpha, x, beta * I), beta = fl32(1 - alpha).  For speculative rows
 //     the update waits for the accepted length a and replays rows 0..a-1 in
-//     order (SPIN digest, arXiv深度剖析: prefix-valid replay).
+//     order (SPIN digest, arXiv深度剖析: prefix-valid replay); under the
+//     row-0 MTP policy row 0 alone is applied (SPIN listing, Table 7).
 //
 // Parallel layout: one warp per block j of a request.  The vertical state of
 // a slot is owned by the slot (its rows run in order inside one thread); the
@@ -58,6 +59,8 @@ cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t s
   return cudaGetLastError();
 }
 
+// R: the most rows one update applies (the call's rows, or 1 under the row-0
+// policy); a.rows, the call's rows, bounds the context and accepted lengths.
 template <int R>
 __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
   pdl_enter();
@@ -69,14 +72,15 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
     const int q = (int)(wid / L.max_blocks);
     const int64_t j = wid % L.max_blocks;
     const int64_t ctx = a.ctx_len[q];
-    if (ctx < 1 || ctx + R - 1 > L.max_slots) continue;
+    if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) continue;
     int acc = R;
     if (a.accepted) {
       acc = a.accepted[q];
-      if (acc < 1 || acc > R) {
+      if (acc < 1 || acc > a.rows) {
         if (j == 0 && lane == 0) raise_error(a.err, ERR_ACCEPTED, q, (uint32_t)acc);
         continue;
       }
+      acc = min(acc, R);
     }
     const int64_t p0 = ctx - 1;
     const int64_t n_last = row_blocks(ctx, acc - 1, L.b);
@@ -156,7 +160,7 @@ cudaError_t launch_ema_update(const EmaArgs& a, cudaStream_t s) {
   int64_t blocks = (warps + 7) / 8;
   if (blocks > 148 * 64) blocks = 148 * 64;
   PdlLaunch l(dim3((unsigned)blocks), dim3(256), 0, s);
-  switch (a.rows) {
+  switch (a.row0 ? 1 : a.rows) {
     case 1: return cudaLaunchKernelEx(&l.cfg, k_ema_update<1>, a);
     case 2: return cudaLaunchKernelEx(&l.cfg, k_ema_update<2>, a);
     case 3: return cudaLaunchKernelEx(&l.cfg, k_ema_update<3>, a);

@@ -28,7 +28,11 @@
 //               quarter its warp may access (lanes 32*(warp%4) ..), hands
 //               the accumulator back as soon as its last columns are in
 //               registers, applies ReLU, head weights and the scale, and
-//               stores the score and the fused EMA update
+//               stores the score and the fused EMA update.  With one CTA
+//               per SM (N > 128) there are four groups; for several query
+//               rows two groups share each tile, one taking the even rows and
+//               the other the odd ones, so an accumulator is read out in half
+//               the time
 // Pipelines: key stages freed as soon as the MMAs have read them (6 per CTA
 // at N = 64, 8 with one CTA per SM); a 16-slot ring of tile info freed by the
 // epilogue; 1 query buffer with two CTAs per SM (2 with one); 4 TMEM
@@ -338,6 +342,10 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   const Ctl ctl{abort_flag, a.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool fused = a.V != nullptr;
+  // With four groups and several rows, two groups share a tile, each taking
+  // every other row: the accumulator (two fit TMEM at N > 128) is read in half
+  // the time, so the MMA waits half as long for it.
+  const int share = (kEpiGroups == 4 && a.rows >= 2) ? 2 : 1;  // groups per tile
 
   // ---- tile prefix over requests (all threads: one load pair each, block
   // scan), barriers ------------------------------------------------------
@@ -367,13 +375,13 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     }
     for (int s = 0; s < kAuxSlots; ++s) {
       mbar_init(B.xf(s), 1);  // the producer's arrive after writing the tile info
-      mbar_init(B.xe(s), 4);  // the four epilogue warps of the group that owns the tile
+      mbar_init(B.xe(s), 4 * share);  // the epilogue warps of the groups that own the tile
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(B.qf(i), 1);
       mbar_init(B.qe(i), 1);
     }
-    for (int i = 0; i < nacc; ++i) mbar_init(B.ae(i), 4);  // the four warps of the group that owns the tile
+    for (int i = 0; i < nacc; ++i) mbar_init(B.ae(i), 4 * share);  // the warps of the groups that own the tile
     mbar_init(B.done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -521,7 +529,9 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   } else {
     // ======================= epilogue (warps 2..9) =======================
     const int ew = warp - 2;              // 0 .. 4*kEpiGroups-1
-    const int group = ew >> 2;
+    const int tgroups = kEpiGroups / share;  // tiles in the epilogue at once
+    const int group = ew / (4 * share);      // tile group: tiles group, group + tgroups, ...
+    const int sub = (ew >> 2) % share;       // rows sub, sub + share, ... of the tile
     const int quarter = warp & 3;         // TMEM lanes this warp may access
     const int m = quarter * 32 + lane;    // accumulator row = tile token
     const int pg_idx = m >> 6, tok = m & 63;
@@ -554,9 +564,9 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     };
     Pre nx;
     bool alive_ = group < n_local && prefetch(group, nx);
-    for (int i = group; alive_ && i < n_local; i += kEpiGroups) {
+    for (int i = group; alive_ && i < n_local; i += tgroups) {
       const Pre cur = nx;
-      if (i + kEpiGroups < n_local && !prefetch(i + kEpiGroups, nx)) break;
+      if (i + tgroups < n_local && !prefetch(i + tgroups, nx)) break;
       const int xs = i % kAuxSlots, acc = i % nacc, stage = i % stages;
       const uint32_t phase = (uint32_t)(i / stages) & 1u;
       if (cur.q != cur_q) {
@@ -571,14 +581,14 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       if (!__all_sync(0xffffffffu, wait_parity(B.e(stage), phase, ctl))) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
-      for (int r = 0; r < a.rows; ++r) {
+      for (int r = sub; r < a.rows; r += share) {
         float part[4] = {0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < L.H; c += 32) {
           uint32_t v[32];
           tmem_ld16(trow + (uint32_t)(r * L.H + c), *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           if (c + 16 < L.H) tmem_ld16(trow + (uint32_t)(r * L.H + c + 16), *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
           tmem_wait_ld();
-          if (r == a.rows - 1 && c + 32 >= L.H) {
+          if (r + share >= a.rows && c + 32 >= L.H) {
             // last accumulator columns are in registers: hand the accumulator
             // (and the tile-info slot, read a tile ago) back before the math
             tc_fence_before();

@@ -9,6 +9,9 @@
 //     of it goes to uniformly random unkept blocks (SPIN digest, arXiv深度剖析;
 //     SPIN listing, Figure 4); each row's top (B_r - n_exp) blocks are unioned
 //     (SPIN listing, Table 7, "Row-local union").  Ties: lower block index.
+//     The row-0 MTP policy (same table) predicts with row 0 alone, keeps the
+//     blocks past row 0's range (the drafts' new keys) and draws the
+//     exploration among row 0's unkept blocks.
 #include <cooperative_groups.h>
 
 #include "spin_internal.cuh"
@@ -34,7 +37,7 @@ __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
   // a0 rides along when asked: the first nvec warp tasks quantise the
   // (request, row, head) query vectors; this kernel is bound by HBM, so they
   // cost next to nothing and the select kernel that follows is spared them
-  const int64_t nvec = a.q8 ? (int64_t)L.Q * R * L.H : 0;
+  const int64_t nvec = a.q8 ? (int64_t)L.Q * a.rows * L.H : 0;
   for (int64_t wid0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
        wid0 < nvec + (int64_t)L.Q * chunks; wid0 += nwarps) {
     if (wid0 < nvec) {
@@ -158,7 +161,7 @@ cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
         : a.pooling == SPIN_POOL_TOP4 ? k_predict_pool<R, SPIN_POOL_TOP4> \
                                       : k_predict_pool<R, SPIN_POOL_MAX>; \
     break;
-  switch (a.rows) {
+  switch (a.mtp_row0 ? 1 : a.rows) {  // R: the rows whose block scores are needed
     SPIN_PREDICT_CASE(1)
     SPIN_PREDICT_CASE(2)
     SPIN_PREDICT_CASE(3)
@@ -390,7 +393,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   } else {
     const int64_t n0 = row_blocks(ctx, 0, L.b);
     const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
-    for (int r = 0; r < a.rows; ++r) {
+    for (int r = 0; r < (a.mtp_row0 ? 1 : a.rows); ++r) {
       const int n = (int)row_blocks(ctx, r, L.b);
       const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
       const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride;
@@ -417,6 +420,10 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
         radix_select_desc(keys, n, all, (uint32_t)n_pred, sh, &T, &eq);
         mark_selected(keys, n, all, T, eq, m, 1, sh);
       }
+    }
+    if (a.mtp_row0) {  // the drafts' new blocks
+      for (int j = (int)n0 + threadIdx.x; j < n_last; j += blockDim.x) m[j] = 1;
+      __syncthreads();
     }
     // exploration among the unkept blocks of the last row's range
     auto cand = [m](int j) { return m[j] == 0; };
@@ -610,7 +617,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
     const int64_t n0 = row_blocks(ctx, 0, L.b);
     const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
     auto all = [](int) { return true; };
-    for (int r = 0; r < a.rows; ++r) {
+    for (int r = 0; r < (a.mtp_row0 ? 1 : a.rows); ++r) {
       const int n = (int)row_blocks(ctx, r, L.b);
       const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
       const int hi = max(0, min(j1, n) - j0);  // this rank's blocks visible to row r
@@ -637,6 +644,10 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
         cl_radix_select_desc(keys, hi, all, (uint32_t)n_pred, sh, sc, &T, &eq);
         cl_mark_selected(keys, hi, all, T, eq, m, 1, sh, sc, r);  // slots 0..3: one per row
       }
+    }
+    if (a.mtp_row0) {  // the drafts' new blocks in this rank's range
+      for (int i = max(0, (int)n0 - j0) + threadIdx.x; i < nl; i += blockDim.x) m[i] = 1;
+      __syncthreads();
     }
     // exploration among the unkept blocks of the last row's range
     int c = 0;

@@ -65,6 +65,7 @@ bool valid_config(const spin_config* c) {
   if (!(c->gamma >= 0.0f && c->gamma <= 1.0f)) return false;
   if (!(c->target_sparsity >= 0.0f && c->target_sparsity < 1.0f)) return false;
   if (c->pooling < SPIN_POOL_MAX || c->pooling > SPIN_POOL_TOP4) return false;
+  if (c->mtp_policy < SPIN_MTP_UNION_PREFIX || c->mtp_policy > SPIN_MTP_ROW0) return false;
   const int64_t max_blocks = (c->max_slots + (int64_t)b - 1) / b;
   if (max_blocks > kMaxBlocksSelect) return false;
   // top-k: bitmap of one (request, row) plus the candidate area on chip
@@ -134,6 +135,7 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   a.layer = layer;
   a.rows = rows;
   a.pooling = st->cfg.pooling;
+  a.mtp_row0 = st->cfg.mtp_policy == SPIN_MTP_ROW0 && rows > 1;
   a.step = step < 0 ? 0 : step;
   a.step_dev = step == SPIN_STEP_DEVICE ? st->step_dev : nullptr;
   a.sparsity = st->sparsity[layer];
@@ -468,6 +470,7 @@ spin_status spin_ema_update(spin_state st, int layer, int rows, const float* sco
   EmaArgs a;
   a.lay = st->lay;
   a.rows = rows;
+  a.row0 = st->cfg.mtp_policy == SPIN_MTP_ROW0 && rows > 1;
   a.scores = scores_dev;
   a.mask = mask_dev;
   a.ctx_len = ctx_len_dev;

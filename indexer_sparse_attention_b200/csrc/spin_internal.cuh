@@ -215,6 +215,7 @@ struct StepArgs {
   int64_t step;
   const int64_t* step_dev;  // non-null: the step is read from the state's counter
   int pooling;              // spin_pooling: block reduction of the predicted scores
+  int mtp_row0;             // SPIN_MTP_ROW0 with rows > 1: row 0 alone predicts
   float sparsity, gamma, alpha;
   uint64_t seed;
   const int32_t* ctx_len;
@@ -299,6 +300,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 struct EmaArgs {
   Layout lay;
   int rows;
+  int row0;           // SPIN_MTP_ROW0: row 0's scores alone update the state
   const float* scores;
   const uint8_t* mask;
   const int32_t* ctx_len;

@@ -37,7 +37,8 @@ class Harness:
         cfg = isa.make_config(num_layers=wl.layers, num_requests=wl.requests, max_slots=wl.max_slots,
                               block_size=wl.b, num_heads=wl.H, head_dim=wl.d, topk=wl.topk, max_rows=wl.rows,
                               key_fp8=wl.key_fp8, q_bf16=wl.q_bf16, alpha=wl.alpha, gamma=wl.gamma,
-                              target_sparsity=wl.sparsity, seed=wl.seed, pooling=wl.pooling)
+                              target_sparsity=wl.sparsity, seed=wl.seed, pooling=wl.pooling,
+                              mtp_policy=wl.mtp_policy)
         self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
         isa.spin_set_score_kernel(self.st, score_kernel)
@@ -111,10 +112,11 @@ class Harness:
         s = float(np.float32(self.sparsity[layer]))
         if s > 0:
             S_gpu = self.st.block_scores()[q, :rows, :nstride].cpu().numpy()
-            for r in range(rows):
+            predicting = 1 if wl.mtp_policy == oracle.MTP_ROW0 else rows   # rows whose scores are computed
+            for r in range(predicting):
                 n = oracle.num_blocks(ctx_len, r, wl.b)
                 assert np.array_equal(S_gpu[r, :n], S_ref[r, :n]), f"block scores differ q={q} r={r}"
-        mask_ref = oracle.select(S_ref, ctx_len, rows, wl.b, s, wl.gamma, wl.seed, q, layer, step)
+        mask_ref = oracle.select(S_ref, ctx_len, rows, wl.b, s, wl.gamma, wl.seed, q, layer, step, wl.mtp_policy)
         mask_gpu = self.mask[q].cpu().numpy()
         assert np.array_equal(mask_gpu, mask_ref), f"mask differs q={q}: {np.nonzero(mask_gpu != mask_ref)[0][:10]}"
         keys, ks, ident = self.pages_of(layer, q)
@@ -152,7 +154,8 @@ class Harness:
             t_ref = oracle.topk_row(row64, mask_ref, ctx_len, r, wl.b, wl.topk)
             assert np.array_equal(topk_gpu[r], t_ref), f"top-k differs q={q} r={r}"
         V1, D1 = V0.copy(), D0.copy()
-        oracle.ema_update(V1, D1, gpu_scores.astype(np.float32), mask_ref, ctx_len, accepted, wl.b, wl.alpha)
+        oracle.ema_update(V1, D1, gpu_scores.astype(np.float32), mask_ref, ctx_len,
+                          oracle.update_rows(wl.mtp_policy, accepted), wl.b, wl.alpha)
         Vg, Dg = self.st.ema(layer)
         assert np.array_equal(Vg[q].cpu().numpy().view(np.uint32), V1.view(np.uint32)), f"V differs q={q}"
         assert np.array_equal(Dg[q].cpu().numpy().view(np.uint32), D1.view(np.uint32)), f"D differs q={q}"

@@ -73,6 +73,7 @@ def test_state_bytes_matches_documented_layout(lib, over):
 @pytest.mark.parametrize("over", [{"block_size": 48}, {"block_size": 8}, {"max_rows": 5}, {"max_rows": 0},
                                   {"target_sparsity": 1.0}, {"target_sparsity": -0.1}, {"gamma": 1.5},
                                   {"num_requests": 0}, {"key_fp8": False, "q_bf16": True}, {"pooling": 3},
+                                  {"mtp_policy": 2}, {"mtp_policy": -1},
                                   {"max_slots": 64 * 50000}, {"alpha": float("nan")}])
 def test_invalid_configs_rejected(lib, over):
     assert isa.spin_state_bytes(_cfg(**over)) == 0

@@ -24,10 +24,11 @@ def _built():
     assert torch.cuda.is_available()
 
 
-def make_state(Q=3, max_slots=8192 + 64, R=1, H=64, d=128, k=256, fp8=True, s=0.5, g=0.05, seed=7, layers=1, b=64):
+def make_state(Q=3, max_slots=8192 + 64, R=1, H=64, d=128, k=256, fp8=True, s=0.5, g=0.05, seed=7, layers=1, b=64,
+               mtp_policy=isa.SPIN_MTP_UNION_PREFIX):
     cfg = isa.make_config(num_layers=layers, num_requests=Q, max_slots=max_slots, block_size=b, num_heads=H,
                           head_dim=d, topk=k, max_rows=R, key_fp8=fp8, q_bf16=fp8, alpha=0.9, gamma=g,
-                          target_sparsity=s, seed=seed)
+                          target_sparsity=s, seed=seed, mtp_policy=mtp_policy)
     return isa.SpinState(cfg)
 
 
@@ -336,6 +337,37 @@ def test_select_cluster_paths_bit_exact(R, s, g):
         for q in range(4):
             S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, 64, st.mask_stride)
             m_ref = oracle.select(S_ref, int(ctx[q]), R, 64, s, g, 7, q, 0, step)
+            assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
+
+
+@pytest.mark.parametrize("R", [2, 4])
+@pytest.mark.parametrize("max_slots", [8192 + 64, 1024 * 1024 + 64])
+def test_mtp_row0_select_bit_exact(R, max_slots):
+    """Row-0 sharing: row 0's block scores, its predicted set, the drafts'
+    new blocks kept and the exploration among row 0's unkept blocks, bit
+    for bit, in the one-CTA select and (1M slots) the cluster select."""
+    rng = np.random.default_rng(R * 7 + max_slots % 97)
+    st = make_state(Q=4, max_slots=max_slots, R=R, s=0.5, g=0.1, k=2048, mtp_policy=isa.SPIN_MTP_ROW0)
+    V, D = st.ema(0)
+    v = rng.integers(0, 4, V.shape).astype(np.float32)    # many equal block scores
+    v[:, -3000:] = np.inf
+    V.copy_(torch.from_numpy(v))
+    d = rng.standard_normal(D.shape).astype(np.float32)
+    d[rng.random(D.shape) < 0.5] = -np.inf
+    D.copy_(torch.from_numpy(d))
+    top = max_slots - 64 - R + 1
+    ctx = np.array([1, top, top // 3 + 37, 64 * (top // 200)], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    for step in [0, 5]:
+        isa.spin_predict_select(st, 0, R, step, ctx_t, mask)
+        assert isa.spin_get_error(st)[0] == 0
+        S_gpu = st.block_scores().cpu().numpy()
+        for q in range(4):
+            S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, 64, st.mask_stride)
+            n0 = oracle.num_blocks(int(ctx[q]), 0, 64)
+            assert np.array_equal(S_gpu[q, 0, :n0].view(np.uint32), S_ref[0, :n0].view(np.uint32)), (q, step)
+            m_ref = oracle.select(S_ref, int(ctx[q]), R, 64, 0.5, 0.1, 7, q, 0, step, oracle.MTP_ROW0)
             assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
 
 

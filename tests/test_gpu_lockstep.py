@@ -79,6 +79,23 @@ def test_mtp_rows_union_and_prefix_valid_replay():
     assert max(realized) <= 0.4 + 1e-9                      # union only adds blocks
 
 
+@pytest.mark.parametrize("defer", [True, False])
+def test_mtp_row0_sharing_and_row0_update(defer):
+    """The baseline MTP policy in lock step: row 0's mask for every row and
+    the EMA update from row 0's scores alone, with deferred accepted lengths
+    and with the update inside the decode step."""
+    wl = workloads.config(3, requests=5, ctx0=(8192, 8190, 64 * 30 + 62, 4000, 129), steps=6,
+                          mtp_policy=isa.SPIN_MTP_ROW0)
+    h = Harness(wl)
+    bootstrap(h)
+    acc = workloads.accepted_lengths(wl, wl.steps).numpy()
+    realized = []
+    for t in range(1, wl.steps):
+        res = h.run_step(0, accepted=acc[t] if defer else None, check=range(5), defer=defer)
+        realized += [1 - r["kept"] / r["n"] for r in res.values()]
+    assert max(realized) <= 0.4 + 1e-9
+
+
 def test_multilayer_per_layer_budget():
     """Ragged long-context workload, scaled: warm-up at uniform 50% with a
     shadow full indexer measuring miss on the GPU, then per-layer budgets."""

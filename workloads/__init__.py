@@ -57,6 +57,7 @@ class Workload:
     accept_probs: Optional[Sequence[float]] = None  # P(a = 1..rows)
     warmup_steps: int = 0         # config with a per-layer budget: uniform-sparsity warm-up steps
     pooling: int = 0              # block reduction of the predicted scores: 0 max, 1 mean, 2 top-4
+    mtp_policy: int = 0           # several rows: 0 row-local union + prefix-valid update, 1 row 0 alone
     spare_slots: int = 0          # extra capacity beyond ctx0 + steps * rows
 
     @property
