@@ -125,14 +125,23 @@ def job_rows_per_s(rows_per_rank: int, world: int, max_ms: float) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi samples (every 50 ms) of this GPU while the timed region runs."""
+    """SM clock, utilisation and clock-event reasons of this GPU, read through
+    NVML from a thread every 5 ms while the timed region runs (one reading at
+    entry and one at exit as well, so a short region still has samples).
+    Falls back to an nvidia-smi process when NVML cannot be opened.  Reads
+    only; changes no setting."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    # clock-event reason bits (NVML): name -> mask
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
 
     def __init__(self, device_index: int):
         self.proc = None
+        self.thread = None
+        self.rows = []
         self.path = tempfile.mktemp(suffix=".csv")
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -140,8 +149,41 @@ class ClockSampler:
         except Exception:
             ident = str(device_index)
         self.ident = ident
+        self.nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(ident)
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+
+    def _read(self):
+        n, h = self.nvml, self.handle
+        try:
+            reasons = n.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            reasons = n.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        return (float(n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)),
+                float(n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)),
+                float(n.nvmlDeviceGetUtilizationRates(h).gpu), int(reasons))
+
+    def _loop(self):
+        import time
+        while not self.stop:
+            try:
+                self.rows.append(self._read())
+            except Exception:
+                return
+            time.sleep(0.005)
 
     def __enter__(self):
+        if self.nvml is not None:
+            import threading
+            self.stop = False
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return self
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.ident}", f"--query-gpu={self.FIELDS}",
@@ -152,6 +194,13 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            try:
+                self.rows.append(self._read())
+            except Exception:
+                pass
+            self.stop = True
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -161,6 +210,15 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self):
+        if self.nvml is not None:
+            if not self.rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+            sm = np.array([r[0] for r in self.rows])
+            util = np.array([r[2] for r in self.rows])
+            loaded = sm[util > 0] if np.any(util > 0) else sm
+            reasons = sorted({k for r in self.rows for k, bit in self.REASONS.items() if r[3] & bit})
+            return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": self.rows[0][1], "reasons": reasons,
+                    "samples": len(self.rows), "samples_under_load": int(loaded.size), "source": "nvml, 5 ms"}
         rows = []
         try:
             for line in open(self.path):
@@ -178,7 +236,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
         return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows), "samples_under_load": int(loaded.size)}
+                "samples": len(rows), "samples_under_load": int(loaded.size), "source": "nvidia-smi, 50 ms"}
 
 
 # ---------------------------------------------------------------------------

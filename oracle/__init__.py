@@ -83,6 +83,11 @@ def _load():
             lib.orc_ema_beta.restype = ctypes.c_float
             lib.orc_ema_update.argtypes = [_f32p, _f32p, _f32p, _u8p, _i64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_float, _i64]
+            lib.orc_slot_prediction.argtypes = [_f32p, _f32p, _i64, ctypes.c_int, _i64, _f32p]
+            lib.orc_random_prediction.argtypes = [_u64, ctypes.c_uint32, ctypes.c_uint32, _u64, _i64, ctypes.c_int,
+                                                  _i64, _f32p]
+            lib.orc_pearson.argtypes = [_f32p, _f32p, _i64]
+            lib.orc_pearson.restype = ctypes.c_double
             lib.orc_miss_fraction.argtypes = [_i32p, ctypes.c_int, _u8p, ctypes.c_int]
             lib.orc_miss_fraction.restype = ctypes.c_double
             lib.orc_layer_sparsity.argtypes = [_f64p, _f64p, _f64p, ctypes.c_int, ctypes.c_double, _f64p]
@@ -247,6 +252,45 @@ def ema_update(V: np.ndarray, D: np.ndarray, scores32: np.ndarray, mask, ctx_len
     mask = _c(mask, np.uint8)
     lib.orc_ema_update(_p(V, _f32p), _p(D, _f32p), _p(s32, _f32p), _p(mask, _u8p), ctx_len,
                        accepted, b, float(alpha), s32.shape[1])
+
+
+# --------------------------------------------------------------------------
+# predictor quality (SPIN listing, Table 1)
+# --------------------------------------------------------------------------
+def slot_prediction(V: np.ndarray, D: np.ndarray, ctx_len: int, rows: int, slot_stride: int) -> np.ndarray:
+    """z = max(V_s, D_{p_r - s}) per visible slot, -inf where not finite;
+    [rows, slot_stride], NaN past each row's position."""
+    lib = _load()
+    V = _c(V, np.float32)
+    D = _c(D, np.float32)
+    out = np.full((rows, slot_stride), np.nan, np.float32)
+    lib.orc_slot_prediction(_p(V, _f32p), _p(D, _f32p), ctx_len, rows, slot_stride, _p(out, _f32p))
+    return out
+
+
+def random_prediction(seed: int, request: int, layer: int, step: int, ctx_len: int, rows: int,
+                      slot_stride: int) -> np.ndarray:
+    lib = _load()
+    out = np.full((rows, slot_stride), np.nan, np.float32)
+    lib.orc_random_prediction(seed, request, layer, step, ctx_len, rows, slot_stride, _p(out, _f32p))
+    return out
+
+
+def pearson(x, y) -> float:
+    """Over the entries where both are finite; 0 if fewer than two or constant."""
+    lib = _load()
+    x = _c(x, np.float32)
+    y = _c(y, np.float32)
+    assert x.shape == y.shape
+    return float(lib.orc_pearson(_p(x, _f32p), _p(y, _f32p), x.size))
+
+
+def topk_visible(values_row, ctx_len: int, row: int, k: int) -> np.ndarray:
+    """Top-k (value desc, lower slot first) over every visible slot of a row:
+    the token top-k with all blocks kept, block size 1."""
+    v = np.asarray(values_row, np.float64)
+    p = ctx_len - 1 + row
+    return topk_row(v, np.ones(p + 1, np.uint8), ctx_len, row, 1, k)
 
 
 def miss_fraction(full_topk, mask, b: int) -> float:

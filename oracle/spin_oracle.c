@@ -475,6 +475,69 @@ ORC_API void orc_ema_update(float* V, float* D, const float* scores32, const uin
 }
 
 /* ------------------------------------------------------------------------ */
+/* Predictor quality ([listing] Table 1: Pearson correlation and top-k recall */
+/* of an indexer prediction against the indexer's scores, for a random       */
+/* baseline, the previous layer and the previous iteration).                 */
+/*                                                                          */
+/* orc_slot_prediction: the SPIN predictor before block pooling, z_{r,s} =   */
+/* max(V_s, D_{p_r - s}) for s <= p_r ([radio] "Title and authors"), and     */
+/* -inf where z is not finite: a slot no step has scored carries the +inf    */
+/* sentinel and no prediction.  out is [rows][slot_stride]; slots past p_r   */
+/* are not written.                                                          */
+/* ------------------------------------------------------------------------ */
+ORC_API void orc_slot_prediction(const float* V, const float* D, int64_t ctx_len, int rows,
+                                 int64_t slot_stride, float* out) {
+  for (int r = 0; r < rows; ++r) {
+    int64_t p = pos_of_row(ctx_len, r);
+    for (int64_t s = 0; s <= p; ++s) {
+      float z = V[s] > D[p - s] ? V[s] : D[p - s];
+      out[(int64_t)r * slot_stride + s] = isfinite(z) ? z : -INFINITY;
+    }
+  }
+}
+
+/* The random baseline: an independent uniform value per slot in [0, 1), the */
+/* top 24 bits of word 0 of Philox4x32-10 at counter (slot, request, layer,  */
+/* step mod 2^32) and key (seed low, seed high) -- the exploration key with  */
+/* the slot in place of the block -- times 2^-24; the same for every row.    */
+ORC_API void orc_random_prediction(uint64_t seed, uint32_t request, uint32_t layer, uint64_t step,
+                                   int64_t ctx_len, int rows, int64_t slot_stride, float* out) {
+  for (int r = 0; r < rows; ++r) {
+    int64_t p = pos_of_row(ctx_len, r);
+    for (int64_t s = 0; s <= p; ++s) {
+      uint32_t w = orc_explore_key(seed, (uint32_t)s, request, layer, step);
+      out[(int64_t)r * slot_stride + s] = (float)((double)(w >> 8) / 16777216.0);
+    }
+  }
+}
+
+/* Pearson correlation of x and y over the entries where both are finite,   */
+/* in double, two passes: the means, then the centred sums.  0 when fewer    */
+/* than two pairs remain or either side is constant on them.                 */
+ORC_API double orc_pearson(const float* x, const float* y, int64_t n) {
+  int64_t m = 0;
+  double sx = 0.0, sy = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    if (!isfinite(x[i]) || !isfinite(y[i])) continue;
+    sx += (double)x[i];
+    sy += (double)y[i];
+    ++m;
+  }
+  if (m < 2) return 0.0;
+  double mx = sx / (double)m, my = sy / (double)m;
+  double sxy = 0.0, sxx = 0.0, syy = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    if (!isfinite(x[i]) || !isfinite(y[i])) continue;
+    double dx = (double)x[i] - mx, dy = (double)y[i] - my;
+    sxy += dx * dy;
+    sxx += dx * dx;
+    syy += dy * dy;
+  }
+  if (sxx == 0.0 || syy == 0.0) return 0.0;
+  return sxy / sqrt(sxx * syy);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Fidelity metric: the fraction of the full indexer's top-k tokens that     */
 /* fall in skipped blocks ([listing] Table 5 caption: mean / p99 miss over   */
 /* eligible sparse decode rows).  full_topk holds k slots padded with -1.    */

@@ -611,3 +611,75 @@ def test_pool_mean_sums_runs_of_eight_then_pairwise(oracle_lib):
     V2 = np.zeros(b, np.float32)
     V2[0], V2[1], V2[8] = 2.0 ** 60, 256.0, -(2.0 ** 60)
     assert oracle_lib.predict_pool(V2, D, b, 1, b, 1, oracle_lib.POOL_MEAN)[0, 0] == np.float32(256.0 / b)
+
+
+# ----------------------------------------------------------------------------
+# predictor quality (SPIN listing, Table 1)
+# ----------------------------------------------------------------------------
+def test_pearson_matches_numpy_corrcoef_on_finite_pairs(oracle_lib):
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal(5000).astype(np.float32)
+    y = (0.3 * x + rng.standard_normal(5000)).astype(np.float32)
+    x[rng.integers(0, 5000, 40)] = -np.inf
+    y[rng.integers(0, 5000, 40)] = np.nan
+    ok = np.isfinite(x) & np.isfinite(y)
+    ref = np.corrcoef(x[ok].astype(np.float64), y[ok].astype(np.float64))[0, 1]
+    assert abs(oracle_lib.pearson(x, y) - ref) < 1e-12
+
+
+def test_pearson_affine_constant_and_short(oracle_lib):
+    x = np.arange(100, dtype=np.float32)
+    assert abs(oracle_lib.pearson(x, 3 * x + 1) - 1.0) < 1e-12
+    assert abs(oracle_lib.pearson(x, -0.5 * x + 7) + 1.0) < 1e-12
+    assert oracle_lib.pearson(x, np.full(100, 2.0, np.float32)) == 0.0
+    one = np.full(100, -np.inf, np.float32)
+    one[5] = 1.0
+    assert oracle_lib.pearson(one, x) == 0.0                  # a single finite pair
+
+
+@pytest.mark.parametrize("ctx_len,rows,b", [(37, 1, 8), (130, 4, 16), (64 * 9 + 1, 3, 64)])
+def test_slot_prediction_pools_to_block_scores(oracle_lib, ctx_len, rows, b):
+    # The block max-pool of the slot prediction is the predicted block score
+    # (pinned above against V's blockwise maximum and the diagonal one-hot);
+    # a slot no step has scored has no prediction.
+    rng = np.random.default_rng(ctx_len)
+    n_stride = -(-(ctx_len + rows) // b) + 1
+    V = rng.standard_normal(n_stride * b).astype(np.float32)
+    D = rng.standard_normal(n_stride * b).astype(np.float32)
+    D[rng.random(D.size) < 0.3] = -np.inf
+    V[ctx_len - 1] = np.inf                                   # the newest slot: never scored
+    z = oracle_lib.slot_prediction(V, D, ctx_len, rows, n_stride * b)
+    S = oracle_lib.predict_pool(V, D, ctx_len, rows, b, n_stride)
+    for r in range(rows):
+        p = ctx_len - 1 + r
+        assert z[r, ctx_len - 1] == -np.inf
+        assert np.all(np.isfinite(np.delete(z[r, : p + 1], ctx_len - 1)))   # V finite elsewhere
+        for j in range(-(-(p + 1) // b)):
+            blk = z[r, j * b: min((j + 1) * b, p + 1)]
+            if ctx_len - 1 in range(j * b, min((j + 1) * b, p + 1)):
+                assert S[r, j] == np.inf                      # the sentinel keeps the block
+            else:
+                assert S[r, j] == blk.max()
+
+
+def test_random_prediction_uniform_uncorrelated_and_table1_recall(oracle_lib):
+    # The random baseline of Table 1 (thelatestinai listing): correlation 0 and
+    # top-k recall k / L in expectation; the pages print 0.022 at AA-LCR's 94k.
+    pages = json.load(open(GOLDEN))["table1_random_recall"]
+    L, k = pages["aa_lcr"]["context_tokens"], pages["k_reading"]
+    assert round(k / L, 3) == pages["aa_lcr"]["recall"]
+    rng = np.random.default_rng(41)
+    scores = rng.standard_normal(L).astype(np.float32)
+    true_top = set(oracle_lib.topk_visible(scores, L, 0, k).tolist())
+    recalls, corr = [], []
+    for step in range(60):
+        u = oracle_lib.random_prediction(5, 1, 2, step, L, 1, L)[0]
+        assert np.all((u >= 0) & (u < 1))
+        corr.append(oracle_lib.pearson(u, scores))
+        recalls.append(len(true_top & set(oracle_lib.topk_visible(u, L, 0, k).tolist())) / k)
+    sigma = math.sqrt(k * (1 - k / L) * (1 - k / L)) / k / math.sqrt(len(recalls))
+    assert abs(np.mean(recalls) - k / L) < 4 * sigma
+    assert abs(np.mean(corr)) < 4 / math.sqrt(L * len(corr))
+    hist = np.histogram(oracle_lib.random_prediction(5, 1, 2, 0, L, 1, L)[0], bins=50, range=(0, 1))[0]
+    e = L / 50
+    assert float(((hist - e) ** 2 / e).sum()) < 3 * 49       # chi-square, 49 dof
