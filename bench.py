@@ -49,7 +49,7 @@ SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write 
 # per kept slot, from one ncu capture of the kernel on 16 requests at 512K, 50% sparsity,
 # fused EMA (traffic grows with kept slots: each is read once), valid for the kernel
 # source with this hash prefix
-SCORE_TRAFFIC = {"src_sha256_16": "e7025aa9a2c3edc6", "bytes_per_kept_slot": 151.15,
+SCORE_TRAFFIC = {"src_sha256_16": "3cac9e62802aec1b", "bytes_per_kept_slot": 151.14,
                  "sources": ("indexer_sparse_attention_b200/csrc/k_score_tc.cu",
                              "indexer_sparse_attention_b200/csrc/spin_internal.cuh")}
 
@@ -71,9 +71,11 @@ def parse():
                    help="block reduction of the predicted scores (max is the method's)")
     p.add_argument("--mtp-policy", choices=list(MTP_POLICIES), default="union-prefix",
                    help="several query rows: row-local union + prefix-valid update (the method's) or row 0 alone")
-    p.add_argument("--ablation", choices=["pooling", "mtp"], default=None,
+    p.add_argument("--ablation", choices=["pooling", "mtp", "predictors"], default=None,
                    help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities; "
-                        "mtp: p99 miss vs realized sparsity of the two MTP policies on the 4-row workload")
+                        "mtp: p99 miss vs realized sparsity of the two MTP policies on the 4-row workload; "
+                        "predictors: Pearson correlation and top-k recall of the random, previous-layer, "
+                        "previous-iteration and SPIN predictors")
     return p.parse_args()
 
 
@@ -934,6 +936,88 @@ def mtp_ablation(args, world, rank, local):
                     "workload's distribution, the same for both policies"}
 
 
+# ---------------------------------------------------------------------------
+# Predictor-quality profile (SPIN listing, Table 1: Pearson correlation and
+# top-k recall per predictor, averaged over layers and decode iterations)
+# ---------------------------------------------------------------------------
+def predictor_profile(args, world, rank, local):
+    """An 8-layer workload with two prompts of Table 1's lengths (94K and
+    9.7K slots) decoded with every block kept.  Before each step of each
+    layer, four predictors of that step's indexer scores are taken: the
+    random baseline, the previous layer's scores of the same step, the
+    previous step's scores of the same layer, and SPIN's z = max(V, D).  Per
+    prompt, the Pearson correlation and the top-k recall of each, averaged
+    over layers and steps 1..T.  Every figure comes from the library's
+    kernels.  One JSON line."""
+    import indexer_sparse_attention_b200 as isa
+    from indexer_sparse_attention_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    isa.load()
+    device = torch.device("cuda", local if world > 1 else 0)
+    T = max(args.steps, 2)
+    total = T + 1
+    base = workloads.config(WORKLOADS["ragged-8Lx8-256K-1M"])
+    wl = workloads.config(WORKLOADS["ragged-8Lx8-256K-1M"], requests=2, ctx0=(94_000, 9_700), steps=total,
+                          seed=base.seed + 1000 * rank, spare_slots=8)
+    run = WorkloadRun(wl, device, total)
+    Ly, Q, R = wl.layers, wl.requests, wl.rows
+    st = run.st
+    run.set_sparsity([0.0] * Ly)
+    allk = torch.ones_like(run.masks[0])
+    names = ("random", "prev_layer", "prev_iter", "spin_ema")
+    corr = {n: [[] for _ in range(Q)] for n in names}
+    recall = {n: [[] for _ in range(Q)] for n in names}
+    r_out = torch.zeros((Q, R), dtype=torch.float64, device=device)
+    ov = torch.zeros((Q, R), dtype=torch.int32, device=device)
+    ptop = torch.empty((Q, R, wl.topk), dtype=torch.int32, device=device)
+    prev = [None] * Ly
+    for t in range(total):
+        cur = [None] * Ly
+        ctx = run.ctx[t]
+        vis = (ctx.long() + R - 1).clamp(max=wl.topk).cpu().numpy()     # k entries a top-k can hold
+        for l in range(Ly):
+            preds = {}
+            if t >= 1:
+                preds["spin_ema"] = st.new_scores()
+                isa.spin_slot_prediction(st, l, R, isa.SPIN_PRED_EMA, t, ctx, preds["spin_ema"])
+                preds["random"] = st.new_scores()
+                isa.spin_slot_prediction(st, l, R, isa.SPIN_PRED_RANDOM, t, ctx, preds["random"])
+                preds["prev_iter"] = prev[l]
+                if l > 0:
+                    preds["prev_layer"] = cur[l - 1]
+            sc = st.new_scores()
+            sc.fill_(float("-inf"))
+            c = run.caches[l]
+            q, w = run.qw[t][l]
+            isa.spin_decode_step(st, l, R, t, c.keys, c.kscale if wl.key_fp8 else None, c.block_table, q, w, ctx,
+                                 False, run.masks[l], run.topks[l], sc)
+            for n, pred in preds.items():
+                isa.spin_pearson(st, R, pred, sc, ctx, r_out)
+                isa.spin_topk(st, R, pred, allk, ctx, ptop)
+                isa.spin_topk_overlap(st, R, ptop, run.topks[l], ov)
+                rr, oo = r_out.cpu().numpy(), ov.cpu().numpy()
+                for qq in range(Q):
+                    corr[n][qq].append(float(rr[qq, 0]))
+                    recall[n][qq].append(float(oo[qq, 0]) / float(vis[qq]))
+            cur[l] = sc
+        prev = cur
+    status, word = isa.spin_get_error(st)
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    prompts = {}
+    for qq, L in enumerate(wl.ctx0):
+        prompts[f"{L // 1000}K"] = {n: {"pearson": float(np.mean(corr[n][qq])), "topk_recall": float(np.mean(recall[n][qq])),
+                                        "samples": len(corr[n][qq])} for n in names}
+    return {"ablation": "predictor quality: Pearson correlation and top-k recall of the indexer scores",
+            "unit": "correlation / recall", "config": {"layers": Ly, "prompts_slots": list(wl.ctx0), "steps": T,
+                                                       "topk": wl.topk, "alpha": wl.alpha, "sparsity": 0.0},
+            "results": prompts,
+            "note": "synthetic keys: each layer draws its own keys, planted directions and vertical slots; "
+                    "the layers share only the position pattern of the diagonal band"}
+
+
 def p99_of(values):
     v = np.sort(np.asarray(values, np.float64))
     return float(v[max(int(np.ceil(0.99 * v.size)), 1) - 1]) if v.size else 0.0
@@ -1027,8 +1111,9 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
-        if args.ablation in ("pooling", "mtp"):
-            out = (pooling_ablation if args.ablation == "pooling" else mtp_ablation)(args, world, rank, local)
+        if args.ablation in ("pooling", "mtp", "predictors"):
+            fn = {"pooling": pooling_ablation, "mtp": mtp_ablation, "predictors": predictor_profile}[args.ablation]
+            out = fn(args, world, rank, local)
             if rank == 0:
                 print(json.dumps(out), flush=True)
             return

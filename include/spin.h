@@ -247,6 +247,44 @@ SPIN_API spin_status spin_decode_step(spin_state st, int layer, int rows, int64_
                              const int32_t* ctx_len_dev, int defer_update, uint8_t* mask_dev,
                              int32_t* topk_dev, float* scores_dev, spin_stream_t stream);
 
+/* Predictor-quality profile (SPIN listing, Table 1 compares predictors of the
+ * indexer's scores by Pearson correlation and top-k recall).
+ *
+ * spin_slot_prediction writes one predictor's value for every visible slot
+ * s <= p_r of every request and row: pred_dev [Q][max_rows][slot_stride] fp32
+ * (the scores layout; slots past p_r are not written).
+ *   SPIN_PRED_EMA     the SPIN predictor before block pooling, z = max(V_s,
+ *                     D_{p_r - s}) from the layer's state; -inf where z is not
+ *                     finite (a slot no step has scored has no prediction).
+ *   SPIN_PRED_RANDOM  the random baseline: the top 24 bits of word 0 of
+ *                     Philox4x32-10 at counter (s, request, layer, step mod
+ *                     2^32), key (seed lo, seed hi), times 2^-24 (uniform in
+ *                     [0, 1)), the same for every row; step >= 0 or
+ *                     SPIN_STEP_DEVICE.
+ * The previous iteration's or the previous layer's scores (a scores buffer of
+ * an earlier spin_decode_step) are predictors as they stand.
+ *
+ * spin_pearson: pearson_dev [Q][rows] double, the Pearson correlation of x_dev
+ * and y_dev (both [Q][max_rows][slot_stride] fp32) over the visible slots of
+ * each (request, row) where both are finite, computed in double in two passes
+ * (means, then centred sums) in a fixed order; 0 when fewer than two such
+ * slots remain or either side is constant on them.
+ *
+ * spin_topk_overlap: overlap_dev [Q][rows] int32, the number of slots that two
+ * top-k lists a_dev, b_dev ([Q][rows][k] int32, ascending, -1 padded, as
+ * spin_topk writes them) share.  The top-k recall of a predictor is the
+ * overlap of its top-k (spin_topk of pred_dev with every block kept) with the
+ * indexer's, divided by k.
+ * A ctx_len out of range sets ERR_CTX_LEN in the device error word and leaves
+ * that request's outputs unwritten (prediction) or 0 (correlation). */
+typedef enum { SPIN_PRED_EMA = 0, SPIN_PRED_RANDOM = 1 } spin_predictor;
+SPIN_API spin_status spin_slot_prediction(spin_state st, int layer, int rows, int kind, int64_t step,
+                                 const int32_t* ctx_len_dev, float* pred_dev, spin_stream_t stream);
+SPIN_API spin_status spin_pearson(spin_state st, int rows, const float* x_dev, const float* y_dev,
+                         const int32_t* ctx_len_dev, double* pearson_dev, spin_stream_t stream);
+SPIN_API spin_status spin_topk_overlap(spin_state st, int rows, const int32_t* a_dev, const int32_t* b_dev,
+                              int32_t* overlap_dev, spin_stream_t stream);
+
 /* Miss count of the fidelity metric (SPIN listing, Table 5 caption): for each
  * (request, row), the number of entries of full_topk_dev [Q][rows][k] (a
  * full-indexer top-k, -1 padded) whose block is skipped in mask_dev.

@@ -25,7 +25,8 @@ __all__ = [
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
     "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_set_kernel_timing_mask",
     "SPIN_STEP_DEVICE", "spin_set_step", "spin_advance_step", "SPIN_POOL_MAX", "SPIN_POOL_MEAN", "SPIN_POOL_TOP4",
-    "SPIN_MTP_UNION_PREFIX", "SPIN_MTP_ROW0",
+    "SPIN_MTP_UNION_PREFIX", "SPIN_MTP_ROW0", "SPIN_PRED_EMA", "SPIN_PRED_RANDOM", "spin_slot_prediction",
+    "spin_pearson", "spin_topk_overlap",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +37,7 @@ SPIN_SCORE_AUTO, SPIN_SCORE_SIMT, SPIN_SCORE_TCGEN05 = 0, 1, 2
 SPIN_STEP_DEVICE = -1  # step argument: read the state's device step counter
 SPIN_POOL_MAX, SPIN_POOL_MEAN, SPIN_POOL_TOP4 = 0, 1, 2  # block reduction of the predicted scores
 SPIN_MTP_UNION_PREFIX, SPIN_MTP_ROW0 = 0, 1  # mask / EMA policy for several query rows
+SPIN_PRED_EMA, SPIN_PRED_RANDOM = 0, 1  # slot predictors of the quality profile
 STATUS_NAMES = {0: "SPIN_OK", 1: "SPIN_EINVAL", 2: "SPIN_ENOMEM", 3: "SPIN_ECUDA", 4: "SPIN_ESTATE",
                 5: "SPIN_ETIMEOUT", 6: "SPIN_EDEVICE", 7: "SPIN_EUNSUPPORTED"}
 
@@ -101,6 +103,9 @@ def load():
         "spin_decode_step": (S, [_vp, ctypes.c_int, ctypes.c_int, _i64, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp,
                                  ctypes.c_int, _vp, _vp, _vp, _vp]),
         "spin_miss_count": (S, [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
+        "spin_slot_prediction": (S, [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64, _vp, _vp, _vp]),
+        "spin_pearson": (S, [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
+        "spin_topk_overlap": (S, [_vp, ctypes.c_int, _vp, _vp, _vp, _vp]),
         "spin_allocate_layer_sparsity": (S, [ctypes.c_int, _vp, _vp, _vp, ctypes.c_double, _vp]),
         "spin_get_error": (S, [_vp, _vp, ctypes.POINTER(_u32)]),
         "spin_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -333,6 +338,23 @@ def spin_miss_count(st: SpinState, rows: int, full_topk, mask, missed, total, st
     _check(load().spin_miss_count(st.handle, rows, _dev(full_topk, "full_topk", torch.int32),
                                   _dev(mask, "mask", torch.uint8), _dev(missed, "missed", torch.int32),
                                   _dev(total, "total", torch.int32), _stream(stream)), "spin_miss_count")
+
+
+def spin_slot_prediction(st: SpinState, layer: int, rows: int, kind: int, step: int, ctx_len, pred,
+                         stream=None) -> None:
+    _check(load().spin_slot_prediction(st.handle, layer, rows, kind, step, _dev(ctx_len, "ctx_len", torch.int32),
+                                       _dev(pred, "pred", torch.float32), _stream(stream)), "spin_slot_prediction")
+
+
+def spin_pearson(st: SpinState, rows: int, x, y, ctx_len, out, stream=None) -> None:
+    _check(load().spin_pearson(st.handle, rows, _dev(x, "x", torch.float32), _dev(y, "y", torch.float32),
+                               _dev(ctx_len, "ctx_len", torch.int32), _dev(out, "out", torch.float64),
+                               _stream(stream)), "spin_pearson")
+
+
+def spin_topk_overlap(st: SpinState, rows: int, a, b, out, stream=None) -> None:
+    _check(load().spin_topk_overlap(st.handle, rows, _dev(a, "a", torch.int32), _dev(b, "b", torch.int32),
+                                    _dev(out, "out", torch.int32), _stream(stream)), "spin_topk_overlap")
 
 
 def spin_allocate_layer_sparsity(miss, blocks, lo, s_glob: float):

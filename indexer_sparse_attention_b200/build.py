@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 BUILD_DIR = os.path.join(ROOT, "_build")
 SO = os.path.join(HERE, "libspin.so")
 SOURCES = ["spin_api.cu", "k_select.cu", "k_score_simt.cu", "k_score_tc.cu", "k_topk.cu", "k_ema.cu",
-           "spin_noalloc.cu"]
+           "spin_noalloc.cu", "k_quality.cu"]
 HEADERS = ["spin_internal.cuh", "block_scan.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

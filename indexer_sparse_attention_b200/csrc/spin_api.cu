@@ -529,6 +529,36 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   return SPIN_OK;
 }
 
+spin_status spin_slot_prediction(spin_state st, int layer, int rows, int kind, int64_t step,
+                                 const int32_t* ctx_len_dev, float* pred_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers || check_rows(st, rows) || step < SPIN_STEP_DEVICE ||
+      (kind != SPIN_PRED_EMA && kind != SPIN_PRED_RANDOM) || !ctx_len_dev || !pred_dev)
+    return SPIN_EINVAL;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  cudaStream_t s = (cudaStream_t)stream;
+  return cuda_status(launch_slot_prediction(st->lay, rows, kind, step < 0 ? 0 : step,
+                                            step == SPIN_STEP_DEVICE ? st->step_dev : nullptr, st->cfg.seed, layer,
+                                            ctx_len_dev, st->V + per_layer * layer, st->D + per_layer * layer,
+                                            pred_dev, st->err, s));
+}
+
+spin_status spin_pearson(spin_state st, int rows, const float* x_dev, const float* y_dev,
+                         const int32_t* ctx_len_dev, double* pearson_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (check_rows(st, rows) || !x_dev || !y_dev || !ctx_len_dev || !pearson_dev) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  return cuda_status(launch_pearson(st->lay, rows, x_dev, y_dev, ctx_len_dev, pearson_dev, st->err, s));
+}
+
+spin_status spin_topk_overlap(spin_state st, int rows, const int32_t* a_dev, const int32_t* b_dev,
+                              int32_t* overlap_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (check_rows(st, rows) || !a_dev || !b_dev || !overlap_dev) return SPIN_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  return cuda_status(launch_topk_overlap(st->lay.Q * rows, st->lay.k, a_dev, b_dev, overlap_dev, s));
+}
+
 spin_status spin_miss_count(spin_state st, int rows, const int32_t* full_topk_dev, const uint8_t* mask_dev,
                             int32_t* missed_dev, int32_t* total_dev, spin_stream_t stream) {
   if (!alive(st)) return SPIN_ESTATE;

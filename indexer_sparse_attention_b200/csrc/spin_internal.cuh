@@ -312,6 +312,14 @@ struct EmaArgs {
 };
 cudaError_t launch_ema_update(const EmaArgs& a, cudaStream_t s);
 
+// Predictor-quality profile (k_quality.cu).
+cudaError_t launch_slot_prediction(const Layout& L, int rows, int kind, int64_t step, const int64_t* step_dev,
+                                   uint64_t seed, int layer, const int32_t* ctx_len, const float* V, const float* D,
+                                   float* pred, ErrWord* err, cudaStream_t s);
+cudaError_t launch_pearson(const Layout& L, int rows, const float* x, const float* y, const int32_t* ctx_len,
+                           double* out, ErrWord* err, cudaStream_t s);
+cudaError_t launch_topk_overlap(int pairs, int k, const int32_t* a, const int32_t* b, int32_t* out, cudaStream_t s);
+
 cudaError_t launch_miss_count(const Layout& lay, int rows, const int32_t* full_topk,
                               const uint8_t* mask, int32_t* missed, int32_t* total,
                               cudaStream_t s);
