@@ -475,11 +475,7 @@ def gpu_arm(args, world, rank, local):
         "metric": METRIC, "value": rows_s, "unit": "rows/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3xe4m3->f32 (selection f32, exact)", "data": "synthetic",
-        "config": {"workload": wl.name, "requests_per_gpu": Q, "context_slots": wl.ctx0[0], "block_size": wl.b,
-                   "heads": wl.H, "head_dim": wl.d, "topk": wl.topk, "target_sparsity": args.sparsity,
-                   "gamma": wl.gamma, "pooling": args.pooling,
-                   "parallelism": f"dp{world} (requests sharded, no collective)",
-                   "l2": "inputs larger than L2: 6.4 GB paged FP8 key cache and 0.4 GB EMA state per GPU"},
+        "config": headline_config(wl, Q, args, world),
         "index_key_gbs": key_gbs,
         "key_roofline_frac": key_gbs / peak,
         "roofline": {"bound": "hbm", "kernel": "k_score_tc (paged FP8 indexer + fused EMA)",
@@ -1076,6 +1072,15 @@ def cpu_baseline(sparsity, seconds):
                       f"after an untimed all-keep bootstrap; fp64 scores, OpenMP over blocks; {dt:.1f} s"}
 
 
+def headline_config(wl, Q, args, world):
+    """The serving workload's config, the same in both arms."""
+    return {"workload": wl.name, "requests_per_gpu": Q, "context_slots": wl.ctx0[0], "block_size": wl.b,
+            "heads": wl.H, "head_dim": wl.d, "topk": wl.topk, "target_sparsity": args.sparsity,
+            "gamma": wl.gamma, "pooling": args.pooling,
+            "parallelism": f"dp{world} (requests sharded, no collective)",
+            "l2": "inputs larger than L2: 6.4 GB paged FP8 key cache and 0.4 GB EMA state per GPU"}
+
+
 def reference_arm(args, world, rank):
     if rank != 0:
         return None
@@ -1092,11 +1097,10 @@ def reference_arm(args, world, rank):
     return {"metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "context_slots": wl.ctx0[0], "target_sparsity": args.sparsity,
-                       "sample": "each step: one request of the 96 (the oracle on host cores)"},
+            "config": headline_config(wl, wl.requests, args, world),
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": threads_used(), "kind": "oracle",
-                             "sample": f"{args.steps} timed steps of 1 request at 512K after "
-                                       f"{args.warmup} warm-up steps"},
+                             "sample": f"each step one request of the 96 at 512K on the host cores: "
+                                       f"{args.steps} timed steps after {args.warmup} warm-up steps"},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
