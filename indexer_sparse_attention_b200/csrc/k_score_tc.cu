@@ -103,9 +103,12 @@ struct Ctl {
 };
 
 // Bounded wait on a phase parity: false on timeout (raises ERR_TIMEOUT and
-// the CTA abort flag) or when another role already aborted.
-__device__ __noinline__ bool wait_parity(uint32_t bar, uint32_t parity, Ctl c) {
-  if (mbar_try_wait(bar, parity)) return true;
+// the CTA abort flag) or when another role already aborted.  The first test
+// is inline; only a phase that is not yet complete calls the out-of-line
+// loop, so a wait that succeeds at once is no function call (a call would
+// make the caller's loads still in flight, such as the next tile's
+// prefetch, complete first).
+__device__ __noinline__ bool wait_parity_slow(uint32_t bar, uint32_t parity, Ctl c) {
   const uint64_t t0 = gtimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -118,6 +121,9 @@ __device__ __noinline__ bool wait_parity(uint32_t bar, uint32_t parity, Ctl c) {
       }
     }
   }
+}
+__device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity, Ctl c) {
+  return mbar_try_wait(bar, parity) || wait_parity_slow(bar, parity, c);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
