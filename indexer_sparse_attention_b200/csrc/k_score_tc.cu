@@ -544,37 +544,69 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     int cur_q = -1;
     float* wcur = wqs + ew * N;           // this warp's copy of the head weights
     const int n_local = g1 - g0;
-    // Per-token operands of a tile, loaded one tile (of this group) ahead.
+    // Per-token operands of a tile.  The tile's metadata comes from the
+    // tile-info ring when the tile is processed (the slot is held until the
+    // hand-back); the three global loads (scale, V, D) are issued two tiles
+    // of this group ahead, because under full load a global load takes longer
+    // than one tile of the epilogue.  Waiting for the info of tile i + 2T
+    // (T = tile groups) cannot deadlock: the producer writes it once the MMAs
+    // of tile i + 2T - stages have completed and the MMAs run up to tile
+    // i + nacc - 1 without this group, and 2T < nacc + stages in every plan.
     struct Pre {
       int q, s, valid, upd, t;
-      int64_t p0;
+      int p0;  // ctx_len - 1 < 2^31 (max_slots is an int32)
       float sigma, v, d;
     };
-    auto prefetch = [&](int i, Pre& r) -> bool {
-      const int xs = i % kAuxSlots;
-      const uint32_t xph = (uint32_t)(i / kAuxSlots) & 1u;
-      if (!__all_sync(0xffffffffu, wait_parity(B.xf(xs), xph, ctl))) return false;
-      const TileInfo* x = aux + xs;
+    struct Side {
+      float sigma, v, d;
+    };
+    auto info_ready = [&](int i) -> bool {
+      return __all_sync(0xffffffffu, wait_parity(B.xf(i & (kAuxSlots - 1)), (uint32_t)(i / kAuxSlots) & 1u, ctl));
+    };
+    auto meta_of = [&](int i, int& pg) -> Pre {  // after info_ready(i)
+      const TileInfo* x = aux + (i & (kAuxSlots - 1));
+      Pre r;
       r.q = x->q;
       r.t = x->t;
       r.p0 = x->ctx - 1;
-      const int pg = x->pg[pg_idx];
+      pg = x->pg[pg_idx];
       const bool present = pg_idx < x->np && pg >= 0;
       r.s = present ? x->j[pg_idx] * kPage + tok : 0;
       r.valid = present && r.s <= r.p0 + (a.rows - 1);
       r.upd = fused && r.valid && r.s <= r.p0;
-      r.sigma = r.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
-      r.v = r.upd ? a.V[(int64_t)r.q * L.slot_stride + r.s] : 0.f;
-      r.d = r.upd ? a.D[(int64_t)r.q * L.slot_stride + (r.p0 - r.s)] : 0.f;
-      return true;
+      return r;
     };
-    Pre nx;
-    bool alive_ = group < n_local && prefetch(group, nx);
+    auto load_side = [&](int i) -> Side {
+      int pg;
+      const Pre m = meta_of(i, pg);
+      Side r;
+      r.sigma = m.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
+      r.v = m.upd ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
+      r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
+      return r;
+    };
+    Side nx1{0.f, 0.f, 0.f}, nx2{0.f, 0.f, 0.f};  // tiles i + T and i + 2T
+    bool alive_ = group < n_local && info_ready(group);
+    if (alive_) nx1 = load_side(group);
+    if (alive_ && group + tgroups < n_local) {
+      alive_ = info_ready(group + tgroups);
+      if (alive_) nx2 = load_side(group + tgroups);
+    }
+    // ring positions of tile i, advanced by T per tile without divisions
+    int acc = group % nacc, stage = group % stages;
+    uint32_t phase = (uint32_t)(group / stages) & 1u;
     for (int i = group; alive_ && i < n_local; i += tgroups) {
-      const Pre cur = nx;
-      if (i + tgroups < n_local && !prefetch(i + tgroups, nx)) break;
-      const int xs = i % kAuxSlots, acc = i % nacc, stage = i % stages;
-      const uint32_t phase = (uint32_t)(i / stages) & 1u;
+      int pg_unused;
+      Pre cur = meta_of(i, pg_unused);
+      cur.sigma = nx1.sigma;
+      cur.v = nx1.v;
+      cur.d = nx1.d;
+      nx1 = nx2;
+      if (i + 2 * tgroups < n_local) {
+        if (!info_ready(i + 2 * tgroups)) break;
+        nx2 = load_side(i + 2 * tgroups);
+      }
+      const int xs = i & (kAuxSlots - 1);
       if (cur.q != cur_q) {
         __syncwarp();
         for (int k = lane; k < N; k += 32) wcur[k] = a.wq[(int64_t)cur.q * N + k];
@@ -634,6 +666,13 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
             a.D[(int64_t)cur.q * L.slot_stride + (cur.p0 - cur.s)] = ema_d(cur.d, score, a.alpha, a.beta);
           }
         }
+      }
+      acc += tgroups;
+      while (acc >= nacc) acc -= nacc;
+      stage += tgroups;
+      while (stage >= stages) {
+        stage -= stages;
+        phase ^= 1u;
       }
     }
   }
