@@ -24,7 +24,7 @@
 //               the accumulator full for the epilogue
 //   warps 2..9  two epilogue groups of four warps, taking alternate tiles; a
 //               thread owns one token: it loads the token's scale and EMA
-//               values one tile ahead, reads its accumulator row from the TMEM
+//               values two tiles ahead, reads its accumulator row from the TMEM
 //               quarter its warp may access (lanes 32*(warp%4) ..), hands
 //               the accumulator back as soon as its last columns are in
 //               registers, applies ReLU, head weights and the scale, and
