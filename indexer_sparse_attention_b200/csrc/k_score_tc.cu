@@ -170,6 +170,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
 // Two independent fp32 fused multiply-adds (round to nearest) in one packed
 // instruction: (a0, a1) += (w0 * x0, w1 * x1), each rounded once as fmaf.
 __device__ __forceinline__ void fma2_rn(float& a0, float& a1, float w0, float w1, float x0, float x1) {
@@ -315,7 +325,9 @@ __device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
   return r;
 }
 
-template <int G>
+// KH: the head count when it is fixed at compile time (64, the DSA indexer's),
+// so that the epilogue's column loops unroll; 0 reads it from the layout.
+template <int G, int KH>
 __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
@@ -323,7 +335,8 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   constexpr int kThreads = threads_for(G);
   constexpr int kEpiGroups = G;
   const Layout L = a.lay;
-  const int N = a.rows * L.H;
+  const int H = KH ? KH : L.H;
+  const int N = a.rows * H;
   const int stages = plan.stages, nacc = plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -621,12 +634,14 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
       for (int r = sub; r < a.rows; r += share) {
         float part[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c = 0; c < L.H; c += 32) {
+        for (int c = 0; c < H; c += 32) {
           uint32_t v[32];
-          tmem_ld16(trow + (uint32_t)(r * L.H + c), *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-          if (c + 16 < L.H) tmem_ld16(trow + (uint32_t)(r * L.H + c + 16), *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+          if (c + 32 <= H)  // 32 columns in one load
+            tmem_ld32(trow + (uint32_t)(r * H + c), v);
+          else
+            tmem_ld16(trow + (uint32_t)(r * H + c), *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           tmem_wait_ld();
-          if (r + share >= a.rows && c + 32 >= L.H) {
+          if (r + share >= a.rows && c + 32 >= H) {
             // last accumulator columns are in registers: hand the accumulator
             // (and the tile-info slot, read a tile ago) back before the math
             tc_fence_before();
@@ -636,8 +651,8 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
               mbar_arrive(B.xe(xs));
             }
           }
-          const float4* wr = reinterpret_cast<const float4*>(wcur + r * L.H + c);
-          const int nu = min(32, L.H - c);  // 16 or 32: H is a multiple of 16
+          const float4* wr = reinterpret_cast<const float4*>(wcur + r * H + c);
+          const int nu = min(32, H - c);  // 16 or 32: H is a multiple of 16
 #pragma unroll
           for (int u = 0; u < 32; u += 4) {
             if (u < nu) {
@@ -717,7 +732,8 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   if (!encode_2d(fn, &tq, a.q8, (uint64_t)L.Q * N, (uint32_t)N)) return cudaErrorInvalidValue;
   const TcPlan plan = tc_plan(N, L.Q);
   const uint32_t smem = smem_layout(N, L.Q, plan.stages, plan.nq, plan.groups).total;
-  auto kernel = plan.groups == 2 ? k_score_tc<2> : k_score_tc<4>;
+  auto kernel = plan.groups == 2 ? (L.H == 64 ? k_score_tc<2, 64> : k_score_tc<2, 0>)
+                                 : (L.H == 64 ? k_score_tc<4, 64> : k_score_tc<4, 0>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;

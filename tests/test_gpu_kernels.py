@@ -117,8 +117,20 @@ def run_score(st, kind, R, cache, q, w, ctx_t, mask, fp8=True):
 @pytest.mark.parametrize("R", [1, 2, 4])
 @pytest.mark.parametrize("kind", [isa.SPIN_SCORE_SIMT, isa.SPIN_SCORE_TCGEN05])
 def test_fp8_scores_vs_oracle(R, kind):
-    rng = np.random.default_rng(R)
-    Q, H, d, max_slots = 3, 64, 128, 64 * 41
+    check_fp8_scores(R, 64, kind, R)
+
+
+@pytest.mark.parametrize("R,H", [(1, 32), (1, 128), (2, 128), (3, 48)])
+def test_tcgen05_other_head_counts(R, H):
+    """Head counts other than 64 take the tcgen05 kernel's generic column
+    loop: N = 32, 128 (two CTAs per SM), 256 and 144 (one CTA per SM, rows
+    split over two epilogue groups; 48 heads end on a 16-column load)."""
+    check_fp8_scores(R, H, isa.SPIN_SCORE_TCGEN05, 100 + H + R)
+
+
+def check_fp8_scores(R, H, kind, seed):
+    rng = np.random.default_rng(seed)
+    Q, d, max_slots = 3, 128, 64 * 41
     st = make_state(Q=Q, max_slots=max_slots, R=R, H=H, d=d)
     wl, cache, q, w = fp8_inputs(Q, R, H, d, max_slots, rng)
     ctx = np.array([64 * 40 + 7 - R + 1, 130, 64 * 23], np.int64)
