@@ -116,3 +116,25 @@ def test_layer_allocator_rejects_bad_input(lib):
         isa.spin_allocate_layer_sparsity([0.1], [100.0], [0.05], 1.0)
     with pytest.raises(isa.SpinError):
         isa.spin_allocate_layer_sparsity([-0.1], [100.0], [0.05], 0.5)
+
+
+def test_null_state_rejected_by_every_entry_point(lib):
+    """Every call that takes a state answers SPIN_ESTATE for a NULL handle,
+    before it touches the device (no GPU needed)."""
+    isa.load()
+    skip = {"spin_state_bytes", "spin_state_create", "spin_topk_noalloc", "spin_allocate_layer_sparsity",
+            "spin_status_string", "spin_state_export_bytes", "spin_score_stride", "spin_mask_stride",
+            "spin_state_destroy"}
+    names = [n for n in isa.__all__ if n.startswith("spin_") and n not in skip]
+    checked = 0
+    for name in names:
+        fn = getattr(lib, name, None)
+        if fn is None or fn.restype is not ctypes.c_int or not fn.argtypes:
+            continue
+        ptr = lambda t: t in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(t, ctypes._Pointer)
+        args = [None] + [None if ptr(t) else 0 for t in fn.argtypes[1:]]
+        assert fn(*args) == 4, name                      # SPIN_ESTATE
+        checked += 1
+    for name in ("spin_slot_prediction", "spin_pearson", "spin_topk_overlap", "spin_decode_step"):
+        assert name in names
+    assert checked >= 20
