@@ -57,7 +57,7 @@ __host__ __device__ __forceinline__ int64_t row_blocks(int64_t ctx_len, int r, i
 }
 
 // Budget of a row and the exploration count (computed in double from the
-// fp32 parameters, exactly as the host and the checker define them).
+// fp32 parameters, the same definition the host code uses).
 __device__ __forceinline__ int64_t block_budget(int64_t n, float s) {
   return n - (int64_t)floor((double)s * (double)n);
 }

@@ -6,7 +6,7 @@
  * library never links, loads or calls it, and it shares no code, header,
  * table or constant generator with the CUDA path.
  *
- * Sources (see the design doc for the full titles of the four pages):
+ * Sources (four web pages on SPIN; short names used below):
  *   [digest]  ai4snews digest of the SPIN paper, sections 核心概要 /
  *             arXiv深度剖析 / 启示与展望
  *   [listing] thelatestinai listing "SaveSPIN: Shadow Predictive Indexer for
@@ -18,8 +18,8 @@
  *
  * The pages do not print the indexer formula; the DSA lightning-indexer form
  * I_{t,s} = sum_h w_{t,h} * ReLU(q_{t,h} . k_s) is taken as the definition.
- * Every reading of a point the pages leave open is listed in the design doc
- * ("Readings").  Each function below says which passage it follows.
+ * Where the pages leave a point open, the function that meets it states the
+ * reading it takes.  Each function below says which passage it follows.
  *
  * Numerics: scores are computed in fp64 from the exact decoded operand
  * values.  The EMA state is fp32 by definition, and its update is written
@@ -115,7 +115,7 @@ ORC_API uint8_t orc_e4m3_encode(double x) {
 
 /* ------------------------------------------------------------------------ */
 /* Query quantisation for the FP8 indexer.  The pages give no precision; the */
-/* reading (R11) quantises each (row, head) query vector to E4M3   */
+/* reading taken here quantises each (row, head) query vector to E4M3       */
 /* with a power-of-two scale 2^e and folds the scale into the head weight:   */
 /* ReLU(c x) = c ReLU(x) for c > 0, so w' = w * 2^e keeps the score the same. */
 /* ------------------------------------------------------------------------ */
@@ -554,7 +554,7 @@ ORC_API double orc_miss_fraction(const int32_t* full_topk, int k, const uint8_t*
 
 /* ------------------------------------------------------------------------ */
 /* Per-layer block budget ([v3] abstract: the block budget is spread across  */
-/* layers by their measured miss rates).  Reading (R16): kept     */
+/* layers by their measured miss rates).  The reading taken here: kept      */
 /* fractions f_l = clamp(c * (m_l + 1e-3), lo_l, 1), with c chosen so that  */
 /* sum_l f_l N_l = (1 - s_glob) sum_l N_l; found by bisection on c.  When   */
 /* even the lower bounds exceed the global budget, f_l = lo_l.  Returns the */

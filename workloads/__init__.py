@@ -8,7 +8,7 @@ lengths.  Every draw comes from a ``torch.Generator`` seeded from
 (workload seed, purpose, layer, request), on the device the caller names, so a
 test or benchmark generates once and hands copies to both sides.
 
-Structure planted in the keys and queries (the recipe is stated in the design doc):
+Structure planted in the keys and queries:
 
 * vertical lines: a fixed set of slots whose keys carry ``3 * u`` while every
   query carries ``sqrt(d) * u`` (u a unit vector per layer and request), so a
