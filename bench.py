@@ -471,6 +471,7 @@ def gpu_arm(args, world, rank, local):
     achieved = kept_slots * SCORE_BYTES_PER_SLOT / (score_avg / 1e3) / 1e9
     traffic_slot = score_traffic_per_slot()
     launches = sum(n for _, n in stages.values())
+    step_tr = step_traffic(int(run.ctx[run.t - 1].long().sum().item()), kept_slots, ms_step, peak)
     out = {
         "metric": METRIC, "value": rows_s, "unit": "rows/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -478,6 +479,7 @@ def gpu_arm(args, world, rank, local):
         "config": headline_config(wl, Q, args, world),
         "index_key_gbs": key_gbs,
         "key_roofline_frac": key_gbs / peak,
+        "step_traffic": step_tr,
         "roofline": {"bound": "hbm", "kernel": "k_score_tc (paged FP8 indexer + fused EMA)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs (copy, MEASURED_PEAKS.json)" if peak_kind == "measured"
@@ -1070,6 +1072,16 @@ def cpu_baseline(sparsity, seconds):
     return {"value": n / dt, "unit": "rows/s", "cores": threads_used(), "kind": "oracle",
             "sample": f"{n} decode steps of 1 of the 96 requests (512K context, {int(sparsity * 100)}% sparsity) "
                       f"after an untimed all-keep bootstrap; fp64 scores, OpenMP over blocks; {dt:.1f} s"}
+
+
+def step_traffic(context_slots, kept_slots, ms_step, peak):
+    """The whole step's algorithmic bytes against the measured copy bandwidth:
+    8 B per slot of context (the predict kernel reads V and D) plus the score
+    kernel's bytes per kept slot (key, scale, score, EMA read and write)."""
+    b = 8 * context_slots + SCORE_BYTES_PER_SLOT * kept_slots
+    gbs = b / (ms_step / 1e3) / 1e9
+    return {"bytes_per_step": b, "gbs": gbs, "frac": gbs / peak,
+            "note": "8 B per slot of context + 152 B per kept slot; the floor of a step"}
 
 
 def headline_config(wl, Q, args, world):

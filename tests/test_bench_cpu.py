@@ -1,0 +1,25 @@
+"""Host-side helpers of bench.py (no GPU): the step-traffic figure and the
+config both arms print."""
+import sys
+import types
+
+import bench
+import workloads
+
+
+def test_step_traffic_closed_form():
+    # 96 requests at 512K and 50%: 8 B per context slot + 152 B per kept slot
+    ctx, kept = 96 * 524_292, 25_170_000
+    t = bench.step_traffic(ctx, kept, 0.8, 6546.6)
+    assert t["bytes_per_step"] == 8 * ctx + 152 * kept
+    assert abs(t["gbs"] - t["bytes_per_step"] / 0.8e-3 / 1e9) < 1e-9
+    assert abs(t["frac"] - t["gbs"] / 6546.6) < 1e-12
+
+
+def test_both_arms_print_the_same_config():
+    args = types.SimpleNamespace(sparsity=0.5, pooling="max")
+    wl = workloads.config(2)
+    a = bench.headline_config(wl, wl.requests, args, 1)
+    b = bench.headline_config(bench.rank_workload(0, 96, 8), 96, args, 1)
+    assert a == b
+    assert a["workload"] == "serve-96x512K" and a["requests_per_gpu"] == 96
