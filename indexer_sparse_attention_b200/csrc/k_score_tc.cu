@@ -559,12 +559,16 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     const int n_local = g1 - g0;
     // Per-token operands of a tile.  The tile's metadata comes from the
     // tile-info ring when the tile is processed (the slot is held until the
-    // hand-back); the three global loads (scale, V, D) are issued two tiles
-    // of this group ahead, because under full load a global load takes longer
-    // than one tile of the epilogue.  Waiting for the info of tile i + 2T
-    // (T = tile groups) cannot deadlock: the producer writes it once the MMAs
-    // of tile i + 2T - stages have completed and the MMAs run up to tile
-    // i + nacc - 1 without this group, and 2T < nacc + stages in every plan.
+    // hand-back); the three global loads (scale, V, D) are issued `dist` tiles
+    // of this group ahead (T = tile groups apart), because under full load a
+    // global load takes longer than one tile of the epilogue.  The wait for
+    // the info of tile i + dist*T must not need this group's hand-back of
+    // tile i: the MMAs run up to tile i + nacc - 1 without it, and the
+    // producer writes the info of tile k once the MMAs of tile k - stages are
+    // done and, at a request change, once the MMA issuer has reached the first
+    // tile of the request nq requests back (one tile before k at the least).
+    // So dist*T < nq + nacc and dist*T < stages + nacc; dist is the largest
+    // of 2, 1, 0 that satisfies both (2 in the one-row plan at N <= 64).
     struct Pre {
       int q, s, valid, upd, t;
       int p0;  // ctx_len - 1 < 2^31 (max_slots is an int32)
@@ -598,27 +602,41 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
       return r;
     };
-    Side nx1{0.f, 0.f, 0.f}, nx2{0.f, 0.f, 0.f};  // tiles i + T and i + 2T
-    bool alive_ = group < n_local && info_ready(group);
-    if (alive_) nx1 = load_side(group);
-    if (alive_ && group + tgroups < n_local) {
+    int dist = 2;
+    while (dist > 0 && !(dist * tgroups < nq + nacc && dist * tgroups < stages + nacc)) --dist;
+    Side q0{0.f, 0.f, 0.f}, q1{0.f, 0.f, 0.f};  // side data of tiles i and i + T
+    bool alive_ = group < n_local;
+    if (alive_ && dist >= 1) {
+      alive_ = info_ready(group);
+      if (alive_) q0 = load_side(group);
+    }
+    if (alive_ && dist == 2 && group + tgroups < n_local) {
       alive_ = info_ready(group + tgroups);
-      if (alive_) nx2 = load_side(group + tgroups);
+      if (alive_) q1 = load_side(group + tgroups);
     }
     // ring positions of tile i, advanced by T per tile without divisions
     int acc = group % nacc, stage = group % stages;
     uint32_t phase = (uint32_t)(group / stages) & 1u;
     for (int i = group; alive_ && i < n_local; i += tgroups) {
+      Side side;
+      if (dist == 0) {
+        if (!info_ready(i)) break;
+        side = load_side(i);
+      } else {
+        side = q0;
+        q0 = q1;
+        const int nxt = i + dist * tgroups;
+        if (nxt < n_local) {
+          if (!info_ready(nxt)) break;
+          const Side ld = load_side(nxt);
+          if (dist == 2) q1 = ld; else q0 = ld;
+        }
+      }
       int pg_unused;
       Pre cur = meta_of(i, pg_unused);
-      cur.sigma = nx1.sigma;
-      cur.v = nx1.v;
-      cur.d = nx1.d;
-      nx1 = nx2;
-      if (i + 2 * tgroups < n_local) {
-        if (!info_ready(i + 2 * tgroups)) break;
-        nx2 = load_side(i + 2 * tgroups);
-      }
+      cur.sigma = side.sigma;
+      cur.v = side.v;
+      cur.d = side.d;
       const int xs = i & (kAuxSlots - 1);
       if (cur.q != cur_q) {
         __syncwarp();

@@ -128,6 +128,40 @@ def test_tcgen05_other_head_counts(R, H):
     check_fp8_scores(R, H, isa.SPIN_SCORE_TCGEN05, 100 + H + R)
 
 
+@pytest.mark.parametrize("R", [2, 4])
+def test_tcgen05_short_requests_between_long_ones(R):
+    """One-tile requests between long ones, so that CTAs meet request changes
+    every few tiles: N = 128 (two CTAs per SM, one query buffer) and N = 256
+    (one CTA per SM, two query buffers).  The epilogue's side-data prefetch
+    must never wait on its own hand-back (a stalled wait would end in
+    ERR_TIMEOUT); scores match the oracle on the short requests and on a
+    sample of the long ones."""
+    rng = np.random.default_rng(40 + R)
+    Q, H, d, max_slots = 5, 64, 128, 64 * 1501
+    st = make_state(Q=Q, max_slots=max_slots, R=R, H=H, d=d)
+    wl, cache, q, w = fp8_inputs(Q, R, H, d, max_slots, rng, permute=False)
+    ctx = np.array([64 * 1500, 100, 64 * 1500, 100, 64 * 1500 - 37], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    m = np.zeros((Q, st.mask_stride), np.uint8)
+    for qq in range(Q):
+        m[qq, : oracle.num_blocks(int(ctx[qq]), R - 1, 64)] = 1
+    scores = run_score(st, isa.SPIN_SCORE_TCGEN05, R, cache, q, w, ctx_t, torch.from_numpy(m).cuda())
+    for qq in range(Q):
+        q8, wq, _ = oracle.quantize_q(q[qq].float().cpu().numpy().astype(np.float64), w[qq].cpu().numpy())
+        keys, ks, ident = workloads.request_pages(cache, qq)
+        n_last = oracle.num_blocks(int(ctx[qq]), R - 1, 64)
+        sub = m[qq].copy()
+        if n_last > 8:                                       # a sample of a long request's blocks
+            sub[:] = 0
+            sub[rng.choice(n_last, 12, replace=False)] = 1
+            sub[n_last - 1] = 1
+        ref = oracle.score_fp8(keys.numpy(), ks.numpy(), ident.numpy(), q8, wq, int(ctx[qq]), sub, st.score_stride)
+        got = scores[qq, :R].cpu().numpy()
+        sc = ~np.isnan(ref)
+        assert sc.sum() > 0
+        assert score_close(got[sc], ref[sc]).all(), qq
+
+
 def check_fp8_scores(R, H, kind, seed):
     rng = np.random.default_rng(seed)
     Q, d, max_slots = 3, 128, 64 * 41
