@@ -486,8 +486,9 @@ def gpu_arm(args, world, rank, local):
                      else "fallback 6650 GB/s", "avg_launch_ms": score_avg,
                      "bytes_per_launch": kept_slots * SCORE_BYTES_PER_SLOT,
                      "traffic": (None if traffic_slot is None else traffic_slot * kept_slots),
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
-                                       "(16-request capture, scaled by kept slots)"},
+                     "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
+                                        "(16-request capture, scaled by kept slots)" if traffic_slot is not None
+                                        else "null: the kernel source has changed since the last ncu capture")},
         "stage_ms_per_step": {k: v[0] / KS for k, v in stage_pass.items() if v[1]},
         "stage_ms_source": f"separate pass of {KS} steps with every launch bracketed by CUDA events",
         "gpu_launches": launches,
