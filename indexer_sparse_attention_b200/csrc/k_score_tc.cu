@@ -269,6 +269,26 @@ __host__ __device__ inline TcPlan tc_plan(int N, int Q) {
   return {kMaxStages, 2, 1, 2, 4};
 }
 
+// Epilogue groups that share one tile: with four groups and several rows two
+// groups split a tile's rows, so an accumulator is read out in half the time.
+__host__ __device__ constexpr int groups_per_tile(int groups, int rows) { return (groups == 4 && rows >= 2) ? 2 : 1; }
+
+// How many tiles (of its own group) ahead an epilogue group issues the side
+// loads (scale, V, D).  The wait for the tile-info of tile i + dist*T
+// (T = tiles in the epilogue at once) must not need this group's hand-back of
+// tile i: the MMAs run up to tile i + nacc - 1 without it, and the producer
+// writes the info of tile k once the MMAs of tile k - stages are done and, at
+// a request change, once the MMA issuer has reached the first tile of the
+// request nq requests back (one tile before k at the least).  So
+// dist*T < nq + nacc and dist*T < stages + nacc; the largest of 2, 1, 0 that
+// satisfies both.  It is a template parameter of the kernel, so that the side
+// data of the tiles ahead stay in fixed registers.
+__host__ __device__ constexpr int prefetch_dist(int tiles_at_once, int nq, int nacc, int stages) {
+  return (2 * tiles_at_once < nq + nacc && 2 * tiles_at_once < stages + nacc)   ? 2
+         : (1 * tiles_at_once < nq + nacc && 1 * tiles_at_once < stages + nacc) ? 1
+                                                                                 : 0;
+}
+
 struct Bars {
   uint32_t full, empty, afull, aempty, qfull, qempty, accempty, done;
   __device__ uint32_t f(int s) const { return full + 8 * s; }
@@ -327,7 +347,8 @@ __device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
 
 // KH: the head count when it is fixed at compile time (64, the DSA indexer's),
 // so that the epilogue's column loops unroll; 0 reads it from the layout.
-template <int G, int KH>
+// DIST: the side-load prefetch distance, prefetch_dist() of the plan.
+template <int G, int KH, int DIST>
 __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
@@ -364,7 +385,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   // With four groups and several rows, two groups share a tile, each taking
   // every other row: the accumulator (two fit TMEM at N > 128) is read in half
   // the time, so the MMA waits half as long for it.
-  const int share = (kEpiGroups == 4 && a.rows >= 2) ? 2 : 1;  // groups per tile
+  const int share = groups_per_tile(kEpiGroups, a.rows);  // groups per tile
 
   // ---- tile prefix over requests (all threads: one load pair each, block
   // scan), barriers ------------------------------------------------------
@@ -559,16 +580,10 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     const int n_local = g1 - g0;
     // Per-token operands of a tile.  The tile's metadata comes from the
     // tile-info ring when the tile is processed (the slot is held until the
-    // hand-back); the three global loads (scale, V, D) are issued `dist` tiles
+    // hand-back); the three global loads (scale, V, D) are issued DIST tiles
     // of this group ahead (T = tile groups apart), because under full load a
-    // global load takes longer than one tile of the epilogue.  The wait for
-    // the info of tile i + dist*T must not need this group's hand-back of
-    // tile i: the MMAs run up to tile i + nacc - 1 without it, and the
-    // producer writes the info of tile k once the MMAs of tile k - stages are
-    // done and, at a request change, once the MMA issuer has reached the first
-    // tile of the request nq requests back (one tile before k at the least).
-    // So dist*T < nq + nacc and dist*T < stages + nacc; dist is the largest
-    // of 2, 1, 0 that satisfies both (2 in the one-row plan at N <= 64).
+    // global load takes longer than one tile of the epilogue.  DIST follows
+    // the rule of prefetch_dist(), which the host checked for this plan.
     struct Pre {
       int q, s, valid, upd, t;
       int p0;  // ctx_len - 1 < 2^31 (max_slots is an int32)
@@ -602,34 +617,40 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
       return r;
     };
-    int dist = 2;
-    while (dist > 0 && !(dist * tgroups < nq + nacc && dist * tgroups < stages + nacc)) --dist;
-    Side q0{0.f, 0.f, 0.f}, q1{0.f, 0.f, 0.f};  // side data of tiles i and i + T
+    Side nx1{0.f, 0.f, 0.f}, nx2{0.f, 0.f, 0.f};  // side data of tiles i and i + T
     bool alive_ = group < n_local;
-    if (alive_ && dist >= 1) {
-      alive_ = info_ready(group);
-      if (alive_) q0 = load_side(group);
+    if constexpr (DIST >= 1) {
+      if (alive_) {
+        alive_ = info_ready(group);
+        if (alive_) nx1 = load_side(group);
+      }
     }
-    if (alive_ && dist == 2 && group + tgroups < n_local) {
-      alive_ = info_ready(group + tgroups);
-      if (alive_) q1 = load_side(group + tgroups);
+    if constexpr (DIST == 2) {
+      if (alive_ && group + tgroups < n_local) {
+        alive_ = info_ready(group + tgroups);
+        if (alive_) nx2 = load_side(group + tgroups);
+      }
     }
     // ring positions of tile i, advanced by T per tile without divisions
     int acc = group % nacc, stage = group % stages;
     uint32_t phase = (uint32_t)(group / stages) & 1u;
     for (int i = group; alive_ && i < n_local; i += tgroups) {
       Side side;
-      if (dist == 0) {
+      if constexpr (DIST == 0) {
         if (!info_ready(i)) break;
         side = load_side(i);
+      } else if constexpr (DIST == 1) {
+        side = nx1;
+        if (i + tgroups < n_local) {
+          if (!info_ready(i + tgroups)) break;
+          nx1 = load_side(i + tgroups);
+        }
       } else {
-        side = q0;
-        q0 = q1;
-        const int nxt = i + dist * tgroups;
-        if (nxt < n_local) {
-          if (!info_ready(nxt)) break;
-          const Side ld = load_side(nxt);
-          if (dist == 2) q1 = ld; else q0 = ld;
+        side = nx1;
+        nx1 = nx2;
+        if (i + 2 * tgroups < n_local) {
+          if (!info_ready(i + 2 * tgroups)) break;
+          nx2 = load_side(i + 2 * tgroups);
         }
       }
       int pg_unused;
@@ -750,8 +771,16 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   if (!encode_2d(fn, &tq, a.q8, (uint64_t)L.Q * N, (uint32_t)N)) return cudaErrorInvalidValue;
   const TcPlan plan = tc_plan(N, L.Q);
   const uint32_t smem = smem_layout(N, L.Q, plan.stages, plan.nq, plan.groups).total;
-  auto kernel = plan.groups == 2 ? (L.H == 64 ? k_score_tc<2, 64> : k_score_tc<2, 0>)
-                                 : (L.H == 64 ? k_score_tc<4, 64> : k_score_tc<4, 0>);
+  const int dist = prefetch_dist(plan.groups / groups_per_tile(plan.groups, a.rows), plan.nq, plan.nacc,
+                                 plan.stages);
+  // the instances the plans reach: two groups with 4 accumulators (N <= 64)
+  // or 2 (N <= 128); four groups sharing tiles (several rows) or not (one row)
+  void (*kernel)(ScoreArgs, TcPlan, const CUtensorMap, const CUtensorMap) = nullptr;
+  if (plan.groups == 2 && dist == 2) kernel = L.H == 64 ? k_score_tc<2, 64, 2> : k_score_tc<2, 0, 2>;
+  if (plan.groups == 2 && dist == 1) kernel = L.H == 64 ? k_score_tc<2, 64, 1> : k_score_tc<2, 0, 1>;
+  if (plan.groups == 4 && dist == 1) kernel = L.H == 64 ? k_score_tc<4, 64, 1> : k_score_tc<4, 0, 1>;
+  if (plan.groups == 4 && dist == 0) kernel = k_score_tc<4, 0, 0>;
+  if (!kernel) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;

@@ -128,11 +128,12 @@ def test_tcgen05_other_head_counts(R, H):
     check_fp8_scores(R, H, isa.SPIN_SCORE_TCGEN05, 100 + H + R)
 
 
-@pytest.mark.parametrize("R", [2, 4])
+@pytest.mark.parametrize("R", [1, 2, 4])
 def test_tcgen05_short_requests_between_long_ones(R):
     """One-tile requests between long ones, so that CTAs meet request changes
-    every few tiles: N = 128 (two CTAs per SM, one query buffer) and N = 256
-    (one CTA per SM, two query buffers).  The epilogue's side-data prefetch
+    every few tiles: N = 64 (two CTAs per SM, one query buffer, side data two
+    tiles ahead), N = 128 (two CTAs per SM, one query buffer, one tile ahead)
+    and N = 256 (one CTA per SM, two query buffers).  The epilogue's side-data prefetch
     must never wait on its own hand-back (a stalled wait would end in
     ERR_TIMEOUT); scores match the oracle on the short requests and on a
     sample of the long ones."""
