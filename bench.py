@@ -71,6 +71,8 @@ def parse():
                    help="block reduction of the predicted scores (max is the method's)")
     p.add_argument("--mtp-policy", choices=list(MTP_POLICIES), default="union-prefix",
                    help="several query rows: row-local union + prefix-valid update (the method's) or row 0 alone")
+    p.add_argument("--no-lookahead", action="store_true",
+                   help="sequential one-row steps: no next-step selection prepared beside the top-k")
     p.add_argument("--ablation", choices=["pooling", "mtp", "predictors"], default=None,
                    help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities; "
                         "mtp: p99 miss vs realized sparsity of the two MTP policies on the 4-row workload; "
@@ -264,7 +266,7 @@ def peaks():
 
 
 class SpinRun:
-    def __init__(self, wl, device, total_steps, pooling=0):
+    def __init__(self, wl, device, total_steps, pooling=0, lookahead=True):
         import indexer_sparse_attention_b200 as isa
         self.isa = isa
         self.wl = wl
@@ -283,6 +285,8 @@ class SpinRun:
                               pooling=pooling)
         self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
+        self.lookahead = lookahead
+        isa.spin_set_lookahead(self.st, lookahead)
         self.mask = self.st.new_mask()
         self.topk = torch.empty((wl.requests, 1, wl.topk), dtype=torch.int32, device=device)
         self.scores = self.st.new_scores()
@@ -435,7 +439,7 @@ def gpu_arm(args, world, rank, local):
     KS = min(K, 40)  # steps of the per-stage timing pass
     total = 1 + (W + K) * (1 + len(sweep)) + 3 + K + KS + 2
     wl = rank_workload(rank, args.requests, total + 8)
-    run = SpinRun(wl, device, total, POOLINGS[args.pooling])
+    run = SpinRun(wl, device, total, POOLINGS[args.pooling], lookahead=not args.no_lookahead)
     Q = wl.requests
     # history bootstrap: all-keep step that fills V and D
     run.set_sparsity(0.0)
@@ -489,8 +493,12 @@ def gpu_arm(args, world, rank, local):
                      "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
                                         "(16-request capture, scaled by kept slots)" if traffic_slot is not None
                                         else "null: the kernel source has changed since the last ncu capture")},
+        "pipelined": ("each step prepares the next step's selection, whose predict kernel runs on a second "
+                      "stream beside the step's top-k (spin_set_lookahead); results are those of the "
+                      "sequential step" if run.lookahead else "no: sequential steps"),
         "stage_ms_per_step": {k: v[0] / KS for k, v in stage_pass.items() if v[1]},
-        "stage_ms_source": f"separate pass of {KS} steps with every launch bracketed by CUDA events",
+        "stage_ms_source": (f"separate pass of {KS} steps with every launch bracketed by CUDA events"
+                            + ("; the next step's predict overlaps the top-k" if run.lookahead else "")),
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
@@ -528,6 +536,9 @@ def graph_pass(run, warmup, steps, world):
     isa, wl = run.isa, run.wl
     t = run.t
     q_buf, w_buf, c_buf = run.q[t].clone(), run.w[t].clone(), run.ctx[t].clone()
+    # the same ctx_len every replay breaks the one-slot-a-step contract of a
+    # pipelined step: replay the sequential step
+    isa.spin_set_lookahead(run.st, False)
     isa.spin_set_step(run.st, t)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
@@ -551,7 +562,8 @@ def graph_pass(run, warmup, steps, world):
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     del graph
     return {"value": job_rows_per_s(wl.requests * steps, world, ms), "unit": "rows/s", "ms_per_step": ms / steps,
-            "note": "one captured graph per step (device step counter), same inputs every replay"}
+            "note": "one captured graph per step (device step counter), same inputs every replay; "
+                    "the sequential step (no lookahead)"}
 
 
 # ---------------------------------------------------------------------------
@@ -604,6 +616,7 @@ class WorkloadRun:
                               seed=wl.seed, pooling=wl.pooling, mtp_policy=wl.mtp_policy)
         self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
+        self.lookahead = False
         self.masks = [self.st.new_mask() for _ in range(Ly)]
         self.topks = [torch.empty((Q, R, wl.topk), dtype=torch.int32, device=device) for _ in range(Ly)]
         self.scores = self.st.new_scores()
@@ -618,7 +631,12 @@ class WorkloadRun:
         for k, v in cfg_fields.items():
             setattr(self.cfg, k, v)
         self.st = self.isa.SpinState(self.cfg, device=self.device)
+        self.isa.spin_set_lookahead(self.st, self.lookahead)
         self.t = 0
+
+    def set_lookahead(self, on):
+        self.lookahead = bool(on)
+        self.isa.spin_set_lookahead(self.st, self.lookahead)
 
     def step(self, layers=None):
         """One decode step of every layer: a0..a5, and for MTP rows the
@@ -691,6 +709,7 @@ def workload_arm(args, world, rank, local):
                           spare_slots=base.rows * 4, pooling=POOLINGS[args.pooling],
                           mtp_policy=MTP_POLICIES[args.mtp_policy])
     run = WorkloadRun(wl, device, total)
+    run.set_lookahead(not args.no_lookahead)   # applies to one-row steps
     Ly, Q, R = wl.layers, wl.requests, wl.rows
     # history bootstrap (all-keep), then the workload's warm-up protocol
     run.set_sparsity([0.0] * Ly)
@@ -780,6 +799,7 @@ def workload_arm(args, world, rank, local):
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "avg_launch_ms": score_avg,
                      "bytes_per_launch": per_launch, "bytes_per_kept_slot": per_slot, "traffic": None},
+        "pipelined": bool(run.lookahead and R == 1 and wl.key_fp8),
         "stage_ms_per_step": {k: v[0] / K for k, v in stages.items() if v[1]},
         "gpu_launches": sum(n for _, n in stages.values()),
         "clocks": clk.summary(),
@@ -961,6 +981,7 @@ def predictor_profile(args, world, rank, local):
     wl = workloads.config(WORKLOADS["ragged-8Lx8-256K-1M"], requests=2, ctx0=(94_000, 9_700), steps=total,
                           seed=base.seed + 1000 * rank, spare_slots=8)
     run = WorkloadRun(wl, device, total)
+    run.set_lookahead(not args.no_lookahead)   # applies to one-row steps
     Ly, Q, R = wl.layers, wl.requests, wl.rows
     st = run.st
     run.set_sparsity([0.0] * Ly)

@@ -25,8 +25,9 @@
  *  - Argument errors are reported synchronously through the return value and
  *    launch nothing.  Errors only visible on the device (a ctx_len past the
  *    capacity, a page id outside the cache, an accepted length outside 1..rows,
- *    a bounded wait that gave up) set a device error word and skip the
- *    affected work; they never trap.  spin_get_error reads and clears it.
+ *    a bounded wait that gave up, a ctx_len other than a prepared selection's)
+ *    set a device error word and skip the affected work; they never trap.
+ *    spin_get_error reads and clears it.
  *  - Results are deterministic for a given (seed, step, inputs).
  *  - A state is not thread-safe; use it from one stream at a time.
  *
@@ -123,8 +124,9 @@ typedef enum { SPIN_MTP_UNION_PREFIX = 0, SPIN_MTP_ROW0 = 1 } spin_mtp_policy;
 typedef struct spin_state_s* spin_state;
 
 /* Bytes of device memory a state needs: EMA states V and D for every layer
- * and request, block-score / work-list / quantised-query / score scratch and
- * the device error word.  Returns 0 for an invalid config. */
+ * and request, block-score / work-list / quantised-query / score scratch, the
+ * per-layer selection a pipelined step prepares (spin_set_lookahead) and the
+ * device error word.  Returns 0 for an invalid config. */
 SPIN_API size_t spin_state_bytes(const spin_config* cfg);
 
 /* Creates a state in the caller's device block dev_mem (>= spin_state_bytes,
@@ -217,13 +219,24 @@ SPIN_API spin_status spin_topk(spin_state st, int rows, const float* scores_dev,
  * exceed 2^20 (e.g. 96 requests at 512K slots with b = 64); larger problems
  * return SPIN_EINVAL.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress), so make that first call before any stream
- * capture.  All calls share the one array: calls that overlap on the GPU (on
- * different streams, or from several host threads) race and must be
- * serialised by the caller. */
+ * capture; a new context on the device (after cudaDeviceReset) is detected
+ * by its context id and the address is looked up again on the next call,
+ * which should then also come before any capture.  All calls share the one
+ * array: calls that overlap on the GPU (on different streams, or from several
+ * host threads) race and must be serialised by the caller.  Device-side
+ * errors (a ctx_len outside 1..max_slots-rows+1 sets bit 0, value 1, of the
+ * error word) leave the rows of that request at -1 and are read with
+ * spin_topk_noalloc_error. */
 SPIN_API spin_status spin_topk_noalloc(int num_requests, int rows, int max_rows, int32_t max_slots,
                                        int block_size, int topk, const float* scores_dev,
                                        const uint8_t* mask_dev, const int32_t* ctx_len_dev,
                                        int32_t* topk_dev, spin_stream_t stream);
+
+/* Error word of the last spin_topk_noalloc call on the current device (the
+ * call clears it when it starts): synchronises the stream, copies the word to
+ * *word_out (may be NULL) and returns SPIN_EDEVICE when a bit is set, else
+ * SPIN_OK.  Not for use during stream capture. */
+SPIN_API spin_status spin_topk_noalloc_error(spin_stream_t stream, uint32_t* word_out);
 
 /* a5: EMA update of V (per slot) and D (per offset p_r - s) from the scores
  * of scored slots only (SPIN digest, 核心概要 / arXiv深度剖析; AI Radio, "The
@@ -246,6 +259,27 @@ SPIN_API spin_status spin_decode_step(spin_state st, int layer, int rows, int64_
                              int32_t bt_stride, const void* q, const float* w,
                              const int32_t* ctx_len_dev, int defer_update, uint8_t* mask_dev,
                              int32_t* topk_dev, float* scores_dev, spin_stream_t stream);
+
+/* Pipelined one-row decode steps (enable = 1; 0 turns it off).  A step's
+ * selection (a1 + a2) depends only on the EMA state, the positions and the
+ * step number, all known once the previous step's score kernel has updated
+ * the state (SPIN digest, arXiv深度剖析: the history comes from earlier
+ * steps' indexer scores).  With lookahead on, spin_decode_step with rows = 1,
+ * no deferred update and FP8 keys on the tensor-core kernel also prepares
+ * the next step's selection of the same layer, for ctx_len + 1 and step + 1
+ * (SPIN_STEP_DEVICE: the counter + 1), running the next step's predict
+ * kernel on a second stream of the state beside this step's top-k; the call
+ * joins that stream back into `stream` before it returns, so its outputs are
+ * ready in stream order as before.  Results are bit-identical to the sequential
+ * step's.  The next call of the layer must then pass ctx_len + 1 for every
+ * request, the next step number and the same target: a different target or
+ * step number (host steps), or an intervening spin_ema_update,
+ * spin_reset_requests or spin_state_import, makes the call select afresh; a
+ * request whose ctx_len is not the prepared one sets ERR_LOOKAHEAD (bit 5,
+ * value 32) in the device error word and comes back unscored with all -1
+ * top-k.  The first call on a state creates the second stream and two events
+ * (no device memory); make it outside stream capture. */
+SPIN_API spin_status spin_set_lookahead(spin_state st, int enable);
 
 /* Predictor-quality profile (SPIN listing, Table 1 compares predictors of the
  * indexer's scores by Pearson correlation and top-k recall).

@@ -23,7 +23,7 @@ __all__ = [
     "spin_decode_step", "spin_miss_count", "spin_allocate_layer_sparsity", "spin_get_error",
     "spin_set_layer_sparsity", "spin_set_score_kernel", "spin_reset_requests", "spin_set_fault_injection",
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
-    "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_set_kernel_timing_mask",
+    "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_topk_noalloc_error", "spin_set_lookahead", "spin_set_kernel_timing_mask",
     "SPIN_STEP_DEVICE", "spin_set_step", "spin_advance_step", "SPIN_POOL_MAX", "SPIN_POOL_MEAN", "SPIN_POOL_TOP4",
     "SPIN_MTP_UNION_PREFIX", "SPIN_MTP_ROW0", "SPIN_PRED_EMA", "SPIN_PRED_RANDOM", "spin_slot_prediction",
     "spin_pearson", "spin_topk_overlap",
@@ -90,6 +90,7 @@ def load():
         "spin_set_kernel_timing": (S, [_vp, ctypes.c_int]),
         "spin_set_kernel_timing_mask": (S, [_vp, _u32]),
         "spin_set_step": (S, [_vp, _i64, _vp]),
+        "spin_set_lookahead": (S, [_vp, ctypes.c_int]),
         "spin_advance_step": (S, [_vp, _vp]),
         "spin_kernel_times": (S, [_vp, _vp, _vp, ctypes.c_int]),
         "spin_reset_requests": (S, [_vp, ctypes.c_int, _vp, ctypes.c_int, _vp]),
@@ -99,6 +100,7 @@ def load():
         "spin_topk": (S, [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
         "spin_topk_noalloc": (S, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32, ctypes.c_int, ctypes.c_int, _vp,
                                   _vp, _vp, _vp, _vp]),
+        "spin_topk_noalloc_error": (S, [_vp, ctypes.POINTER(_u32)]),
         "spin_ema_update": (S, [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]),
         "spin_decode_step": (S, [_vp, ctypes.c_int, ctypes.c_int, _i64, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp,
                                  ctypes.c_int, _vp, _vp, _vp, _vp]),
@@ -256,6 +258,13 @@ def spin_set_step(st: SpinState, step: int, stream=None) -> None:
     _check(load().spin_set_step(st.handle, int(step), _stream(stream)), "spin_set_step")
 
 
+def spin_set_lookahead(st: SpinState, enable: bool = True) -> None:
+    """Pipelined one-row decode steps: each step prepares the next step's
+    selection, its predict kernel on a second stream beside the step's top-k
+    (see include/spin.h)."""
+    _check(load().spin_set_lookahead(st.handle, 1 if enable else 0), "spin_set_lookahead")
+
+
 def spin_advance_step(st: SpinState, stream=None) -> None:
     _check(load().spin_advance_step(st.handle, _stream(stream)), "spin_advance_step")
 
@@ -315,6 +324,14 @@ def spin_topk_noalloc(num_requests: int, rows: int, max_rows: int, max_slots: in
                                     _dev(scores, "scores", torch.float32), _dev(mask, "mask", torch.uint8),
                                     _dev(ctx_len, "ctx_len", torch.int32), _dev(topk, "topk", torch.int32),
                                     _stream(stream)), "spin_topk_noalloc")
+
+
+def spin_topk_noalloc_error(stream=None):
+    """Returns (status, raw device error word) of the last spin_topk_noalloc
+    call on the current device; synchronises the stream."""
+    word = _u32()
+    status = load().spin_topk_noalloc_error(_stream(stream), ctypes.byref(word))
+    return int(status), int(word.value)
 
 
 def spin_ema_update(st: SpinState, layer: int, rows: int, scores, mask, ctx_len, accepted=None,

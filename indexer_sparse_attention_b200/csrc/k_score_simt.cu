@@ -2,7 +2,8 @@
 //
 // a0: each (row, head) query vector is quantised to E4M3 with a power-of-two
 //     scale folded into the head weight (quantize_vec); the decode step does
-//     this inside its select kernel, the standalone score call here.
+//     this inside its predict or select kernel, the standalone score call and
+//     the pipelined decode step (spin_set_lookahead) here.
 // a3: I_{r,s} = sigma_s * sum_h w'_{r,h} * ReLU(q8_{r,h} . k8_s) over the slots
 //     of kept blocks with s <= p_r (SPIN listing, Abstract; SPIN digest,
 //     arXiv深度剖析: the indexer input is pruned to the kept blocks).  fp32 keys:
@@ -17,6 +18,7 @@ namespace spin {
 
 // One warp per (request, row, head).
 __global__ void __launch_bounds__(256) k_quantize_q(ScoreArgs a) {
+  pdl_enter();  // q8 and wq may still be read by the previous score launch
   const Layout L = a.lay;
   const int64_t nvec = (int64_t)L.Q * a.rows * L.H;
   const int64_t v = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -26,8 +28,8 @@ __global__ void __launch_bounds__(256) k_quantize_q(ScoreArgs a) {
 
 cudaError_t launch_quantize_q(const ScoreArgs& a, cudaStream_t s) {
   const int64_t nvec = (int64_t)a.lay.Q * a.rows * a.lay.H;
-  k_quantize_q<<<(unsigned)((nvec + 7) / 8), 256, 0, s>>>(a);
-  return cudaGetLastError();
+  PdlLaunch l(dim3((unsigned)((nvec + 7) / 8)), dim3(256), 0, s);
+  return cudaLaunchKernelEx(&l.cfg, k_quantize_q, a);
 }
 
 // ---------------------------------------------------------------------------

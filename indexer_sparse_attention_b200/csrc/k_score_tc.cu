@@ -397,7 +397,12 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       int v = 0;
       if (q < L.Q) {
         const int64_t ctx = a.ctx_len[q];
-        const bool ok = ctx >= 1 && ctx + a.rows - 1 <= L.max_slots;
+        bool ok = ctx >= 1 && ctx + a.rows - 1 <= L.max_slots;
+        if (ok && a.ctx_sel && a.ctx_sel[q] != ctx) {  // the prepared selection is for another ctx_len
+          ok = false;
+          if (blockIdx.x == 0) raise_error(a.err, ERR_LOOKAHEAD, q, (uint32_t)ctx);
+        }
+        if (a.ctx_next && blockIdx.x == 0) a.ctx_next[q] = (int32_t)(ctx + 1);
         v = ok ? (a.kept[q] + 1) / 2 : 0;
       }
       int tot;

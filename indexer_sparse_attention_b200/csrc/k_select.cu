@@ -14,49 +14,52 @@
 //     exploration among row 0's unkept blocks.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "spin_internal.cuh"
 #include "block_scan.cuh"
 
 namespace spin {
 
 // ---------------------------------------------------------------------------
-// a1: one warp per 256-slot chunk of one request; a lane takes 8 consecutive
-// slots (two float4 loads of V and the D window its rows need, all issued
-// before any use), and the b/8 lanes of a block reduce with shuffles.
-// Block sizes 16..256 (powers of two).
+// a1: grid column x = request; its blocks' warps take 256-slot chunks of that
+// request in turn (no division per chunk).  A lane takes 8 consecutive slots:
+// two float4 loads of V and the D window its rows need (offsets p0-i0-7 ..
+// p0-i0+R-1) as aligned float4 loads, all issued before any use; the b/8
+// lanes of a block reduce with shuffles.  When a0 rides along, the row's
+// first warps quantise that request's (row, head) query vectors first: the
+// kernel is bound by HBM, so they cost next to nothing and the select kernel
+// that follows is spared them.  Block sizes 16..256 (powers of two).
 // ---------------------------------------------------------------------------
 template <int R, int P>
-__global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
+__global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
   pdl_enter();
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
   const int lb = __ffs(L.b) - 1;
   const int lpb = L.b >> 3;  // lanes per block
-  const int64_t chunks = (L.slot_stride + 255) / 256;
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  // a0 rides along when asked: the first nvec warp tasks quantise the
-  // (request, row, head) query vectors; this kernel is bound by HBM, so they
-  // cost next to nothing and the select kernel that follows is spared them
-  const int64_t nvec = a.q8 ? (int64_t)L.Q * a.rows * L.H : 0;
-  for (int64_t wid0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       wid0 < nvec + (int64_t)L.Q * chunks; wid0 += nwarps) {
-    if (wid0 < nvec) {
-      quantize_vec(a.q, a.w, a.q_bf16, L.d, wid0, a.q8, a.wq);
-      continue;
-    }
-    const int64_t wid = wid0 - nvec;
-    const int q = (int)(wid / chunks);
-    const int64_t c = wid % chunks;
-    const int64_t ctx = a.ctx_len[q];
-    if (ctx < 1 || ctx + R - 1 > L.max_slots) continue;  // warp-uniform; select reports it
-    const int64_t n_last = row_blocks(ctx, R - 1, L.b);
-    if (c * 256 >= n_last * L.b) continue;                 // warp-uniform
-    const int64_t p0 = ctx - 1;
-    const int64_t i0 = c * 256 + lane * 8;
+  const int q = blockIdx.x;
+  const int wpr = (int)gridDim.y * (blockDim.x >> 5);                   // warps of this request
+  const int wr = (int)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);  // this warp among them
+  if (a.q8) {
+    const int nv = a.rows * L.H;
+    for (int v = wr; v < nv; v += wpr) quantize_vec(a.q, a.w, a.q_bf16, L.d, (int64_t)q * nv + v, a.q8, a.wq);
+  }
+  const int64_t ctx = a.ctx_len[q];
+  if (ctx < 1 || ctx + R - 1 > L.max_slots) return;  // block-uniform; select reports it
+  const int64_t n_last = row_blocks(ctx, R - 1, L.b);
+  const int nchunks = (int)((n_last * L.b + 255) / 256);
+  const int64_t p0 = ctx - 1;
+  const float* V = a.V + (int64_t)q * L.slot_stride;
+  const float* D = a.D + (int64_t)q * L.slot_stride;
+  // the D window of every lane starts at p0 - i0 - 7 with i0 = 0 mod 8: its
+  // offset from a 16-byte boundary is the same for all lanes
+  const int sh = (int)((p0 + 1) & 3);
+  constexpr int kNV = (R + 7 + 3 + 3) / 4;  // float4 loads covering R + 7 values at any offset
+  for (int c = wr; c < nchunks; c += wpr) {
+    const int64_t i0 = (int64_t)c * 256 + lane * 8;
     const int64_t j = i0 >> lb;
     const bool active = j < n_last && i0 <= p0 + R - 1;
-    const float* V = a.V + (int64_t)q * L.slot_stride;
-    const float* D = a.D + (int64_t)q * L.slot_stride;
     float vv[8];
     float dw[R + 7];  // D at offsets p0 - i0 - 7 .. p0 - i0 + R - 1
 #pragma unroll
@@ -68,10 +71,29 @@ __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
       const float4 v1 = __ldg(reinterpret_cast<const float4*>(V + i0 + 4));
       vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
       vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+      const int64_t ob = p0 - i0 - 7 - sh;  // 16-byte aligned start of the window
+      if (ob >= 0 && ob + 4 * kNV <= L.slot_stride) {
+        float buf[4 * kNV];
 #pragma unroll
-      for (int t = 0; t < R + 7; ++t) {
-        const int64_t di = p0 - i0 - 7 + t;
-        if (di >= 0) dw[t] = __ldg(D + di);
+        for (int u = 0; u < kNV; ++u) {
+          const float4 d4 = __ldg(reinterpret_cast<const float4*>(D + ob) + u);
+          buf[4 * u] = d4.x; buf[4 * u + 1] = d4.y; buf[4 * u + 2] = d4.z; buf[4 * u + 3] = d4.w;
+        }
+#define SPIN_DW_FROM(S)                                       \
+  _Pragma("unroll") for (int t = 0; t < R + 7; ++t) dw[t] = buf[t + (S)];
+        switch (sh) {  // warp-uniform
+          case 0: SPIN_DW_FROM(0) break;
+          case 1: SPIN_DW_FROM(1) break;
+          case 2: SPIN_DW_FROM(2) break;
+          default: SPIN_DW_FROM(3) break;
+        }
+#undef SPIN_DW_FROM
+      } else {  // the window reaches below offset 0 (the newest slots) or past the row
+#pragma unroll
+        for (int t = 0; t < R + 7; ++t) {
+          const int64_t di = p0 - i0 - 7 + t;
+          if (di >= 0) dw[t] = __ldg(D + di);
+        }
       }
     }
 #pragma unroll
@@ -149,11 +171,14 @@ __global__ void __launch_bounds__(256) k_predict_pool(StepArgs a) {
 }
 
 cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
+  // one wave (4 blocks of 256 threads per SM at <= 64 registers) over all
+  // requests, each request's chunks shared by the gx blocks of its column
   const int64_t chunks = (a.lay.slot_stride + 255) / 256;
-  const int64_t warps = (int64_t)a.lay.Q * chunks + (a.q8 ? (int64_t)a.lay.Q * a.rows * a.lay.H : 0);
-  int64_t blocks = (warps + 7) / 8;
-  if (blocks > 148 * 32) blocks = 148 * 32;
-  PdlLaunch l(dim3((unsigned)blocks), dim3(256), 0, s);
+  int64_t gx = (148 * 4) / a.lay.Q;
+  gx = std::min<int64_t>(gx, (chunks + 7) / 8);
+  gx = std::max<int64_t>(std::min<int64_t>(gx, 65535), 1);
+  PdlLaunch l(dim3((unsigned)a.lay.Q, (unsigned)gx), dim3(256), 0, s);
+  l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
   void (*k)(StepArgs) = nullptr;
 #define SPIN_PREDICT_CASE(R)                                            \
   case R:                                                               \
@@ -357,7 +382,7 @@ __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t
 __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   pdl_enter();
   StepArgs a = a_in;
-  if (a.step_dev) a.step = *a.step_dev;  // the state's counter (read after the predecessors finished)
+  if (a.step_dev) a.step = *a.step_dev + a.step_add;  // the state's counter (read after the predecessors finished)
   const Layout L = a.lay;
   const int q = blockIdx.x;
   extern __shared__ __align__(16) uint8_t dyn[];
@@ -377,12 +402,14 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   uint8_t* mask_row = a.mask + (int64_t)q * L.max_blocks;
   if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {
     if (threadIdx.x == 0) {
-      raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
+      if (!a.quiet) raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
       a.kept[q] = 0;
+      if (a.ctx_sel) a.ctx_sel[q] = -1;
     }
     for (int64_t j = threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = 0;
     return;
   }
+  if (a.ctx_sel && threadIdx.x == 0) a.ctx_sel[q] = (int32_t)ctx;
   const int n_last = (int)row_blocks(ctx, a.rows - 1, L.b);
   for (int j = threadIdx.x; j < n_last; j += blockDim.x) m[j] = 0;
   __syncthreads();
@@ -574,7 +601,7 @@ __device__ void cl_mark_selected(const uint32_t* keys, int hi, Valid valid, uint
 __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
   pdl_enter();
   StepArgs a = a_in;
-  if (a.step_dev) a.step = *a.step_dev;  // the state's counter (read after the predecessors finished)
+  if (a.step_dev) a.step = *a.step_dev + a.step_add;  // the state's counter (read after the predecessors finished)
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
@@ -596,13 +623,15 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
   uint8_t* mask_row = a.mask + (int64_t)q * L.max_blocks;
   if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {  // alike in every rank
     if (cr == 0 && threadIdx.x == 0) {
-      raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
+      if (!a.quiet) raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
       a.kept[q] = 0;
+      if (a.ctx_sel) a.ctx_sel[q] = -1;
     }
     const int z0 = range_lo((int)L.max_blocks, cr, C), z1 = range_lo((int)L.max_blocks, cr + 1, C);
     for (int j = z0 + threadIdx.x; j < z1; j += blockDim.x) mask_row[j] = 0;
     return;
   }
+  if (a.ctx_sel && cr == 0 && threadIdx.x == 0) a.ctx_sel[q] = (int32_t)ctx;
   const int n_last = (int)row_blocks(ctx, a.rows - 1, L.b);
   const int j0 = range_lo(n_last, cr, C), j1 = range_lo(n_last, cr + 1, C);
   const int nl = j1 - j0;  // this rank's blocks: j = j0 + i
@@ -763,6 +792,7 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   while (C < 8 && a.lay.Q * C * 2 <= sms && a.lay.max_blocks >= (int64_t)C * 2 * 2048) C *= 2;
   if (C > 1) {
     PdlLaunch l(dim3(a.lay.Q * C), dim3(kSelThreads), smem, s);
+    l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
     l.attr[1].id = cudaLaunchAttributeClusterDimension;
     l.attr[1].val.clusterDim.x = (unsigned)C;
     l.attr[1].val.clusterDim.y = 1;
@@ -774,6 +804,7 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
     cudaGetLastError();  // this shape cannot be placed
   }
   PdlLaunch l(dim3(a.lay.Q), dim3(kSelThreads), smem, s);
+  l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
   return cudaLaunchKernelEx(&l.cfg, k_select, a);
 }
 

@@ -718,10 +718,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   const unsigned rid = blockIdx.x / (unsigned)C;
   const int q = rid / a.rows, r = rid % a.rows;
   int32_t* out = a.topk + ((int64_t)q * a.rows + r) * L.k;
+  if (a.mask_src && r == 0 && cr == 0)  // the selection's mask row, to the caller's buffer
+    for (int64_t j = threadIdx.x; j < L.max_blocks; j += blockDim.x)
+      a.mask_dst[(int64_t)q * L.max_blocks + j] = a.mask_src[(int64_t)q * L.max_blocks + j];
   __shared__ TopkShared sh;
   extern __shared__ __align__(16) uint8_t dyn[];
   const int64_t ctx = a.ctx_len[q];
-  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {
+  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots || (a.ctx_sel && a.ctx_sel[q] != ctx)) {
     if (cr == 0)
       for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;

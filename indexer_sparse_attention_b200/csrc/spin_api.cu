@@ -39,6 +39,23 @@ struct spin_state_s {
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
   int64_t launches[8];
+  // Lookahead (spin_set_lookahead): each one-row decode step also prepares
+  // the next step's selection of its layer, so that the step's top-k runs on
+  // a second stream beside the next step's predict kernel.
+  int lookahead;
+  cudaStream_t side;                 // the next step's predict runs here (created on first use)
+  cudaEvent_t ev_scored, ev_pred;    // fork after the score kernel, join after the side stream's predict
+  struct Prepared {
+    bool ready;
+    int64_t step;                    // the step the selection is for (SPIN_STEP_DEVICE: the counter's)
+    float sparsity;                  // the layer's target it was made with
+  };
+  std::vector<Prepared> prep;        // per layer
+  int32_t* la_work;                  // [L][Q][blk_stride] kept block ids of the prepared selection
+  int32_t* la_kept;                  // [L][Q]
+  uint8_t* la_mask;                  // [L][Q][max_blocks]
+  int32_t* la_ctx;                   // [L][Q] ctx_len each request's selection was made for (-1: none)
+  int32_t* ctx_next;                 // [Q] ctx_len + 1, written by the score kernel
   uint32_t magic;
 };
 
@@ -97,7 +114,7 @@ Layout make_layout(const spin_config* c) {
 int64_t gmax_stride(const Layout& L) { return L.blk_stride * std::max(1, L.b / 32); }
 
 struct Carve {
-  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, step, total;
+  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, step, la_work, la_kept, la_mask, la_ctx, ctx_next, total;
 };
 
 Carve carve(const Layout& L) {
@@ -115,6 +132,11 @@ Carve carve(const Layout& L) {
   k.scores = take((size_t)L.Q * L.R * L.slot_stride * 4);
   k.gmax = take((size_t)L.Q * L.R * gmax_stride(L) * 4);
   k.step = take(sizeof(int64_t));
+  k.la_work = take((size_t)L.L * L.Q * L.blk_stride * 4);
+  k.la_kept = take((size_t)L.L * L.Q * 4);
+  k.la_mask = take((size_t)L.L * L.Q * L.max_blocks);
+  k.la_ctx = take((size_t)L.L * L.Q * 4);
+  k.ctx_next = take((size_t)L.Q * 4);
   k.total = off;
   return k;
 }
@@ -138,6 +160,10 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   a.mtp_row0 = st->cfg.mtp_policy == SPIN_MTP_ROW0 && rows > 1;
   a.step = step < 0 ? 0 : step;
   a.step_dev = step == SPIN_STEP_DEVICE ? st->step_dev : nullptr;
+  a.step_add = 0;
+  a.ctx_sel = nullptr;
+  a.quiet = 0;
+  a.no_pdl = 0;
   a.sparsity = st->sparsity[layer];
   a.gamma = st->cfg.gamma;
   a.alpha = st->cfg.alpha;
@@ -194,10 +220,19 @@ cudaError_t staged(spin_state st, int stage, cudaStream_t s, F launch) {
 }
 
 // Quantise (FP8 keys) and score the kept blocks listed in st->work / st->kept.
+// The kept-block list a score reads, and the checks of a prepared selection.
+struct Selection {
+  const int32_t* work;
+  const int32_t* kept;
+  const int32_t* ctx_sel;  // or null
+  int32_t* ctx_next;       // or null
+};
+
 spin_status run_score(spin_state st, int layer, int rows, const void* keys, const float* key_scale,
                       int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
                       const float* w, const int32_t* ctx_len, const uint8_t* mask, float* scores,
-                      bool fuse_ema, cudaStream_t stream, bool* wrote_gmax = nullptr, bool quantized = false) {
+                      bool fuse_ema, cudaStream_t stream, bool* wrote_gmax = nullptr, bool quantized = false,
+                      const Selection* sel = nullptr) {
   ScoreArgs a;
   a.lay = st->lay;
   a.rows = rows;
@@ -212,8 +247,10 @@ spin_status run_score(spin_state st, int layer, int rows, const void* keys, cons
   a.w = w;
   a.ctx_len = ctx_len;
   a.mask = mask;
-  a.work = st->work;
-  a.kept = st->kept;
+  a.work = sel ? sel->work : st->work;
+  a.kept = sel ? sel->kept : st->kept;
+  a.ctx_sel = sel ? sel->ctx_sel : nullptr;
+  a.ctx_next = sel ? sel->ctx_next : nullptr;
   a.q8 = st->q8;
   a.wq = st->wq;
   a.scores = scores;
@@ -246,6 +283,85 @@ spin_status run_score(spin_state st, int layer, int rows, const void* keys, cons
 
 spin_status check_rows(spin_state st, int rows) {
   return (rows >= 1 && rows <= st->cfg.max_rows) ? SPIN_OK : SPIN_EINVAL;
+}
+
+// The pipelined one-row decode step (spin_set_lookahead).  The step's
+// selection was prepared by the previous step of this layer (or is made here
+// when there is none, or it was made for another step or target):
+//   stream:  a0 -> score + fused EMA (writes ctx_len + 1) -> top-k (+ mask) -> [join] -> select(next)
+//   side:                                      [fork] -> predict(next) --------^
+// The next step's predict reads only V and D, which the score kernel has
+// finished, and writes only the block scores, so it runs beside this step's
+// top-k; the next selection overwrites the kept lists the top-k reads, so it
+// follows the top-k.  The top-k is launched first, directly behind the score
+// kernel, so that its CTAs are placed before the predict kernel's fill the
+// SMs.  Results are those of the sequential step: the next selection is
+// computed from the same state, positions (ctx_len + 1) and step number as the
+// next call would compute it.
+spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const void* keys, const float* key_scale,
+                                  int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
+                                  const float* w, const int32_t* ctx_len, uint8_t* mask_dev, int32_t* topk_dev,
+                                  float* scores, cudaStream_t s) {
+  const Layout& L = st->lay;
+  spin_state_s::Prepared& P = st->prep[layer];
+  const float sp = st->sparsity[layer];
+  int32_t* work = st->la_work + (size_t)layer * L.Q * L.blk_stride;
+  int32_t* kept = st->la_kept + (size_t)layer * L.Q;
+  uint8_t* lmask = st->la_mask + (size_t)layer * L.Q * L.max_blocks;
+  int32_t* lctx = st->la_ctx + (size_t)layer * L.Q;
+  const int64_t next = step == SPIN_STEP_DEVICE ? SPIN_STEP_DEVICE : step + 1;
+  auto select_args = [&](const int32_t* ctx, int64_t stp, bool ahead) {
+    StepArgs a = step_args(st, layer, 1, stp, ctx, lmask);
+    a.step_add = (ahead && stp == SPIN_STEP_DEVICE) ? 1 : 0;
+    a.work = work;
+    a.kept = kept;
+    a.ctx_sel = lctx;
+    a.quiet = ahead ? 1 : 0;
+    return a;
+  };
+  spin_status r;
+  P.ready = P.ready && P.sparsity == sp && P.step == step;
+  if (!P.ready) {  // no selection prepared for this step: make it now
+    StepArgs a = select_args(ctx_len, step, false);
+    if (sp > 0.0f) {
+      r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
+      if (r != SPIN_OK) return r;
+    }
+    r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
+    if (r != SPIN_OK) return r;
+  }
+  P.ready = false;  // consumed below; set again once the next one is issued
+  const Selection sel{work, kept, lctx, st->ctx_next};
+  bool gm = false;
+  r = run_score(st, layer, 1, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len, lmask, scores,
+                true, s, &gm, false, &sel);
+  if (r != SPIN_OK) return r;
+  // fork: the next step's predict on the side stream
+  StepArgs a = select_args(st->ctx_next, next, true);
+  a.no_pdl = 1;  // both launches below follow a wait on the other stream's event
+  cudaError_t e = cudaEventRecord(st->ev_scored, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->side, st->ev_scored, 0);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (sp > 0.0f) {
+    r = cuda_status(staged(st, kPredict, st->side, [&] { return launch_predict_pool(a, st->side); }));
+    if (r != SPIN_OK) return r;
+  }
+  e = cudaEventRecord(st->ev_pred, st->side);  // the predict's end
+  if (e != cudaSuccess) return cuda_status(e);
+  // this step's top-k, which also hands the selection's mask to the caller
+  TopkArgs t{L, 1, scores, mask_dev, ctx_len, work, kept, topk_dev, st->err, gm ? st->gmax : nullptr,
+             st->gstride, lctx, lmask, mask_dev};
+  r = cuda_status(staged(st, kTopk, s, [&] { return launch_topk(t, s); }));
+  if (r != SPIN_OK) return r;
+  // join, then the next step's selection
+  e = cudaStreamWaitEvent(s, st->ev_pred, 0);
+  if (e != cudaSuccess) return cuda_status(e);
+  r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
+  if (r != SPIN_OK) return r;
+  P.ready = true;
+  P.step = next;
+  P.sparsity = sp;
+  return SPIN_OK;
 }
 
 }  // namespace
@@ -283,6 +399,15 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->gmax = (float*)(st->base + k.gmax);
   st->gstride = gmax_stride(L);
   st->step_dev = (int64_t*)(st->base + k.step);
+  st->la_work = (int32_t*)(st->base + k.la_work);
+  st->la_kept = (int32_t*)(st->base + k.la_kept);
+  st->la_mask = (uint8_t*)(st->base + k.la_mask);
+  st->la_ctx = (int32_t*)(st->base + k.la_ctx);
+  st->ctx_next = (int32_t*)(st->base + k.ctx_next);
+  st->lookahead = 0;
+  st->side = nullptr;
+  st->ev_scored = st->ev_pred = nullptr;
+  st->prep.assign(cfg->num_layers, spin_state_s::Prepared{false, 0, 0.0f});
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
   st->inject = 0;
@@ -315,6 +440,9 @@ spin_status spin_state_destroy(spin_state st) {
     cudaEventDestroy(r.b);
   }
   for (auto e : st->pool) cudaEventDestroy(e);
+  if (st->ev_scored) cudaEventDestroy(st->ev_scored);
+  if (st->ev_pred) cudaEventDestroy(st->ev_pred);
+  if (st->side) cudaStreamDestroy(st->side);
   st->magic = 0;
   delete st;
   return SPIN_OK;
@@ -326,7 +454,7 @@ spin_status spin_set_layer_sparsity(spin_state st, const float* s_host) {
   for (int l = 0; l < st->cfg.num_layers; ++l)
     if (!(s_host[l] >= 0.0f && s_host[l] < 1.0f)) return SPIN_EINVAL;
   st->sparsity.assign(s_host, s_host + st->cfg.num_layers);
-  return SPIN_OK;
+  return SPIN_OK;  // a prepared selection made with another target is dropped at its next use
 }
 
 spin_status spin_set_score_kernel(spin_state st, int kind) {
@@ -336,6 +464,20 @@ spin_status spin_set_score_kernel(spin_state st, int kind) {
                                       st->encode_fn))
     return SPIN_EUNSUPPORTED;
   st->score_kernel = kind;
+  return SPIN_OK;
+}
+
+spin_status spin_set_lookahead(spin_state st, int enable) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (enable != 0 && enable != 1) return SPIN_EINVAL;
+  if (enable && !st->side) {
+    cudaError_t e = cudaStreamCreateWithFlags(&st->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_scored, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_pred, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  st->lookahead = enable;
+  for (auto& p : st->prep) p.ready = false;
   return SPIN_OK;
 }
 
@@ -402,6 +544,8 @@ spin_status spin_reset_requests(spin_state st, int layer, const int32_t* req_hos
     if (req_host[i] < 0 || req_host[i] >= st->cfg.num_requests) return SPIN_EINVAL;
   cudaStream_t s = (cudaStream_t)stream;
   const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  for (int l = 0; l < st->cfg.num_layers; ++l)
+    if (layer < 0 || l == layer) st->prep[l].ready = false;   // the state changes under the prepared selection
   for (int i0 = 0; i0 < n; i0 += ReqList::kMax) {
     ReqList list;
     list.n = std::min(n - i0, ReqList::kMax);
@@ -482,6 +626,7 @@ spin_status spin_ema_update(spin_state st, int layer, int rows, const float* sco
   a.beta = beta_of(st->cfg.alpha);
   a.err = st->err;
   cudaStream_t s = (cudaStream_t)stream;
+  st->prep[layer].ready = false;
   return cuda_status(staged(st, kEma, s, [&] { return launch_ema_update(a, s); }));
 }
 
@@ -500,8 +645,12 @@ spin_status spin_decode_step(spin_state st, int layer, int rows, int64_t step, c
   if (defer_update && !scores_dev) return SPIN_EINVAL;
   float* scores = scores_dev ? scores_dev : st->scores;
   cudaStream_t s = (cudaStream_t)stream;
-  StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
   const bool fp8 = st->cfg.key_dtype == SPIN_FP8_E4M3;
+  if (st->lookahead && rows == 1 && !defer_update && fp8 && use_tc(st, 1))
+    return decode_step_lookahead(st, layer, step, keys, key_scale, num_pages, block_table, bt_stride, q, w,
+                                 ctx_len_dev, mask_dev, topk_dev, scores, s);
+  st->prep[layer].ready = false;  // this step's EMA update moves the state under any prepared selection
+  StepArgs a = step_args(st, layer, rows, step, ctx_len_dev, mask_dev);
   if (fp8) {  // a0 rides in the predict kernel, or in select when there is no prediction
     a.q = q;
     a.w = w;
@@ -666,6 +815,7 @@ spin_status spin_state_import(spin_state st, const void* host, size_t bytes, spi
   const size_t half = spin_state_export_bytes(st) / 2;
   if (!host || bytes < 2 * half) return SPIN_EINVAL;
   cudaStream_t s = (cudaStream_t)stream;
+  for (auto& p : st->prep) p.ready = false;
   cudaError_t e = cudaMemcpyAsync(st->V, host, half, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->D, (const char*)host + half, half, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -20,6 +20,7 @@ enum : uint32_t {
   ERR_ACCEPTED = 1u << 2,     // accepted length outside 1..rows
   ERR_TIMEOUT = 1u << 3,      // a bounded mbarrier wait gave up
   ERR_CAPACITY = 1u << 4,     // a shape exceeded a kernel's on-chip capacity
+  ERR_LOOKAHEAD = 1u << 5,    // ctx_len differs from the one a prepared selection was made for
 };
 
 // Error word block: [0] flags, [1] first offending request, [2] first value.
@@ -214,6 +215,7 @@ struct StepArgs {
   int layer, rows;
   int64_t step;
   const int64_t* step_dev;  // non-null: the step is read from the state's counter
+  int64_t step_add;         // added to the counter's step (a selection prepared one step ahead)
   int pooling;              // spin_pooling: block reduction of the predicted scores
   int mtp_row0;             // SPIN_MTP_ROW0 with rows > 1: row 0 alone predicts
   float sparsity, gamma, alpha;
@@ -223,6 +225,11 @@ struct StepArgs {
   float* S;
   int32_t* work;      // [Q][blk_stride] kept block ids, ascending
   int32_t* kept;      // [Q] kept counts
+  int32_t* ctx_sel;   // [Q] out, or null: the ctx_len each request's selection was made for (-1: none)
+  int quiet;          // a selection prepared one step ahead: an out-of-range ctx_len is no error
+                      // (the request gets no selection, ctx_sel -1)
+  int no_pdl;         // launch as an ordinary dependent (after a wait on another stream's event)
+
   float* V;           // layer base [Q][slot_stride]
   float* D;
   ErrWord* err;
@@ -273,6 +280,9 @@ struct ScoreArgs {
   float* D;
   float alpha, beta;   // beta = fl32(1 - alpha), computed once on the host
   int inject;          // test hook: withhold the first key stage of CTA 0
+  const int32_t* ctx_sel;  // [Q] or null: the ctx_len the selection was made for; a request whose
+                           // ctx_len differs raises ERR_LOOKAHEAD and is not scored
+  int32_t* ctx_next;       // [Q] or null: written with ctx_len + 1 (the next step's, one row a step)
   float* gmax;         // [Q][R][gstride] max score of each 32-slot group of the
   int64_t gstride;     // kept-slot order (tensor-core kernel only), or null
 };
@@ -294,6 +304,9 @@ struct TopkArgs {
   ErrWord* err;
   const float* gmax;  // group maxima written by the score kernel, or null
   int64_t gstride;
+  const int32_t* ctx_sel;  // [Q] or null: a request whose ctx_len differs comes back all -1
+  const uint8_t* mask_src; // [Q][max_blocks] or null: copied to mask_dst (a prepared selection's mask
+  uint8_t* mask_dst;       // handed to the caller by the top-k launch)
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 

@@ -28,24 +28,65 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-int32_t* g_ptr[kMaxDevices] = {nullptr};
+struct Cached {
+  unsigned long long ctx_id;  // unique id of the context the address belongs to
+  int32_t* ptr;
+};
+Cached g_cache[kMaxDevices] = {};
 
-// Device address of the array on the current device, resolved once per device
-// with that device current (in host code the symbol itself is only a
-// stand-in, not a device address).
+typedef int (*CtxGetCurrentFn)(void**);
+typedef int (*CtxGetIdFn)(void*, unsigned long long*);
+
+// Unique id of the current context (cuCtxGetCurrent + cuCtxGetId through the
+// runtime's driver entry points), or 0 when it cannot be read.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    cudaDriverEntryPointQueryResult q1, q2;
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+        q2 == cudaDriverEntryPointSuccess) {
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(f1);
+      get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    cudaGetLastError();
+  }
+  if (!get_cur || !get_id) return 0;
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+  return id;
+}
+
+// Device address of the array on the current device, resolved with that
+// device current (in host code the symbol itself is only a stand-in, not a
+// device address).  The address is cached per device together with the id of
+// the context it was resolved in; a new context on the device (after
+// cudaDeviceReset, for example) loads the module again, so the address is
+// resolved again.  If the context id cannot be read, it is resolved on every
+// call.
 cudaError_t scratch_on_current_device(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_ptr[dev]) {
+  Cached& c = g_cache[dev];
+  unsigned long long id = current_ctx_id();
+  if (!c.ptr || id == 0 || id != c.ctx_id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the primary context current if needed
     if (e != cudaSuccess) return e;
-    g_ptr[dev] = static_cast<int32_t*>(p);
+    c.ptr = static_cast<int32_t*>(p);
+    c.ctx_id = id ? id : current_ctx_id();
   }
-  *out = g_ptr[dev];
+  *out = c.ptr;
   return cudaSuccess;
 }
 
@@ -101,4 +142,22 @@ extern "C" SPIN_API spin_status spin_topk_noalloc(int num_requests, int rows, in
     return SPIN_ECUDA;
   }
   return SPIN_OK;
+}
+
+// Reads the error word the last spin_topk_noalloc call on this device left in
+// the fixed array.  Synchronises the stream first.
+extern "C" SPIN_API spin_status spin_topk_noalloc_error(spin_stream_t stream, uint32_t* word_out) {
+  int32_t* base = nullptr;
+  cudaError_t e = scratch_on_current_device(&base);
+  cudaStream_t s = (cudaStream_t)stream;
+  ErrWord h{};
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, base, sizeof(ErrWord), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "libspin: CUDA error %s\n", cudaGetErrorString(e));
+    return SPIN_ECUDA;
+  }
+  if (word_out) *word_out = h.flags;
+  return h.flags ? SPIN_EDEVICE : SPIN_OK;
 }

@@ -66,6 +66,8 @@ def _load():
             lib.orc_predict_pool.argtypes = [_f32p, _f32p, _i64, ctypes.c_int, ctypes.c_int, _i64, _f32p]
             lib.orc_predict_pool_mode.argtypes = [_f32p, _f32p, _i64, ctypes.c_int, ctypes.c_int, _i64, ctypes.c_int,
                                                   _f32p]
+            lib.orc_mean_exact.argtypes = [_f32p, ctypes.c_int]
+            lib.orc_mean_exact.restype = ctypes.c_float
             lib.orc_budget.argtypes = [_i64, ctypes.c_double]
             lib.orc_budget.restype = _i64
             lib.orc_explore_count.argtypes = [_i64, ctypes.c_double]
@@ -163,6 +165,13 @@ def quantize_q(q: np.ndarray, w: np.ndarray):
 
 
 POOL_MAX, POOL_MEAN, POOL_TOP4 = 0, 1, 2
+
+
+def mean_exact(z) -> np.float32:
+    """The mean of 1..256 floats: the exact sum over the count, rounded once
+    to the nearest float (the definition the Mean and Top-4 pools use)."""
+    z = _c(np.atleast_1d(z), np.float32)
+    return np.float32(_load().orc_mean_exact(_p(z, _f32p), int(z.size)))
 
 
 def predict_pool(V: np.ndarray, D: np.ndarray, ctx_len: int, rows: int, b: int, n_stride: int, pooling: int = 0):

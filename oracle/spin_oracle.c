@@ -186,18 +186,113 @@ ORC_API void orc_predict_pool(const float* V, const float* D, int64_t ctx_len, i
 /* Block-reduction variants of the pool ([listing] Figure 3: "Mean and Top-4
  * compared with Max pooling"; the pages do not define them, so these are the
  * plainest readings).  Over the block's visible slots of row r:
- *   Mean  = (sum of z) / count,
- *   Top-4 = (sum of the min(4, count) largest z) / min(4, count),
- * each computed in double in a fixed order and rounded once to float: the
- * Mean sums every run of 8 consecutive slots in slot order, then adds the
- * runs' sums pairwise (runs 2k and 2k+1, then pairs of pairs, ...); the
- * Top-4 adds its values from the largest down.  +inf (a never-observed slot)
- * makes either +inf.  mode 0 is the max-pool above. */
-static double orc_tree_sum(double* c, int n) {  /* n a power of two */
-  for (int w = 1; w < n; w *= 2)
-    for (int u = 0; u + w < n; u += 2 * w) c[u] = c[u] + c[u + w];
-  return c[0];
+ *   Mean  = the mean of z: (sum of z) / count,
+ *   Top-4 = the mean of the min(4, count) largest z,
+ * each the exact value rounded once to the nearest float (ties to even), so
+ * that no summation order enters the definition.  +inf (a never-observed
+ * slot) makes the result +inf; -inf with no +inf makes it -inf; both, or a
+ * NaN, make it NaN.  mode 0 is the max-pool above.
+ *
+ * The exact sum: every finite float is an integer multiple of 2^-149, and
+ * |z| < 2^128, so a sum of at most 256 of them is an integer N (in units of
+ * 2^-149) below 2^285.  N is held in ten base-2^32 digits, each digit kept in
+ * an int64 so that signed digits and up to 2^31 additions need no carry until
+ * the end. */
+typedef struct {
+  int64_t d[10];
+} orc_exact_sum;
+
+static void orc_exact_add(orc_exact_sum* a, float x) {
+  if (x == 0.0f) return;
+  int e;
+  const double f = frexp((double)x, &e);      /* x = f 2^e, 0.5 <= |f| < 1 */
+  int64_t m = (int64_t)ldexp(f, 24);           /* exact: a float has 24 bits */
+  int shift = e - 24 + 149;                    /* x = m 2^(shift - 149) */
+  if (shift < 0) {                             /* subnormal: the low bits of m are zero */
+    m /= ((int64_t)1 << -shift);
+    shift = 0;
+  }
+  const int k = shift / 32, off = shift % 32;
+  const int neg = m < 0;
+  const uint64_t mag = (uint64_t)(neg ? -m : m) << off;   /* < 2^56 */
+  const int64_t lo = (int64_t)(mag & 0xFFFFFFFFu), hi = (int64_t)(mag >> 32);
+  a->d[k] += neg ? -lo : lo;
+  if (hi) a->d[k + 1] += neg ? -hi : hi;
 }
+
+/* The exact sum divided by cnt (1..256), rounded once to the nearest float. */
+static float orc_exact_mean(const orc_exact_sum* a, int cnt) {
+  int64_t d[11];
+  for (int k = 0; k < 10; ++k) d[k] = a->d[k];
+  d[10] = 0;
+  for (int k = 0; k < 10; ++k) {               /* digits to [0, 2^32), the sign to the top */
+    int64_t c = d[k] >> 32;                    /* floor division by 2^32 */
+    d[k] -= c * ((int64_t)1 << 32);
+    d[k + 1] += c;
+  }
+  int neg = d[10] < 0;
+  if (neg) {                                   /* magnitude of a negative sum: -N */
+    int64_t borrow = 0;
+    for (int k = 0; k < 11; ++k) {
+      int64_t v = -d[k] - borrow;
+      borrow = 0;
+      if (v < 0 && k < 10) { v += ((int64_t)1 << 32); borrow = 1; }
+      d[k] = v;
+    }
+  }
+  /* quotient and remainder of N / cnt, most significant digit first */
+  uint64_t q[10];
+  uint64_t rem = 0;
+  for (int k = 9; k >= 0; --k) {
+    const uint64_t cur = (rem << 32) | (uint64_t)d[k];
+    q[k] = cur / (uint64_t)cnt;
+    rem = cur % (uint64_t)cnt;
+  }
+  int top = -1;                                /* bit length of the quotient */
+  for (int k = 9; k >= 0 && top < 0; --k)
+    if (q[k]) {
+      int b = 31;
+      while (!((q[k] >> b) & 1u)) --b;
+      top = 32 * k + b + 1;
+    }
+  if (top < 0) {                               /* below one unit: 0 or 2^-149 */
+    float r = (2 * rem > (uint64_t)cnt) ? ldexpf(1.0f, -149) : 0.0f;
+    return neg ? -r : r;
+  }
+  /* a float keeps 24 significant bits; below 2^24 units (the subnormals and
+   * the lowest normal binade) its spacing is one unit */
+  const int sh = top > 24 ? top - 24 : 0;
+  uint64_t kept = 0;                           /* bits [sh, top) of the quotient */
+  for (int bit = top - 1; bit >= sh; --bit) kept = (kept << 1) | ((q[bit / 32] >> (bit % 32)) & 1u);
+  int up;
+  if (sh == 0) {
+    up = (2 * rem > (uint64_t)cnt) || (2 * rem == (uint64_t)cnt && (kept & 1u));
+  } else {
+    const int half = (int)((q[(sh - 1) / 32] >> ((sh - 1) % 32)) & 1u);
+    int below = rem != 0;                      /* anything under the half bit */
+    for (int bit = sh - 2; bit >= 0 && !below; --bit) below = (q[bit / 32] >> (bit % 32)) & 1u;
+    up = half && (below || (kept & 1u));
+  }
+  const double v = ldexp((double)(kept + (uint64_t)up), sh - 149);   /* exact; a float */
+  return neg ? -(float)v : (float)v;
+}
+
+static float orc_mean_of(const float* z, int cnt) {
+  int pinf = 0, ninf = 0, nan = 0;
+  orc_exact_sum a;
+  memset(&a, 0, sizeof(a));
+  for (int u = 0; u < cnt; ++u) {
+    if (isnan(z[u])) nan = 1;
+    else if (isinf(z[u])) { if (z[u] > 0) pinf = 1; else ninf = 1; }
+    else orc_exact_add(&a, z[u]);
+  }
+  if (nan || (pinf && ninf)) return NAN;
+  if (pinf) return INFINITY;
+  if (ninf) return -INFINITY;
+  return orc_exact_mean(&a, cnt);
+}
+
+ORC_API float orc_mean_exact(const float* z, int cnt) { return cnt >= 1 && cnt <= 256 ? orc_mean_of(z, cnt) : NAN; }
 
 ORC_API void orc_predict_pool_mode(const float* V, const float* D, int64_t ctx_len, int rows, int b,
                                    int64_t n_stride, int mode, float* S) {
@@ -205,38 +300,22 @@ ORC_API void orc_predict_pool_mode(const float* V, const float* D, int64_t ctx_l
     orc_predict_pool(V, D, ctx_len, rows, b, n_stride, S);
     return;
   }
-  double runs[32];  /* b <= 256: at most 32 runs of 8 slots */
+  float z[256];  /* b <= 256 */
   for (int r = 0; r < rows; ++r) {
     int64_t p = pos_of_row(ctx_len, r);
     int64_t n = nblocks_of_row(ctx_len, r, b);
     for (int64_t j = 0; j < n; ++j) {
       int count = 0;
-      float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      int nr = b / 8;
-      for (int u = 0; u < nr; ++u) runs[u] = 0.0;
-      for (int64_t i = j * b; i < (j + 1) * b && i <= p; ++i) {
-        float z = fmaxf(V[i], D[p - i]);
-        ++count;
-        runs[(i - j * b) / 8] += (double)z;
-        /* insert into the descending top-4 */
-        for (int k = 0; k < 4; ++k) {
-          if (z > top[k]) {
-            for (int m = 3; m > k; --m) top[m] = top[m - 1];
-            top[k] = z;
-            break;
-          }
-        }
-      }
-      double v;
-      if (mode == 1) {
-        v = orc_tree_sum(runs, nr) / (double)count;
-      } else {
+      for (int64_t i = j * b; i < (j + 1) * b && i <= p; ++i) z[count++] = fmaxf(V[i], D[p - i]);
+      if (mode == 2) {
+        /* the min(4, count) largest: a partial selection sort, descending */
         int m = count < 4 ? count : 4;
-        double t = 0.0;
-        for (int k = 0; k < m; ++k) t += (double)top[k];
-        v = t / (double)m;
+        for (int k = 0; k < m; ++k)
+          for (int u = k + 1; u < count; ++u)
+            if (z[u] > z[k]) { float t = z[k]; z[k] = z[u]; z[u] = t; }
+        count = m;
       }
-      S[(int64_t)r * n_stride + j] = (float)v;
+      S[(int64_t)r * n_stride + j] = orc_mean_of(z, count);
     }
   }
 }

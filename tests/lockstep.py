@@ -25,9 +25,24 @@ def score_close(gpu, ref):
     return np.abs(gpu - ref) <= ATOL + RTOL * np.abs(ref)
 
 
+def pool_close(gpu, ref, zabs_mean=0.0):
+    """Mean and Top-4 block scores.  The oracle's value is the exact mean
+    rounded once; the kernel sums in double in a fixed order (at most 256
+    terms, error <= 255 * 2^-53 * sum|z|) and rounds once to float, so it is
+    within one float ulp of the oracle's, plus 2^-45 * mean|z| where z takes
+    both signs.  Equal infinities and NaNs match."""
+    gpu = np.asarray(gpu, np.float32)
+    ref = np.asarray(ref, np.float32)
+    same = (gpu.view(np.uint32) == ref.view(np.uint32)) | (np.isnan(gpu) & np.isnan(ref))
+    with np.errstate(invalid="ignore", over="ignore"):
+        tol = np.spacing(np.abs(ref)).astype(np.float64) + 2.0 ** -45 * np.asarray(zabs_mean, np.float64)
+        close = np.abs(gpu.astype(np.float64) - ref.astype(np.float64)) <= tol
+    return same | close
+
+
 class Harness:
     def __init__(self, wl: workloads.Workload, device="cuda", score_kernel=isa.SPIN_SCORE_AUTO, positions=None,
-                 layers=None):
+                 layers=None, lookahead=False):
         self.wl = wl
         self.device = device
         self.layers = list(range(wl.layers)) if layers is None else layers
@@ -42,6 +57,9 @@ class Harness:
         self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
         isa.spin_set_score_kernel(self.st, score_kernel)
+        self.lookahead = lookahead
+        if lookahead:
+            isa.spin_set_lookahead(self.st, True)
         self.committed = np.array(wl.ctx0, np.int64)
         self.mask = self.st.new_mask()
         self.topk = None
@@ -110,13 +128,22 @@ class Harness:
         nstride = self.st.mask_stride
         S_ref = oracle.predict_pool(V0, D0, ctx_len, rows, wl.b, nstride, wl.pooling)
         s = float(np.float32(self.sparsity[layer]))
-        if s > 0:
+        S_sel = S_ref
+        pipelined = self.lookahead and rows == 1 and wl.key_fp8
+        if s > 0 and not pipelined:   # pipelined: the buffer already holds the next step's scores
             S_gpu = self.st.block_scores()[q, :rows, :nstride].cpu().numpy()
             predicting = 1 if wl.mtp_policy == oracle.MTP_ROW0 else rows   # rows whose scores are computed
             for r in range(predicting):
                 n = oracle.num_blocks(ctx_len, r, wl.b)
-                assert np.array_equal(S_gpu[r, :n], S_ref[r, :n]), f"block scores differ q={q} r={r}"
-        mask_ref = oracle.select(S_ref, ctx_len, rows, wl.b, s, wl.gamma, wl.seed, q, layer, step, wl.mtp_policy)
+                if wl.pooling == oracle.POOL_MAX:   # a max is exact: bit for bit
+                    assert np.array_equal(S_gpu[r, :n], S_ref[r, :n]), f"block scores differ q={q} r={r}"
+                else:                               # z >= 0 here (EMA of non-negative scores)
+                    assert pool_close(S_gpu[r, :n], S_ref[r, :n]).all(), f"block scores differ q={q} r={r}"
+            if wl.pooling != oracle.POOL_MAX:
+                # the selection is an integer decision taken from the block
+                # scores: the oracle takes it from the GPU's
+                S_sel = S_gpu
+        mask_ref = oracle.select(S_sel, ctx_len, rows, wl.b, s, wl.gamma, wl.seed, q, layer, step, wl.mtp_policy)
         mask_gpu = self.mask[q].cpu().numpy()
         assert np.array_equal(mask_gpu, mask_ref), f"mask differs q={q}: {np.nonzero(mask_gpu != mask_ref)[0][:10]}"
         keys, ks, ident = self.pages_of(layer, q)
@@ -159,5 +186,64 @@ class Harness:
         Vg, Dg = self.st.ema(layer)
         assert np.array_equal(Vg[q].cpu().numpy().view(np.uint32), V1.view(np.uint32)), f"V differs q={q}"
         assert np.array_equal(Dg[q].cpu().numpy().view(np.uint32), D1.view(np.uint32)), f"D differs q={q}"
+        if pipelined and s > 0 and ctx_len + 1 <= self.cfg.max_slots:
+            # the block scores of the next step (one slot more), predicted from
+            # the state this step left behind
+            S_next = oracle.predict_pool(V1, D1, ctx_len + 1, 1, wl.b, nstride, wl.pooling)
+            n = oracle.num_blocks(ctx_len + 1, 0, wl.b)
+            S_gpu = self.st.block_scores()[q, 0, :nstride].cpu().numpy()
+            if wl.pooling == oracle.POOL_MAX:
+                assert np.array_equal(S_gpu[:n], S_next[0, :n]), f"next step's block scores differ q={q}"
+            else:
+                assert pool_close(S_gpu[:n], S_next[0, :n]).all(), f"next step's block scores differ q={q}"
         n_last = oracle.num_blocks(ctx_len, rows - 1, wl.b)
         return {"kept": int(np.count_nonzero(mask_ref)), "n": n_last, "scored_checked": int(scored.sum())}
+
+
+def run_multilayer(h: Harness, check, check_warmup, sample_blocks=None):
+    """The per-layer budget protocol of the multi-layer workload: an all-keep
+    step on every layer, warm-up steps at the uniform target with a shadow
+    full indexer measuring each layer's miss rate on the GPU, the water-filled
+    per-layer sparsities (library against oracle), then the remaining steps
+    with them.  Every layer of a step sees the same token.  Lock-step checks
+    on `check_warmup` requests during warm-up and `check` afterwards."""
+    wl = h.wl
+    for layer in range(wl.layers):
+        keep = list(h.sparsity)
+        h.set_sparsity([0.0] * wl.layers)
+        h.run_step(layer, check=check_warmup, step=0, sample_blocks=sample_blocks)
+        h.committed -= 1                                    # every layer sees the same token
+        h.set_sparsity(keep)
+    h.committed += 1
+    miss = np.zeros(wl.layers)
+    Q, k = wl.requests, wl.topk
+    full_scores = h.st.new_scores()
+    full_topk = torch.empty((Q, 1, k), dtype=torch.int32, device=h.device)
+    missed = torch.zeros((Q, 1), dtype=torch.int32, device=h.device)
+    total = torch.zeros((Q, 1), dtype=torch.int32, device=h.device)
+    for t in range(1, 1 + wl.warmup_steps):
+        for layer in range(wl.layers):
+            h.run_step(layer, check=check_warmup, step=t, sample_blocks=sample_blocks)
+            h.committed -= 1
+            qstep, wstep, ctx = h.step_inputs(layer, 1)
+            cache = h.caches[layer]
+            allk = torch.ones_like(h.mask)
+            isa.spin_indexer_score(h.st, layer, 1, cache.keys, cache.kscale, cache.block_table, qstep, wstep, ctx,
+                                   allk, full_scores)
+            isa.spin_topk(h.st, 1, full_scores, allk, ctx, full_topk)
+            isa.spin_miss_count(h.st, 1, full_topk, h.mask, missed, total)
+            miss[layer] += (missed.double() / total.double()).mean().item()
+        h.committed += 1
+    miss /= wl.warmup_steps
+    blocks = np.array([sum(-(-(c + 1) // wl.b) for c in h.committed)] * wl.layers, np.float64)
+    lo = np.full(wl.layers, 0.05)
+    s = isa.spin_allocate_layer_sparsity(miss, blocks, lo, wl.sparsity)
+    ref = oracle.layer_sparsity(miss, blocks, lo, wl.sparsity)
+    assert np.allclose(s, ref, atol=2e-6)
+    h.set_sparsity(s)
+    for t in range(1 + wl.warmup_steps, wl.steps):
+        for layer in range(wl.layers):
+            h.run_step(layer, check=check, step=t, sample_blocks=sample_blocks)
+            h.committed -= 1
+        h.committed += 1
+    return s, miss

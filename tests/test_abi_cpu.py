@@ -54,7 +54,9 @@ def _expected_bytes(L, Q, R, H, d, b, max_slots):
     slot = mb * b
     blk = -(-mb // 16) * 16
     parts = [16, L * Q * slot * 4, L * Q * slot * 4, Q * R * blk * 4, Q * blk * 4, Q * 4, Q * R * H * d,
-             Q * R * H * 4, Q * R * slot * 4, Q * R * blk * max(1, b // 32) * 4, 8]
+             Q * R * H * 4, Q * R * slot * 4, Q * R * blk * max(1, b // 32) * 4, 8,
+             # the selection a pipelined step prepares for the next one, per layer, and ctx_len + 1
+             L * Q * blk * 4, L * Q * 4, L * Q * mb, L * Q * 4, Q * 4]
     return sum(a(p) for p in parts)
 
 
@@ -122,7 +124,8 @@ def test_null_state_rejected_by_every_entry_point(lib):
     """Every call that takes a state answers SPIN_ESTATE for a NULL handle,
     before it touches the device (no GPU needed)."""
     isa.load()
-    skip = {"spin_state_bytes", "spin_state_create", "spin_topk_noalloc", "spin_allocate_layer_sparsity",
+    skip = {"spin_state_bytes", "spin_state_create", "spin_topk_noalloc", "spin_topk_noalloc_error",
+            "spin_allocate_layer_sparsity",
             "spin_status_string", "spin_state_export_bytes", "spin_score_stride", "spin_mask_stride",
             "spin_state_destroy"}
     names = [n for n in isa.__all__ if n.startswith("spin_") and n not in skip]

@@ -9,7 +9,7 @@ import torch
 import indexer_sparse_attention_b200 as isa
 import oracle
 import workloads
-from lockstep import Harness, score_close
+from lockstep import Harness, run_multilayer, score_close
 
 pytestmark = pytest.mark.gpu
 
@@ -100,45 +100,7 @@ def test_multilayer_per_layer_budget():
     """Ragged long-context workload, scaled: warm-up at uniform 50% with a
     shadow full indexer measuring miss on the GPU, then per-layer budgets."""
     wl = workloads.config(4, layers=2, requests=3, ctx0=(70000, 40000, 100000), steps=6, warmup_steps=2)
-    h = Harness(wl)
-    for layer in range(wl.layers):
-        keep = list(h.sparsity)
-        h.set_sparsity([0.0] * wl.layers)
-        h.run_step(layer, check=[0], step=0)
-        h.committed -= 1                                    # every layer sees the same token
-        h.set_sparsity(keep)
-    h.committed += 1
-    miss = np.zeros(wl.layers)
-    Q, k = wl.requests, wl.topk
-    full_scores = h.st.new_scores()
-    full_topk = torch.empty((Q, 1, k), dtype=torch.int32, device="cuda")
-    missed = torch.zeros((Q, 1), dtype=torch.int32, device="cuda")
-    total = torch.zeros((Q, 1), dtype=torch.int32, device="cuda")
-    for t in range(1, 1 + wl.warmup_steps):
-        for layer in range(wl.layers):
-            h.run_step(layer, check=[1], step=t)
-            h.committed -= 1
-            qstep, wstep, ctx = h.step_inputs(layer, 1)
-            cache = h.caches[layer]
-            allk = torch.ones_like(h.mask)
-            isa.spin_indexer_score(h.st, layer, 1, cache.keys, cache.kscale, cache.block_table, qstep, wstep, ctx,
-                                   allk, full_scores)
-            isa.spin_topk(h.st, 1, full_scores, allk, ctx, full_topk)
-            isa.spin_miss_count(h.st, 1, full_topk, h.mask, missed, total)
-            miss[layer] += (missed.double() / total.double()).mean().item()
-        h.committed += 1
-    miss /= wl.warmup_steps
-    blocks = np.array([sum(-(-(c + 1) // 64) for c in h.committed)] * wl.layers, np.float64)
-    lo = np.full(wl.layers, 0.05)
-    s = isa.spin_allocate_layer_sparsity(miss, blocks, lo, 0.5)
-    ref = oracle.layer_sparsity(miss, blocks, lo, 0.5)
-    assert np.allclose(s, ref, atol=2e-6)
-    h.set_sparsity(s)
-    for t in range(1 + wl.warmup_steps, wl.steps):
-        for layer in range(wl.layers):
-            h.run_step(layer, check=range(Q), step=t)
-            h.committed -= 1
-        h.committed += 1
+    run_multilayer(Harness(wl), check=range(wl.requests), check_warmup=[1])
 
 
 def test_serving_full_size_sampled():

@@ -1,0 +1,174 @@
+"""Pipelined one-row decode steps (spin_set_lookahead): each step prepares the
+next step's selection from the state its score kernel leaves behind and runs
+its own top-k on a second stream beside the next step's predict kernel.  The
+results must be those of the sequential step, bit for bit: the same masks,
+top-k indices and EMA state, in lock step with the oracle, replayed from a CUDA
+graph, and with a request whose ctx_len breaks the one-slot-a-step contract
+reported in the device error word."""
+import numpy as np
+import pytest
+import torch
+
+import indexer_sparse_attention_b200 as isa
+import oracle
+import workloads
+from lockstep import Harness
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from indexer_sparse_attention_b200 import build
+    build.build()
+    oracle.build()
+
+
+def _wl(steps=9):
+    return workloads.config(2, requests=5, ctx0=(70_000, 130, 64 * 700 - 1, 90_011, 64 * 64), steps=steps,
+                            sparsity=0.5)
+
+
+def _states(wl):
+    out = []
+    for la in (False, True):
+        cfg = isa.make_config(num_layers=1, num_requests=wl.requests, max_slots=wl.max_slots, topk=wl.topk,
+                              target_sparsity=wl.sparsity, gamma=wl.gamma, seed=wl.seed)
+        st = isa.SpinState(cfg)
+        if la:
+            isa.spin_set_lookahead(st, True)
+        out.append(st)
+    return out
+
+
+@pytest.mark.parametrize("device_step", [False, True])
+def test_lookahead_matches_sequential_steps(device_step):
+    """Sparsity schedule with an all-keep bootstrap, target changes (the
+    prepared selection is dropped and made afresh) and an all-keep step in
+    the middle; explicit step numbers or the device counter."""
+    wl = _wl()
+    cache = workloads.make_key_cache(wl, 0, "cuda")
+    q_all, w_all = workloads.make_queries(wl, 0, wl.steps, "cuda")
+    ctx0 = torch.tensor(wl.ctx0, dtype=torch.int64, device="cuda")
+    Q, k = wl.requests, wl.topk
+    seq, la = _states(wl)
+    for st in (seq, la):
+        isa.spin_set_step(st, 0)
+    sched = [0.0, 0.5, 0.5, 0.5, 0.4, 0.4, 0.0, 0.5, 0.5]
+    for t, s in enumerate(sched):
+        q, w = q_all[:, t:t + 1].contiguous(), w_all[:, t:t + 1].contiguous()
+        ctx = (ctx0 + t + 1).to(torch.int32)
+        outs = []
+        for st in (seq, la):
+            isa.spin_set_layer_sparsity(st, [s])
+            mask = st.new_mask()
+            topk = torch.full((Q, 1, k), -7, dtype=torch.int32, device="cuda")
+            step = isa.SPIN_STEP_DEVICE if device_step else t
+            isa.spin_decode_step(st, 0, 1, step, cache.keys, cache.kscale, cache.block_table, q, w, ctx, False,
+                                 mask, topk)
+            if device_step:
+                isa.spin_advance_step(st)
+            outs.append((mask, topk))
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0][0], outs[1][0]), f"mask differs at step {t}"
+        assert torch.equal(outs[0][1], outs[1][1]), f"top-k differs at step {t}"
+        for a, b in zip(seq.ema(0), la.ema(0)):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32)), f"state differs at step {t}"
+    assert isa.spin_get_error(seq)[0] == 0 and isa.spin_get_error(la)[0] == 0
+
+
+def test_lookahead_lock_step_with_oracle():
+    """Pipelined steps of the serving shape in lock step with the oracle; the
+    block-score buffer is checked as the next step's prediction from the
+    state each step leaves behind."""
+    wl = _wl(steps=6)
+    h = Harness(wl, lookahead=True)
+    h.set_sparsity([0.0])
+    h.run_step(0, check=range(wl.requests))
+    h.set_sparsity([0.5])
+    for _ in range(wl.steps - 1):
+        h.run_step(0, check=range(wl.requests))
+
+
+def test_lookahead_graph_replay():
+    """One pipelined step captured with the device step counter (after an
+    eager pipelined step prepared the first selection), replayed with each
+    step's inputs: the same results as sequential eager steps."""
+    wl = _wl(steps=6)
+    cache = workloads.make_key_cache(wl, 0, "cuda")
+    q_all, w_all = workloads.make_queries(wl, 0, wl.steps, "cuda")
+    ctx0 = torch.tensor(wl.ctx0, dtype=torch.int64, device="cuda")
+    Q, k = wl.requests, wl.topk
+    seq, la = _states(wl)
+
+    def inputs(t):
+        return q_all[:, t:t + 1].contiguous(), w_all[:, t:t + 1].contiguous(), (ctx0 + t + 1).to(torch.int32)
+
+    eager = []
+    for t in range(wl.steps):
+        mask = seq.new_mask()
+        topk = torch.empty((Q, 1, k), dtype=torch.int32, device="cuda")
+        q, w, ctx = inputs(t)
+        isa.spin_decode_step(seq, 0, 1, t, cache.keys, cache.kscale, cache.block_table, q, w, ctx, False, mask, topk)
+        eager.append((mask.clone(), topk.clone()))
+    q_buf, w_buf, ctx_buf = (x.clone() for x in inputs(0))
+    mask_g = la.new_mask()
+    topk_g = torch.empty((Q, 1, k), dtype=torch.int32, device="cuda")
+    isa.spin_set_step(la, 0)
+    isa.spin_decode_step(la, 0, 1, isa.SPIN_STEP_DEVICE, cache.keys, cache.kscale, cache.block_table, q_buf, w_buf,
+                         ctx_buf, False, mask_g, topk_g)
+    isa.spin_advance_step(la)
+    torch.cuda.synchronize()
+    assert torch.equal(mask_g, eager[0][0]) and torch.equal(topk_g, eager[0][1])
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        isa.spin_decode_step(la, 0, 1, isa.SPIN_STEP_DEVICE, cache.keys, cache.kscale, cache.block_table, q_buf,
+                             w_buf, ctx_buf, False, mask_g, topk_g)
+        isa.spin_advance_step(la)
+    for t in range(1, wl.steps):
+        q, w, ctx = inputs(t)
+        q_buf.copy_(q)
+        w_buf.copy_(w)
+        ctx_buf.copy_(ctx)
+        graph.replay()
+        assert torch.equal(mask_g, eager[t][0]), t
+        assert torch.equal(topk_g, eager[t][1]), t
+    torch.cuda.synchronize()
+    assert isa.spin_get_error(la)[0] == 0
+    for a, b in zip(seq.ema(0), la.ema(0)):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    del graph
+
+
+def test_lookahead_reports_a_broken_ctx_contract():
+    """A request whose next ctx_len is not the prepared one (here: the same
+    ctx_len again) is not scored: ERR_LOOKAHEAD is raised and its top-k rows
+    are -1; the other requests match the sequential step."""
+    wl = _wl(steps=3)
+    cache = workloads.make_key_cache(wl, 0, "cuda")
+    q_all, w_all = workloads.make_queries(wl, 0, wl.steps, "cuda")
+    ctx0 = torch.tensor(wl.ctx0, dtype=torch.int64, device="cuda")
+    Q, k = wl.requests, wl.topk
+    seq, la = _states(wl)
+    for t in range(2):
+        q, w = q_all[:, t:t + 1].contiguous(), w_all[:, t:t + 1].contiguous()
+        ctx = (ctx0 + t + 1).to(torch.int32)
+        if t == 1:
+            ctx_la = ctx.clone()
+            ctx_la[2] -= 1                                  # request 2 does not advance
+        res = []
+        for st, c in ((seq, ctx), (la, ctx if t == 0 else ctx_la)):
+            mask = st.new_mask()
+            topk = torch.empty((Q, 1, k), dtype=torch.int32, device="cuda")
+            isa.spin_decode_step(st, 0, 1, t, cache.keys, cache.kscale, cache.block_table, q, w, c, False, mask,
+                                 topk)
+            res.append(topk)
+        status, word = isa.spin_get_error(la)
+        if t == 0:
+            assert status == 0
+            continue
+        assert isa.STATUS_NAMES[status] == "SPIN_EDEVICE" and word & 32, (status, word)
+        assert torch.all(res[1][2] == -1)
+        keep = [0, 1, 3, 4]
+        assert torch.equal(res[0][keep], res[1][keep])
+    assert isa.spin_get_error(seq)[0] == 0

@@ -8,6 +8,8 @@ import json
 import math
 import os
 
+from fractions import Fraction
+
 import numpy as np
 import pytest
 import torch
@@ -593,24 +595,95 @@ def test_pool_variants_order_and_sentinels(oracle_lib):
     p = n - 1
     i = np.arange(64 * (nb - 1), n)
     z = np.maximum(V[i], D[p - i]).astype(np.float64)
-    assert len(i) == 3 and S[2][nb - 1] == np.float32(z.mean())
+    assert len(i) == 3 and S[2][nb - 1] == _exact_mean(z)
 
 
-def test_pool_mean_sums_runs_of_eight_then_pairwise(oracle_lib):
-    """The Mean's fixed order: each run of 8 slots is summed in slot order,
-    then the runs are added pairwise.  With z spanning 2^60 the order shows:
-    a 1.0 in the run of 2^60 is absorbed (the double ulp there is 2^8), so
-    runs (2^60 + 1) and (-2^60 + 1) sum to 0, where a single left-to-right sum
-    over the block would give 1."""
+def _f32_nearest(fr):
+    """A rational rounded to the nearest float32, ties to even, by integer
+    arithmetic on the exact value (no float operation rounds on the way)."""
+    if fr == 0:
+        return np.float32(0.0)
+    sign = -1.0 if fr < 0 else 1.0
+    a = abs(fr)
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    if a < Fraction(2) ** e:
+        e -= 1
+    while a >= Fraction(2) ** (e + 1):
+        e += 1
+    ulp_exp = max(e, -126) - 23                                   # spacing of floats at a
+    n = a / Fraction(2) ** ulp_exp
+    k = n.numerator // n.denominator
+    rest = n - k
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and k % 2 == 1):
+        k += 1
+    return np.float32(sign * float(k) * 2.0 ** ulp_exp)        # exact: k <= 2^24
+
+
+def _exact_mean(z):
+    z = [float(np.float32(v)) for v in z]
+    return _f32_nearest(sum((Fraction(v) for v in z), Fraction(0)) / len(z))
+
+
+def test_f32_nearest_reference_on_known_values():
+    # the reference rounding itself, on values whose float is known
+    assert _f32_nearest(Fraction(1, 3)) == np.float32(1.0 / 3.0)
+    mid = Fraction(1) + Fraction(1, 2 ** 24)                    # halfway between 1 and 1 + 2^-23
+    assert _f32_nearest(mid) == np.float32(1.0)                 # ties to even
+    assert _f32_nearest(mid + Fraction(1, 2 ** 60)) == np.nextafter(np.float32(1), np.float32(2))
+    assert _f32_nearest(Fraction(3, 2 ** 150)) == np.float32(2.0 ** -148)   # 1.5 units -> 2 (even)
+    assert _f32_nearest(Fraction(1, 2 ** 150)) == np.float32(0.0)          # half a unit -> 0 (even)
+
+
+def test_mean_exact_against_rational_arithmetic(oracle_lib):
+    """The pools' mean is the exact sum over the count rounded once: checked
+    against exact rational arithmetic on values spanning the float range
+    (2^-149 .. 2^120, mixed signs, up to 256 values), where any fixed double
+    summation order would lose bits."""
+    rng = np.random.default_rng(77)
+    for trial in range(400):
+        n = int(rng.integers(1, 257))
+        kind = trial % 4
+        if kind == 0:    # one exponent band: a sum in double would be exact
+            z = rng.uniform(0, 50, n)
+        elif kind == 1:  # wide spread, both signs
+            z = rng.standard_normal(n) * 2.0 ** rng.integers(-140, 120, n)
+        elif kind == 2:  # subnormals and tiny values
+            z = rng.integers(-2 ** 20, 2 ** 20, n) * 2.0 ** -149
+        else:            # large values that cancel, plus small ones
+            z = np.concatenate([[2.0 ** 100, -(2.0 ** 100)], rng.uniform(-1, 1, n - 2)]) if n > 2 else [1.0] * n
+        z = np.asarray(z, np.float32)
+        got = oracle_lib.mean_exact(z)
+        ref = _exact_mean(z)
+        assert got.view(np.uint32) == ref.view(np.uint32), (trial, got, ref)
+        perm = rng.permutation(z.size)
+        assert oracle_lib.mean_exact(z[perm]).view(np.uint32) == got.view(np.uint32)   # no order enters
+
+
+def test_pool_mean_and_top4_exact_on_wide_values(oracle_lib):
+    """The block Mean and Top-4 on z spanning 2^60 equal the exact rational
+    values: with z = (2^60, 1, -2^60, 1, 0, ...) over 16 slots the mean is
+    2/16 exactly (a left-to-right double sum would absorb the first 1)."""
     b = 16
     D = np.full(b, -np.inf, np.float32)
     V = np.zeros(b, np.float32)
     V[0], V[1], V[8], V[9] = 2.0 ** 60, 1.0, -(2.0 ** 60), 1.0
-    assert oracle_lib.predict_pool(V, D, b, 1, b, 1, oracle_lib.POOL_MEAN)[0, 0] == np.float32(0.0)
-    # a value of one ulp survives its run: (2^60 + 256) + (-2^60) = 256
-    V2 = np.zeros(b, np.float32)
-    V2[0], V2[1], V2[8] = 2.0 ** 60, 256.0, -(2.0 ** 60)
-    assert oracle_lib.predict_pool(V2, D, b, 1, b, 1, oracle_lib.POOL_MEAN)[0, 0] == np.float32(256.0 / b)
+    assert oracle_lib.predict_pool(V, D, b, 1, b, 1, oracle_lib.POOL_MEAN)[0, 0] == np.float32(2.0 / 16)
+    # top-4 of the same block: 2^60, 1, 1, 0 -> (2^60 + 2) / 4 rounds to 2^58
+    assert oracle_lib.predict_pool(V, D, b, 1, b, 1, oracle_lib.POOL_TOP4)[0, 0] == np.float32(2.0 ** 58)
+    rng = np.random.default_rng(9)
+    n = 64 * 9 + 5
+    V = (rng.standard_normal(n + 4) * 2.0 ** rng.integers(-60, 60, n + 4)).astype(np.float32)
+    D = (rng.standard_normal(n + 4) * 2.0 ** rng.integers(-60, 60, n + 4)).astype(np.float32)
+    for rows in (1, 3):
+        Sm = oracle_lib.predict_pool(V, D, n, rows, 64, 16, oracle_lib.POOL_MEAN)
+        St = oracle_lib.predict_pool(V, D, n, rows, 64, 16, oracle_lib.POOL_TOP4)
+        for r in range(rows):
+            p = n - 1 + r
+            for j in range(oracle_lib.num_blocks(n, r, 64)):
+                i = np.arange(j * 64, min((j + 1) * 64, p + 1))
+                z = np.maximum(V[i], D[p - i])
+                assert Sm[r, j].view(np.uint32) == _exact_mean(z).view(np.uint32), (r, j)
+                assert St[r, j].view(np.uint32) == _exact_mean(np.sort(z)[::-1][:4]).view(np.uint32), (r, j)
 
 
 # ----------------------------------------------------------------------------

@@ -1,48 +1,73 @@
 """The allocation-free top-k entry point (spin_topk_noalloc), for callers that
 cannot give the library any device memory -- code running under CUDA graph
-capture, or hosts that own every byte of device memory.  It must return
-exactly what the state-based spin_topk returns for the same inputs, on
-consecutive calls that reuse its fixed scratch, and refuse problems larger
-than that scratch.  Kept in a file of its own that pytest collects last."""
+capture, or hosts that own every byte of device memory.  Its output must be
+the oracle's token top-k (higher score first, ties to the lower slot,
+ascending, padded with -1) on consecutive calls that reuse its fixed scratch;
+a request whose ctx_len is out of range comes back all -1 with bit 0 of the
+error word set, readable through spin_topk_noalloc_error; problems larger than
+the scratch are refused.  Kept in a file of its own that pytest collects last."""
 import numpy as np
 import pytest
 import torch
 
 import indexer_sparse_attention_b200 as isa
+import oracle
+
+B = 64
 
 
-def _inputs(rng, st, Q, R, ctx):
-    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.55).astype(np.uint8)
+def _inputs(rng, Q, R, max_slots, ctx):
+    n_max = -(-max_slots // B)
+    m = (rng.uniform(size=(Q, n_max)) < 0.55).astype(np.uint8)
     for q in range(Q):
-        m[q, -(-(int(ctx[q]) + R - 1) // 64):] = 0
-    vals = rng.standard_normal((Q, st.cfg.max_rows, st.score_stride)).astype(np.float32) * 8
+        if 1 <= ctx[q] <= max_slots - R + 1:
+            m[q, oracle.num_blocks(int(ctx[q]), R - 1, B):] = 0
+    vals = rng.standard_normal((Q, R, n_max * B)).astype(np.float32) * 8
     vals[:, :, ::7] = np.round(vals[:, :, ::7])                 # plenty of exact ties
-    return torch.from_numpy(m).cuda(), torch.from_numpy(vals).cuda()
+    return m, vals
+
+
+def _oracle_topk(vals, m, ctx, R, k, max_slots):
+    Q = vals.shape[0]
+    out = np.full((Q, R, k), -1, np.int32)
+    for q in range(Q):
+        if not (1 <= ctx[q] <= max_slots - R + 1):
+            continue                                         # out of range: all -1
+        for r in range(R):
+            out[q, r] = oracle.topk_row(vals[q, r].astype(np.float64), m[q], int(ctx[q]), r, B, k)
+    return out
+
+
+def _run(Q, R, k, max_slots, m, vals, ctx):
+    got = torch.full((Q, R, k), -7, dtype=torch.int32, device="cuda")
+    isa.spin_topk_noalloc(Q, R, R, max_slots, B, k, torch.from_numpy(vals).cuda(), torch.from_numpy(m).cuda(),
+                          torch.from_numpy(ctx.astype(np.int32)).cuda(), got)
+    status, word = isa.spin_topk_noalloc_error()
+    return got.cpu().numpy(), status, word
 
 
 @pytest.mark.gpu
-def test_noalloc_topk_matches_state_topk_on_consecutive_calls():
+def test_noalloc_topk_matches_oracle_and_reports_device_errors():
     from indexer_sparse_attention_b200 import build
     build.build()
+    oracle.build()
     Q, R, k, max_slots = 7, 2, 512, 64 * 300 + 5
-    cfg = isa.make_config(num_layers=1, num_requests=Q, max_slots=max_slots, topk=k, max_rows=R)
-    st = isa.SpinState(cfg)
     rng = np.random.default_rng(2024)
-    for call in range(2):
-        ctx = np.array([max_slots - R + 1, 1, 130, 64 * 77, 64 * 299 + 3, 5000, 64 * 8], np.int64)
-        if call == 1:
-            ctx = ctx[::-1].copy()
-            ctx[0] = max_slots - R + 1
-        ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
-        mask, scores = _inputs(rng, st, Q, R, ctx)
-        ref = torch.full((Q, R, k), -7, dtype=torch.int32, device="cuda")
-        got = torch.full((Q, R, k), -7, dtype=torch.int32, device="cuda")
-        isa.spin_topk(st, R, scores, mask, ctx_t, ref)
-        isa.spin_topk_noalloc(Q, R, R, max_slots, 64, k, scores, mask, ctx_t, got)
-        torch.cuda.synchronize()
-        assert isa.spin_get_error(st)[0] == 0
+    base = np.array([max_slots - R + 1, 1, 130, 64 * 77, 64 * 299 + 3, 5000, 64 * 8], np.int64)
+    cases = [base, base[::-1].copy(), base.copy()]
+    cases[1][0] = max_slots - R + 1
+    cases[2][3] = max_slots                                  # past the last position two rows can take
+    for call, ctx in enumerate(cases):
+        m, vals = _inputs(rng, Q, R, max_slots, ctx)
+        got, status, word = _run(Q, R, k, max_slots, m, vals, ctx)
+        ref = _oracle_topk(vals, m, ctx, R, k, max_slots)
         # integer outputs: the tolerance is exact equality
-        assert torch.equal(got, ref), f"call {call}: {(got != ref).sum().item()} entries differ"
+        assert np.array_equal(got, ref), f"call {call}: {(got != ref).sum()} entries differ"
+        if call < 2:
+            assert status == 0 and word == 0, (call, status, word)   # cleared at the start of each call
+        else:
+            assert (got[3] == -1).all()
+            assert isa.STATUS_NAMES[status] == "SPIN_EDEVICE" and word & 1, (status, word)
 
 
 @pytest.mark.gpu
