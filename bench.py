@@ -71,8 +71,9 @@ def parse():
                    help="block reduction of the predicted scores (max is the method's)")
     p.add_argument("--mtp-policy", choices=list(MTP_POLICIES), default="union-prefix",
                    help="several query rows: row-local union + prefix-valid update (the method's) or row 0 alone")
-    p.add_argument("--no-lookahead", action="store_true",
-                   help="sequential one-row steps: no next-step selection prepared beside the top-k")
+    p.add_argument("--lookahead", action="store_true",
+                   help="pipelined one-row steps (spin_set_lookahead): each step prepares the next step's "
+                        "selection, whose select kernel runs beside the step's top-k")
     p.add_argument("--ablation", choices=["pooling", "mtp", "predictors"], default=None,
                    help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities; "
                         "mtp: p99 miss vs realized sparsity of the two MTP policies on the 4-row workload; "
@@ -266,7 +267,7 @@ def peaks():
 
 
 class SpinRun:
-    def __init__(self, wl, device, total_steps, pooling=0, lookahead=True):
+    def __init__(self, wl, device, total_steps, pooling=0, lookahead=False):
         import indexer_sparse_attention_b200 as isa
         self.isa = isa
         self.wl = wl
@@ -439,7 +440,7 @@ def gpu_arm(args, world, rank, local):
     KS = min(K, 40)  # steps of the per-stage timing pass
     total = 1 + (W + K) * (1 + len(sweep)) + 3 + K + KS + 2
     wl = rank_workload(rank, args.requests, total + 8)
-    run = SpinRun(wl, device, total, POOLINGS[args.pooling], lookahead=not args.no_lookahead)
+    run = SpinRun(wl, device, total, POOLINGS[args.pooling], lookahead=args.lookahead)
     Q = wl.requests
     # history bootstrap: all-keep step that fills V and D
     run.set_sparsity(0.0)
@@ -493,12 +494,12 @@ def gpu_arm(args, world, rank, local):
                      "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
                                         "(16-request capture, scaled by kept slots)" if traffic_slot is not None
                                         else "null: the kernel source has changed since the last ncu capture")},
-        "pipelined": ("each step prepares the next step's selection, whose predict kernel runs on a second "
-                      "stream beside the step's top-k (spin_set_lookahead); results are those of the "
+        "pipelined": ("each step prepares the next step's selection, whose select kernel runs beside the "
+                      "step's top-k on a second stream (spin_set_lookahead); results are those of the "
                       "sequential step" if run.lookahead else "no: sequential steps"),
         "stage_ms_per_step": {k: v[0] / KS for k, v in stage_pass.items() if v[1]},
         "stage_ms_source": (f"separate pass of {KS} steps with every launch bracketed by CUDA events"
-                            + ("; the next step's predict overlaps the top-k" if run.lookahead else "")),
+                            + ("; the top-k overlaps the next step's select" if run.lookahead else "")),
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
@@ -709,7 +710,7 @@ def workload_arm(args, world, rank, local):
                           spare_slots=base.rows * 4, pooling=POOLINGS[args.pooling],
                           mtp_policy=MTP_POLICIES[args.mtp_policy])
     run = WorkloadRun(wl, device, total)
-    run.set_lookahead(not args.no_lookahead)   # applies to one-row steps
+    run.set_lookahead(args.lookahead)   # applies to one-row steps
     Ly, Q, R = wl.layers, wl.requests, wl.rows
     # history bootstrap (all-keep), then the workload's warm-up protocol
     run.set_sparsity([0.0] * Ly)
@@ -981,7 +982,7 @@ def predictor_profile(args, world, rank, local):
     wl = workloads.config(WORKLOADS["ragged-8Lx8-256K-1M"], requests=2, ctx0=(94_000, 9_700), steps=total,
                           seed=base.seed + 1000 * rank, spare_slots=8)
     run = WorkloadRun(wl, device, total)
-    run.set_lookahead(not args.no_lookahead)   # applies to one-row steps
+    run.set_lookahead(args.lookahead)   # applies to one-row steps
     Ly, Q, R = wl.layers, wl.requests, wl.rows
     st = run.st
     run.set_sparsity([0.0] * Ly)

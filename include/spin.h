@@ -267,10 +267,11 @@ SPIN_API spin_status spin_decode_step(spin_state st, int layer, int rows, int64_
  * steps' indexer scores).  With lookahead on, spin_decode_step with rows = 1,
  * no deferred update and FP8 keys on the tensor-core kernel also prepares
  * the next step's selection of the same layer, for ctx_len + 1 and step + 1
- * (SPIN_STEP_DEVICE: the counter + 1), running the next step's predict
- * kernel on a second stream of the state beside this step's top-k; the call
- * joins that stream back into `stream` before it returns, so its outputs are
- * ready in stream order as before.  Results are bit-identical to the sequential
+ * (SPIN_STEP_DEVICE: the counter + 1).  The next step's predict kernel runs
+ * right after the score kernel, and this step's top-k then runs on a second
+ * stream of the state beside the next step's select; the call joins that
+ * stream back into `stream` before it returns, so its outputs are ready in
+ * stream order as before.  Results are bit-identical to the sequential
  * step's.  The next call of the layer must then pass ctx_len + 1 for every
  * request, the next step number and the same target: a different target or
  * step number (host steps), or an intervening spin_ema_update,

@@ -260,8 +260,8 @@ def spin_set_step(st: SpinState, step: int, stream=None) -> None:
 
 def spin_set_lookahead(st: SpinState, enable: bool = True) -> None:
     """Pipelined one-row decode steps: each step prepares the next step's
-    selection, its predict kernel on a second stream beside the step's top-k
-    (see include/spin.h)."""
+    selection, whose select kernel runs beside the step's top-k on a second
+    stream (see include/spin.h)."""
     _check(load().spin_set_lookahead(st.handle, 1 if enable else 0), "spin_set_lookahead")
 
 

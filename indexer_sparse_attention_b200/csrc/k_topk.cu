@@ -66,6 +66,7 @@ struct TopkCtx {
   const float* sc;
   const int32_t* work;
   int nk, lb, bmask, p, n_elem, nwords;
+  int bits_cap;     // words of the bitmap area
   uint32_t* bits;
   uint32_t* hist;   // kBins
   uint32_t* ckey;   // kCandCap (aliases hist)
@@ -392,21 +393,36 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
     }
   }
   // compact the qualifying group ids to the front, in place (a round reads
-  // before it writes, and writes only reach indices already read)
+  // before it writes, and writes only reach indices already read); one
+  // shared atomic per warp and round
   if (threadIdx.x == 0) sh.n_eq = 0;
   __syncthreads();
-  for (int base = 0; base < n_groups; base += blockDim.x) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int base = 0; base < n_groups; base += blockDim.x) {  // block-uniform trip count
     const int g = base + threadIdx.x;
     const bool take = g < n_groups && gk[g] >= M;
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
     __syncthreads();
-    if (take) gk[atomicAdd(&sh.n_eq, 1)] = (uint32_t)g;
+    if (bal) {
+      uint32_t at = 0;
+      if (lane == 0) at = atomicAdd((uint32_t*)&sh.n_eq, (uint32_t)__popc(bal));
+      at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+      if (take) gk[at] = (uint32_t)g;
+    }
     __syncthreads();
   }
   const int n_q = sh.n_eq;
   if (threadIdx.x == 0) sh.n_cand = 0;
   __syncthreads();
-  // gather: a warp takes 32 groups at a time, 8 lanes x float4 per group
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // gather: a warp takes 32 groups at a time, 8 lanes x float4 per group.
+  // Pass 1 keeps no score: each lane records which of its 32 values reach M
+  // (4 bits per float4) in the free part of the bitmap area, so every pass
+  // issues its eight loads with nothing held from the pass before.  Pass 2
+  // reads the taken values again (from L2) and appends them.
+  const int q_al = (n_q + 31) & ~31;
+  uint32_t* tmask = gk + q_al;  // one word per lane per warp pass: entry base + lane
+  const bool two_pass = 2 * q_al <= c.bits_cap;
+  int my_cnt = 0;
   for (int base = warp * 32; base < n_q; base += nw * 32) {
     int e0[8];
     float4 v[8];
@@ -428,8 +444,6 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
         }
       }
     }
-    // every take of this pass in one 32-bit mask per lane (4 bits per step),
-    // then one warp scan and one shared atomic for the whole pass
     uint32_t takes = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -438,6 +452,12 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
       for (int k = 0; k < 4; ++k)
         if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << (4 * u + k);
     }
+    if (two_pass) {
+      tmask[base + lane] = takes;
+      my_cnt += __popc(takes);
+      continue;
+    }
+    // one pass (no room for the masks): append now
     const int n_my = __popc(takes);
     if (!__any_sync(0xffffffffu, n_my != 0)) continue;
     int incl = n_my;
@@ -461,6 +481,33 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
           }
           ++at;
         }
+      }
+    }
+  }
+  if (two_pass) {
+    // this lane's places in the candidate list: one atomic per warp
+    int incl = my_cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int at = 0;
+    if (lane == 31 && incl) at = atomicAdd(&sh.n_cand, incl);
+    at = __shfl_sync(0xffffffffu, at, 31) + incl - my_cnt;
+    for (int base = warp * 32; base < n_q; base += nw * 32) {
+      uint32_t takes = tmask[base + lane];
+      while (takes) {
+        const int bit = __ffs(takes) - 1;
+        takes &= takes - 1;
+        const int u = bit >> 2, k = bit & 3;
+        const int e = (int)gk[base + u * 4 + (lane >> 3)] * 32 + (lane & 7) * 4 + k;
+        const int s = (c.work[e >> c.lb] << c.lb) + (e & c.bmask);
+        if (at < kCandCap) {
+          c.ckey[at] = fkey(c.sc[s]);
+          c.cpos[at] = (uint32_t)e;
+        }
+        ++at;
       }
     }
   }
@@ -718,9 +765,6 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   const unsigned rid = blockIdx.x / (unsigned)C;
   const int q = rid / a.rows, r = rid % a.rows;
   int32_t* out = a.topk + ((int64_t)q * a.rows + r) * L.k;
-  if (a.mask_src && r == 0 && cr == 0)  // the selection's mask row, to the caller's buffer
-    for (int64_t j = threadIdx.x; j < L.max_blocks; j += blockDim.x)
-      a.mask_dst[(int64_t)q * L.max_blocks + j] = a.mask_src[(int64_t)q * L.max_blocks + j];
   __shared__ TopkShared sh;
   extern __shared__ __align__(16) uint8_t dyn[];
   const int64_t ctx = a.ctx_len[q];
@@ -739,6 +783,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   c.n_elem = c.nk << c.lb;
   c.nwords = (c.n_elem + 31) / 32;
   c.bits = reinterpret_cast<uint32_t*>(dyn);
+  c.bits_cap = (int)(topk_bitmap_bytes(L) / 4);
   uint8_t* area = dyn + topk_bitmap_bytes(L);
   c.hist = reinterpret_cast<uint32_t*>(area);
   c.ckey = reinterpret_cast<uint32_t*>(area);

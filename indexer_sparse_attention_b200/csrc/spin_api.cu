@@ -43,8 +43,8 @@ struct spin_state_s {
   // the next step's selection of its layer, so that the step's top-k runs on
   // a second stream beside the next step's predict kernel.
   int lookahead;
-  cudaStream_t side;                 // the next step's predict runs here (created on first use)
-  cudaEvent_t ev_scored, ev_pred;    // fork after the score kernel, join after the side stream's predict
+  cudaStream_t side;                 // this step's top-k runs here (created on first use)
+  cudaEvent_t ev_scored, ev_pred, ev_copied, ev_topk;  // see decode_step_lookahead
   struct Prepared {
     bool ready;
     int64_t step;                    // the step the selection is for (SPIN_STEP_DEVICE: the counter's)
@@ -56,6 +56,9 @@ struct spin_state_s {
   uint8_t* la_mask;                  // [L][Q][max_blocks]
   int32_t* la_ctx;                   // [L][Q] ctx_len each request's selection was made for (-1: none)
   int32_t* ctx_next;                 // [Q] ctx_len + 1, written by the score kernel
+  int32_t* tk_work;                  // [Q][blk_stride] the top-k's copy of the selection it reads, so that
+  int32_t* tk_kept;                  // [Q]   the next selection can be written while it runs
+  int32_t* tk_ctx;                   // [Q]
   uint32_t magic;
 };
 
@@ -114,7 +117,8 @@ Layout make_layout(const spin_config* c) {
 int64_t gmax_stride(const Layout& L) { return L.blk_stride * std::max(1, L.b / 32); }
 
 struct Carve {
-  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, step, la_work, la_kept, la_mask, la_ctx, ctx_next, total;
+  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, step, la_work, la_kept, la_mask, la_ctx, ctx_next, tk_work,
+      tk_kept, tk_ctx, total;
 };
 
 Carve carve(const Layout& L) {
@@ -137,6 +141,9 @@ Carve carve(const Layout& L) {
   k.la_mask = take((size_t)L.L * L.Q * L.max_blocks);
   k.la_ctx = take((size_t)L.L * L.Q * 4);
   k.ctx_next = take((size_t)L.Q * 4);
+  k.tk_work = take((size_t)L.Q * L.blk_stride * 4);
+  k.tk_kept = take((size_t)L.Q * 4);
+  k.tk_ctx = take((size_t)L.Q * 4);
   k.total = off;
   return k;
 }
@@ -288,16 +295,15 @@ spin_status check_rows(spin_state st, int rows) {
 // The pipelined one-row decode step (spin_set_lookahead).  The step's
 // selection was prepared by the previous step of this layer (or is made here
 // when there is none, or it was made for another step or target):
-//   stream:  a0 -> score + fused EMA (writes ctx_len + 1) -> top-k (+ mask) -> [join] -> select(next)
-//   side:                                      [fork] -> predict(next) --------^
+//   stream:  a0 -> score + fused EMA (writes ctx_len + 1) -> predict(next) ----> select(next) -> [join]
+//   side:                                  [fork] -> copy selection, mask ---^ -> top-k --------^
 // The next step's predict reads only V and D, which the score kernel has
-// finished, and writes only the block scores, so it runs beside this step's
-// top-k; the next selection overwrites the kept lists the top-k reads, so it
-// follows the top-k.  The top-k is launched first, directly behind the score
-// kernel, so that its CTAs are placed before the predict kernel's fill the
-// SMs.  Results are those of the sequential step: the next selection is
-// computed from the same state, positions (ctx_len + 1) and step number as the
-// next call would compute it.
+// finished, and has the GPU to itself; then this step's top-k and the next
+// step's select, both latency-bound with one CTA per request, run side by
+// side.  The top-k reads a copy of the kept lists, taken while the predict
+// runs, because the next select overwrites them.  Results are those of the
+// sequential step: the next selection is computed from the same state,
+// positions (ctx_len + 1) and step number as the next call would compute it.
 spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const void* keys, const float* key_scale,
                                   int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
                                   const float* w, const int32_t* ctx_len, uint8_t* mask_dev, int32_t* topk_dev,
@@ -336,28 +342,39 @@ spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const 
   r = run_score(st, layer, 1, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len, lmask, scores,
                 true, s, &gm, false, &sel);
   if (r != SPIN_OK) return r;
-  // fork: the next step's predict on the side stream
-  StepArgs a = select_args(st->ctx_next, next, true);
-  a.no_pdl = 1;  // both launches below follow a wait on the other stream's event
+  // fork: the side stream copies the selection the top-k reads, and the mask
   cudaError_t e = cudaEventRecord(st->ev_scored, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st->side, st->ev_scored, 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->tk_work, work, (size_t)L.Q * L.blk_stride * 4, cudaMemcpyDeviceToDevice, st->side);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->tk_kept, kept, (size_t)L.Q * 4, cudaMemcpyDeviceToDevice, st->side);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->tk_ctx, lctx, (size_t)L.Q * 4, cudaMemcpyDeviceToDevice, st->side);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(mask_dev, lmask, (size_t)L.Q * L.max_blocks, cudaMemcpyDeviceToDevice, st->side);
+  if (e == cudaSuccess) e = cudaEventRecord(st->ev_copied, st->side);
   if (e != cudaSuccess) return cuda_status(e);
+  // the next step's predict, alone on the GPU
+  StepArgs a = select_args(st->ctx_next, next, true);
   if (sp > 0.0f) {
-    r = cuda_status(staged(st, kPredict, st->side, [&] { return launch_predict_pool(a, st->side); }));
+    r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
     if (r != SPIN_OK) return r;
   }
-  e = cudaEventRecord(st->ev_pred, st->side);  // the predict's end
+  e = cudaEventRecord(st->ev_pred, s);
+  // this step's top-k, once the predict is done, beside the next select
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->side, st->ev_pred, 0);
   if (e != cudaSuccess) return cuda_status(e);
-  // this step's top-k, which also hands the selection's mask to the caller
-  TopkArgs t{L, 1, scores, mask_dev, ctx_len, work, kept, topk_dev, st->err, gm ? st->gmax : nullptr,
-             st->gstride, lctx, lmask, mask_dev};
-  r = cuda_status(staged(st, kTopk, s, [&] { return launch_topk(t, s); }));
+  TopkArgs t{L, 1, scores, mask_dev, ctx_len, st->tk_work, st->tk_kept, topk_dev, st->err, gm ? st->gmax : nullptr,
+             st->gstride, st->tk_ctx};
+  r = cuda_status(staged(st, kTopk, st->side, [&] { return launch_topk(t, st->side); }));
   if (r != SPIN_OK) return r;
-  // join, then the next step's selection
-  e = cudaStreamWaitEvent(s, st->ev_pred, 0);
+  e = cudaEventRecord(st->ev_topk, st->side);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->ev_copied, 0);  // the kept lists are copied
   if (e != cudaSuccess) return cuda_status(e);
+  a.no_pdl = 1;  // follows a wait on the other stream's event
   r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
   if (r != SPIN_OK) return r;
+  e = cudaStreamWaitEvent(s, st->ev_topk, 0);  // join
+  if (e != cudaSuccess) return cuda_status(e);
   P.ready = true;
   P.step = next;
   P.sparsity = sp;
@@ -404,9 +421,12 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->la_mask = (uint8_t*)(st->base + k.la_mask);
   st->la_ctx = (int32_t*)(st->base + k.la_ctx);
   st->ctx_next = (int32_t*)(st->base + k.ctx_next);
+  st->tk_work = (int32_t*)(st->base + k.tk_work);
+  st->tk_kept = (int32_t*)(st->base + k.tk_kept);
+  st->tk_ctx = (int32_t*)(st->base + k.tk_ctx);
   st->lookahead = 0;
   st->side = nullptr;
-  st->ev_scored = st->ev_pred = nullptr;
+  st->ev_scored = st->ev_pred = st->ev_copied = st->ev_topk = nullptr;
   st->prep.assign(cfg->num_layers, spin_state_s::Prepared{false, 0, 0.0f});
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
@@ -440,8 +460,8 @@ spin_status spin_state_destroy(spin_state st) {
     cudaEventDestroy(r.b);
   }
   for (auto e : st->pool) cudaEventDestroy(e);
-  if (st->ev_scored) cudaEventDestroy(st->ev_scored);
-  if (st->ev_pred) cudaEventDestroy(st->ev_pred);
+  for (cudaEvent_t e : {st->ev_scored, st->ev_pred, st->ev_copied, st->ev_topk})
+    if (e) cudaEventDestroy(e);
   if (st->side) cudaStreamDestroy(st->side);
   st->magic = 0;
   delete st;
@@ -474,6 +494,8 @@ spin_status spin_set_lookahead(spin_state st, int enable) {
     cudaError_t e = cudaStreamCreateWithFlags(&st->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_scored, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_pred, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_copied, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_topk, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_status(e);
   }
   st->lookahead = enable;

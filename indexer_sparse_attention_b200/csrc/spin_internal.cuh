@@ -305,8 +305,6 @@ struct TopkArgs {
   const float* gmax;  // group maxima written by the score kernel, or null
   int64_t gstride;
   const int32_t* ctx_sel;  // [Q] or null: a request whose ctx_len differs comes back all -1
-  const uint8_t* mask_src; // [Q][max_blocks] or null: copied to mask_dst (a prepared selection's mask
-  uint8_t* mask_dst;       // handed to the caller by the top-k launch)
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 

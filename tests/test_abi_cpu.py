@@ -56,7 +56,8 @@ def _expected_bytes(L, Q, R, H, d, b, max_slots):
     parts = [16, L * Q * slot * 4, L * Q * slot * 4, Q * R * blk * 4, Q * blk * 4, Q * 4, Q * R * H * d,
              Q * R * H * 4, Q * R * slot * 4, Q * R * blk * max(1, b // 32) * 4, 8,
              # the selection a pipelined step prepares for the next one, per layer, and ctx_len + 1
-             L * Q * blk * 4, L * Q * 4, L * Q * mb, L * Q * 4, Q * 4]
+             L * Q * blk * 4, L * Q * 4, L * Q * mb, L * Q * 4, Q * 4,
+             Q * blk * 4, Q * 4, Q * 4]  # and the top-k's copy of the kept lists
     return sum(a(p) for p in parts)
 
 
