@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_shard_requests_and_take_max_time():
     world, port = 2, _free_port()
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)

@@ -120,7 +120,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 3])
 def test_sharded_steps_equal_the_unsharded_oracle(world):
     port = _free_port()
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)
