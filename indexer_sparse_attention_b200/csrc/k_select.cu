@@ -270,62 +270,41 @@ __device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t
 }
 
 constexpr int kExpCap = 2048;
-constexpr int kRankMax = 512;  // longest list ranked by counting
 
 // The `take` entries of list[0 .. cnt) first by (key, block index) go to
-// mark(block): ranked by counting for up to kRankMax entries, by a bitonic
-// sort for longer lists.  `rank` holds cnt ints of scratch.  All threads of
-// the CTA call it.
+// mark(block): a radix select of the largest ~key (the smallest key) over
+// the list, then the entries past the threshold, and the lowest blocks among
+// those equal to it.  `scratch` holds cnt words.  All threads of the CTA call
+// it; 1 <= take <= cnt.
 template <class Mark>
-__device__ void draw_from_list(uint2* list, int cnt, int take, int* rank, Mark mark) {
-  if (cnt <= kRankMax) {
-    // exact rank of every entry: `parts` threads per entry each count a
-    // slice of the list (cnt^2 comparisons: cheaper than a sort's barriers
-    // for short lists)
-    int parts = 1;
-    while (parts * 2 * cnt <= (int)blockDim.x) parts *= 2;
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) rank[i] = 0;
-    __syncthreads();
-    const int i = (int)threadIdx.x / parts, part = (int)threadIdx.x % parts;
-    if (i < cnt) {
-      const uint2 me = list[i];
-      const int k0 = (int)((int64_t)cnt * part / parts), k1 = (int)((int64_t)cnt * (part + 1) / parts);
-      int below = 0;
-      for (int k = k0; k < k1; ++k) {
-        const uint2 o = list[k];
-        below += (o.x < me.x) || (o.x == me.x && o.y < me.y);
-      }
-      if (below) atomicAdd(&rank[i], below);
-    }
-    __syncthreads();
-    for (int i2 = threadIdx.x; i2 < cnt; i2 += blockDim.x)
-      if (rank[i2] < take) mark((int)list[i2].y);
-    __syncthreads();
-    return;
-  }
-  // longer lists: bitonic sort by (key, block), padded to a power of two with
-  // entries that sort last; the first `take` entries are the draw
-  int n2 = 1;
-  while (n2 < cnt) n2 <<= 1;
-  for (int i = cnt + (int)threadIdx.x; i < n2; i += blockDim.x) list[i] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+__device__ void draw_from_list(const uint2* list, int cnt, int take, int* scratch, Mark mark, SelShared& sh) {
+  uint32_t* nk = reinterpret_cast<uint32_t*>(scratch);
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) nk[i] = ~list[i].x;
   __syncthreads();
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const uint2 x = list[i], y = list[ixj];
-          const bool gt = x.x > y.x || (x.x == y.x && x.y > y.y);
-          if (gt == ((i & k) == 0)) {
-            list[i] = y;
-            list[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
+  uint32_t T, eq_take;
+  radix_select_desc(nk, cnt, [](int) { return true; }, (uint32_t)take, sh, &T, &eq_take);
+  if (threadIdx.x == 0) sh.digit[0] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+    if (nk[i] > T) mark((int)list[i].y);
+    else if (nk[i] == T) atomicAdd(&sh.digit[0], 1u);
+  }
+  __syncthreads();
+  const uint32_t n_eq = sh.digit[0];
+  if (n_eq == eq_take) {
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x)
+      if (nk[i] == T) mark((int)list[i].y);
+  } else if (threadIdx.x == 0) {
+    // equal 32-bit keys: the eq_take lowest blocks among them, one at a time
+    uint32_t last = 0;
+    for (uint32_t t = 0; t < eq_take; ++t) {
+      uint32_t best = 0xFFFFFFFFu;
+      for (int i = 0; i < cnt; ++i)
+        if (nk[i] == T && list[i].y < best && (t == 0 || list[i].y > last)) best = list[i].y;
+      mark((int)best);
+      last = best;
     }
   }
-  for (int i = threadIdx.x; i < take; i += blockDim.x) mark((int)list[i].y);
   __syncthreads();
 }
 
@@ -362,20 +341,25 @@ __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last
   __syncthreads();
   const int cnt = (int)sh.digit[0];
   if (cnt < take || cnt > kExpCap) return false;  // uniform: every thread reads the same count
-  draw_from_list(list, cnt, take, rank, [m](int j) { m[j] = 2; });
+  draw_from_list(list, cnt, take, rank, [m](int j) { m[j] = 2; }, sh);
   return true;
 }
 
-// Ordered compaction of the kept blocks of one request into its work list.
-__device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t* kept, int* scan) {
+// Ordered compaction of the kept blocks of one request into its work list;
+// with mask_out, the labels of blocks 0 .. n_last-1 are written there too.
+__device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t* kept, int* scan,
+                            uint8_t* mask_out = nullptr) {
   const int chunk = (n_last + blockDim.x - 1) / blockDim.x;
   const int lo = threadIdx.x * chunk, hi = min(n_last, lo + chunk);
   int c = 0;
   for (int j = lo; j < hi; ++j) c += m[j] != 0;
   int total;
   int pos = block_exclusive_scan(c, scan, &total);
-  for (int j = lo; j < hi; ++j)
-    if (m[j]) work[pos++] = j;
+  for (int j = lo; j < hi; ++j) {
+    const uint8_t v = m[j];
+    if (mask_out) mask_out[j] = v;
+    if (v) work[pos++] = j;
+  }
   if (threadIdx.x == 0) *kept = total;
 }
 
@@ -454,10 +438,15 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
     }
     // exploration among the unkept blocks of the last row's range
     auto cand = [m](int j) { return m[j] == 0; };
-    int c = 0;
-    for (int j = threadIdx.x; j < n_last; j += blockDim.x) c += (m[j] == 0);
     int n_cand;
-    block_exclusive_scan(c, sh.scan, &n_cand);
+    if (a.rows == 1) {  // one row: exactly min(max(n_pred, 0), n) blocks are predicted
+      const int64_t n_pred = block_budget(n_last, a.sparsity) - n_exp;
+      n_cand = n_last - (int)(n_pred < 0 ? 0 : n_pred > n_last ? n_last : n_pred);
+    } else {
+      int c = 0;
+      for (int j = threadIdx.x; j < n_last; j += blockDim.x) c += (m[j] == 0);
+      block_exclusive_scan(c, sh.scan, &n_cand);
+    }
     const int64_t take = n_exp < n_cand ? n_exp : n_cand;
     if (take == n_cand) {
       for (int j = threadIdx.x; j < n_last; j += blockDim.x)
@@ -494,8 +483,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
       }
     }
   }
-  for (int64_t j = threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = j < n_last ? m[j] : 0;
-  compact_row(m, n_last, a.work + (int64_t)q * L.blk_stride, a.kept + q, sh.scan);
+  for (int64_t j = n_last + threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = 0;
+  compact_row(m, n_last, a.work + (int64_t)q * L.blk_stride, a.kept + q, sh.scan, mask_row);
 }
 
 // ---------------------------------------------------------------------------
@@ -724,7 +713,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
             int owner = C - 1;
             while (owner > 0 && range_lo(n_last, owner, C) > j) --owner;
             cl.map_shared_rank(m, owner)[j - range_lo(n_last, owner, C)] = 2;
-          });
+          }, sh);
         }
         cl.sync();  // the drawn blocks are marked in every owner's mask
       } else {
