@@ -9,7 +9,7 @@
 //     order (SPIN digest, arXiv深度剖析: prefix-valid replay); under the
 //     row-0 MTP policy row 0 alone is applied (SPIN listing, Table 7).
 //
-// Parallel layout: one warp per block j of a request.  The vertical state of
+// Parallel layout: one warp per block j of a request at a time.  The vertical state of
 // a slot is owned by the slot (its rows run in order inside one thread); the
 // diagonal state D_delta is owned by the block of row 0's slot
 // s_0 = p_0 - delta, and its rows r = 0..a-1 (slot s_0 + r) run in order
@@ -61,30 +61,29 @@ cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t s
 
 // R: the most rows one update applies (the call's rows, or 1 under the row-0
 // policy); a.rows, the call's rows, bounds the context and accepted lengths.
+// Grid: column x = request, its gridDim.y blocks' warps take the request's
+// blocks j in turn (no division per block).
 template <int R>
 __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
   pdl_enter();
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
-  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       wid < (int64_t)L.Q * L.max_blocks; wid += nw) {
-    const int q = (int)(wid / L.max_blocks);
-    const int64_t j = wid % L.max_blocks;
-    const int64_t ctx = a.ctx_len[q];
-    if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) continue;
-    int acc = R;
-    if (a.accepted) {
-      acc = a.accepted[q];
-      if (acc < 1 || acc > a.rows) {
-        if (j == 0 && lane == 0) raise_error(a.err, ERR_ACCEPTED, q, (uint32_t)acc);
-        continue;
-      }
-      acc = min(acc, R);
+  const int q = blockIdx.x;
+  const int64_t ctx = a.ctx_len[q];
+  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) return;  // block-uniform
+  int acc = R;
+  if (a.accepted) {
+    acc = a.accepted[q];
+    if (acc < 1 || acc > a.rows) {
+      if (blockIdx.y == 0 && threadIdx.x == 0) raise_error(a.err, ERR_ACCEPTED, q, (uint32_t)acc);
+      return;
     }
-    const int64_t p0 = ctx - 1;
-    const int64_t n_last = row_blocks(ctx, acc - 1, L.b);
-    if (j >= n_last) continue;
+    acc = min(acc, R);
+  }
+  const int64_t p0 = ctx - 1;
+  const int64_t n_last = row_blocks(ctx, acc - 1, L.b);
+  const int wpr = (int)gridDim.y * (blockDim.x >> 5);
+  for (int64_t j = (int64_t)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5); j < n_last; j += wpr) {
     const uint8_t* mask = a.mask + (int64_t)q * L.max_blocks;
     const bool kj = mask[j] != 0;
     const bool kj1 = (R > 1) && (j + 1 < n_last) && mask[j + 1] != 0;
@@ -156,10 +155,11 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
 }
 
 cudaError_t launch_ema_update(const EmaArgs& a, cudaStream_t s) {
-  int64_t warps = (int64_t)a.lay.Q * a.lay.max_blocks;
-  int64_t blocks = (warps + 7) / 8;
-  if (blocks > 148 * 64) blocks = 148 * 64;
-  PdlLaunch l(dim3((unsigned)blocks), dim3(256), 0, s);
+  // about 8 blocks of 256 threads per SM over all requests
+  int64_t gy = (148 * 8 + a.lay.Q - 1) / a.lay.Q;
+  gy = std::min<int64_t>(gy, (a.lay.max_blocks + 7) / 8);
+  gy = std::max<int64_t>(std::min<int64_t>(gy, 65535), 1);
+  PdlLaunch l(dim3((unsigned)a.lay.Q, (unsigned)gy), dim3(256), 0, s);
   switch (a.row0 ? 1 : a.rows) {
     case 1: return cudaLaunchKernelEx(&l.cfg, k_ema_update<1>, a);
     case 2: return cudaLaunchKernelEx(&l.cfg, k_ema_update<2>, a);
