@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
   }
   const int64_t p0 = ctx - 1;
   const int64_t n_last = row_blocks(ctx, acc - 1, L.b);
+  const int lb = __ffs(L.b) - 1;  // the block size is a power of two
   const int wpr = (int)gridDim.y * (blockDim.x >> 5);
   for (int64_t j = (int64_t)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5); j < n_last; j += wpr) {
     const uint8_t* mask = a.mask + (int64_t)q * L.max_blocks;
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
         for (int r = 0; r < R; ++r) {
           use_v[h][r] = do_v[h] && r < acc && s <= p0 + r;
           const int64_t sr = s + r;  // row r's slot for delta: in block j, or past its end in block j + 1
-          use_d[h][r] = do_d[h] && r < acc && ((sr / L.b == j) ? kj : kj1);
+          use_d[h][r] = do_d[h] && r < acc && (((sr >> lb) == j) ? kj : kj1);
           sv[h][r] = use_v[h][r] ? sc[(int64_t)r * L.slot_stride + s] : 0.f;
           sd[h][r] = use_d[h][r] ? sc[(int64_t)r * L.slot_stride + sr] : 0.f;
         }
