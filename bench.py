@@ -473,10 +473,11 @@ def gpu_arm(args, world, rank, local):
     peak, peak_kind = peaks()
     score_ms, score_n = stages["score"]
     score_avg = score_ms / max(score_n, 1)
-    achieved = kept_slots * SCORE_BYTES_PER_SLOT / (score_avg / 1e3) / 1e9
+    score_b = score_bytes_per_slot(1, True, True, 128, args.pooling == "max")
+    achieved = kept_slots * score_b / (score_avg / 1e3) / 1e9
     traffic_slot = score_traffic_per_slot()
     launches = sum(n for _, n in stages.values())
-    step_tr = step_traffic(int(run.ctx[run.t - 1].long().sum().item()), kept_slots, ms_step, peak)
+    step_tr = step_traffic(int(run.ctx[run.t - 1].long().sum().item()), kept_slots, ms_step, peak, args.pooling)
     out = {
         "metric": METRIC, "value": rows_s, "unit": "rows/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -489,7 +490,7 @@ def gpu_arm(args, world, rank, local):
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs (copy, MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s", "avg_launch_ms": score_avg,
-                     "bytes_per_launch": kept_slots * SCORE_BYTES_PER_SLOT,
+                     "bytes_per_launch": kept_slots * score_b,
                      "traffic": (None if traffic_slot is None else traffic_slot * kept_slots),
                      "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
                                         "(16-request capture, scaled by kept slots)" if traffic_slot is not None
@@ -582,12 +583,12 @@ def graph_pass(run, warmup, steps, world):
 L2_BYTES = 126 * 1024 * 1024
 
 
-def score_bytes_per_slot(rows: int, fused: bool, key_fp8: bool, d: int) -> int:
+def score_bytes_per_slot(rows: int, fused: bool, key_fp8: bool, d: int, vmax: bool = False) -> float:
     """Algorithmic bytes of the score kernel per kept slot: the key row and
-    its scale, one score per row, and (fused, one row) the EMA read/write of
-    V and D."""
+    its scale, one score per row, (fused, one row) the EMA read/write of V
+    and D, and with it (max pooling) V's maximum of each 32 kept slots."""
     key = (d + 4) if key_fp8 else 4 * d
-    return key + 4 * rows + (16 if fused else 0)
+    return key + 4 * rows + (16 if fused else 0) + (4 / 32 if fused and vmax else 0)
 
 
 class WorkloadRun:
@@ -782,7 +783,7 @@ def workload_arm(args, world, rank, local):
     rows_step = Q * R
     peak, peak_kind = peaks()
     fused = R == 1
-    per_slot = score_bytes_per_slot(R, fused, wl.key_fp8, wl.d)
+    per_slot = score_bytes_per_slot(R, fused, wl.key_fp8, wl.d, args.pooling == "max" and wl.b >= 32)
     key_slot = (wl.d + 4) if wl.key_fp8 else 4 * wl.d
     score_ms, score_n = stages["score"]
     score_avg = score_ms / max(score_n, 1)
@@ -1105,14 +1106,17 @@ def cpu_baseline(sparsity, seconds):
                       f"after an untimed all-keep bootstrap; fp64 scores, OpenMP over blocks; {dt:.1f} s"}
 
 
-def step_traffic(context_slots, kept_slots, ms_step, peak):
+def step_traffic(context_slots, kept_slots, ms_step, peak, pooling="max"):
     """The whole step's algorithmic bytes against the measured copy bandwidth:
-    8 B per slot of context (the predict kernel reads V and D) plus the score
+    per slot of context, what the predict kernel reads (max pooling: D and
+    V's maximum per 32 slots, 4.125 B; otherwise V and D, 8 B), plus the score
     kernel's bytes per kept slot (key, scale, score, EMA read and write)."""
-    b = 8 * context_slots + SCORE_BYTES_PER_SLOT * kept_slots
+    ctx_b = 4 + 4 / 32 if pooling == "max" else 8
+    kept_b = score_bytes_per_slot(1, True, True, 128, pooling == "max")
+    b = ctx_b * context_slots + kept_b * kept_slots
     gbs = b / (ms_step / 1e3) / 1e9
     return {"bytes_per_step": b, "gbs": gbs, "frac": gbs / peak,
-            "note": "8 B per slot of context + 152 B per kept slot; the floor of a step"}
+            "note": f"{ctx_b:g} B per slot of context + {kept_b:g} B per kept slot; the floor of a step"}
 
 
 def headline_config(wl, Q, args, world):

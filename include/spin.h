@@ -124,7 +124,9 @@ typedef enum { SPIN_MTP_UNION_PREFIX = 0, SPIN_MTP_ROW0 = 1 } spin_mtp_policy;
 typedef struct spin_state_s* spin_state;
 
 /* Bytes of device memory a state needs: EMA states V and D for every layer
- * and request, block-score / work-list / quantised-query / score scratch, the
+ * and request (with max pooling and block_size >= 32 also V's maximum over
+ * each aligned 32-slot group, which the prediction reads in place of V for
+ * the blocks below the newest one), block-score / work-list / quantised-query / score scratch, the
  * per-layer selection a pipelined step prepares (spin_set_lookahead) and the
  * device error word.  Returns 0 for an invalid config. */
 SPIN_API size_t spin_state_bytes(const spin_config* cfg);
@@ -372,14 +374,26 @@ SPIN_API size_t spin_state_export_bytes(spin_state st);
 SPIN_API spin_status spin_state_export(spin_state st, void* host, size_t bytes, spin_stream_t stream);
 SPIN_API spin_status spin_state_import(spin_state st, const void* host, size_t bytes, spin_stream_t stream);
 
+/* After writing V (or D) of the EMA state through the pointers spin_state_ema
+ * returns, the caller calls this before the next library call that reads the
+ * state: it recomputes V's 32-slot group maxima of `layer` (layer -1: every
+ * layer) on `stream`, and drops any selection a pipelined step prepared.
+ * Every library call that writes V keeps them current by itself. */
+SPIN_API spin_status spin_state_refresh(spin_state st, int layer, spin_stream_t stream);
+
 /* Inspection: device pointers into the state block.
- *   spin_state_ema: V, D of `layer`, each [Q][*stride] fp32.
+ *   spin_state_ema: V, D of `layer`, each [Q][*stride] fp32.  Writing through
+ *     them is allowed, followed by spin_state_refresh.
+ *   spin_state_vmax: V's group maxima of `layer`, [Q][*stride] fp32 with
+ *     (*vmax)[q][g] = max(V[q][32 g .. 32 g + 31]); NULL and stride 0 when the
+ *     state keeps none (block_size 16, or a pooling other than max).
  *   spin_state_block_scores: S [Q][max_rows][*stride] fp32 of the last predict.
  *   spin_state_qquant: quantised queries [Q][max_rows][H][d] E4M3 and their
  *   folded head weights [Q][max_rows][H] fp32 of the last FP8 score call.
  *   spin_score_stride: slot stride of a score row (ceil(max_slots/b)*b);
  *   spin_mask_stride: block stride of a mask row (ceil(max_slots/b)). */
 SPIN_API spin_status spin_state_ema(spin_state st, int layer, float** V, float** D, int64_t* stride);
+SPIN_API spin_status spin_state_vmax(spin_state st, int layer, const float** vmax, int64_t* stride);
 SPIN_API spin_status spin_state_block_scores(spin_state st, const float** S, int64_t* stride);
 SPIN_API spin_status spin_state_qquant(spin_state st, const uint8_t** q8, const float** wq);
 SPIN_API int64_t spin_score_stride(spin_state st);

@@ -115,6 +115,8 @@ def load():
         "spin_state_export": (S, [_vp, _vp, ctypes.c_size_t, _vp]),
         "spin_state_import": (S, [_vp, _vp, ctypes.c_size_t, _vp]),
         "spin_state_ema": (S, [_vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
+        "spin_state_vmax": (S, [_vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
+        "spin_state_refresh": (S, [_vp, ctypes.c_int, _vp]),
         "spin_state_block_scores": (S, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
         "spin_state_qquant": (S, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
         "spin_score_stride": (_i64, [_vp]),
@@ -198,6 +200,19 @@ class SpinState:
         Q = self.cfg.num_requests
         return (self._view(V.value, Q * st.value, torch.float32, (Q, st.value)),
                 self._view(D.value, Q * st.value, torch.float32, (Q, st.value)))
+
+    def vmax(self, layer: int):
+        """V's 32-slot group maxima of a layer, [Q][slot_stride / 32], or None."""
+        p, st = _vp(), _i64()
+        _check(load().spin_state_vmax(self.handle, layer, ctypes.byref(p), ctypes.byref(st)), "spin_state_vmax")
+        if not p.value:
+            return None
+        Q = self.cfg.num_requests
+        return self._view(p.value, Q * st.value, torch.float32, (Q, st.value))
+
+    def refresh(self, layer: int = -1, stream=None):
+        """After writing V or D through ema(): brings the state's derived data up to date."""
+        _check(load().spin_state_refresh(self.handle, layer, _stream(stream)), "spin_state_refresh")
 
     def block_scores(self):
         S, st = _vp(), _i64()

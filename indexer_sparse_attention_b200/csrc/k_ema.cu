@@ -15,24 +15,55 @@
 // s_0 = p_0 - delta, and its rows r = 0..a-1 (slot s_0 + r) run in order
 // inside one thread.  Offsets delta > p_0 (only later rows see them) belong to
 // block 0.  Every (row, slot) pair is applied exactly once, in row order.
+//
+// Group maxima of V: where the state keeps vmax[g] = max(V[32 g .. 32 g + 31])
+// (the max-pooled prediction reads them in place of V: max over a block of
+// max(V_i, D_{p-i}) is the max of V's maximum and D's), every writer of V
+// brings the groups it wrote up to date: the replay kernel from the values in
+// its registers, the fills with +inf, k_vmax_refresh after a bulk write.
 #include <algorithm>
 
 #include "spin_internal.cuh"
 
 namespace spin {
 
-__global__ void k_fill(float* V, float* D, int64_t n) {
+__global__ void k_fill(float* V, float* D, int64_t n, float* vmax, int64_t nv) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     V[i] = __int_as_float(0x7f800000);
     D[i] = __int_as_float(0xff800000);
   }
+  if (vmax)
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += (int64_t)gridDim.x * blockDim.x)
+      vmax[i] = __int_as_float(0x7f800000);
 }
 
-cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s) {
+cudaError_t launch_init_state(float* V, float* D, int64_t n, float* vmax, int64_t nv, cudaStream_t s) {
   int64_t blocks = (n + 255) / 256;
   if (blocks > 148 * 32) blocks = 148 * 32;
   if (blocks < 1) blocks = 1;
-  k_fill<<<(int)blocks, 256, 0, s>>>(V, D, n);
+  k_fill<<<(int)blocks, 256, 0, s>>>(V, D, n, vmax, nv);
+  return cudaGetLastError();
+}
+
+// One warp per 32-slot group: a coalesced 128-byte row of V and a warp max.
+__global__ void __launch_bounds__(256) k_vmax_refresh(const float* V, float* vmax, int64_t rows, int64_t slot_stride,
+                                                      int64_t vg_stride) {
+  const int lane = threadIdx.x & 31;
+  const int64_t groups = rows * vg_stride;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < groups; g += warps) {
+    const int64_t row = g / vg_stride, c = g - row * vg_stride;
+    const float x = warp_max(V[row * slot_stride + c * 32 + lane]);
+    if (lane == 0) vmax[g] = x;
+  }
+}
+
+cudaError_t launch_vmax_refresh(const float* V, float* vmax, int64_t rows, int64_t slot_stride, int64_t vg_stride,
+                                cudaStream_t s) {
+  if (!vmax || rows < 1 || vg_stride < 1) return cudaSuccess;
+  int64_t blocks = (rows * vg_stride + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_vmax_refresh<<<(int)blocks, 256, 0, s>>>(V, vmax, rows, slot_stride, vg_stride);
   return cudaGetLastError();
 }
 
@@ -43,19 +74,26 @@ cudaError_t launch_step_op(int64_t* p, bool set, int64_t value, cudaStream_t s) 
   return cudaGetLastError();
 }
 
-__global__ void k_reset_rows(float* V, float* D, ReqList list, int64_t stride) {
+__global__ void k_reset_rows(float* V, float* D, float* vmax, ReqList list, int64_t stride, int64_t vg_stride) {
   for (int k = blockIdx.y; k < list.n; k += gridDim.y) {
     const int64_t base = (int64_t)list.ids[k] * stride;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < stride; i += (int64_t)gridDim.x * blockDim.x) {
       V[base + i] = __int_as_float(0x7f800000);
       D[base + i] = __int_as_float(0xff800000);
     }
+    if (vmax) {
+      const int64_t vb = (int64_t)list.ids[k] * vg_stride;
+      for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < vg_stride;
+           i += (int64_t)gridDim.x * blockDim.x)
+        vmax[vb + i] = __int_as_float(0x7f800000);
+    }
   }
 }
 
-cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t stride, cudaStream_t s) {
+cudaError_t launch_reset_rows(float* V, float* D, float* vmax, const ReqList& list, int64_t stride,
+                              int64_t vg_stride, cudaStream_t s) {
   dim3 grid((unsigned)std::min<int64_t>((stride + 255) / 256, 1024), (unsigned)list.n);
-  k_reset_rows<<<grid, 256, 0, s>>>(V, D, list, stride);
+  k_reset_rows<<<grid, 256, 0, s>>>(V, D, vmax, list, stride, vg_stride);
   return cudaGetLastError();
 }
 
@@ -132,6 +170,17 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
         }
         if (tv) V[sl[h]] = v[h];
         if (td) D[p0 - sl[h]] = dv[h];
+      }
+      // a kept block's 32-slot groups: every lane holds its slot's V, new or
+      // not (vmax is kept only for b >= 32, so the whole warp is here)
+      if (a.vmax && kj) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (i0 - lane + 32 * h < L.b) {  // warp-uniform
+            const float g = warp_max(v[h]);
+            if (lane == 0) a.vmax[(int64_t)q * L.vg_stride + (sl[h] >> 5)] = g;
+          }
+        }
       }
     }
     // offsets delta = p0 + m (m >= 1): seen only by rows r >= m at slot r - m

@@ -118,6 +118,15 @@ __global__ void __launch_bounds__(kSimtThreads) k_score_simt(ScoreArgs a) {
         }
       }
     }
+    if (a.vmax) {  // kernel-uniform: the block's 32-slot groups of V, after its update
+      __syncthreads();
+      const int lane = threadIdx.x & 31;
+      const float* V = a.V + (int64_t)q * L.slot_stride + (int64_t)j * L.b;
+      for (int g = threadIdx.x >> 5; g < L.b / 32; g += kSimtThreads / 32) {
+        const float x = warp_max(V[g * 32 + lane]);
+        if (lane == 0) a.vmax[(int64_t)q * L.vg_stride + (((int64_t)j * L.b) >> 5) + g] = x;
+      }
+    }
   }
 }
 

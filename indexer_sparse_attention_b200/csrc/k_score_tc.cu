@@ -28,7 +28,9 @@
 //               quarter its warp may access (lanes 32*(warp%4) ..), hands
 //               the accumulator back as soon as its last columns are in
 //               registers, applies ReLU, head weights and the scale, and
-//               stores the score and the fused EMA update.  With one CTA
+//               stores the score and the fused EMA update (a warp's 32
+//               tokens are one aligned group of V, whose maximum it also
+//               stores for the next prediction).  With one CTA
 //               per SM (N > 128) there are four groups; for several query
 //               rows two groups share each tile, one taking the even rows and
 //               the other the odd ones, so an accumulator is read out in half
@@ -590,7 +592,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     // global load takes longer than one tile of the epilogue.  DIST follows
     // the rule of prefetch_dist(), which the host checked for this plan.
     struct Pre {
-      int q, s, valid, upd, t;
+      int q, s, pres, valid, upd, t;
       int p0;  // ctx_len - 1 < 2^31 (max_slots is an int32)
       float sigma, v, d;
     };
@@ -609,6 +611,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       pg = x->pg[pg_idx];
       const bool present = pg_idx < x->np && pg >= 0;
       r.s = present ? x->j[pg_idx] * kPage + tok : 0;
+      r.pres = present;
       r.valid = present && r.s <= r.p0 + (a.rows - 1);
       r.upd = fused && r.valid && r.s <= r.p0;
       return r;
@@ -618,7 +621,8 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       const Pre m = meta_of(i, pg);
       Side r;
       r.sigma = m.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
-      r.v = m.upd ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
+      // V of the page's slots past the context too, for its group maxima
+      r.v = (m.upd || (a.vmax && m.pres)) ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
       r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
       return r;
     };
@@ -712,18 +716,23 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
         const bool scored = cur.valid && cur.s <= cur.p0 + r;
         if (a.gmax) {
           // max over this warp's 32 slots = group 4t + quarter of the kept-slot order
-          float g = scored ? sum * cur.sigma : __int_as_float(0xff800000);
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
+          const float g = warp_max(scored ? sum * cur.sigma : __int_as_float(0xff800000));
           if (lane == 0) a.gmax[((int64_t)cur.q * L.R + r) * a.gstride + 4 * cur.t + quarter] = g;
         }
+        float vnew = cur.v;
         if (scored) {
           const float score = sum * cur.sigma;
           a.scores[((int64_t)cur.q * L.R + r) * L.slot_stride + cur.s] = score;
           if (cur.upd && r == 0) {
-            a.V[(int64_t)cur.q * L.slot_stride + cur.s] = ema_v(cur.v, score, a.alpha, a.beta);
+            vnew = ema_v(cur.v, score, a.alpha, a.beta);
+            a.V[(int64_t)cur.q * L.slot_stride + cur.s] = vnew;
             a.D[(int64_t)cur.q * L.slot_stride + (cur.p0 - cur.s)] = ema_d(cur.d, score, a.alpha, a.beta);
           }
+        }
+        if (a.vmax && r == 0 && cur.pres) {
+          // this warp's 32 slots are one aligned group of V (present is warp-uniform)
+          const float g = warp_max(vnew);
+          if (lane == 0) a.vmax[(int64_t)cur.q * L.vg_stride + (cur.s >> 5)] = g;
         }
       }
       acc += tgroups;

@@ -4,7 +4,8 @@
 // a1: z_{r,i} = max(V_i, D_{p_r - i}) and S_{r,j} = max over the valid slots
 //     of block j (AI Radio episode, "Title and authors"; SPIN digest,
 //     arXiv深度剖析: per-slot and per-offset EMA states).  HBM-bound: 8 bytes
-//     per slot of context (V and D read once for all rows).
+//     per slot of context (V and D read once for all rows); with max pooling,
+//     4 bytes of D plus 4 bytes of V's maximum per 32 slots.
 // a2: block budget B_r = n_r - floor(s n_r); a share n_exp = floor(gamma B_0)
 //     of it goes to uniformly random unkept blocks (SPIN digest, arXiv深度剖析;
 //     SPIN listing, Figure 4); each row's top (B_r - n_exp) blocks are unioned
@@ -22,22 +23,32 @@
 namespace spin {
 
 // ---------------------------------------------------------------------------
-// a1: grid column x = request; its blocks' warps take 256-slot chunks of that
-// request in turn (no division per chunk).  A lane takes 8 consecutive slots:
-// two float4 loads of V and the D window its rows need (offsets p0-i0-7 ..
-// p0-i0+R-1) as aligned float4 loads, all issued before any use; the b/8
-// lanes of a block reduce with shuffles.  When a0 rides along, the row's
+// a1: grid column x = request; its blocks' warps take 32*SPL-slot chunks of
+// that request in turn (no division per chunk).  A lane takes SPL consecutive
+// slots: their V (SPL/4 float4 loads, or one group maximum, below) and the D
+// window its rows need (offsets p0-i0-(SPL-1) .. p0-i0+R-1) as aligned float4
+// loads, all issued before any use; the b/SPL lanes of a block reduce with
+// shuffles.  A warp's chunk is one round trip to memory, so the slots per
+// lane set the bytes in flight: 16 for max pooling at R <= 2, whose V part is
+// mostly one group maximum, 8 otherwise.  When a0 rides along, the row's
 // first warps quantise that request's (row, head) query vectors first: the
-// kernel is bound by HBM, so they cost next to nothing and the select kernel
-// that follows is spared them.  Block sizes 16..256 (powers of two).
+// kernel is bound by memory, so they cost next to nothing and the select
+// kernel that follows is spared them.  Block sizes 16..256 (powers of two).
 // ---------------------------------------------------------------------------
+template <int R, int P>
+struct PredictShape {
+  static constexpr int SPL = (P == SPIN_POOL_MAX && R <= 2) ? 16 : 8;  // slots per lane
+  static constexpr int CH = 32 * SPL;                                   // slots per warp chunk
+};
+
 template <int R, int P>
 __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
   pdl_enter();
+  constexpr int SPL = PredictShape<R, P>::SPL, CH = PredictShape<R, P>::CH;
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
   const int lb = __ffs(L.b) - 1;
-  const int lpb = L.b >> 3;  // lanes per block
+  const int lpb = L.b >= SPL ? L.b / SPL : 1;  // lanes per block
   const int q = blockIdx.x;
   const int wpr = (int)gridDim.y * (blockDim.x >> 5);                   // warps of this request
   const int wr = (int)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);  // this warp among them
@@ -48,30 +59,44 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
   const int64_t ctx = a.ctx_len[q];
   if (ctx < 1 || ctx + R - 1 > L.max_slots) return;  // block-uniform; select reports it
   const int64_t n_last = row_blocks(ctx, R - 1, L.b);
-  const int nchunks = (int)((n_last * L.b + 255) / 256);
+  const int nchunks = (int)((n_last * L.b + CH - 1) / CH);
   const int64_t p0 = ctx - 1;
   const float* V = a.V + (int64_t)q * L.slot_stride;
   const float* D = a.D + (int64_t)q * L.slot_stride;
-  // the D window of every lane starts at p0 - i0 - 7 with i0 = 0 mod 8: its
-  // offset from a 16-byte boundary is the same for all lanes
+  // Max pooling with V's group maxima kept: a block whose every slot is
+  // visible to every row (j < ctx / b) takes V's part from its 32-slot group
+  // maxima, since the max over the block of max(V_i, D_{p-i}) is the larger
+  // of V's maximum and D's; V itself is read only for the last blocks.
+  const float* VG = (P == SPIN_POOL_MAX && a.vmax) ? a.vmax + (int64_t)q * L.vg_stride : nullptr;
+  const int64_t n_full = ctx >> lb;
+  // the D window of every lane starts at p0 - i0 - (SPL-1) with i0 = 0 mod
+  // SPL: its offset from a 16-byte boundary is the same for all lanes
   const int sh = (int)((p0 + 1) & 3);
-  constexpr int kNV = (R + 7 + 3 + 3) / 4;  // float4 loads covering R + 7 values at any offset
+  constexpr int kW = R + SPL - 1;            // D values a lane's rows need
+  constexpr int kNV = (kW + 3 + 3) / 4;      // float4 loads covering them at any offset
   for (int c = wr; c < nchunks; c += wpr) {
-    const int64_t i0 = (int64_t)c * 256 + lane * 8;
+    const int64_t i0 = (int64_t)c * CH + lane * SPL;
     const int64_t j = i0 >> lb;
     const bool active = j < n_last && i0 <= p0 + R - 1;
-    float vv[8];
-    float dw[R + 7];  // D at offsets p0 - i0 - 7 .. p0 - i0 + R - 1
+    float vv[SPL];
+    float dw[kW];  // D at offsets p0 - i0 - (SPL-1) .. p0 - i0 + R - 1
 #pragma unroll
-    for (int k = 0; k < 8; ++k) vv[k] = __int_as_float(0xff800000);
+    for (int k = 0; k < SPL; ++k) vv[k] = __int_as_float(0xff800000);
 #pragma unroll
-    for (int t = 0; t < R + 7; ++t) dw[t] = __int_as_float(0xff800000);
+    for (int t = 0; t < kW; ++t) dw[t] = __int_as_float(0xff800000);
     if (active) {
-      const float4 v0 = __ldg(reinterpret_cast<const float4*>(V + i0));
-      const float4 v1 = __ldg(reinterpret_cast<const float4*>(V + i0 + 4));
-      vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
-      vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
-      const int64_t ob = p0 - i0 - 7 - sh;  // 16-byte aligned start of the window
+      if (VG && j < n_full) {  // the lane's slots lie in one group of a full block
+        const float g = __ldg(VG + (i0 >> 5));
+#pragma unroll
+        for (int k = 0; k < SPL; ++k) vv[k] = g;
+      } else {
+#pragma unroll
+        for (int u = 0; u < SPL / 4; ++u) {
+          const float4 v4 = __ldg(reinterpret_cast<const float4*>(V + i0) + u);
+          vv[4 * u] = v4.x; vv[4 * u + 1] = v4.y; vv[4 * u + 2] = v4.z; vv[4 * u + 3] = v4.w;
+        }
+      }
+      const int64_t ob = p0 - i0 - (SPL - 1) - sh;  // 16-byte aligned start of the window
       if (ob >= 0 && ob + 4 * kNV <= L.slot_stride) {
         float buf[4 * kNV];
 #pragma unroll
@@ -80,7 +105,7 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
           buf[4 * u] = d4.x; buf[4 * u + 1] = d4.y; buf[4 * u + 2] = d4.z; buf[4 * u + 3] = d4.w;
         }
 #define SPIN_DW_FROM(S)                                       \
-  _Pragma("unroll") for (int t = 0; t < R + 7; ++t) dw[t] = buf[t + (S)];
+  _Pragma("unroll") for (int t = 0; t < kW; ++t) dw[t] = buf[t + (S)];
         switch (sh) {  // warp-uniform
           case 0: SPIN_DW_FROM(0) break;
           case 1: SPIN_DW_FROM(1) break;
@@ -90,32 +115,32 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
 #undef SPIN_DW_FROM
       } else {  // the window reaches below offset 0 (the newest slots) or past the row
 #pragma unroll
-        for (int t = 0; t < R + 7; ++t) {
-          const int64_t di = p0 - i0 - 7 + t;
+        for (int t = 0; t < kW; ++t) {
+          const int64_t di = p0 - i0 - (SPL - 1) + t;
           if (di >= 0) dw[t] = __ldg(D + di);
         }
       }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      // this lane's slots i0 .. i0+7 visible to row r: z = max(V_i, D_{p_r - i}),
-      // slot i0+k at offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + 7]
+      // this lane's slots i0 .. i0+SPL-1 visible to row r: z = max(V_i, D_{p_r - i}),
+      // slot i0+k at offset p_r - (i0+k) = p0 - i0 + r - k  -> dw[r - k + SPL - 1]
       float x;
       if (P == SPIN_POOL_MAX) {
         x = __int_as_float(0xff800000);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (active && i0 + k <= p0 + r) x = fmaxf(x, fmaxf(vv[k], dw[r - k + 7]));
+        for (int k = 0; k < SPL; ++k)
+          if (active && i0 + k <= p0 + r) x = fmaxf(x, fmaxf(vv[k], dw[r - k + SPL - 1]));
         for (int o = lpb >> 1; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
       } else if (P == SPIN_POOL_MEAN) {
-        // the run of 8 slots in slot order, then runs added pairwise (lanes
+        // the run of SPL slots in slot order, then runs added pairwise (lanes
         // l and l^1, then pairs of pairs, ...): the order the reduction fixes
         double sum = 0.0;
         int cnt = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < SPL; ++k)
           if (active && i0 + k <= p0 + r) {
-            sum += (double)fmaxf(vv[k], dw[r - k + 7]);
+            sum += (double)fmaxf(vv[k], dw[r - k + SPL - 1]);
             ++cnt;
           }
         for (int o = 1; o < lpb; o <<= 1) {
@@ -130,9 +155,9 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
                       __int_as_float(0xff800000)};
         int cnt = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < SPL; ++k)
           if (active && i0 + k <= p0 + r) {
-            float z = fmaxf(vv[k], dw[r - k + 7]);
+            float z = fmaxf(vv[k], dw[r - k + SPL - 1]);
             ++cnt;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {  // insert, keeping t descending
@@ -173,7 +198,7 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
 cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   // one wave (4 blocks of 256 threads per SM at <= 64 registers) over all
   // requests, each request's chunks shared by the gx blocks of its column
-  const int64_t chunks = (a.lay.slot_stride + 255) / 256;
+  const int64_t chunks = (a.lay.slot_stride + 255) / 256;  // of the 8-slot-per-lane shape
   int64_t gx = (148 * 4) / a.lay.Q;
   gx = std::min<int64_t>(gx, (chunks + 7) / 8);
   gx = std::max<int64_t>(std::min<int64_t>(gx, 65535), 1);

@@ -20,6 +20,7 @@ struct spin_state_s {
   ErrWord* err;
   float* V;       // [L][Q][slot_stride]
   float* D;
+  float* vmax;    // [L][Q][vg_stride] max of V over each aligned 32-slot group, or null
   float* S;       // [Q][R][blk_stride]
   int32_t* work;  // [Q][blk_stride]
   int32_t* kept;  // [Q]
@@ -110,6 +111,8 @@ Layout make_layout(const spin_config* c) {
   L.max_blocks = (c->max_slots + (int64_t)c->block_size - 1) / c->block_size;
   L.slot_stride = L.max_blocks * c->block_size;
   L.blk_stride = (L.max_blocks + 15) / 16 * 16;
+  // V's 32-slot group maxima: read by the max-pooled prediction in place of V
+  L.vg_stride = (c->block_size >= 32 && c->pooling == SPIN_POOL_MAX) ? L.slot_stride / 32 : 0;
   return L;
 }
 
@@ -117,7 +120,7 @@ Layout make_layout(const spin_config* c) {
 int64_t gmax_stride(const Layout& L) { return L.blk_stride * std::max(1, L.b / 32); }
 
 struct Carve {
-  size_t err, V, D, S, work, kept, q8, wq, scores, gmax, step, la_work, la_kept, la_mask, la_ctx, ctx_next, tk_work,
+  size_t err, V, D, vmax, S, work, kept, q8, wq, scores, gmax, step, la_work, la_kept, la_mask, la_ctx, ctx_next, tk_work,
       tk_kept, tk_ctx, total;
 };
 
@@ -128,6 +131,7 @@ Carve carve(const Layout& L) {
   k.err = take(sizeof(ErrWord));
   k.V = take((size_t)L.L * L.Q * L.slot_stride * 4);
   k.D = take((size_t)L.L * L.Q * L.slot_stride * 4);
+  k.vmax = take((size_t)L.L * L.Q * L.vg_stride * 4);
   k.S = take((size_t)L.Q * L.R * L.blk_stride * 4);
   k.work = take((size_t)L.Q * L.blk_stride * 4);
   k.kept = take((size_t)L.Q * 4);
@@ -158,6 +162,10 @@ spin_status cuda_status(cudaError_t e) {
 
 float beta_of(float alpha) { return (float)(1.0 - (double)alpha); }
 
+float* vmax_of(spin_state st, int layer) {
+  return st->vmax ? st->vmax + (size_t)st->lay.Q * st->lay.vg_stride * layer : nullptr;
+}
+
 StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32_t* ctx_len, uint8_t* mask) {
   StepArgs a;
   a.lay = st->lay;
@@ -183,6 +191,7 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
   a.V = st->V + per_layer * layer;
   a.D = st->D + per_layer * layer;
+  a.vmax = vmax_of(st, layer);
   a.err = st->err;
   a.q = nullptr;
   a.w = nullptr;
@@ -265,6 +274,7 @@ spin_status run_score(spin_state st, int layer, int rows, const void* keys, cons
   const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
   a.V = fuse_ema ? st->V + per_layer * layer : nullptr;
   a.D = fuse_ema ? st->D + per_layer * layer : nullptr;
+  a.vmax = fuse_ema ? vmax_of(st, layer) : nullptr;
   a.alpha = st->cfg.alpha;
   a.beta = beta_of(st->cfg.alpha);
   a.inject = 0;
@@ -407,6 +417,7 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->err = (ErrWord*)(st->base + k.err);
   st->V = (float*)(st->base + k.V);
   st->D = (float*)(st->base + k.D);
+  st->vmax = L.vg_stride ? (float*)(st->base + k.vmax) : nullptr;
   st->S = (float*)(st->base + k.S);
   st->work = (int32_t*)(st->base + k.work);
   st->kept = (int32_t*)(st->base + k.kept);
@@ -442,7 +453,9 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   cudaGetLastError();
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(st->err, 0, sizeof(ErrWord), s);
-  if (e == cudaSuccess) e = launch_init_state(st->V, st->D, (int64_t)L.L * L.Q * L.slot_stride, s);
+  if (e == cudaSuccess)
+    e = launch_init_state(st->V, st->D, (int64_t)L.L * L.Q * L.slot_stride, st->vmax,
+                          (int64_t)L.L * L.Q * L.vg_stride, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(st->step_dev, 0, sizeof(int64_t), s);
   if (e != cudaSuccess) {
     delete st;
@@ -574,7 +587,8 @@ spin_status spin_reset_requests(spin_state st, int layer, const int32_t* req_hos
     for (int i = 0; i < list.n; ++i) list.ids[i] = req_host[i0 + i];
     for (int l = 0; l < st->cfg.num_layers; ++l) {
       if (layer >= 0 && l != layer) continue;
-      cudaError_t e = launch_reset_rows(st->V + per_layer * l, st->D + per_layer * l, list, st->lay.slot_stride, s);
+      cudaError_t e = launch_reset_rows(st->V + per_layer * l, st->D + per_layer * l, vmax_of(st, l), list,
+                                        st->lay.slot_stride, st->lay.vg_stride, s);
       if (e != cudaSuccess) return cuda_status(e);
     }
   }
@@ -644,6 +658,7 @@ spin_status spin_ema_update(spin_state st, int layer, int rows, const float* sco
   const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
   a.V = st->V + per_layer * layer;
   a.D = st->D + per_layer * layer;
+  a.vmax = vmax_of(st, layer);
   a.alpha = st->cfg.alpha;
   a.beta = beta_of(st->cfg.alpha);
   a.err = st->err;
@@ -840,8 +855,23 @@ spin_status spin_state_import(spin_state st, const void* host, size_t bytes, spi
   for (auto& p : st->prep) p.ready = false;
   cudaError_t e = cudaMemcpyAsync(st->V, host, half, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->D, (const char*)host + half, half, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = launch_vmax_refresh(st->V, st->vmax, (int64_t)st->lay.L * st->lay.Q, st->lay.slot_stride, st->lay.vg_stride, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_status(e);
+}
+
+spin_status spin_state_refresh(spin_state st, int layer, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < -1 || layer >= st->cfg.num_layers) return SPIN_EINVAL;
+  for (int l = 0; l < st->cfg.num_layers; ++l)
+    if (layer < 0 || l == layer) st->prep[l].ready = false;  // the state changed under the prepared selection
+  if (!st->vmax) return SPIN_OK;
+  const int64_t layers = layer < 0 ? st->lay.L : 1;
+  const size_t per_layer = (size_t)st->lay.Q * st->lay.slot_stride;
+  const float* V = st->V + per_layer * (layer < 0 ? 0 : layer);
+  return cuda_status(launch_vmax_refresh(V, vmax_of(st, layer < 0 ? 0 : layer), layers * st->lay.Q,
+                                         st->lay.slot_stride, st->lay.vg_stride, (cudaStream_t)stream));
 }
 
 spin_status spin_state_ema(spin_state st, int layer, float** V, float** D, int64_t* stride) {
@@ -851,6 +881,14 @@ spin_status spin_state_ema(spin_state st, int layer, float** V, float** D, int64
   if (V) *V = st->V + per_layer * layer;
   if (D) *D = st->D + per_layer * layer;
   if (stride) *stride = st->lay.slot_stride;
+  return SPIN_OK;
+}
+
+spin_status spin_state_vmax(spin_state st, int layer, const float** vmax, int64_t* stride) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (layer < 0 || layer >= st->cfg.num_layers) return SPIN_EINVAL;
+  if (vmax) *vmax = vmax_of(st, layer);
+  if (stride) *stride = st->lay.vg_stride;
   return SPIN_OK;
 }
 

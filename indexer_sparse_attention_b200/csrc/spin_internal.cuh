@@ -47,6 +47,8 @@ struct Layout {
   int64_t max_blocks;    // ceil(max_slots / b)
   int64_t slot_stride;   // max_blocks * b  (a score / V / D row)
   int64_t blk_stride;    // max_blocks rounded up to 16 (mask, S, work-list rows)
+  int64_t vg_stride;     // slot_stride / 32 (a row of V's 32-slot group maxima), or 0 when
+                         // they are not kept (block size 16, or a pooling other than max)
 };
 
 // ---------------------------------------------------------------------------
@@ -102,6 +104,14 @@ __device__ __forceinline__ uint32_t explore_key(uint64_t seed, uint32_t j, uint3
   uint4 r = philox4x32_10(make_uint4(j, req, layer, (uint32_t)step),
                           make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
   return r.x;
+}
+
+// Maximum of x over the 32 lanes of a warp, all of them active: one
+// redux.sync on sm_100a.  The callers' values are never NaN.
+__device__ __forceinline__ float warp_max(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // EMA update with never-observed sentinels (+inf for V, -inf for D).
@@ -232,6 +242,7 @@ struct StepArgs {
 
   float* V;           // layer base [Q][slot_stride]
   float* D;
+  const float* vmax;  // layer base [Q][vg_stride]: max of V over each aligned 32-slot group, or null
   ErrWord* err;
   // a0 folded into the select kernel (decode step with FP8 keys), or q8 null
   const void* q;      // [Q][rows][H][d]
@@ -241,7 +252,11 @@ struct StepArgs {
   float* wq;
 };
 
-cudaError_t launch_init_state(float* V, float* D, int64_t n, cudaStream_t s);
+// V = +inf, D = -inf over n slots, and vmax (nv groups, or null) = +inf.
+cudaError_t launch_init_state(float* V, float* D, int64_t n, float* vmax, int64_t nv, cudaStream_t s);
+// vmax[g] = max(V[32 g .. 32 g + 31]) for rows rows of V (stride slot_stride) and vmax (stride vg_stride).
+cudaError_t launch_vmax_refresh(const float* V, float* vmax, int64_t rows, int64_t slot_stride, int64_t vg_stride,
+                                cudaStream_t s);
 // Sets (*p = value) or advances (*p += 1) the device step counter.
 cudaError_t launch_step_op(int64_t* p, bool set, int64_t value, cudaStream_t s);
 struct ReqList {
@@ -249,7 +264,8 @@ struct ReqList {
   int32_t ids[kMax];
   int n;
 };
-cudaError_t launch_reset_rows(float* V, float* D, const ReqList& list, int64_t stride, cudaStream_t s);
+cudaError_t launch_reset_rows(float* V, float* D, float* vmax, const ReqList& list, int64_t stride,
+                              int64_t vg_stride, cudaStream_t s);
 cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s);
 cudaError_t launch_select(const StepArgs& a, cudaStream_t s);
 cudaError_t launch_compact(const Layout& L, int rows, const int32_t* ctx_len, const uint8_t* mask,
@@ -278,6 +294,7 @@ struct ScoreArgs {
   // fused EMA (rows == 1 only): V, D of the layer, or null
   float* V;
   float* D;
+  float* vmax;         // with V: V's 32-slot group maxima of the layer, kept current, or null
   float alpha, beta;   // beta = fl32(1 - alpha), computed once on the host
   int inject;          // test hook: withhold the first key stage of CTA 0
   const int32_t* ctx_sel;  // [Q] or null: the ctx_len the selection was made for; a request whose
@@ -318,6 +335,7 @@ struct EmaArgs {
   const int32_t* accepted;
   float* V;
   float* D;
+  float* vmax;        // V's 32-slot group maxima of the layer, kept current, or null
   float alpha, beta;
   ErrWord* err;
 };

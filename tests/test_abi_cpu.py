@@ -48,12 +48,13 @@ def _cfg(**over):
     return isa.make_config(**base)
 
 
-def _expected_bytes(L, Q, R, H, d, b, max_slots):
+def _expected_bytes(L, Q, R, H, d, b, max_slots, pooling=0):
     a = lambda x: (x + 255) // 256 * 256
     mb = -(-max_slots // b)
     slot = mb * b
     blk = -(-mb // 16) * 16
-    parts = [16, L * Q * slot * 4, L * Q * slot * 4, Q * R * blk * 4, Q * blk * 4, Q * 4, Q * R * H * d,
+    vg = slot // 32 if (b >= 32 and pooling == isa.SPIN_POOL_MAX) else 0  # V's 32-slot group maxima
+    parts = [16, L * Q * slot * 4, L * Q * slot * 4, L * Q * vg * 4, Q * R * blk * 4, Q * blk * 4, Q * 4, Q * R * H * d,
              Q * R * H * 4, Q * R * slot * 4, Q * R * blk * max(1, b // 32) * 4, 8,
              # the selection a pipelined step prepares for the next one, per layer, and ctx_len + 1
              L * Q * blk * 4, L * Q * 4, L * Q * mb, L * Q * 4, Q * 4,
@@ -64,12 +65,14 @@ def _expected_bytes(L, Q, R, H, d, b, max_slots):
 @pytest.mark.parametrize("over", [{}, {"max_rows": 4, "num_requests": 32, "max_slots": 131072 + 128},
                                   {"num_layers": 8, "num_requests": 8, "max_slots": 1048576 + 64},
                                   {"key_fp8": False, "q_bf16": False, "num_heads": 8, "head_dim": 64,
-                                   "num_requests": 1, "max_slots": 4096 + 32, "topk": 256}])
+                                   "num_requests": 1, "max_slots": 4096 + 32, "topk": 256},
+                                  {"block_size": 16, "max_slots": 4096 + 16}, {"block_size": 32},
+                                  {"pooling": 1}, {"pooling": 2, "block_size": 256}])
 def test_state_bytes_matches_documented_layout(lib, over):
     cfg = _cfg(**over)
     got = isa.spin_state_bytes(cfg)
     exp = _expected_bytes(cfg.num_layers, cfg.num_requests, cfg.max_rows, cfg.num_heads, cfg.head_dim,
-                          cfg.block_size, cfg.max_slots)
+                          cfg.block_size, cfg.max_slots, cfg.pooling)
     assert got == exp
 
 

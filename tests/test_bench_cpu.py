@@ -8,12 +8,16 @@ import workloads
 
 
 def test_step_traffic_closed_form():
-    # 96 requests at 512K and 50%: 8 B per context slot + 152 B per kept slot
+    # 96 requests at 512K and 50%.  Max pooling: the predict kernel reads D
+    # and one V maximum per 32 slots (4.125 B per context slot); the score
+    # kernel moves 152 B per kept slot plus one V maximum per 32 kept slots.
     ctx, kept = 96 * 524_292, 25_170_000
     t = bench.step_traffic(ctx, kept, 0.8, 6546.6)
-    assert t["bytes_per_step"] == 8 * ctx + 152 * kept
+    assert t["bytes_per_step"] == 4.125 * ctx + 152.125 * kept
     assert abs(t["gbs"] - t["bytes_per_step"] / 0.8e-3 / 1e9) < 1e-9
     assert abs(t["frac"] - t["gbs"] / 6546.6) < 1e-12
+    # other poolings read V and D whole: 8 B per context slot
+    assert bench.step_traffic(ctx, kept, 0.8, 6546.6, "mean")["bytes_per_step"] == 8 * ctx + 152 * kept
 
 
 def test_both_arms_print_the_same_config():

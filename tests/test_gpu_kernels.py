@@ -42,6 +42,7 @@ def random_state(st, layer, rng, frac_sentinel=0.1):
     v = np.round(v / 4) * 4
     V.copy_(torch.from_numpy(v))
     D.copy_(torch.from_numpy(dd))
+    st.refresh()  # V and D were written through the views
     torch.cuda.synchronize()
 
 
@@ -82,6 +83,7 @@ def test_select_large_request_with_infinite_and_tied_scores(g):
     v[:, -5000:] = np.inf
     V.copy_(torch.from_numpy(v))
     D.fill_(-np.inf)
+    st.refresh()  # V and D were written through the views
     ctx = np.array([1024 * 1024 + 1, 300000], np.int64)
     ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
     mask = st.new_mask()
@@ -375,6 +377,7 @@ def test_select_cluster_paths_bit_exact(R, s, g):
     d = rng.standard_normal(D.shape).astype(np.float32)
     d[rng.random(D.shape) < 0.5] = -np.inf
     D.copy_(torch.from_numpy(d))
+    st.refresh()  # V and D were written through the views
     ctx = np.array([1, 1024 * 1024 - R + 1, 300_000 + 37, 64 * 5000], np.int64)
     ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
     mask = st.new_mask()
@@ -402,6 +405,7 @@ def test_mtp_row0_select_bit_exact(R, max_slots):
     d = rng.standard_normal(D.shape).astype(np.float32)
     d[rng.random(D.shape) < 0.5] = -np.inf
     D.copy_(torch.from_numpy(d))
+    st.refresh()  # V and D were written through the views
     top = max_slots - 64 - R + 1
     ctx = np.array([1, top, top // 3 + 37, 64 * (top // 200)], np.int64)
     ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
@@ -441,6 +445,7 @@ def test_pooling_variants_vs_exact_mean(pooling, R, b, spread):
     d = (rng.standard_normal(D.shape) * scale).astype(np.float32)
     d[rng.random(D.shape) < 0.3] = -np.inf
     D.copy_(torch.from_numpy(d))
+    st.refresh()  # V and D were written through the views
     ctx = np.array([1, 37 * b + 5, max_slots - R + 1], np.int64)
     ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
     mask = st.new_mask()

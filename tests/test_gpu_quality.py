@@ -38,6 +38,7 @@ def test_slot_predictions_bit_exact(R):
     d = (rng.standard_normal(D.shape) * 5).astype(np.float32)
     d[rng.random(D.shape) < 0.3] = -np.inf
     D.copy_(torch.from_numpy(d))
+    st.refresh()  # V and D were written through the views
     ctx = np.array([1, 64 * 137 + 29, max_slots - R + 1], np.int64)
     ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
     stride = st.score_stride
@@ -122,6 +123,7 @@ def test_predictor_topk_and_recall_end_to_end():
     v[:, 40_000:] = np.inf
     V.copy_(torch.from_numpy(v))
     D.copy_(torch.from_numpy(rng.standard_normal(D.shape).astype(np.float32)))
+    st.refresh()  # V and D were written through the views
     ctx = np.array([64 * 700 + 5, 30_001], np.int64)
     ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
     scores = st.new_scores()
