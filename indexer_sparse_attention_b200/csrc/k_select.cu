@@ -23,28 +23,21 @@
 namespace spin {
 
 // ---------------------------------------------------------------------------
-// a1: grid column x = request; its blocks' warps take 32*SPL-slot chunks of
-// that request in turn (no division per chunk).  A lane takes SPL consecutive
-// slots: their V (SPL/4 float4 loads, or one group maximum, below) and the D
-// window its rows need (offsets p0-i0-(SPL-1) .. p0-i0+R-1) as aligned float4
-// loads, all issued before any use; the b/SPL lanes of a block reduce with
-// shuffles.  A warp's chunk is one round trip to memory, so the slots per
-// lane set the bytes in flight: 16 for max pooling at R <= 2, whose V part is
-// mostly one group maximum, 8 otherwise.  When a0 rides along, the row's
-// first warps quantise that request's (row, head) query vectors first: the
-// kernel is bound by memory, so they cost next to nothing and the select
-// kernel that follows is spared them.  Block sizes 16..256 (powers of two).
+// a1 for Mean and Top-4 pooling, and for max pooling at block size 16 (no
+// group maxima): grid column x = request; its blocks' warps take 256-slot
+// chunks of that request in turn (no division per chunk).  A lane takes
+// SPL = 8 consecutive slots: two float4 loads of V and the D window its rows
+// need (offsets p0-i0-7 .. p0-i0+R-1) as aligned float4 loads, all issued
+// before any use; the b/8 lanes of a block reduce with shuffles.  When a0
+// rides along, the row's first warps quantise that request's (row, head)
+// query vectors first: the kernel is bound by memory, so they cost next to
+// nothing and the select kernel that follows is spared them.  Block sizes
+// 16..256 (powers of two).
 // ---------------------------------------------------------------------------
-template <int R, int P>
-struct PredictShape {
-  static constexpr int SPL = (P == SPIN_POOL_MAX && R <= 2) ? 16 : 8;  // slots per lane
-  static constexpr int CH = 32 * SPL;                                   // slots per warp chunk
-};
-
 template <int R, int P>
 __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
   pdl_enter();
-  constexpr int SPL = PredictShape<R, P>::SPL, CH = PredictShape<R, P>::CH;
+  constexpr int SPL = 8, CH = 32 * SPL;
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
   const int lb = __ffs(L.b) - 1;
@@ -63,12 +56,6 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
   const int64_t p0 = ctx - 1;
   const float* V = a.V + (int64_t)q * L.slot_stride;
   const float* D = a.D + (int64_t)q * L.slot_stride;
-  // Max pooling with V's group maxima kept: a block whose every slot is
-  // visible to every row (j < ctx / b) takes V's part from its 32-slot group
-  // maxima, since the max over the block of max(V_i, D_{p-i}) is the larger
-  // of V's maximum and D's; V itself is read only for the last blocks.
-  const float* VG = (P == SPIN_POOL_MAX && a.vmax) ? a.vmax + (int64_t)q * L.vg_stride : nullptr;
-  const int64_t n_full = ctx >> lb;
   // the D window of every lane starts at p0 - i0 - (SPL-1) with i0 = 0 mod
   // SPL: its offset from a 16-byte boundary is the same for all lanes
   const int sh = (int)((p0 + 1) & 3);
@@ -85,16 +72,10 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
 #pragma unroll
     for (int t = 0; t < kW; ++t) dw[t] = __int_as_float(0xff800000);
     if (active) {
-      if (VG && j < n_full) {  // the lane's slots lie in one group of a full block
-        const float g = __ldg(VG + (i0 >> 5));
 #pragma unroll
-        for (int k = 0; k < SPL; ++k) vv[k] = g;
-      } else {
-#pragma unroll
-        for (int u = 0; u < SPL / 4; ++u) {
-          const float4 v4 = __ldg(reinterpret_cast<const float4*>(V + i0) + u);
-          vv[4 * u] = v4.x; vv[4 * u + 1] = v4.y; vv[4 * u + 2] = v4.z; vv[4 * u + 3] = v4.w;
-        }
+      for (int u = 0; u < SPL / 4; ++u) {
+        const float4 v4 = __ldg(reinterpret_cast<const float4*>(V + i0) + u);
+        vv[4 * u] = v4.x; vv[4 * u + 1] = v4.y; vv[4 * u + 2] = v4.z; vv[4 * u + 3] = v4.w;
       }
       const int64_t ob = p0 - i0 - (SPL - 1) - sh;  // 16-byte aligned start of the window
       if (ob >= 0 && ob + 4 * kNV <= L.slot_stride) {
@@ -195,16 +176,250 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// a1 for one row (R = 1), max pooling, V's group maxima kept, block size
+// B in {32, 64, 128, 256}: every load is coalesced.  A warp takes 1,024
+// slots, NB = 1024 / B blocks J0 .. J0+NB-1.  In offset space (delta = p0 - i)
+// those blocks are one run of 1,024 offsets, and block J0+NB-1-s is its s-th
+// run of B offsets.  The warp loads the run as eight float4 per lane from a
+// 16-byte boundary (the run starts sh = (p0 + 1) mod 4 past it) plus one
+// float4 past its end: every load instruction reads 512 contiguous bytes.
+// A lane's float4 f holds run positions 4f - sh .. 4f + 3 - sh; its last
+// 4 - sh values and the first sh values of float4 f + 1 (one shuffle down)
+// are run positions 4f .. 4f + 3, all in run block floor(4f / B), so the B/4
+// lanes of a block reduce with xor shuffles and no value crosses a block
+// edge.  V's part: one group maximum per lane (32 groups per chunk, one
+// coalesced load), the group of the newest slot read from V itself; a
+// block's groups reduce with shuffles.  Lanes 0 .. NB-1 store the chunk's
+// block scores, one coalesced store.
+// ---------------------------------------------------------------------------
+template <int B>
+__global__ void __launch_bounds__(256, 4) k_predict_max_r1(StepArgs a) {
+  pdl_enter();
+  constexpr int NB = 1024 / B;                 // blocks per chunk
+  constexpr int LPS = B / 4 < 32 ? B / 4 : 32;  // lanes of a block's run in one load instruction
+  constexpr int IPB = B / 4 > 32 ? B / 128 : 1;  // load instructions per block (B = 256: 2)
+  constexpr int SPI = 32 / LPS;                // blocks per load instruction
+  constexpr int GPB = B / 32;                  // V groups per block
+  const Layout L = a.lay;
+  const int lane = threadIdx.x & 31;
+  const int q = blockIdx.x;
+  const int wpr = (int)gridDim.y * (blockDim.x >> 5);
+  const int wr = (int)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (a.q8) {
+    const int nv = a.rows * L.H;
+    for (int v = wr; v < nv; v += wpr) quantize_vec(a.q, a.w, a.q_bf16, L.d, (int64_t)q * nv + v, a.q8, a.wq);
+  }
+  const int64_t ctx = a.ctx_len[q];
+  if (ctx < 1 || ctx > L.max_slots) return;  // block-uniform; select reports it
+  const int64_t n_last = (ctx + B - 1) / B;
+  const int nchunks = (int)((n_last + NB - 1) / NB);
+  const int64_t p0 = ctx - 1;
+  const float* V = a.V + (int64_t)q * L.slot_stride;
+  const float* D = a.D + (int64_t)q * L.slot_stride;
+  const float* VG = a.vmax + (int64_t)q * L.vg_stride;
+  const int sh = (int)((p0 + 1) & 3);
+  const float kNeg = __int_as_float(0xff800000);
+  for (int c = wr; c < nchunks; c += wpr) {
+    const int64_t J0 = (int64_t)c * NB;
+    const int64_t A = p0 + 1 - (J0 + NB) * B - sh;  // 16-byte boundary at or below the run's start
+    float4 x[9];
+#pragma unroll
+    for (int u = 0; u < 9; ++u) {
+      const int64_t o = A + 128 * u + 4 * lane;  // a float4 lies wholly inside or outside [0, stride)
+      x[u] = make_float4(kNeg, kNeg, kNeg, kNeg);
+      if ((u < 8 || lane == 0) && o >= 0 && o < L.slot_stride) x[u] = __ldg(reinterpret_cast<const float4*>(D + o));
+    }
+    // V's part: lane = group g0 + lane of the chunk; groups past the newest
+    // slot see nothing, and the newest slot's group gp is read from V itself
+    // (the whole warp: one coalesced load of its visible values)
+    const int64_t g0 = (J0 * B) >> 5, g = g0 + lane, gp = p0 >> 5;
+    float vg = kNeg;
+    if (g < gp) vg = __ldg(VG + g);
+    if (gp >= g0 && gp < g0 + 32) {  // warp-uniform
+      const int64_t i = 32 * gp + lane;
+      const float m = warp_max(i <= p0 ? __ldg(V + i) : kNeg);
+      if (g == gp) vg = m;
+    }
+    // run-aligned float4 maxima: hi = values e >= sh of x[u], lo = values e < sh
+    float hi[9], lo[9];
+#pragma unroll
+    for (int u = 0; u < 9; ++u) {
+      const float e[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+      float h = kNeg, l = kNeg;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k >= sh) h = fmaxf(h, e[k]);
+        else l = fmaxf(l, e[k]);
+      }
+      hi[u] = h;
+      lo[u] = l;
+    }
+    float seg[8];  // block maxima of D per load instruction (each lane of a block's lanes)
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float nxt = __shfl_down_sync(0xffffffffu, lo[u], 1);
+      const float wrap = __shfl_sync(0xffffffffu, lo[u + 1], 0);  // lane 31: the next instruction's lane 0
+      if (lane == 31) nxt = wrap;
+      float m = fmaxf(hi[u], nxt);
+#pragma unroll
+      for (int o = LPS >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      seg[u] = m;
+    }
+    // lane k < NB gathers block J0 + k, run block s = NB - 1 - k
+    const int k = lane;
+    const int s = NB - 1 - k;
+    float res = kNeg;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int src = IPB == 1 ? ((s & (SPI - 1)) * LPS) & 31 : 0;
+      const float v = __shfl_sync(0xffffffffu, seg[u], src);
+      const bool mine = IPB == 1 ? (u == s / SPI) : (u / IPB == s);
+      if (k < NB && mine) res = fmaxf(res, v);
+    }
+#pragma unroll
+    for (int o = GPB >> 1; o >= 1; o >>= 1) vg = fmaxf(vg, __shfl_xor_sync(0xffffffffu, vg, o));
+    const float vb = __shfl_sync(0xffffffffu, vg, (k * GPB) & 31);
+    if (k < NB && J0 + k < n_last) a.S[(int64_t)q * L.R * L.blk_stride + J0 + k] = fmaxf(res, vb);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a1 for max pooling with V's 32-slot group maxima kept (block size >= 32).
+// The max over a block of max(V_i, D_{p_r-i}) is the larger of V's maximum
+// and D's, so a lane takes one aligned group of 32 slots i0 .. i0+31:
+//   V's part: the group's maximum when the whole group is visible (i0 + 31
+//     <= p0), else -- only in the group of the newest slots -- the max of
+//     its visible V values, read directly;
+//   D's part: row r needs offsets p_r - i0 - 31 .. p_r - i0, so the rows
+//     share one window of 31 + R values of D, loaded as aligned float4 (its
+//     offset from a 16-byte boundary is the same for every lane) and reduced
+//     once over the part all rows share.
+// A warp's chunk is 1,024 slots: 4.1 B of memory per slot (D and one group
+// maximum) in 10 loads per lane, one round trip.  The b/32 lanes of a block
+// reduce with shuffles.  a0 rides along as in k_predict_pool.
+// ---------------------------------------------------------------------------
+// Row maxima of D from the window buf[S .. S + 30 + R]: row r takes
+// buf[S + r .. S + r + 31].
+template <int S, int R>
+__device__ __forceinline__ void d_row_max(const float* buf, float* dmax) {
+  float common = buf[S + R - 1];
+#pragma unroll
+  for (int t = S + R; t <= S + 31; ++t) common = fmaxf(common, buf[t]);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float x = common;
+#pragma unroll
+    for (int t = S + r; t < S + R - 1; ++t) x = fmaxf(x, buf[t]);    // head only row r sees
+#pragma unroll
+    for (int t = S + 32; t <= S + 31 + r; ++t) x = fmaxf(x, buf[t]);  // tail only row r sees
+    dmax[r] = x;
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(256, 4) k_predict_max(StepArgs a) {
+  pdl_enter();
+  const Layout L = a.lay;
+  const int lane = threadIdx.x & 31;
+  const int lb = __ffs(L.b) - 1;
+  const int lpb = L.b >> 5;  // lanes per block
+  const int q = blockIdx.x;
+  const int wpr = (int)gridDim.y * (blockDim.x >> 5);
+  const int wr = (int)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (a.q8) {
+    const int nv = a.rows * L.H;
+    for (int v = wr; v < nv; v += wpr) quantize_vec(a.q, a.w, a.q_bf16, L.d, (int64_t)q * nv + v, a.q8, a.wq);
+  }
+  const int64_t ctx = a.ctx_len[q];
+  if (ctx < 1 || ctx + R - 1 > L.max_slots) return;  // block-uniform; select reports it
+  const int64_t n_last = row_blocks(ctx, R - 1, L.b);
+  const int nchunks = (int)((n_last * L.b + 1023) / 1024);
+  const int64_t p0 = ctx - 1;
+  const float* V = a.V + (int64_t)q * L.slot_stride;
+  const float* D = a.D + (int64_t)q * L.slot_stride;
+  const float* VG = a.vmax + (int64_t)q * L.vg_stride;
+  const int sh = (int)((p0 + 1) & 3);       // (p0 - i0 - 31) mod 4, the same for every lane
+  constexpr int kNV = (31 + R + 3 + 3) / 4;  // float4 loads covering 31 + R values at any offset
+  for (int c = wr; c < nchunks; c += wpr) {
+    const int64_t i0 = (int64_t)c * 1024 + lane * 32;
+    const int64_t j = i0 >> lb;
+    const bool active = j < n_last && i0 <= p0 + R - 1;
+    float x[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) x[r] = __int_as_float(0xff800000);
+    if (active) {
+      const bool whole = i0 + 31 <= p0;
+      const float g = whole ? __ldg(VG + (i0 >> 5)) : __int_as_float(0xff800000);
+      float buf[4 * kNV];  // D at offsets ob .. ob + 4 kNV - 1
+      const int64_t ob = p0 - i0 - 31 - sh;
+      if (ob >= 0 && ob + 4 * kNV <= L.slot_stride) {
+#pragma unroll
+        for (int u = 0; u < kNV; ++u) {
+          const float4 d4 = __ldg(reinterpret_cast<const float4*>(D + ob) + u);
+          buf[4 * u] = d4.x; buf[4 * u + 1] = d4.y; buf[4 * u + 2] = d4.z; buf[4 * u + 3] = d4.w;
+        }
+      } else {  // the newest slots (offsets below 0 are past the row) or the end of the row
+#pragma unroll
+        for (int t = 0; t < 4 * kNV; ++t) {
+          const int64_t di = ob + t;
+          buf[t] = (di >= 0 && di < L.slot_stride) ? __ldg(D + di) : __int_as_float(0xff800000);
+        }
+      }
+      float dmax[R];
+      switch (sh) {  // warp-uniform
+        case 0: d_row_max<0, R>(buf, dmax); break;
+        case 1: d_row_max<1, R>(buf, dmax); break;
+        case 2: d_row_max<2, R>(buf, dmax); break;
+        default: d_row_max<3, R>(buf, dmax); break;
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) x[r] = fmaxf(g, dmax[r]);
+      if (!whole) {  // the group of the newest slots: V's visible values
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 v4 = __ldg(reinterpret_cast<const float4*>(V + i0) + u);
+          const float vals[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+              if (i0 + 4 * u + e <= p0 + r) x[r] = fmaxf(x[r], vals[e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float y = x[r];
+      for (int o = lpb >> 1; o >= 1; o >>= 1) y = fmaxf(y, __shfl_xor_sync(0xffffffffu, y, o));
+      if (active && (lane & (lpb - 1)) == 0 && j < row_blocks(ctx, r, L.b))
+        a.S[((int64_t)q * L.R + r) * L.blk_stride + j] = y;
+    }
+  }
+}
+
 cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   // one wave (4 blocks of 256 threads per SM at <= 64 registers) over all
   // requests, each request's chunks shared by the gx blocks of its column
-  const int64_t chunks = (a.lay.slot_stride + 255) / 256;  // of the 8-slot-per-lane shape
+  const int64_t chunks = (a.lay.slot_stride + 255) / 256;
   int64_t gx = (148 * 4) / a.lay.Q;
   gx = std::min<int64_t>(gx, (chunks + 7) / 8);
   gx = std::max<int64_t>(std::min<int64_t>(gx, 65535), 1);
   PdlLaunch l(dim3((unsigned)a.lay.Q, (unsigned)gx), dim3(256), 0, s);
   l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
   void (*k)(StepArgs) = nullptr;
+  if (a.pooling == SPIN_POOL_MAX && a.vmax) {  // V's group maxima kept (block size >= 32)
+    switch (a.mtp_row0 ? 1 : a.rows) {
+      case 1:
+        k = a.lay.b == 32 ? k_predict_max_r1<32> : a.lay.b == 64 ? k_predict_max_r1<64>
+          : a.lay.b == 128 ? k_predict_max_r1<128> : k_predict_max_r1<256>;
+        break;
+      case 2: k = k_predict_max<2>; break;
+      case 3: k = k_predict_max<3>; break;
+      default: k = k_predict_max<4>;
+    }
+    return cudaLaunchKernelEx(&l.cfg, k, a);
+  }
 #define SPIN_PREDICT_CASE(R)                                            \
   case R:                                                               \
     k = a.pooling == SPIN_POOL_MEAN   ? k_predict_pool<R, SPIN_POOL_MEAN> \

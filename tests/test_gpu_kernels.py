@@ -70,6 +70,35 @@ def test_predict_select_bit_exact(R, s, g):
             assert np.array_equal(mask[q].cpu().numpy(), m_ref), (q, step)
 
 
+@pytest.mark.parametrize("R", [1, 2, 3, 4])
+@pytest.mark.parametrize("b", [16, 32, 128, 256])
+def test_max_pooling_block_sizes_bit_exact(R, b):
+    """Max pooling at every block size: b = 16 keeps no group maxima (V is
+    read slot by slot), b >= 32 takes V's part from the 32-slot group maxima
+    except in the group of the newest slots.  Contexts end on, just before
+    and just after 32-slot and block boundaries; the block scores and the
+    mask equal the oracle's bit for bit."""
+    rng = np.random.default_rng(R * 31 + b)
+    max_slots = 300 * b + 64
+    st = make_state(Q=6, max_slots=max_slots, R=R, H=16, s=0.5, g=0.1, b=b)  # H: a valid config at b = 256
+    random_state(st, 0, rng)
+    top = max_slots - R + 1
+    ctx = np.array([1, 31, 32 * 7 + 1, b * 40, b * 97 + 33, top], np.int64)
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    isa.spin_predict_select(st, 0, R, 4, ctx_t, mask)
+    assert isa.spin_get_error(st)[0] == 0
+    V, D = st.ema(0)
+    S_gpu = st.block_scores().cpu().numpy()
+    for q in range(len(ctx)):
+        S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, b, st.mask_stride)
+        for r in range(R):
+            n = oracle.num_blocks(int(ctx[q]), r, b)
+            assert np.array_equal(S_gpu[q, r, :n].view(np.uint32), S_ref[r, :n].view(np.uint32)), (q, r)
+        m_ref = oracle.select(S_ref, int(ctx[q]), R, b, 0.5, 0.1, 7, q, 0, 4)
+        assert np.array_equal(mask[q].cpu().numpy(), m_ref), q
+
+
 @pytest.mark.parametrize("g", [0.1, 0.3])
 def test_select_large_request_with_infinite_and_tied_scores(g):
     # one 1M-slot request: 16,385 blocks, many equal block scores.  The
