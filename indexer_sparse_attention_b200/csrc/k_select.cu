@@ -408,12 +408,19 @@ cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   PdlLaunch l(dim3((unsigned)a.lay.Q, (unsigned)gx), dim3(256), 0, s);
   l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
   void (*k)(StepArgs) = nullptr;
+  if (a.pooling == SPIN_POOL_MAX && a.vmax && (a.mtp_row0 || a.rows == 1)) {
+    // one 1,024-slot chunk per warp, many short blocks: the hardware hands
+    // them to SMs as they free up, so the kernel also fills the SMs another
+    // stream's kernel leaves idle
+    const int64_t cy = (a.lay.slot_stride + 8 * 1024 - 1) / (8 * 1024);
+    PdlLaunch m(dim3((unsigned)a.lay.Q, (unsigned)std::min<int64_t>(cy, 65535)), dim3(256), 0, s);
+    m.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
+    k = a.lay.b == 32 ? k_predict_max_r1<32> : a.lay.b == 64 ? k_predict_max_r1<64>
+      : a.lay.b == 128 ? k_predict_max_r1<128> : k_predict_max_r1<256>;
+    return cudaLaunchKernelEx(&m.cfg, k, a);
+  }
   if (a.pooling == SPIN_POOL_MAX && a.vmax) {  // V's group maxima kept (block size >= 32)
-    switch (a.mtp_row0 ? 1 : a.rows) {
-      case 1:
-        k = a.lay.b == 32 ? k_predict_max_r1<32> : a.lay.b == 64 ? k_predict_max_r1<64>
-          : a.lay.b == 128 ? k_predict_max_r1<128> : k_predict_max_r1<256>;
-        break;
+    switch (a.rows) {
       case 2: k = k_predict_max<2>; break;
       case 3: k = k_predict_max<3>; break;
       default: k = k_predict_max<4>;

@@ -45,7 +45,7 @@ struct spin_state_s {
   // a second stream beside the next step's predict kernel.
   int lookahead;
   cudaStream_t side;                 // this step's top-k runs here (created on first use)
-  cudaEvent_t ev_scored, ev_pred, ev_copied, ev_topk;  // see decode_step_lookahead
+  cudaEvent_t ev_scored, ev_copied, ev_topk;  // see decode_step_lookahead
   struct Prepared {
     bool ready;
     int64_t step;                    // the step the selection is for (SPIN_STEP_DEVICE: the counter's)
@@ -305,15 +305,16 @@ spin_status check_rows(spin_state st, int rows) {
 // The pipelined one-row decode step (spin_set_lookahead).  The step's
 // selection was prepared by the previous step of this layer (or is made here
 // when there is none, or it was made for another step or target):
-//   stream:  a0 -> score + fused EMA (writes ctx_len + 1) -> predict(next) ----> select(next) -> [join]
-//   side:                                  [fork] -> copy selection, mask ---^ -> top-k --------^
+//   stream:  a0 -> score + fused EMA (writes ctx_len + 1) -> predict(next) -------> select(next) -> [join]
+//   side:                                  [fork] -> copy selection, mask -> top-k ---^ ------------^
 // The next step's predict reads only V and D, which the score kernel has
-// finished, and has the GPU to itself; then this step's top-k and the next
-// step's select, both latency-bound with one CTA per request, run side by
-// side.  The top-k reads a copy of the kept lists, taken while the predict
-// runs, because the next select overwrites them.  Results are those of the
-// sequential step: the next selection is computed from the same state,
-// positions (ctx_len + 1) and step number as the next call would compute it.
+// finished; its many short blocks take the SMs the top-k (one CTA per
+// request) leaves idle, and the next select follows once the kept lists are
+// copied.  The top-k reads that copy, because the next select overwrites
+// them.  Results are those of the sequential step: the next selection is
+// computed from the same state, positions (ctx_len + 1) and step number as
+// the next call would compute it.  The step's query quantisation (a0) cannot
+// ride in the predict here, which runs a step ahead: it is a launch of its own.
 spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const void* keys, const float* key_scale,
                                   int32_t num_pages, const int32_t* block_table, int32_t bt_stride, const void* q,
                                   const float* w, const int32_t* ctx_len, uint8_t* mask_dev, int32_t* topk_dev,
@@ -363,20 +364,17 @@ spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const 
     e = cudaMemcpyAsync(mask_dev, lmask, (size_t)L.Q * L.max_blocks, cudaMemcpyDeviceToDevice, st->side);
   if (e == cudaSuccess) e = cudaEventRecord(st->ev_copied, st->side);
   if (e != cudaSuccess) return cuda_status(e);
-  // the next step's predict, alone on the GPU
+  // this step's top-k on the side stream; the next step's predict fills the
+  // SMs the top-k leaves idle, then the next select runs
+  TopkArgs t{L, 1, scores, mask_dev, ctx_len, st->tk_work, st->tk_kept, topk_dev, st->err, gm ? st->gmax : nullptr,
+             st->gstride, st->tk_ctx};
+  r = cuda_status(staged(st, kTopk, st->side, [&] { return launch_topk(t, st->side); }));
+  if (r != SPIN_OK) return r;
   StepArgs a = select_args(st->ctx_next, next, true);
   if (sp > 0.0f) {
     r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
     if (r != SPIN_OK) return r;
   }
-  e = cudaEventRecord(st->ev_pred, s);
-  // this step's top-k, once the predict is done, beside the next select
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->side, st->ev_pred, 0);
-  if (e != cudaSuccess) return cuda_status(e);
-  TopkArgs t{L, 1, scores, mask_dev, ctx_len, st->tk_work, st->tk_kept, topk_dev, st->err, gm ? st->gmax : nullptr,
-             st->gstride, st->tk_ctx};
-  r = cuda_status(staged(st, kTopk, st->side, [&] { return launch_topk(t, st->side); }));
-  if (r != SPIN_OK) return r;
   e = cudaEventRecord(st->ev_topk, st->side);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->ev_copied, 0);  // the kept lists are copied
   if (e != cudaSuccess) return cuda_status(e);
@@ -437,7 +435,7 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->tk_ctx = (int32_t*)(st->base + k.tk_ctx);
   st->lookahead = 0;
   st->side = nullptr;
-  st->ev_scored = st->ev_pred = st->ev_copied = st->ev_topk = nullptr;
+  st->ev_scored = st->ev_copied = st->ev_topk = nullptr;
   st->prep.assign(cfg->num_layers, spin_state_s::Prepared{false, 0, 0.0f});
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
@@ -473,7 +471,7 @@ spin_status spin_state_destroy(spin_state st) {
     cudaEventDestroy(r.b);
   }
   for (auto e : st->pool) cudaEventDestroy(e);
-  for (cudaEvent_t e : {st->ev_scored, st->ev_pred, st->ev_copied, st->ev_topk})
+  for (cudaEvent_t e : {st->ev_scored, st->ev_copied, st->ev_topk})
     if (e) cudaEventDestroy(e);
   if (st->side) cudaStreamDestroy(st->side);
   st->magic = 0;
@@ -506,7 +504,6 @@ spin_status spin_set_lookahead(spin_state st, int enable) {
   if (enable && !st->side) {
     cudaError_t e = cudaStreamCreateWithFlags(&st->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_scored, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_pred, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_copied, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_topk, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_status(e);
