@@ -558,9 +558,8 @@ __device__ void draw_from_list(const uint2* list, int cnt, int take, int* scratc
 // Exploration draw by a short list: the Philox keys are uniform, so the
 // `take` smallest of n_cand lie below t = (1.25 take + 64) / n_cand * 2^32
 // with overwhelming probability.  Candidates under t are appended to a
-// shared list (one atomic per warp), each entry is ranked by (key, block
-// index) -- by counting for short lists, by a bitonic sort for long ones --
-// and the first `take` blocks are explored.  Returns false -- nothing marked -- when the list holds fewer
+// shared list (one atomic per warp), and a radix select over the list takes
+// its `take` smallest (key, block index) pairs.  Returns false -- nothing marked -- when the list holds fewer
 // than `take` entries or overflows, and the caller runs the radix select.
 
 __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last, int take, int n_cand,
@@ -570,20 +569,30 @@ __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last
   if (threadIdx.x == 0) sh.digit[0] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  for (int j0 = 0; j0 < n_last; j0 += blockDim.x) {  // warp-uniform trip count
-    const int j = j0 + (int)threadIdx.x;
-    uint32_t u = 0;
-    bool in = false;
-    if (j < n_last && m[j] == 0) {
-      u = explore_key(a.seed, (uint32_t)j, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
-      in = (uint64_t)u < t;
+  // a thread takes blocks 4i .. 4i+3: one Philox gives their four keys
+  for (int i0 = 0; 4 * i0 < n_last; i0 += blockDim.x) {  // warp-uniform trip count
+    const int i = i0 + (int)threadIdx.x;
+    bool c4[4];
+    bool any = false;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = 4 * i + k;
+      c4[k] = j < n_last && m[j] == 0;
+      any |= c4[k];
     }
-    const uint32_t bal = __ballot_sync(0xffffffffu, in);
-    if (!bal) continue;
-    uint32_t at = 0;
-    if (lane == 0) at = atomicAdd(&sh.digit[0], (uint32_t)__popc(bal));
-    at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
-    if (in && at < (uint32_t)kExpCap) list[at] = make_uint2(u, (uint32_t)j);
+    const uint4 w = any ? explore_keys4(a.seed, (uint32_t)i, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step)
+                        : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t u = word_of(w, k);
+      const bool in = c4[k] && (uint64_t)u < t;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (!bal) continue;
+      uint32_t at = 0;
+      if (lane == 0) at = atomicAdd(&sh.digit[0], (uint32_t)__popc(bal));
+      at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+      if (in && at < (uint32_t)kExpCap) list[at] = make_uint2(u, (uint32_t)(4 * i + k));
+    }
   }
   __syncthreads();
   const int cnt = (int)sh.digit[0];
@@ -594,18 +603,29 @@ __device__ bool explore_by_list(const StepArgs& a, int q, uint8_t* m, int n_last
 
 // Ordered compaction of the kept blocks of one request into its work list;
 // with mask_out, the labels of blocks 0 .. n_last-1 are written there too.
+// With stage (shared memory, n_last ints), the list is built there and both
+// outputs go out with coalesced stores.
 __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t* kept, int* scan,
-                            uint8_t* mask_out = nullptr) {
+                            uint8_t* mask_out = nullptr, int32_t* stage = nullptr) {
   const int chunk = (n_last + blockDim.x - 1) / blockDim.x;
   const int lo = threadIdx.x * chunk, hi = min(n_last, lo + chunk);
   int c = 0;
   for (int j = lo; j < hi; ++j) c += m[j] != 0;
   int total;
   int pos = block_exclusive_scan(c, scan, &total);
-  for (int j = lo; j < hi; ++j) {
-    const uint8_t v = m[j];
-    if (mask_out) mask_out[j] = v;
-    if (v) work[pos++] = j;
+  if (stage) {
+    for (int j = lo; j < hi; ++j)
+      if (m[j]) stage[pos++] = j;
+    if (mask_out)
+      for (int j = threadIdx.x; j < n_last; j += blockDim.x) mask_out[j] = m[j];
+    __syncthreads();
+    for (int i = threadIdx.x; i < total; i += blockDim.x) work[i] = stage[i];
+  } else {
+    for (int j = lo; j < hi; ++j) {
+      const uint8_t v = m[j];
+      if (mask_out) mask_out[j] = v;
+      if (v) work[pos++] = j;
+    }
   }
   if (threadIdx.x == 0) *kept = total;
 }
@@ -703,8 +723,12 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
                                            reinterpret_cast<int*>(keys), sh)) {  // block keys are spent
       // done: the `take` smallest keys came from the short list
     } else if (take > 0) {
-      for (int j = threadIdx.x; j < n_last; j += blockDim.x)
-        keys[j] = ~explore_key(a.seed, (uint32_t)j, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
+      for (int i = threadIdx.x; 4 * i < n_last; i += blockDim.x) {
+        const uint4 w = explore_keys4(a.seed, (uint32_t)i, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (4 * i + k < n_last) keys[4 * i + k] = ~word_of(w, k);
+      }
       __syncthreads();
       {
         uint32_t T, eq;
@@ -731,7 +755,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
     }
   }
   for (int64_t j = n_last + threadIdx.x; j < L.max_blocks; j += blockDim.x) mask_row[j] = 0;
-  compact_row(m, n_last, a.work + (int64_t)q * L.blk_stride, a.kept + q, sh.scan, mask_row);
+  compact_row(m, n_last, a.work + (int64_t)q * L.blk_stride, a.kept + q, sh.scan, mask_row,
+              reinterpret_cast<int32_t*>(keys));  // the block keys are spent
 }
 
 // ---------------------------------------------------------------------------

@@ -97,13 +97,19 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
   return c;
 }
 
-// Exploration key of block j: word 0 of Philox at counter
-// (j, request, layer, step mod 2^32) under key (seed lo, seed hi).
+// Exploration keys of blocks 4i .. 4i+3: words 0..3 of Philox at counter
+// (i, request, layer, step mod 2^32) under key (seed lo, seed hi); block j
+// takes word j mod 4 of counter j div 4.
+__device__ __forceinline__ uint4 explore_keys4(uint64_t seed, uint32_t i, uint32_t req, uint32_t layer,
+                                               uint64_t step) {
+  return philox4x32_10(make_uint4(i, req, layer, (uint32_t)step), make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
+}
+__device__ __forceinline__ uint32_t word_of(uint4 w, int k) {
+  return k == 0 ? w.x : k == 1 ? w.y : k == 2 ? w.z : w.w;
+}
 __device__ __forceinline__ uint32_t explore_key(uint64_t seed, uint32_t j, uint32_t req,
                                                 uint32_t layer, uint64_t step) {
-  uint4 r = philox4x32_10(make_uint4(j, req, layer, (uint32_t)step),
-                          make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
-  return r.x;
+  return word_of(explore_keys4(seed, j >> 2, req, layer, step), (int)(j & 3));
 }
 
 // Maximum of x over the 32 lanes of a warp, all of them active: one

@@ -61,18 +61,20 @@ ORC_API void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2
   out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
-/* Exploration key of logical block j: word 0 of Philox4x32-10 with counter
- * (j, request, layer, step mod 2^32) and key (seed low, seed high).  Random
- * exploration reserves part of the block budget for uniformly random unkept
- * blocks ([digest] arXiv深度剖析; [listing] Figure 4); drawing the blocks with
- * the smallest i.i.d. uniform keys is a uniform draw without replacement. */
+/* Exploration key of logical block j: word (j mod 4) of Philox4x32-10 with
+ * counter (j div 4, request, layer, step mod 2^32) and key (seed low, seed
+ * high) -- one generator call gives the keys of four consecutive blocks.
+ * Random exploration reserves part of the block budget for uniformly random
+ * unkept blocks ([digest] arXiv深度剖析; [listing] Figure 4); drawing the
+ * blocks with the smallest i.i.d. uniform keys is a uniform draw without
+ * replacement. */
 ORC_API uint32_t orc_explore_key(uint64_t seed, uint32_t block, uint32_t request,
                                  uint32_t layer, uint64_t step) {
-  uint32_t ctr[4] = {block, request, layer, (uint32_t)step};
+  uint32_t ctr[4] = {block >> 2, request, layer, (uint32_t)step};
   uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
   uint32_t out[4];
   orc_philox4x32_10(ctr, key, out);
-  return out[0];
+  return out[block & 3u];
 }
 
 /* ------------------------------------------------------------------------ */
@@ -576,9 +578,9 @@ ORC_API void orc_slot_prediction(const float* V, const float* D, int64_t ctx_len
 }
 
 /* The random baseline: an independent uniform value per slot in [0, 1), the */
-/* top 24 bits of word 0 of Philox4x32-10 at counter (slot, request, layer,  */
-/* step mod 2^32) and key (seed low, seed high) -- the exploration key with  */
-/* the slot in place of the block -- times 2^-24; the same for every row.    */
+/* top 24 bits of the exploration key with the slot in place of the block    */
+/* (word s mod 4 of Philox4x32-10 at counter (s div 4, request, layer, step  */
+/* mod 2^32), key (seed low, seed high)) times 2^-24; the same for every row. */
 ORC_API void orc_random_prediction(uint64_t seed, uint32_t request, uint32_t layer, uint64_t step,
                                    int64_t ctx_len, int rows, int64_t slot_stride, float* out) {
   for (int r = 0; r < rows; ++r) {

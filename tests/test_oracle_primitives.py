@@ -48,11 +48,13 @@ def test_philox_matches_curand_host_generator(oracle_lib, seed):
         assert list(got) == list(ref[i]), (seed, i)
 
 
-def test_explore_key_is_word0_of_counter_block_req_layer_step(oracle_lib):
+def test_explore_key_is_word_j_mod_4_of_counter_j_div_4_req_layer_step(oracle_lib):
     seed = 0xDEADBEEF12345678
-    got = oracle_lib.explore_key(seed, 5, 7, 3, (1 << 32) + 9)
-    ref = oracle_lib.philox4x32_10([5, 7, 3, 9], [seed & 0xFFFFFFFF, seed >> 32])[0]
-    assert got == ref
+    key = [seed & 0xFFFFFFFF, seed >> 32]
+    for j in (0, 5, 6, 7, 8, 4099):
+        got = oracle_lib.explore_key(seed, j, 7, 3, (1 << 32) + 9)
+        ref = oracle_lib.philox4x32_10([j // 4, 7, 3, 9], key)[j % 4]
+        assert got == ref, j
 
 
 def test_explore_keys_uniform_chi_square(oracle_lib):
