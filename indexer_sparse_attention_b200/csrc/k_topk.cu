@@ -331,6 +331,26 @@ __device__ uint32_t select_candidates(const TopkCtx& c, int n_cand, int want, To
 // 13-bit histogram bin that holds the want-th largest group key, with the bin
 // window placed just below the leading bits all group keys share.  The group
 // keys and then the compacted group list live in the bitmap area.
+// The float whose key is M (the inverse of fkey, M never a NaN pattern): for
+// every score x, fkey(x) >= M exactly when x >= key_float(M), -0 and +0 alike.
+__device__ __forceinline__ float key_float(uint32_t M) {
+  return __uint_as_float((M & 0x80000000u) ? (M & 0x7FFFFFFFu) : ~M);
+}
+
+// Bit 4u + k: the k-th score of float4 v[u] (slot s0[u] + k, s0[u] < 0 for
+// none) is visible (slot <= p) and at least Mf.
+__device__ __forceinline__ uint32_t takes_at_least(const float4 (&v)[8], const int (&s0)[8], int p, float Mf) {
+  uint32_t takes = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int nv = s0[u] < 0 ? 0 : min(4, p - s0[u] + 1);  // visible values of this float4
+    const uint32_t ge = (v[u].x >= Mf ? 1u : 0u) | (v[u].y >= Mf ? 2u : 0u) | (v[u].z >= Mf ? 4u : 0u) |
+                        (v[u].w >= Mf ? 8u : 0u);
+    takes |= (ge & ((1u << nv) - 1u)) << (4 * u);
+  }
+  return takes;
+}
+
 __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want, TopkShared& sh) {
   const int n_groups = (c.n_elem + 31) / 32;  // == c.nwords
   uint32_t* gk = c.bits;
@@ -412,6 +432,7 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
     __syncthreads();
   }
   const int n_q = sh.n_eq;
+  const float Mf = key_float(M);
   if (threadIdx.x == 0) sh.n_cand = 0;
   __syncthreads();
   // gather: a warp takes 32 groups at a time, 8 lanes x float4 per group.
@@ -444,14 +465,7 @@ __device__ int collect_from_groups(const TopkCtx& c, const float* gmax, int want
         }
       }
     }
-    uint32_t takes = 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << (4 * u + k);
-    }
+    const uint32_t takes = takes_at_least(v, s0, c.p, Mf);
     if (two_pass) {
       tmask[base + lane] = takes;
       my_cnt += __popc(takes);
@@ -602,6 +616,7 @@ __device__ __forceinline__ int collect_from_groups_cluster(const TopkCtx& c, con
   }
   cl.sync();
   const uint32_t M = sh.M;
+  const float Mf = key_float(M);
   // this share's qualifying groups to the front of gk, in place (a round
   // reads before it writes, and writes only reach indices already read)
   for (int base = 0; base < n_my; base += blockDim.x) {
@@ -637,14 +652,7 @@ __device__ __forceinline__ int collect_from_groups_cluster(const TopkCtx& c, con
         }
       }
     }
-    uint32_t takes = 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (s0[u] >= 0 && s0[u] + k <= c.p && fkey(vals[k]) >= M) takes |= 1u << (4 * u + k);
-    }
+    const uint32_t takes = takes_at_least(v, s0, c.p, Mf);
     const int n_t = __popc(takes);
     if (!__any_sync(0xffffffffu, n_t != 0)) continue;
     int incl = n_t;
