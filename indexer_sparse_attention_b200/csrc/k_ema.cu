@@ -122,84 +122,97 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
   const int64_t n_last = row_blocks(ctx, acc - 1, L.b);
   const int lb = __ffs(L.b) - 1;  // the block size is a power of two
   const int wpr = (int)gridDim.y * (blockDim.x >> 5);
-  for (int64_t j = (int64_t)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5); j < n_last; j += wpr) {
-    const uint8_t* mask = a.mask + (int64_t)q * L.max_blocks;
-    const bool kj = mask[j] != 0;
-    const bool kj1 = (R > 1) && (j + 1 < n_last) && mask[j + 1] != 0;
-    if (!kj && !kj1 && !(R > 1 && j == 0)) continue;
-    float* V = a.V + (int64_t)q * L.slot_stride;
-    float* D = a.D + (int64_t)q * L.slot_stride;
-    const float* sc = a.scores + (int64_t)q * L.R * L.slot_stride;
-    // Two slots per lane per pass (i, i + 32): every load of the pass is
-    // issued before the first store, so the pass costs one memory latency.
-    for (int i0 = lane; i0 < L.b; i0 += 64) {
-      float v[2], dv[2], sv[2][R], sd[2][R];
-      bool do_v[2], do_d[2], use_v[2][R], use_d[2][R];
-      int64_t sl[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int i = i0 + 32 * h;
-        sl[h] = j * L.b + i;
-        const int64_t s = sl[h];
-        do_v[h] = i < L.b && kj;                         // vertical state of slot s
-        do_d[h] = i < L.b && s <= p0 && (kj || kj1);     // diagonal state delta = p0 - s
-        v[h] = do_v[h] ? V[s] : 0.f;
-        dv[h] = do_d[h] ? D[p0 - s] : 0.f;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          use_v[h][r] = do_v[h] && r < acc && s <= p0 + r;
-          const int64_t sr = s + r;  // row r's slot for delta: in block j, or past its end in block j + 1
-          use_d[h][r] = do_d[h] && r < acc && (((sr >> lb) == j) ? kj : kj1);
-          sv[h][r] = use_v[h][r] ? sc[(int64_t)r * L.slot_stride + s] : 0.f;
-          sd[h][r] = use_d[h][r] ? sc[(int64_t)r * L.slot_stride + sr] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        bool tv = false, td = false;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {  // rows in order
-          if (use_v[h][r]) {
-            v[h] = ema_v(v[h], sv[h][r], a.alpha, a.beta);
-            tv = true;
-          }
-          if (use_d[h][r]) {
-            dv[h] = ema_d(dv[h], sd[h][r], a.alpha, a.beta);
-            td = true;
-          }
-        }
-        if (tv) V[sl[h]] = v[h];
-        if (td) D[p0 - sl[h]] = dv[h];
-      }
-      // a kept block's 32-slot groups: every lane holds its slot's V, new or
-      // not (vmax is kept only for b >= 32, so the whole warp is here)
-      if (a.vmax && kj) {
+  const int64_t j_first = (int64_t)blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const uint8_t* mask = a.mask + (int64_t)q * L.max_blocks;
+  // The warp's blocks j_first + t wpr, 32 at a time: lane t reads the mask of
+  // block t (and of the next block), so the blocks to update are known
+  // before the first one is loaded.
+  for (int64_t jb = j_first; jb < n_last; jb += 32 * (int64_t)wpr) {
+    const int64_t jl = jb + (int64_t)lane * wpr;
+    const bool ml = jl < n_last && mask[jl] != 0;
+    const bool ml1 = (R > 1) && jl + 1 < n_last && mask[jl + 1] != 0;
+    const uint32_t bk = __ballot_sync(0xffffffffu, ml), bk1 = __ballot_sync(0xffffffffu, ml1);
+    uint32_t todo = bk | bk1 | ((R > 1 && jb == 0) ? 1u : 0u);  // block 0 holds the offsets past p0
+    while (todo) {
+      const int t = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int64_t j = jb + (int64_t)t * wpr;
+      const bool kj = (bk >> t) & 1u;
+      const bool kj1 = (bk1 >> t) & 1u;
+      float* V = a.V + (int64_t)q * L.slot_stride;
+      float* D = a.D + (int64_t)q * L.slot_stride;
+      const float* sc = a.scores + (int64_t)q * L.R * L.slot_stride;
+      // Two slots per lane per pass (i, i + 32): every load of the pass is
+      // issued before the first store, so the pass costs one memory latency.
+      for (int i0 = lane; i0 < L.b; i0 += 64) {
+        float v[2], dv[2], sv[2][R], sd[2][R];
+        bool do_v[2], do_d[2], use_v[2][R], use_d[2][R];
+        int64_t sl[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (i0 - lane + 32 * h < L.b) {  // warp-uniform
-            const float g = warp_max(v[h]);
-            if (lane == 0) a.vmax[(int64_t)q * L.vg_stride + (sl[h] >> 5)] = g;
-          }
-        }
-      }
-    }
-    // offsets delta = p0 + m (m >= 1): seen only by rows r >= m at slot r - m
-    if (R > 1 && j == 0 && lane < R - 1) {
-      const int m = lane + 1;
-      const int64_t dlt = p0 + m;
-      float dv = D[dlt];
-      bool touched = false;
+          const int i = i0 + 32 * h;
+          sl[h] = j * L.b + i;
+          const int64_t s = sl[h];
+          do_v[h] = i < L.b && kj;                         // vertical state of slot s
+          do_d[h] = i < L.b && s <= p0 && (kj || kj1);     // diagonal state delta = p0 - s
+          v[h] = do_v[h] ? V[s] : 0.f;
+          dv[h] = do_d[h] ? D[p0 - s] : 0.f;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (r >= m && r < acc) {
-          const int64_t sr = r - m;  // in block 0 (r < R <= 4 < b)
-          if (kj) {
-            dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
-            touched = true;
+          for (int r = 0; r < R; ++r) {
+            use_v[h][r] = do_v[h] && r < acc && s <= p0 + r;
+            const int64_t sr = s + r;  // row r's slot for delta: in block j, or past its end in block j + 1
+            use_d[h][r] = do_d[h] && r < acc && (((sr >> lb) == j) ? kj : kj1);
+            sv[h][r] = use_v[h][r] ? sc[(int64_t)r * L.slot_stride + s] : 0.f;
+            sd[h][r] = use_d[h][r] ? sc[(int64_t)r * L.slot_stride + sr] : 0.f;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          bool tv = false, td = false;
+#pragma unroll
+          for (int r = 0; r < R; ++r) {  // rows in order
+            if (use_v[h][r]) {
+              v[h] = ema_v(v[h], sv[h][r], a.alpha, a.beta);
+              tv = true;
+            }
+            if (use_d[h][r]) {
+              dv[h] = ema_d(dv[h], sd[h][r], a.alpha, a.beta);
+              td = true;
+            }
+          }
+          if (tv) V[sl[h]] = v[h];
+          if (td) D[p0 - sl[h]] = dv[h];
+        }
+        // a kept block's 32-slot groups: every lane holds its slot's V, new or
+        // not (vmax is kept only for b >= 32, so the whole warp is here)
+        if (a.vmax && kj) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (i0 - lane + 32 * h < L.b) {  // warp-uniform
+              const float g = warp_max(v[h]);
+              if (lane == 0) a.vmax[(int64_t)q * L.vg_stride + (sl[h] >> 5)] = g;
+            }
           }
         }
       }
-      if (touched) D[dlt] = dv;
+      // offsets delta = p0 + m (m >= 1): seen only by rows r >= m at slot r - m
+      if (R > 1 && j == 0 && lane < R - 1) {
+        const int m = lane + 1;
+        const int64_t dlt = p0 + m;
+        float dv = D[dlt];
+        bool touched = false;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (r >= m && r < acc) {
+            const int64_t sr = r - m;  // in block 0 (r < R <= 4 < b)
+            if (kj) {
+              dv = ema_d(dv, sc[(int64_t)r * L.slot_stride + sr], a.alpha, a.beta);
+              touched = true;
+            }
+          }
+        }
+        if (touched) D[dlt] = dv;
+      }
     }
   }
 }

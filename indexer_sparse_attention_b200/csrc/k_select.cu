@@ -460,8 +460,22 @@ constexpr int kSelThreads = 1024;
 struct SelShared {
   uint32_t hist[256];
   uint32_t digit[2];
+  uint32_t digit_r[4][2];  // per-row digits of the batched radix passes
   int scan[33];
 };
+
+// Shared memory of the one-CTA select: block keys, labels and the
+// exploration list; with several predicting rows whose keys fit next to
+// them, every row's keys too, so the rows' radix passes run together.
+constexpr size_t kSelBatchCap = 160 * 1024;
+__host__ __device__ inline size_t select_smem(int64_t blk_stride, int rows) {
+  const size_t base = (size_t)blk_stride * 5 + (size_t)2048 * 8;  // keys, labels, kExpCap (key, block) pairs
+  const size_t extra = (size_t)rows * 4 * (size_t)blk_stride;
+  return (rows > 1 && base + extra <= kSelBatchCap) ? base + extra : base;
+}
+__host__ __device__ inline bool select_batched(int64_t blk_stride, int rows) {
+  return rows > 1 && (size_t)blk_stride * 5 + (size_t)2048 * 8 + (size_t)rows * 4 * blk_stride <= kSelBatchCap;
+}
 
 // Radix select over keys[0..n) restricted to elements with valid(j).  `want`
 // must be in [1, #valid].  Returns T and the number of elements equal to T
@@ -493,6 +507,48 @@ __device__ void radix_select_desc(const uint32_t* keys, int n, Valid valid, uint
 // Marks m[j] = label for the top `want` valid elements (keys > T, then the
 // lowest-index keys == T).  Each thread walks a contiguous chunk so that the
 // "lowest index" order is a block scan.
+// The radix passes of several rows at once.  Row r's keys are kb[r stride
+// + j], j < n_r; rows with want_r = 0 take no select.  One sweep over every
+// row's keys per 8-bit digit fills a histogram per row, and one warp per row
+// finds its digit.  Each row gets the T and eq of radix_select_desc.  The
+// per-row values live in scalars (a row index selects among them), so
+// nothing goes to local memory.
+__device__ void radix_select_rows(const uint32_t* kb, int stride, int pr, const int (&n)[4], const uint32_t (&want)[4],
+                                  uint32_t (*hist)[256], SelShared& sh, uint32_t (&T)[4], uint32_t (&eq)[4]) {
+  uint32_t p0 = 0, p1 = 0, p2 = 0, p3 = 0;
+  uint32_t m0 = want[0], m1 = want[1], m2 = want[2], m3 = want[3];
+  uint32_t pmask = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < pr * 256; i += blockDim.x) hist[i >> 8][i & 255] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < pr * stride; i += blockDim.x) {
+      const int r = (i >= stride) + (i >= 2 * stride) + (i >= 3 * stride);
+      const int j = i - r * stride;
+      const int nr = r == 0 ? n[0] : r == 1 ? n[1] : r == 2 ? n[2] : n[3];
+      const uint32_t rem = r == 0 ? m0 : r == 1 ? m1 : r == 2 ? m2 : m3;
+      const uint32_t pre = r == 0 ? p0 : r == 1 ? p1 : r == 2 ? p2 : p3;
+      if (j >= nr || rem == 0) continue;
+      const uint32_t k = kb[i];
+      if ((k & pmask) == pre) atomicAdd(&hist[r][(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    const int w = threadIdx.x >> 5;
+    if (w < pr) {
+      const uint32_t rem = w == 0 ? m0 : w == 1 ? m1 : w == 2 ? m2 : m3;
+      if (rem != 0) warp_find_digit_desc<256>(hist[w], rem, sh.digit_r[w]);
+    }
+    __syncthreads();
+    if (m0) { p0 |= sh.digit_r[0][0] << shift; m0 = sh.digit_r[0][1]; }
+    if (pr > 1 && m1) { p1 |= sh.digit_r[1][0] << shift; m1 = sh.digit_r[1][1]; }
+    if (pr > 2 && m2) { p2 |= sh.digit_r[2][0] << shift; m2 = sh.digit_r[2][1]; }
+    if (pr > 3 && m3) { p3 |= sh.digit_r[3][0] << shift; m3 = sh.digit_r[3][1]; }
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  T[0] = p0; T[1] = p1; T[2] = p2; T[3] = p3;
+  eq[0] = m0; eq[1] = m1; eq[2] = m2; eq[3] = m3;
+}
+
 template <class Valid>
 __device__ void mark_selected(const uint32_t* keys, int n, Valid valid, uint32_t T, uint32_t eq_take,
                               uint8_t* m, uint8_t label, SelShared& sh) {
@@ -641,6 +697,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   uint8_t* m = dyn + 4 * L.blk_stride;
   uint2* list = reinterpret_cast<uint2*>(dyn + 5 * L.blk_stride);  // kExpCap (key, block) pairs
   __shared__ SelShared sh;
+  __shared__ uint32_t hist_r[4][256];
 
   if (a.q8) {
     // a0 for this request's (row, head) vectors, one warp each; the score
@@ -671,7 +728,35 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   } else {
     const int64_t n0 = row_blocks(ctx, 0, L.b);
     const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
-    for (int r = 0; r < (a.mtp_row0 ? 1 : a.rows); ++r) {
+    const int pr = a.mtp_row0 ? 1 : a.rows;  // rows whose predicted sets are unioned
+    if (pr > 1 && select_batched(L.blk_stride, a.rows)) {
+      // every row's keys on chip (row r at kb + r blk_stride), the rows'
+      // radix passes together
+      uint32_t* kb = reinterpret_cast<uint32_t*>(dyn + select_smem(L.blk_stride, 1));
+      const int stride = (int)L.blk_stride;
+      int nrow[4] = {0, 0, 0, 0};
+      uint32_t want[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (r >= pr) break;
+        nrow[r] = (int)row_blocks(ctx, r, L.b);
+        const int64_t n_pred = block_budget(nrow[r], a.sparsity) - n_exp;
+        want[r] = (n_pred > 0 && n_pred < nrow[r]) ? (uint32_t)n_pred : 0u;
+        const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride;
+        for (int j = threadIdx.x; j < nrow[r]; j += blockDim.x) {
+          kb[r * stride + j] = fkey(S[j]);
+          if (n_pred >= nrow[r]) m[j] = 1;  // this row keeps all its blocks
+        }
+      }
+      __syncthreads();
+      uint32_t T[4], eq[4];
+      radix_select_rows(kb, stride, pr, nrow, want, hist_r, sh, T, eq);
+      auto all = [](int) { return true; };
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (r < pr && want[r]) mark_selected(kb + r * stride, nrow[r], all, T[r], eq[r], m, 1, sh);
+    }
+    for (int r = 0; r < pr && !(pr > 1 && select_batched(L.blk_stride, a.rows)); ++r) {
       const int n = (int)row_blocks(ctx, r, L.b);
       const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
       const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride;
@@ -1038,7 +1123,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
 }
 
 cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)a.lay.blk_stride * 5 + (size_t)kExpCap * sizeof(uint2);
+  static_assert(kExpCap * sizeof(uint2) == 2048 * 8, "select_smem counts kExpCap entries");
+  const size_t smem = select_smem(a.lay.blk_stride, a.mtp_row0 ? 1 : a.rows);
   cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -843,7 +843,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
     if (total <= kCandCap) {
       n_cand = collect_ge(c, 0u, sh);  // everything fits
     } else {
-      if (a.gmax && c.nwords > want) {
+      // The group path pays when the wanted scores lie in a small share of
+      // the groups.  With fewer than two groups per wanted score nearly every
+      // group qualifies, the candidates overflow the on-chip list, and the
+      // sampled threshold below is taken anyway.
+      if (a.gmax && c.nwords >= 2 * want) {
         const float* gm = a.gmax + ((int64_t)q * L.R + r) * a.gstride;
         if constexpr (kCluster) {
           n_cand = collect_from_groups_cluster(c, gm, want, sh);
@@ -853,7 +857,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
         }
       }
       if constexpr (kCluster) {
-        if (!(a.gmax && c.nwords > want)) {  // every rank takes this branch alike
+        if (!(a.gmax && c.nwords >= 2 * want)) {  // every rank takes this branch alike
           n_cand = collect_sampled_cluster(c, want, total, sh);
           if (n_cand == -2) return;
         }
