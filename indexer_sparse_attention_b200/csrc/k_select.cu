@@ -1046,20 +1046,32 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
       uint32_t* list_n0 = &cl.map_shared_rank(&sc, 0)->list_n;
       uint2* list0 = cl.map_shared_rank(list, 0);
       const int lane = threadIdx.x & 31;
-      for (int i0 = 0; i0 < nl; i0 += blockDim.x) {  // warp-uniform trip count
-        const int i = i0 + (int)threadIdx.x;
-        uint32_t u = 0;
-        bool in = false;
-        if (i < nl && m[i] == 0) {
-          u = explore_key(a.seed, (uint32_t)(j0 + i), (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step);
-          in = (uint64_t)u < t;
+      // a thread takes the blocks 4c .. 4c+3 of one Philox call that lie in
+      // this rank's range
+      const int c0 = j0 >> 2, nq = ((j0 + nl + 3) >> 2) - c0;
+      for (int i0 = 0; i0 < nq; i0 += blockDim.x) {  // warp-uniform trip count
+        const int cq = c0 + i0 + (int)threadIdx.x;
+        bool c4[4];
+        bool any = false;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = 4 * cq + k - j0;
+          c4[k] = i0 + (int)threadIdx.x < nq && i >= 0 && i < nl && m[i] == 0;
+          any |= c4[k];
         }
-        const uint32_t bal = __ballot_sync(0xffffffffu, in);
-        if (!bal) continue;
-        uint32_t at = 0;
-        if (lane == 0) at = atomicAdd(list_n0, (uint32_t)__popc(bal));
-        at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
-        if (in && at < (uint32_t)kExpCap) list0[at] = make_uint2(u, (uint32_t)(j0 + i));
+        const uint4 w = any ? explore_keys4(a.seed, (uint32_t)cq, (uint32_t)q, (uint32_t)a.layer, (uint64_t)a.step)
+                            : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t u = word_of(w, k);
+          const bool in = c4[k] && (uint64_t)u < t;
+          const uint32_t bal = __ballot_sync(0xffffffffu, in);
+          if (!bal) continue;
+          uint32_t at = 0;
+          if (lane == 0) at = atomicAdd(list_n0, (uint32_t)__popc(bal));
+          at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+          if (in && at < (uint32_t)kExpCap) list0[at] = make_uint2(u, (uint32_t)(4 * cq + k));
+        }
       }
       cl.sync();
       const int cnt = (int)*list_n0;  // alike in every rank
@@ -1114,10 +1126,15 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
   int local_kept, total_kept;
   int pos = block_exclusive_scan(kc, sh.scan, &local_kept);
   cl.sync();  // slot 2 / 3 readers of earlier phases are done
-  pos += cl_rank_prefix(local_kept, 2, sc, &total_kept);
-  int32_t* work = a.work + (int64_t)q * L.blk_stride;
+  const int base = cl_rank_prefix(local_kept, 2, sc, &total_kept);
+  // this rank's part of the list staged in shared memory (the block keys are
+  // spent), then stored coalesced
+  int32_t* stage = reinterpret_cast<int32_t*>(keys);
   for (int i = lo; i < up; ++i)
-    if (m[i]) work[pos++] = j0 + i;
+    if (m[i]) stage[pos++] = j0 + i;
+  __syncthreads();
+  int32_t* work = a.work + (int64_t)q * L.blk_stride + base;
+  for (int i = threadIdx.x; i < local_kept; i += blockDim.x) work[i] = stage[i];
   if (cr == 0 && threadIdx.x == 0) a.kept[q] = total_kept;
   cl.sync();  // no rank leaves while another may still read its counters
 }

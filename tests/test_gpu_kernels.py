@@ -391,6 +391,35 @@ def test_kernel_timing_mask_times_only_named_stages():
         isa.spin_set_kernel_timing_mask(st, ["no such stage"])
 
 
+@pytest.mark.parametrize("R", [2, 4])
+def test_select_rows_long_context_bit_exact(R):
+    """640K slots with too many requests for clusters (74), so one CTA per
+    request: two rows' block keys still fit on chip together and their radix
+    passes run together; four rows' do not, and the rows' selects run one
+    after another.  The union masks equal the oracle's bit for bit."""
+    rng = np.random.default_rng(R + 40)
+    max_slots = 640 * 1024 + 64
+    st = make_state(Q=74, max_slots=max_slots, R=R, H=16, s=0.5, g=0.1, k=2048)
+    V, D = st.ema(0)
+    v = rng.integers(0, 6, V.shape).astype(np.float32)    # many equal block scores
+    v[:, -3000:] = np.inf
+    V.copy_(torch.from_numpy(v))
+    d = rng.standard_normal(D.shape).astype(np.float32)
+    d[rng.random(D.shape) < 0.5] = -np.inf
+    D.copy_(torch.from_numpy(d))
+    st.refresh()  # V and D were written through the views
+    ctx = np.full(74, max_slots - 64 - R + 1, np.int64)
+    ctx[1], ctx[2], ctx[3] = 1, 300_000 + 37, 64 * 5000
+    ctx_t = torch.from_numpy(ctx).to(torch.int32).cuda()
+    mask = st.new_mask()
+    isa.spin_predict_select(st, 0, R, 6, ctx_t, mask)
+    assert isa.spin_get_error(st)[0] == 0
+    for q in range(4):
+        S_ref = oracle.predict_pool(V[q].cpu().numpy(), D[q].cpu().numpy(), int(ctx[q]), R, 64, st.mask_stride)
+        m_ref = oracle.select(S_ref, int(ctx[q]), R, 64, 0.5, 0.1, 7, q, 0, 6)
+        assert np.array_equal(mask[q].cpu().numpy(), m_ref), q
+
+
 @pytest.mark.parametrize("R", [1, 2, 4])
 @pytest.mark.parametrize("s,g", [(0.5, 0.05), (0.4, 0.3), (0.0, 0.05), (0.3, 0.0), (0.999, 0.5)])
 def test_select_cluster_paths_bit_exact(R, s, g):
