@@ -591,23 +591,52 @@ __device__ __forceinline__ int collect_from_groups_cluster(const TopkCtx& c, con
     }
   }
   cl.sync();
+  // The cluster's histogram: rank k sums slice k of the bins over the ranks
+  // into its own copy of that slice (no rank reads another's slice of its
+  // own bins), with the slice's total beside it; rank 0 then finds the slice
+  // that holds the wanted rank, and the bin inside it.
+  const int per = kBins / C, b0 = cr * per;  // C is 2, 4 or 8
+  if (diff) {
+    int cnt = 0;
+    for (int b = b0 + threadIdx.x; b < b0 + per; b += blockDim.x) {
+      uint32_t t = 0;
+      for (int k = 0; k < C; ++k) t += cl.map_shared_rank(c.hist, k)[b];
+      c.hist[b] = t;
+      cnt += (int)t;
+    }
+    int slice_total;
+    block_exclusive_scan(cnt, sh.scan, &slice_total);
+    if (threadIdx.x == 0) sh.total = slice_total;  // the kernel keeps its own copy of the scored total
+  }
+  cl.sync();
   if (cr == 0) {
     uint32_t M = all_or == 0u ? kEmptyGroup : all_and;
     if (diff) {
-      // the cluster's histogram, bin by bin, into rank 0's
-      int cnt = 0;
-      for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
-        uint32_t t = c.hist[i];
-        for (int k = 1; k < C; ++k) t += cl.map_shared_rank(c.hist, k)[i];
-        c.hist[i] = t;
-        cnt += (int)t;
+      if (threadIdx.x == 0) {
+        uint32_t above = 0;
+        int hit = -1;
+        for (int k = C - 1; k >= 0; --k) {  // the largest keys sit in the last slice
+          const uint32_t t = (uint32_t)cl.map_shared_rank(&sh, k)->total;
+          if (above + t >= (uint32_t)want) {
+            hit = k;
+            break;
+          }
+          above += t;
+        }
+        sh.digit[0] = (uint32_t)hit;
+        sh.digit[1] = above;
       }
-      int n_scored_groups;
-      block_exclusive_scan(cnt, sh.scan, &n_scored_groups);
-      if (n_scored_groups >= want) {
-        block_find_bin_desc(c.hist, kBins, (uint32_t)want, sh);
+      __syncthreads();
+      const int hit = (int)sh.digit[0];
+      const uint32_t above = sh.digit[1];
+      __syncthreads();
+      if (hit >= 0) {
+        if (hit != 0)  // that slice's merged bins, from their owner
+          for (int b = threadIdx.x; b < per; b += blockDim.x) c.hist[b] = cl.map_shared_rank(c.hist, hit)[hit * per + b];
+        __syncthreads();
+        block_find_bin_desc(c.hist, per, (uint32_t)want - above, sh);
         const uint32_t high = shift + 13 >= 32 ? 0u : (all_and & ~((1u << (shift + 13)) - 1u));
-        M = high | (sh.digit[0] << shift);
+        M = high | ((uint32_t)(hit * per + (int)sh.digit[0]) << shift);
       } else {
         M = all_and;  // fewer scored groups than wanted: every scored group qualifies
       }
