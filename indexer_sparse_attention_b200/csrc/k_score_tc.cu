@@ -350,7 +350,8 @@ __device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
 // KH: the head count when it is fixed at compile time (64, the DSA indexer's),
 // so that the epilogue's column loops unroll; 0 reads it from the layout.
 // DIST: the side-load prefetch distance, prefetch_dist() of the plan.
-template <int G, int KH, int DIST>
+// R1: one query row, known at compile time (the fused one-row step).
+template <int G, int KH, int DIST, int R1 = 0>
 __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
@@ -359,7 +360,8 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   constexpr int kEpiGroups = G;
   const Layout L = a.lay;
   const int H = KH ? KH : L.H;
-  const int N = a.rows * H;
+  const int rows = R1 ? 1 : a.rows;
+  const int N = rows * H;
   const int stages = plan.stages, nacc = plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   // With four groups and several rows, two groups share a tile, each taking
   // every other row: the accumulator (two fit TMEM at N > 128) is read in half
   // the time, so the MMA waits half as long for it.
-  const int share = groups_per_tile(kEpiGroups, a.rows);  // groups per tile
+  const int share = groups_per_tile(kEpiGroups, rows);  // groups per tile
 
   // ---- tile prefix over requests (all threads: one load pair each, block
   // scan), barriers ------------------------------------------------------
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       int v = 0;
       if (q < L.Q) {
         const int64_t ctx = a.ctx_len[q];
-        bool ok = ctx >= 1 && ctx + a.rows - 1 <= L.max_slots;
+        bool ok = ctx >= 1 && ctx + rows - 1 <= L.max_slots;
         if (ok && a.ctx_sel && a.ctx_sel[q] != ctx) {  // the prepared selection is for another ctx_len
           ok = false;
           if (blockIdx.x == 0) raise_error(a.err, ERR_LOOKAHEAD, q, (uint32_t)ctx);
@@ -612,7 +614,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       const bool present = pg_idx < x->np && pg >= 0;
       r.s = present ? x->j[pg_idx] * kPage + tok : 0;
       r.pres = present;
-      r.valid = present && r.s <= r.p0 + (a.rows - 1);
+      r.valid = present && r.s <= r.p0 + (rows - 1);
       r.upd = fused && r.valid && r.s <= r.p0;
       return r;
     };
@@ -680,7 +682,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       if (!__all_sync(0xffffffffu, wait_parity(B.e(stage), phase, ctl))) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
-      for (int r = sub; r < a.rows; r += share) {
+      for (int r = sub; r < rows; r += share) {
         float part[4] = {0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < H; c += 32) {
           uint32_t v[32];
@@ -689,7 +691,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
           else
             tmem_ld16(trow + (uint32_t)(r * H + c), *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           tmem_wait_ld();
-          if (r + share >= a.rows && c + 32 >= H) {
+          if (r + share >= rows && c + 32 >= H) {
             // last accumulator columns are in registers: hand the accumulator
             // (and the tile-info slot, read a tile ago) back before the math
             tc_fence_before();
@@ -790,7 +792,8 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   // the instances the plans reach: two groups with 4 accumulators (N <= 64)
   // or 2 (N <= 128); four groups sharing tiles (several rows) or not (one row)
   void (*kernel)(ScoreArgs, TcPlan, const CUtensorMap, const CUtensorMap) = nullptr;
-  if (plan.groups == 2 && dist == 2) kernel = L.H == 64 ? k_score_tc<2, 64, 2> : k_score_tc<2, 0, 2>;
+  if (plan.groups == 2 && dist == 2)
+    kernel = L.H == 64 ? (a.rows == 1 ? k_score_tc<2, 64, 2, 1> : k_score_tc<2, 64, 2>) : k_score_tc<2, 0, 2>;
   if (plan.groups == 2 && dist == 1) kernel = L.H == 64 ? k_score_tc<2, 64, 1> : k_score_tc<2, 0, 1>;
   if (plan.groups == 4 && dist == 1) kernel = L.H == 64 ? k_score_tc<4, 64, 1> : k_score_tc<4, 0, 1>;
   if (plan.groups == 4 && dist == 0) kernel = k_score_tc<4, 0, 0>;
