@@ -350,8 +350,9 @@ __device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
 // KH: the head count when it is fixed at compile time (64, the DSA indexer's),
 // so that the epilogue's column loops unroll; 0 reads it from the layout.
 // DIST: the side-load prefetch distance, prefetch_dist() of the plan.
-// R1: one query row, known at compile time (the fused one-row step).
-template <int G, int KH, int DIST, int R1 = 0>
+// RC: the number of query rows when fixed at compile time (0: a.rows), so
+// that the epilogue's row loop and its per-row conditions fold.
+template <int G, int KH, int DIST, int RC = 0>
 __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   constexpr int kEpiGroups = G;
   const Layout L = a.lay;
   const int H = KH ? KH : L.H;
-  const int rows = R1 ? 1 : a.rows;
+  const int rows = RC ? RC : a.rows;
   const int N = rows * H;
   const int stages = plan.stages, nacc = plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -795,7 +796,8 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   if (plan.groups == 2 && dist == 2)
     kernel = L.H == 64 ? (a.rows == 1 ? k_score_tc<2, 64, 2, 1> : k_score_tc<2, 64, 2>) : k_score_tc<2, 0, 2>;
   if (plan.groups == 2 && dist == 1) kernel = L.H == 64 ? k_score_tc<2, 64, 1> : k_score_tc<2, 0, 1>;
-  if (plan.groups == 4 && dist == 1) kernel = L.H == 64 ? k_score_tc<4, 64, 1> : k_score_tc<4, 0, 1>;
+  if (plan.groups == 4 && dist == 1)
+    kernel = L.H == 64 ? (a.rows == 4 ? k_score_tc<4, 64, 1, 4> : k_score_tc<4, 64, 1>) : k_score_tc<4, 0, 1>;
   if (plan.groups == 4 && dist == 0) kernel = k_score_tc<4, 0, 0>;
   if (!kernel) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
