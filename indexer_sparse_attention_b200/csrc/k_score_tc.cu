@@ -351,8 +351,9 @@ __device__ __forceinline__ TileMeta shfl_meta(const TileMeta& m, int src) {
 // so that the epilogue's column loops unroll; 0 reads it from the layout.
 // DIST: the side-load prefetch distance, prefetch_dist() of the plan.
 // RC: the number of query rows when fixed at compile time (0: a.rows), so
-// that the epilogue's row loop and its per-row conditions fold.
-template <int G, int KH, int DIST, int RC = 0>
+// that the epilogue's row loop and its per-row conditions fold.  FU: the
+// fused EMA update known at compile time (1 on, 0 off, -1: a.V decides).
+template <int G, int KH, int DIST, int RC = 0, int FU = -1>
 __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
     k_score_tc(ScoreArgs a, TcPlan plan, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_q) {
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   B.done = B.accempty + 8 * kMaxAcc;
   const Ctl ctl{abort_flag, a.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool fused = a.V != nullptr;
+  const bool fused = FU >= 0 ? FU == 1 : a.V != nullptr;
   // With four groups and several rows, two groups share a tile, each taking
   // every other row: the accumulator (two fit TMEM at N > 128) is read in half
   // the time, so the MMA waits half as long for it.
@@ -625,7 +626,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       Side r;
       r.sigma = m.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
       // V of the page's slots past the context too, for its group maxima
-      r.v = (m.upd || (a.vmax && m.pres)) ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
+      r.v = (m.upd || (fused && a.vmax && m.pres)) ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
       r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
       return r;
     };
@@ -732,7 +733,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
             a.D[(int64_t)cur.q * L.slot_stride + (cur.p0 - cur.s)] = ema_d(cur.d, score, a.alpha, a.beta);
           }
         }
-        if (a.vmax && r == 0 && cur.pres) {
+        if (fused && a.vmax && r == 0 && cur.pres) {
           // this warp's 32 slots are one aligned group of V (present is warp-uniform)
           const float g = warp_max(vnew);
           if (lane == 0) a.vmax[(int64_t)cur.q * L.vg_stride + (cur.s >> 5)] = g;
@@ -794,7 +795,10 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   // or 2 (N <= 128); four groups sharing tiles (several rows) or not (one row)
   void (*kernel)(ScoreArgs, TcPlan, const CUtensorMap, const CUtensorMap) = nullptr;
   if (plan.groups == 2 && dist == 2)
-    kernel = L.H == 64 ? (a.rows == 1 ? k_score_tc<2, 64, 2, 1> : k_score_tc<2, 64, 2>) : k_score_tc<2, 0, 2>;
+    kernel = L.H != 64 ? k_score_tc<2, 0, 2>
+             : a.rows != 1 ? k_score_tc<2, 64, 2>
+             : a.V        ? k_score_tc<2, 64, 2, 1, 1>
+                          : k_score_tc<2, 64, 2, 1, 0>;
   if (plan.groups == 2 && dist == 1) kernel = L.H == 64 ? k_score_tc<2, 64, 1> : k_score_tc<2, 0, 1>;
   if (plan.groups == 4 && dist == 1)
     kernel = L.H == 64 ? (a.rows == 4 ? k_score_tc<4, 64, 1, 4> : k_score_tc<4, 64, 1>) : k_score_tc<4, 0, 1>;
