@@ -49,7 +49,7 @@ SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write 
 # per kept slot, from one ncu capture of the kernel on 16 requests at 512K, 50% sparsity,
 # fused EMA (traffic grows with kept slots: each is read once), valid for the kernel
 # source with this hash prefix
-SCORE_TRAFFIC = {"src_sha256_16": "c786f7ba10ee1679", "bytes_per_kept_slot": 151.41,
+SCORE_TRAFFIC = {"src_sha256_16": "49036cef2a6a88d6", "bytes_per_kept_slot": 151.49,
                  "sources": ("indexer_sparse_attention_b200/csrc/k_score_tc.cu",
                              "indexer_sparse_attention_b200/csrc/spin_internal.cuh")}
 
