@@ -686,11 +686,14 @@ __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t
   if (threadIdx.x == 0) *kept = total;
 }
 
+// R1: one query row known at compile time (the decode step's common case).
+template <int R1>
 __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   pdl_enter();
   StepArgs a = a_in;
   if (a.step_dev) a.step = *a.step_dev + a.step_add;  // the state's counter (read after the predecessors finished)
   const Layout L = a.lay;
+  const int rows = R1 ? 1 : a.rows;
   const int q = blockIdx.x;
   extern __shared__ __align__(16) uint8_t dyn[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);
@@ -702,13 +705,13 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   if (a.q8) {
     // a0 for this request's (row, head) vectors, one warp each; the score
     // kernel reads them after this kernel
-    const int nv = a.rows * L.H, warp = threadIdx.x >> 5;
+    const int nv = rows * L.H, warp = threadIdx.x >> 5;
     for (int i = warp; i < nv; i += kSelThreads / 32)
       quantize_vec(a.q, a.w, a.q_bf16, L.d, (int64_t)q * nv + i, a.q8, a.wq);
   }
   const int64_t ctx = a.ctx_len[q];
   uint8_t* mask_row = a.mask + (int64_t)q * L.max_blocks;
-  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots) {
+  if (ctx < 1 || ctx + rows - 1 > L.max_slots) {
     if (threadIdx.x == 0) {
       if (!a.quiet) raise_error(a.err, ERR_CTX_LEN, q, (uint32_t)ctx);
       a.kept[q] = 0;
@@ -718,7 +721,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
     return;
   }
   if (a.ctx_sel && threadIdx.x == 0) a.ctx_sel[q] = (int32_t)ctx;
-  const int n_last = (int)row_blocks(ctx, a.rows - 1, L.b);
+  const int n_last = (int)row_blocks(ctx, rows - 1, L.b);
   for (int j = threadIdx.x; j < n_last; j += blockDim.x) m[j] = 0;
   __syncthreads();
 
@@ -728,8 +731,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   } else {
     const int64_t n0 = row_blocks(ctx, 0, L.b);
     const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
-    const int pr = a.mtp_row0 ? 1 : a.rows;  // rows whose predicted sets are unioned
-    if (pr > 1 && select_batched(L.blk_stride, a.rows)) {
+    const int pr = (R1 || a.mtp_row0) ? 1 : rows;  // rows whose predicted sets are unioned
+    if (pr > 1 && select_batched(L.blk_stride, rows)) {
       // every row's keys on chip (row r at kb + r blk_stride), the rows'
       // radix passes together
       uint32_t* kb = reinterpret_cast<uint32_t*>(dyn + select_smem(L.blk_stride, 1));
@@ -756,7 +759,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
       for (int r = 0; r < 4; ++r)
         if (r < pr && want[r]) mark_selected(kb + r * stride, nrow[r], all, T[r], eq[r], m, 1, sh);
     }
-    for (int r = 0; r < pr && !(pr > 1 && select_batched(L.blk_stride, a.rows)); ++r) {
+    for (int r = 0; r < pr && !(pr > 1 && select_batched(L.blk_stride, rows)); ++r) {
       const int n = (int)row_blocks(ctx, r, L.b);
       const int64_t n_pred = block_budget(n, a.sparsity) - n_exp;
       const float* S = a.S + ((int64_t)q * L.R + r) * L.blk_stride;
@@ -791,7 +794,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
     // exploration among the unkept blocks of the last row's range
     auto cand = [m](int j) { return m[j] == 0; };
     int n_cand;
-    if (a.rows == 1) {  // one row: exactly min(max(n_pred, 0), n) blocks are predicted
+    if (rows == 1) {  // one row: exactly min(max(n_pred, 0), n) blocks are predicted
       const int64_t n_pred = block_budget(n_last, a.sparsity) - n_exp;
       n_cand = n_last - (int)(n_pred < 0 ? 0 : n_pred > n_last ? n_last : n_pred);
     } else {
@@ -1142,7 +1145,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(StepArgs a_in) {
 cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   static_assert(kExpCap * sizeof(uint2) == 2048 * 8, "select_smem counts kExpCap entries");
   const size_t smem = select_smem(a.lay.blk_stride, a.mtp_row0 ? 1 : a.rows);
-  cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_select<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Few requests with long contexts leave most SMs idle: a cluster of up to 8
@@ -1169,7 +1173,7 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   }
   PdlLaunch l(dim3(a.lay.Q), dim3(kSelThreads), smem, s);
   l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
-  return cudaLaunchKernelEx(&l.cfg, k_select, a);
+  return cudaLaunchKernelEx(&l.cfg, a.rows == 1 ? k_select<1> : k_select<0>, a);
 }
 
 // ---------------------------------------------------------------------------
