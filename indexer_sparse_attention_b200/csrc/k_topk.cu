@@ -792,7 +792,9 @@ __device__ __forceinline__ int collect_sampled_cluster(const TopkCtx& c, int wan
 
 // kCluster: launched with a cluster of C CTAs per (request, row), which share
 // the group path; otherwise one CTA per pair.
-template <bool kCluster>
+// R1B64: one row and 64-slot blocks known at compile time (the decode
+// step's common case), so the position arithmetic of every pass folds.
+template <bool kCluster, int R1B64 = 0>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   pdl_enter();
   const Layout L = a.lay;
@@ -800,12 +802,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   const int C = kCluster ? (int)cg::this_cluster().num_blocks() : 1;
   const int cr = kCluster ? (int)cg::this_cluster().block_rank() : 0;
   const unsigned rid = blockIdx.x / (unsigned)C;
-  const int q = rid / a.rows, r = rid % a.rows;
-  int32_t* out = a.topk + ((int64_t)q * a.rows + r) * L.k;
+  const int rows = R1B64 ? 1 : a.rows;
+  const int q = rid / rows, r = rid % rows;
+  int32_t* out = a.topk + ((int64_t)q * rows + r) * L.k;
   __shared__ TopkShared sh;
   extern __shared__ __align__(16) uint8_t dyn[];
   const int64_t ctx = a.ctx_len[q];
-  if (ctx < 1 || ctx + a.rows - 1 > L.max_slots || (a.ctx_sel && a.ctx_sel[q] != ctx)) {
+  if (ctx < 1 || ctx + rows - 1 > L.max_slots || (a.ctx_sel && a.ctx_sel[q] != ctx)) {
     if (cr == 0)
       for (int t = threadIdx.x; t < L.k; t += blockDim.x) out[t] = -1;
     return;
@@ -815,8 +818,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(TopkArgs a) {
   c.nk = a.kept[q];
   c.work = a.work + (int64_t)q * L.blk_stride;
   c.sc = a.scores + ((int64_t)q * L.R + r) * L.slot_stride;
-  c.lb = __ffs(L.b) - 1;  // block size is a power of two
-  c.bmask = L.b - 1;
+  c.lb = R1B64 ? 6 : __ffs(L.b) - 1;  // block size is a power of two
+  c.bmask = R1B64 ? 63 : L.b - 1;
   c.n_elem = c.nk << c.lb;
   c.nwords = (c.n_elem + 31) / 32;
   c.bits = reinterpret_cast<uint32_t*>(dyn);
@@ -1048,6 +1051,7 @@ size_t topk_smem_bytes(const Layout& L) {
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const size_t smem = topk_smem_bytes(a.lay);
   cudaError_t e = cudaFuncSetAttribute(k_topk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_topk<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Few (request, row) pairs leave most SMs idle: give each a cluster of up to
@@ -1080,7 +1084,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     cudaGetLastError();  // this shape cannot be placed: one CTA per pair
   }
   PdlLaunch l(dim3(pairs), dim3(kTopkThreads), smem, s);
-  return cudaLaunchKernelEx(&l.cfg, k_topk<false>, a);
+  return cudaLaunchKernelEx(&l.cfg, (a.rows == 1 && a.lay.b == 64) ? k_topk<false, 1> : k_topk<false>, a);
 }
 
 }  // namespace spin
