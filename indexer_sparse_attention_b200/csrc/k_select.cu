@@ -686,14 +686,15 @@ __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t
   if (threadIdx.x == 0) *kept = total;
 }
 
-// R1: one query row known at compile time (the decode step's common case).
-template <int R1>
+// RC: the number of query rows when fixed at compile time (0: a.rows); the
+// decode step's one row and the MTP step's four have their own instances.
+template <int RC>
 __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   pdl_enter();
   StepArgs a = a_in;
   if (a.step_dev) a.step = *a.step_dev + a.step_add;  // the state's counter (read after the predecessors finished)
   const Layout L = a.lay;
-  const int rows = R1 ? 1 : a.rows;
+  const int rows = RC ? RC : a.rows;
   const int q = blockIdx.x;
   extern __shared__ __align__(16) uint8_t dyn[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);
@@ -731,7 +732,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   } else {
     const int64_t n0 = row_blocks(ctx, 0, L.b);
     const int64_t n_exp = explore_count(block_budget(n0, a.sparsity), a.gamma);
-    const int pr = (R1 || a.mtp_row0) ? 1 : rows;  // rows whose predicted sets are unioned
+    const int pr = (RC == 1 || a.mtp_row0) ? 1 : rows;  // rows whose predicted sets are unioned
     if (pr > 1 && select_batched(L.blk_stride, rows)) {
       // every row's keys on chip (row r at kb + r blk_stride), the rows'
       // radix passes together
@@ -1147,6 +1148,7 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   const size_t smem = select_smem(a.lay.blk_stride, a.mtp_row0 ? 1 : a.rows);
   cudaError_t e = cudaFuncSetAttribute(k_select<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Few requests with long contexts leave most SMs idle: a cluster of up to 8
@@ -1173,7 +1175,7 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   }
   PdlLaunch l(dim3(a.lay.Q), dim3(kSelThreads), smem, s);
   l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
-  return cudaLaunchKernelEx(&l.cfg, a.rows == 1 ? k_select<1> : k_select<0>, a);
+  return cudaLaunchKernelEx(&l.cfg, a.rows == 1 ? k_select<1> : a.rows == 4 ? k_select<4> : k_select<0>, a);
 }
 
 // ---------------------------------------------------------------------------
