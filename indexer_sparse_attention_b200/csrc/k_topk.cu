@@ -6,9 +6,12 @@
 // One CTA (1024 threads) per (request, row).  Scores are compared through
 // their order-preserving 32-bit keys.
 //  1. Candidates.  When the score kernel left the maximum of every 32 slots
-//     (the fused decode step), M = the k-th largest group maximum bounds the
-//     k-th score from below; only the groups whose maximum is >= M are read
-//     and their scores >= M kept.  Otherwise a lower threshold comes from the
+//     (the fused decode step) and there are at least two groups per wanted
+//     score, M = the k-th largest group maximum bounds the k-th score from
+//     below; only the groups whose maximum is >= M are read and their scores
+//     >= M kept (compared with the float whose key is M).  With fewer groups
+//     nearly all of them qualify and the list would overflow, so, as without
+//     group maxima, a lower threshold comes from the
 //     13-bit histogram of a fixed 1/16 sample (about 1.3 k keys expected
 //     above it) and one pass over all scored slots keeps the keys above it.
 //     Candidates are (key, position in the ascending kept-slot order) in
