@@ -45,6 +45,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "block_scan.cuh"
 #include "spin_internal.cuh"
@@ -600,9 +601,15 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       int p0;  // ctx_len - 1 < 2^31 (max_slots is an int32)
       float sigma, v, d;
     };
-    struct Side {
+    struct SideData {
       float sigma, v, d;
     };
+    // With four groups (one CTA per SM, several rows) a tile's metadata is
+    // carried from its side loads to its processing, so the tile-info slot is
+    // read once; with two groups the registers are scarcer (two CTAs per SM,
+    // two tiles of prefetch) and it is read again.
+    constexpr bool kCarry = G == 4;
+    using Side = std::conditional_t<kCarry, Pre, SideData>;
     auto info_ready = [&](int i) -> bool {
       return __all_sync(0xffffffffu, wait_parity(B.xf(i & (kAuxSlots - 1)), (uint32_t)(i / kAuxSlots) & 1u, ctl));
     };
@@ -624,13 +631,24 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       int pg;
       const Pre m = meta_of(i, pg);
       Side r;
-      r.sigma = m.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
-      // V of the page's slots past the context too, for its group maxima
-      r.v = (m.upd || (fused && a.vmax && m.pres)) ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
-      r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
+      if constexpr (kCarry) {
+        r = m;
+        // safe addresses instead of predicates, so that nothing waits for
+        // the loads before the tile that uses them: a value that is not
+        // needed (the scale of an invalid slot, V or D of a slot that is not
+        // updated) is read from a valid place and never used
+        r.sigma = __ldg(a.kscale + (int64_t)(m.valid ? pg : 0) * kPage + tok);
+        r.v = fused ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
+        r.d = fused ? a.D[(int64_t)m.q * L.slot_stride + (m.upd ? m.p0 - m.s : 0)] : 0.f;
+      } else {
+        r.sigma = m.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
+        // V of the page's slots past the context too, for its group maxima
+        r.v = (m.upd || (fused && a.vmax && m.pres)) ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
+        r.d = m.upd ? a.D[(int64_t)m.q * L.slot_stride + (m.p0 - m.s)] : 0.f;
+      }
       return r;
     };
-    Side nx1{0.f, 0.f, 0.f}, nx2{0.f, 0.f, 0.f};  // side data of tiles i and i + T
+    Side nx1{}, nx2{};  // side data of tiles i and i + T
     bool alive_ = group < n_local;
     if constexpr (DIST >= 1) {
       if (alive_) {
@@ -666,11 +684,16 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
           nx2 = load_side(i + 2 * tgroups);
         }
       }
-      int pg_unused;
-      Pre cur = meta_of(i, pg_unused);
-      cur.sigma = side.sigma;
-      cur.v = side.v;
-      cur.d = side.d;
+      Pre cur;
+      if constexpr (kCarry) {
+        cur = side;
+      } else {
+        int pg_unused;
+        cur = meta_of(i, pg_unused);
+        cur.sigma = side.sigma;
+        cur.v = side.v;
+        cur.d = side.d;
+      }
       const int xs = i & (kAuxSlots - 1);
       if (cur.q != cur_q) {
         __syncwarp();
@@ -684,7 +707,15 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       if (!__all_sync(0xffffffffu, wait_parity(B.e(stage), phase, ctl))) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
-      for (int r = sub; r < rows; r += share) {
+      // this warp's rows sub, sub + share, ...; with the row count fixed at
+      // compile time the loop unrolls, and one row's reduction and stores
+      // overlap the next row's accumulator loads
+      constexpr int kRowsPerWarp = RC ? (RC + groups_per_tile(G, RC) - 1) / groups_per_tile(G, RC) : 0;
+      const int nrw = kRowsPerWarp ? kRowsPerWarp : (rows - sub + share - 1) / share;
+#pragma unroll
+      for (int k = 0; k < nrw; ++k) {
+        const int r = sub + k * share;
+        if (kRowsPerWarp && r >= rows) break;
         float part[4] = {0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < H; c += 32) {
           uint32_t v[32];
