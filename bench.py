@@ -46,10 +46,12 @@ WORKLOADS = {"serve-96x512K": 2, "mtp-32x128K-r4": 3, "ragged-8Lx8-256K-1M": 4, 
 KEY_BYTES_PER_SLOT = 128 + 4            # E4M3 key row + fp32 scale
 SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write of V and D
 # DRAM traffic of one k_score_tc launch (dram__bytes_read.sum + dram__bytes_write.sum)
-# per kept slot, from one ncu capture of the kernel on 16 requests at 512K, 50% sparsity,
-# fused EMA (traffic grows with kept slots: each is read once), valid for the kernel
-# source with this hash prefix
-SCORE_TRAFFIC = {"src_sha256_16": "49036cef2a6a88d6", "bytes_per_kept_slot": 151.49,
+# per kept slot, from one ncu capture per launch plan (traffic grows with kept slots:
+# each is read once), valid for the kernel source with this hash prefix:
+#   "fused-r1": 16 requests at 512K, 50% sparsity, one row, fused EMA;
+#   "deferred-r4": 32 requests at 128K, 40% sparsity, four MTP rows, no EMA in the launch
+SCORE_TRAFFIC = {"src_sha256_16": "fa9ad90adac50265",
+                 "bytes_per_kept_slot": {"fused-r1": 151.37, "deferred-r4": 146.33},
                  "sources": ("indexer_sparse_attention_b200/csrc/k_score_tc.cu",
                              "indexer_sparse_attention_b200/csrc/spin_internal.cuh")}
 
@@ -247,15 +249,18 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def score_traffic_per_slot():
-    """The captured DRAM bytes per kept slot, or None once the kernel source
-    differs from the one the counters were taken on."""
+def score_traffic_per_slot(plan="fused-r1"):
+    """The captured DRAM bytes per kept slot of a launch plan, or None for a
+    plan without a capture or once the kernel source differs from the one the
+    counters were taken on."""
     import hashlib
     h = hashlib.sha256()
     for f in SCORE_TRAFFIC["sources"]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    return SCORE_TRAFFIC["bytes_per_kept_slot"] if h.hexdigest()[:16] == SCORE_TRAFFIC["src_sha256_16"] else None
+    if h.hexdigest()[:16] != SCORE_TRAFFIC["src_sha256_16"]:
+        return None
+    return SCORE_TRAFFIC["bytes_per_kept_slot"].get(plan)
 
 
 def peaks():
@@ -789,6 +794,9 @@ def workload_arm(args, world, rank, local):
     score_avg = score_ms / max(score_n, 1)
     per_launch = kept / Ly * per_slot
     achieved = per_launch / (score_avg / 1e3) / 1e9
+    # the MTP plan with a capture: four rows of 64 heads, FP8 keys, EMA deferred
+    plan = "deferred-r4" if (R == 4 and wl.key_fp8 and wl.H == 64 and wl.d == 128) else None
+    traffic_slot = score_traffic_per_slot(plan) if plan else None
     out = {
         "metric": METRIC, "value": job_rows_per_s(rows_step * K, world, ms),
         "unit": "rows/s" if Ly == 1 else f"rows/s (a row passes all {Ly} layers)",
@@ -808,7 +816,11 @@ def workload_arm(args, world, rank, local):
         "roofline": {"bound": "hbm", "kernel": ("k_score_tc" if wl.key_fp8 else "k_score_simt"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "avg_launch_ms": score_avg,
-                     "bytes_per_launch": per_launch, "bytes_per_kept_slot": per_slot, "traffic": None},
+                     "bytes_per_launch": per_launch, "bytes_per_kept_slot": per_slot,
+                     "traffic": None if traffic_slot is None else traffic_slot * kept / Ly,
+                     "traffic_source": (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per kept slot "
+                                        f"({plan} capture, scaled by kept slots)" if traffic_slot is not None
+                                        else "null: no capture of this launch plan on the current kernel source")},
         "pipelined": bool(run.lookahead and R == 1 and wl.key_fp8),
         "stage_ms_per_step": {k: v[0] / K for k, v in stages.items() if v[1]},
         "gpu_launches": sum(n for _, n in stages.values()),

@@ -365,11 +365,12 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
   const int H = KH ? KH : L.H;
   const int rows = RC ? RC : a.rows;
   const int N = rows * H;
-  const int stages = plan.stages, nacc = plan.nacc;
+  // the four-group plan is always 8 stages, 2 accumulators, 2 query buffers
+  const int stages = G == 4 ? kMaxStages : plan.stages, nacc = G == 4 ? 2 : plan.nacc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const SmemLayout lay = smem_layout(N, L.Q, stages, plan.nq, G);
-  const int nq = plan.nq;
+  const int nq = G == 4 ? 2 : plan.nq;
   const uint32_t sbase = smem_u32(smem);
   TileInfo* aux = reinterpret_cast<TileInfo*>(smem + lay.aux);
   int* prefix = reinterpret_cast<int*>(smem + lay.prefix);
@@ -819,6 +820,8 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
   if (!encode_2d(fn, &tk, a.keys, (uint64_t)a.num_pages * kPage, kPage)) return cudaErrorInvalidValue;
   if (!encode_2d(fn, &tq, a.q8, (uint64_t)L.Q * N, (uint32_t)N)) return cudaErrorInvalidValue;
   const TcPlan plan = tc_plan(N, L.Q);
+  if (plan.groups == 4 && (plan.stages != kMaxStages || plan.nacc != 2 || plan.nq != 2))
+    return cudaErrorInvalidValue;  // the four-group kernels take this plan as constants
   const uint32_t smem = smem_layout(N, L.Q, plan.stages, plan.nq, plan.groups).total;
   const int dist = prefetch_dist(plan.groups / groups_per_tile(plan.groups, a.rows), plan.nq, plan.nacc,
                                  plan.stages);
@@ -832,7 +835,10 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
                           : k_score_tc<2, 64, 2, 1, 0>;
   if (plan.groups == 2 && dist == 1) kernel = L.H == 64 ? k_score_tc<2, 64, 1> : k_score_tc<2, 0, 1>;
   if (plan.groups == 4 && dist == 1)
-    kernel = L.H == 64 ? (a.rows == 4 ? k_score_tc<4, 64, 1, 4> : k_score_tc<4, 64, 1>) : k_score_tc<4, 0, 1>;
+    kernel = L.H != 64    ? k_score_tc<4, 0, 1>
+             : a.rows != 4 ? k_score_tc<4, 64, 1>
+             : a.V         ? k_score_tc<4, 64, 1, 4, 1>
+                           : k_score_tc<4, 64, 1, 4, 0>;
   if (plan.groups == 4 && dist == 0) kernel = k_score_tc<4, 0, 0>;
   if (!kernel) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
