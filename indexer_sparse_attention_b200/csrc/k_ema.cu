@@ -102,7 +102,7 @@ cudaError_t launch_reset_rows(float* V, float* D, float* vmax, const ReqList& li
 // Grid: column x = request, its gridDim.y blocks' warps take the request's
 // blocks j in turn (no division per block).
 template <int R>
-__global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
+__global__ void __launch_bounds__(256, 4) k_ema_update(EmaArgs a) {
   pdl_enter();
   const Layout L = a.lay;
   const int lane = threadIdx.x & 31;
@@ -142,6 +142,44 @@ __global__ void __launch_bounds__(256) k_ema_update(EmaArgs a) {
       float* V = a.V + (int64_t)q * L.slot_stride;
       float* D = a.D + (int64_t)q * L.slot_stride;
       const float* sc = a.scores + (int64_t)q * L.R * L.slot_stride;
+      if (R > 1 && L.b == 64 && j > 0 && kj && kj1 && (j + 1) * 64 - 1 <= p0) {
+        // A kept block (not block 0) below p0 whose successor is kept too:
+        // every accepted row updates V and D of every slot, so only r < acc
+        // (uniform) is tested.  Two slots per lane; offsets in 32 bits.
+        const int s0 = (int)(j * 64) + lane, p = (int)p0;
+        float v[2], dv[2], sv[2][R], sd[2][R];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          v[h] = V[s0 + 32 * h];
+          dv[h] = D[p - (s0 + 32 * h)];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const float* sr = sc + (int64_t)r * L.slot_stride;
+            sv[h][r] = r < acc ? sr[s0 + 32 * h] : 0.f;
+            sd[h][r] = r < acc ? sr[s0 + 32 * h + r] : 0.f;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int r = 0; r < R; ++r) {  // rows in order
+            if (r < acc) {
+              v[h] = ema_v(v[h], sv[h][r], a.alpha, a.beta);
+              dv[h] = ema_d(dv[h], sd[h][r], a.alpha, a.beta);
+            }
+          }
+          V[s0 + 32 * h] = v[h];
+          D[p - (s0 + 32 * h)] = dv[h];
+        }
+        if (a.vmax) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float g = warp_max(v[h]);
+            if (lane == 0) a.vmax[(int64_t)q * L.vg_stride + ((s0 - lane + 32 * h) >> 5)] = g;
+          }
+        }
+        continue;  // (block 0, which also holds the offsets past p0, takes the general path)
+      }
       // Two slots per lane per pass (i, i + 32): every load of the pass is
       // issued before the first store, so the pass costs one memory latency.
       for (int i0 = lane; i0 < L.b; i0 += 64) {
