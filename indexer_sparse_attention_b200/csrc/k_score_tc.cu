@@ -835,10 +835,8 @@ cudaError_t launch_score_tc(const ScoreArgs& a, void* encode_fn, cudaStream_t s)
                           : k_score_tc<2, 64, 2, 1, 0>;
   if (plan.groups == 2 && dist == 1) kernel = L.H == 64 ? k_score_tc<2, 64, 1> : k_score_tc<2, 0, 1>;
   if (plan.groups == 4 && dist == 1)
-    kernel = L.H != 64    ? k_score_tc<4, 0, 1>
-             : a.rows != 4 ? k_score_tc<4, 64, 1>
-             : a.V         ? k_score_tc<4, 64, 1, 4, 1>
-                           : k_score_tc<4, 64, 1, 4, 0>;
+    // (the EMA is fused for one row only, so four rows come without V)
+    kernel = L.H != 64 ? k_score_tc<4, 0, 1> : (a.rows == 4 && !a.V) ? k_score_tc<4, 64, 1, 4, 0> : k_score_tc<4, 64, 1>;
   if (plan.groups == 4 && dist == 0) kernel = k_score_tc<4, 0, 0>;
   if (!kernel) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
