@@ -285,13 +285,16 @@ def test_topk_bit_exact(R, kind):
 
 
 @pytest.mark.parametrize("R", [1, 2, 3, 4])
-def test_ema_update_prefix_valid_bit_exact(R):
-    rng = np.random.default_rng(40 + R)
+@pytest.mark.parametrize("kept", [0.5, 0.9])
+def test_ema_update_prefix_valid_bit_exact(R, kept):
+    # at 90% most blocks are kept with a kept successor: the replay's path
+    # for those blocks (only r < a tested) against the general one
+    rng = np.random.default_rng(40 + R + int(100 * kept))
     Q = 6
     st = make_state(Q=Q, max_slots=64 * 60, R=R)
     random_state(st, 0, rng, frac_sentinel=0.3)
     ctx = np.array([64 * 60 - R + 1, 64 * 10 + 1, 64 * 10, 1, 65, 64 * 33 + 17], np.int64)
-    m = (rng.uniform(size=(Q, st.mask_stride)) < 0.5).astype(np.uint8)
+    m = (rng.uniform(size=(Q, st.mask_stride)) < kept).astype(np.uint8)
     for qq in range(Q):
         m[qq, oracle.num_blocks(int(ctx[qq]), R - 1, 64):] = 0
     acc = rng.integers(1, R + 1, Q).astype(np.int32)
