@@ -76,6 +76,9 @@ def parse():
     p.add_argument("--lookahead", action="store_true",
                    help="pipelined one-row steps (spin_set_lookahead): each step prepares the next step's "
                         "selection, whose select kernel runs beside the step's top-k")
+    p.add_argument("--prepare-layers", action="store_true",
+                   help="with --lookahead on a multi-layer workload: every layer's selection of a step is made "
+                        "at once (spin_prepare_selections) before the first layer's step")
     p.add_argument("--ablation", choices=["pooling", "mtp", "predictors"], default=None,
                    help="pooling: miss and step time of max / mean / top-4 pooling over target sparsities; "
                         "mtp: p99 miss vs realized sparsity of the two MTP policies on the 4-row workload; "
@@ -632,6 +635,7 @@ class WorkloadRun:
         self.cfg = cfg
         self.st = isa.SpinState(cfg, device=device)
         self.lookahead = False
+        self.prepare = False              # spin_prepare_selections before each step's layers
         self.masks = [self.st.new_mask() for _ in range(Ly)]
         self.topks = [torch.empty((Q, R, wl.topk), dtype=torch.int32, device=device) for _ in range(Ly)]
         self.scores = self.st.new_scores()
@@ -658,6 +662,8 @@ class WorkloadRun:
         prefix-valid EMA replay once the accepted lengths are known."""
         isa, wl, t = self.isa, self.wl, self.t
         R = wl.rows
+        if self.prepare and self.lookahead and layers is None:
+            isa.spin_prepare_selections(self.st, t, self.ctx[t])
         for l in (range(wl.layers) if layers is None else layers):
             c = self.caches[l]
             q, w = self.qw[t][l]
@@ -725,6 +731,7 @@ def workload_arm(args, world, rank, local):
                           mtp_policy=MTP_POLICIES[args.mtp_policy])
     run = WorkloadRun(wl, device, total)
     run.set_lookahead(args.lookahead)   # applies to one-row steps
+    run.prepare = bool(args.prepare_layers and args.lookahead and wl.rows == 1 and wl.key_fp8)
     Ly, Q, R = wl.layers, wl.requests, wl.rows
     # history bootstrap (all-keep), then the workload's warm-up protocol
     run.set_sparsity([0.0] * Ly)
@@ -822,6 +829,7 @@ def workload_arm(args, world, rank, local):
                                         f"({plan} capture, scaled by kept slots)" if traffic_slot is not None
                                         else "null: no capture of this launch plan on the current kernel source")},
         "pipelined": bool(run.lookahead and R == 1 and wl.key_fp8),
+        "layers_prepared_at_once": bool(run.prepare),
         "stage_ms_per_step": {k: v[0] / K for k, v in stages.items() if v[1]},
         "gpu_launches": sum(n for _, n in stages.values()),
         "clocks": clk.summary(),

@@ -127,8 +127,10 @@ typedef struct spin_state_s* spin_state;
  * and request (with max pooling and block_size >= 32 also V's maximum over
  * each aligned 32-slot group, which the prediction reads in place of V for
  * the blocks below the newest one), block-score / work-list / quantised-query / score scratch, the
- * per-layer selection a pipelined step prepares (spin_set_lookahead) and the
- * device error word.  Returns 0 for an invalid config. */
+ * per-layer selection a pipelined step prepares (spin_set_lookahead), one
+ * row of block scores for each of min(num_layers, 4) streams of
+ * spin_prepare_selections, and the device error word.  Returns 0 for an
+ * invalid config. */
 SPIN_API size_t spin_state_bytes(const spin_config* cfg);
 
 /* Creates a state in the caller's device block dev_mem (>= spin_state_bytes,
@@ -283,6 +285,29 @@ SPIN_API spin_status spin_decode_step(spin_state st, int layer, int rows, int64_
  * top-k.  The first call on a state creates the second stream and two events
  * (no device memory); make it outside stream capture. */
 SPIN_API spin_status spin_set_lookahead(spin_state st, int enable);
+
+/* Every layer's one-row selection of one step, made at once (SPIN digest,
+ * arXiv深度剖析: a layer's selection comes from its own EMA history, the
+ * positions and the step, not from the step's queries, so the selections of
+ * all layers are known before the first layer's indexer runs).  Needs
+ * lookahead on (spin_set_lookahead; else SPIN_EINVAL).  For each layer, with
+ * its current target, the predict and select kernels of rows = 1 run for
+ * `step` (>= 0, or SPIN_STEP_DEVICE: the counter's current value) at
+ * ctx_len_dev [Q] (device, slots visible to row 0), into the per-layer slots
+ * the pipelined step uses; the layers are spread over up to four streams of
+ * the state, forked from and joined back into `stream` (the first call
+ * creates the streams and five events, no device memory; make it outside
+ * stream capture).  A layer's next spin_decode_step with rows = 1, no
+ * deferred update, that step, the same ctx_len and the same target then
+ * scores this selection, runs its top-k on `stream` and prepares no next
+ * selection; results are bit-identical to the sequential step's.  A request
+ * whose ctx_len differs at the step sets ERR_LOOKAHEAD as for the pipelined
+ * step; a different step or target, spin_ema_update, spin_reset_requests or
+ * spin_state_import makes the step select afresh.  Argument errors return
+ * SPIN_EINVAL and launch nothing; device-side errors go to the error word as
+ * for spin_predict_select. */
+SPIN_API spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* ctx_len_dev,
+                                             spin_stream_t stream);
 
 /* Predictor-quality profile (SPIN listing, Table 1 compares predictors of the
  * indexer's scores by Pearson correlation and top-k recall).

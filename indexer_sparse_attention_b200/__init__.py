@@ -23,7 +23,7 @@ __all__ = [
     "spin_decode_step", "spin_miss_count", "spin_allocate_layer_sparsity", "spin_get_error",
     "spin_set_layer_sparsity", "spin_set_score_kernel", "spin_reset_requests", "spin_set_fault_injection",
     "spin_state_export", "spin_state_import", "spin_status_string", "spin_set_kernel_timing",
-    "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_topk_noalloc_error", "spin_set_lookahead", "spin_set_kernel_timing_mask",
+    "spin_kernel_times", "STAGES", "spin_topk_noalloc", "spin_topk_noalloc_error", "spin_set_lookahead", "spin_prepare_selections", "spin_set_kernel_timing_mask",
     "SPIN_STEP_DEVICE", "spin_set_step", "spin_advance_step", "SPIN_POOL_MAX", "SPIN_POOL_MEAN", "SPIN_POOL_TOP4",
     "SPIN_MTP_UNION_PREFIX", "SPIN_MTP_ROW0", "SPIN_PRED_EMA", "SPIN_PRED_RANDOM", "spin_slot_prediction",
     "spin_pearson", "spin_topk_overlap",
@@ -91,6 +91,7 @@ def load():
         "spin_set_kernel_timing_mask": (S, [_vp, _u32]),
         "spin_set_step": (S, [_vp, _i64, _vp]),
         "spin_set_lookahead": (S, [_vp, ctypes.c_int]),
+        "spin_prepare_selections": (S, [_vp, _i64, _vp, _vp]),
         "spin_advance_step": (S, [_vp, _vp]),
         "spin_kernel_times": (S, [_vp, _vp, _vp, ctypes.c_int]),
         "spin_reset_requests": (S, [_vp, ctypes.c_int, _vp, ctypes.c_int, _vp]),
@@ -308,6 +309,14 @@ def spin_reset_requests(st: SpinState, layer: int, requests, stream=None) -> Non
     req = (ctypes.c_int32 * len(requests))(*[int(r) for r in requests])
     _check(load().spin_reset_requests(st.handle, layer, ctypes.cast(req, _vp), len(requests), _stream(stream)),
            "spin_reset_requests")
+
+
+def spin_prepare_selections(st: SpinState, step: int, ctx_len: torch.Tensor, stream=None) -> None:
+    """Every layer's one-row selection of `step`, made at once on the state's
+    prepare streams; each layer's next pipelined decode step scores it (see
+    include/spin.h)."""
+    _check(load().spin_prepare_selections(st.handle, step, _dev(ctx_len, "ctx_len", torch.int32), _stream(stream)),
+           "spin_prepare_selections")
 
 
 def spin_predict_select(st: SpinState, layer: int, rows: int, step: int, ctx_len: torch.Tensor,

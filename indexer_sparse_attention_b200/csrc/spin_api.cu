@@ -12,6 +12,9 @@
 
 using namespace spin;
 
+// Streams spin_prepare_selections spreads the layers over (created on first use).
+constexpr int kPrepStreams = 4;
+
 struct spin_state_s {
   spin_config cfg;
   Layout lay;
@@ -50,6 +53,7 @@ struct spin_state_s {
     bool ready;
     int64_t step;                    // the step the selection is for (SPIN_STEP_DEVICE: the counter's)
     float sparsity;                  // the layer's target it was made with
+    bool batch;                      // made by spin_prepare_selections: the step prepares no next one
   };
   std::vector<Prepared> prep;        // per layer
   int32_t* la_work;                  // [L][Q][blk_stride] kept block ids of the prepared selection
@@ -60,6 +64,12 @@ struct spin_state_s {
   int32_t* tk_work;                  // [Q][blk_stride] the top-k's copy of the selection it reads, so that
   int32_t* tk_kept;                  // [Q]   the next selection can be written while it runs
   int32_t* tk_ctx;                   // [Q]
+  // spin_prepare_selections: every layer's predict + select on prep_k
+  // streams at once, each stream with its own block-score scratch
+  int prep_k;
+  float* prep_S;                     // [prep_k][Q][blk_stride]
+  cudaStream_t pstream[kPrepStreams];
+  cudaEvent_t pev[kPrepStreams + 1]; // [0]: the fork; [1 + i]: stream i done
   uint32_t magic;
 };
 
@@ -121,8 +131,10 @@ int64_t gmax_stride(const Layout& L) { return L.blk_stride * std::max(1, L.b / 3
 
 struct Carve {
   size_t err, V, D, vmax, S, work, kept, q8, wq, scores, gmax, step, la_work, la_kept, la_mask, la_ctx, ctx_next, tk_work,
-      tk_kept, tk_ctx, total;
+      tk_kept, tk_ctx, prep_S, total;
 };
+
+int prep_streams(const Layout& L) { return (int)std::min<int64_t>(L.L, kPrepStreams); }
 
 Carve carve(const Layout& L) {
   Carve k;
@@ -148,6 +160,7 @@ Carve carve(const Layout& L) {
   k.tk_work = take((size_t)L.Q * L.blk_stride * 4);
   k.tk_kept = take((size_t)L.Q * 4);
   k.tk_ctx = take((size_t)L.Q * 4);
+  k.prep_S = take((size_t)prep_streams(L) * L.Q * L.blk_stride * 4);
   k.total = off;
   return k;
 }
@@ -338,6 +351,7 @@ spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const 
   };
   spin_status r;
   P.ready = P.ready && P.sparsity == sp && P.step == step;
+  const bool batch = P.ready && P.batch;  // made by spin_prepare_selections for this step alone
   if (!P.ready) {  // no selection prepared for this step: make it now
     StepArgs a = select_args(ctx_len, step, false);
     if (sp > 0.0f) {
@@ -353,6 +367,16 @@ spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const 
   r = run_score(st, layer, 1, keys, key_scale, num_pages, block_table, bt_stride, q, w, ctx_len, lmask, scores,
                 true, s, &gm, false, &sel);
   if (r != SPIN_OK) return r;
+  if (batch) {
+    // the next selection of this layer comes from the next spin_prepare_selections:
+    // the top-k reads this one in place, on this stream
+    P.batch = false;
+    cudaError_t e = cudaMemcpyAsync(mask_dev, lmask, (size_t)L.Q * L.max_blocks, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    TopkArgs t{L, 1, scores, mask_dev, ctx_len, work, kept, topk_dev, st->err, gm ? st->gmax : nullptr,
+               st->gstride, lctx};
+    return cuda_status(staged(st, kTopk, s, [&] { return launch_topk(t, s); }));
+  }
   // fork: the side stream copies the selection the top-k reads, and the mask
   cudaError_t e = cudaEventRecord(st->ev_scored, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st->side, st->ev_scored, 0);
@@ -386,6 +410,7 @@ spin_status decode_step_lookahead(spin_state st, int layer, int64_t step, const 
   P.ready = true;
   P.step = next;
   P.sparsity = sp;
+  P.batch = false;
   return SPIN_OK;
 }
 
@@ -433,10 +458,14 @@ spin_status spin_state_create(const spin_config* cfg, void* dev_mem, size_t byte
   st->tk_work = (int32_t*)(st->base + k.tk_work);
   st->tk_kept = (int32_t*)(st->base + k.tk_kept);
   st->tk_ctx = (int32_t*)(st->base + k.tk_ctx);
+  st->prep_k = prep_streams(L);
+  st->prep_S = (float*)(st->base + k.prep_S);
+  for (int i = 0; i < kPrepStreams; ++i) st->pstream[i] = nullptr;
+  for (int i = 0; i <= kPrepStreams; ++i) st->pev[i] = nullptr;
   st->lookahead = 0;
   st->side = nullptr;
   st->ev_scored = st->ev_copied = st->ev_topk = nullptr;
-  st->prep.assign(cfg->num_layers, spin_state_s::Prepared{false, 0, 0.0f});
+  st->prep.assign(cfg->num_layers, spin_state_s::Prepared{false, 0, 0.0f, false});
   st->sparsity.assign(cfg->num_layers, cfg->target_sparsity);
   st->score_kernel = SPIN_SCORE_AUTO;
   st->inject = 0;
@@ -474,6 +503,10 @@ spin_status spin_state_destroy(spin_state st) {
   for (cudaEvent_t e : {st->ev_scored, st->ev_copied, st->ev_topk})
     if (e) cudaEventDestroy(e);
   if (st->side) cudaStreamDestroy(st->side);
+  for (int i = 0; i <= kPrepStreams; ++i)
+    if (st->pev[i]) cudaEventDestroy(st->pev[i]);
+  for (int i = 0; i < kPrepStreams; ++i)
+    if (st->pstream[i]) cudaStreamDestroy(st->pstream[i]);
   st->magic = 0;
   delete st;
   return SPIN_OK;
@@ -511,6 +544,50 @@ spin_status spin_set_lookahead(spin_state st, int enable) {
   st->lookahead = enable;
   for (auto& p : st->prep) p.ready = false;
   return SPIN_OK;
+}
+
+spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* ctx_len_dev, spin_stream_t stream) {
+  if (!alive(st)) return SPIN_ESTATE;
+  if (!st->lookahead || !ctx_len_dev || (step < 0 && step != SPIN_STEP_DEVICE)) return SPIN_EINVAL;
+  const Layout& L = st->lay;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i <= st->prep_k && e == cudaSuccess; ++i)
+    if (!st->pev[i]) e = cudaEventCreateWithFlags(&st->pev[i], cudaEventDisableTiming);
+  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i)
+    if (!st->pstream[i]) e = cudaStreamCreateWithFlags(&st->pstream[i], cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventRecord(st->pev[0], s);  // fork: after everything before on `stream`
+  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(st->pstream[i], st->pev[0], 0);
+  if (e != cudaSuccess) return cuda_status(e);
+  // layer l on stream l mod prep_k, whose block scores only its own layers use
+  for (int layer = 0; layer < L.L; ++layer) {
+    const int i = layer % st->prep_k;
+    cudaStream_t ps = st->pstream[i];
+    spin_state_s::Prepared& P = st->prep[layer];
+    P.ready = false;
+    StepArgs a = step_args(st, layer, 1, step, ctx_len_dev, st->la_mask + (size_t)layer * L.Q * L.max_blocks);
+    a.S = st->prep_S + (size_t)i * L.Q * L.blk_stride;
+    a.work = st->la_work + (size_t)layer * L.Q * L.blk_stride;
+    a.kept = st->la_kept + (size_t)layer * L.Q;
+    a.ctx_sel = st->la_ctx + (size_t)layer * L.Q;
+    a.no_pdl = layer < st->prep_k ? 1 : 0;  // a stream's first launch follows the fork's wait
+    spin_status r = SPIN_OK;
+    if (a.sparsity > 0.0f) {
+      r = cuda_status(staged(st, kPredict, ps, [&] { return launch_predict_pool(a, ps); }));
+      a.no_pdl = 0;
+    }
+    if (r == SPIN_OK) r = cuda_status(staged(st, kSelect, ps, [&] { return launch_select(a, ps); }));
+    if (r != SPIN_OK) return r;
+    P.ready = true;
+    P.batch = true;
+    P.step = step;
+    P.sparsity = st->sparsity[layer];
+  }
+  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) {  // join
+    e = cudaEventRecord(st->pev[1 + i], st->pstream[i]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->pev[1 + i], 0);
+  }
+  return cuda_status(e);
 }
 
 spin_status spin_set_step(spin_state st, int64_t step, spin_stream_t stream) {

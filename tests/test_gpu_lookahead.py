@@ -172,3 +172,77 @@ def test_lookahead_reports_a_broken_ctx_contract():
         keep = [0, 1, 3, 4]
         assert torch.equal(res[0][keep], res[1][keep])
     assert isa.spin_get_error(seq)[0] == 0
+
+
+@pytest.mark.parametrize("device_step", [False, True])
+def test_prepared_selections_match_sequential_steps(device_step):
+    """spin_prepare_selections makes every layer's selection of a step up
+    front, over up to four streams (five layers: one stream takes two), and
+    each layer's step then scores it.  Masks, top-k and EMA state equal the
+    sequential steps', also on steps without a preparation (the pipelined
+    path runs instead), after a target change that drops a prepared
+    selection, and on all-keep steps."""
+    wl = _wl(steps=7)
+    Ly = 5
+    caches = [workloads.make_key_cache(wl, l, "cuda") for l in range(Ly)]
+    qw = [workloads.make_queries(wl, l, wl.steps, "cuda") for l in range(Ly)]
+    ctx0 = torch.tensor(wl.ctx0, dtype=torch.int64, device="cuda")
+    Q, k = wl.requests, wl.topk
+    sts = []
+    for prep in (False, True):
+        cfg = isa.make_config(num_layers=Ly, num_requests=wl.requests, max_slots=wl.max_slots, topk=wl.topk,
+                              target_sparsity=wl.sparsity, gamma=wl.gamma, seed=wl.seed)
+        st = isa.SpinState(cfg)
+        if prep:
+            isa.spin_set_lookahead(st, True)
+        isa.spin_set_step(st, 0)
+        sts.append(st)
+    seq, pre = sts
+    base = [0.5, 0.4, 0.6, 0.5, 0.3]
+    sched = [[0.0] * Ly, base, base, [0.0] + base[1:], base, base, base]
+    prepared = {1, 2, 3, 5, 6}            # step 4 takes the pipelined path
+    for t in range(wl.steps):
+        ctx = (ctx0 + t + 1).to(torch.int32)
+        step = isa.SPIN_STEP_DEVICE if device_step else t
+        for st in sts:
+            isa.spin_set_layer_sparsity(st, sched[t])
+        if t in prepared:
+            isa.spin_prepare_selections(pre, step, ctx)
+        if t == 5:                        # layer 2's target changes after its preparation
+            changed = list(sched[t])
+            changed[2] = 0.45
+            for st in sts:
+                isa.spin_set_layer_sparsity(st, changed)
+        for l in range(Ly):
+            q, w = qw[l][0][:, t:t + 1].contiguous(), qw[l][1][:, t:t + 1].contiguous()
+            c = caches[l]
+            outs = []
+            for st in sts:
+                mask = st.new_mask()
+                topk = torch.full((Q, 1, k), -7, dtype=torch.int32, device="cuda")
+                isa.spin_decode_step(st, l, 1, step, c.keys, c.kscale, c.block_table, q, w, ctx, False, mask, topk)
+                outs.append((mask, topk))
+            torch.cuda.synchronize()
+            assert torch.equal(outs[0][0], outs[1][0]), f"mask differs at step {t}, layer {l}"
+            assert torch.equal(outs[0][1], outs[1][1]), f"top-k differs at step {t}, layer {l}"
+        if device_step:
+            for st in sts:
+                isa.spin_advance_step(st)
+        for l in range(Ly):
+            for a, b in zip(seq.ema(l), pre.ema(l)):
+                assert torch.equal(a.view(torch.int32), b.view(torch.int32)), f"state differs at step {t}, layer {l}"
+    assert isa.spin_get_error(seq)[0] == 0 and isa.spin_get_error(pre)[0] == 0
+
+
+def test_prepare_selections_needs_lookahead():
+    cfg = isa.make_config(num_layers=2, num_requests=2, max_slots=64 * 40, topk=256)
+    st = isa.SpinState(cfg)
+    ctx = torch.full((2,), 100, dtype=torch.int32, device="cuda")
+    with pytest.raises(isa.SpinError):
+        isa.spin_prepare_selections(st, 0, ctx)
+    isa.spin_set_lookahead(st, True)
+    with pytest.raises(isa.SpinError):
+        isa.spin_prepare_selections(st, -5, ctx)
+    isa.spin_prepare_selections(st, 0, ctx)
+    torch.cuda.synchronize()
+    assert isa.spin_get_error(st)[0] == 0
