@@ -128,7 +128,7 @@ typedef struct spin_state_s* spin_state;
  * each aligned 32-slot group, which the prediction reads in place of V for
  * the blocks below the newest one), block-score / work-list / quantised-query / score scratch, the
  * per-layer selection a pipelined step prepares (spin_set_lookahead), one
- * row of block scores for each of min(num_layers, 4) streams of
+ * row of block scores for each of min(num_layers, 8) streams of
  * spin_prepare_selections, and the device error word.  Returns 0 for an
  * invalid config. */
 SPIN_API size_t spin_state_bytes(const spin_config* cfg);
@@ -294,9 +294,9 @@ SPIN_API spin_status spin_set_lookahead(spin_state st, int enable);
  * its current target, the predict and select kernels of rows = 1 run for
  * `step` (>= 0, or SPIN_STEP_DEVICE: the counter's current value) at
  * ctx_len_dev [Q] (device, slots visible to row 0), into the per-layer slots
- * the pipelined step uses; the layers are spread over up to four streams of
+ * the pipelined step uses; the layers are spread over up to eight streams of
  * the state, forked from and joined back into `stream` (the first call
- * creates the streams and five events, no device memory; make it outside
+ * creates the streams and nine events, no device memory; make it outside
  * stream capture).  A layer's next spin_decode_step with rows = 1, no
  * deferred update, that step, the same ctx_len and the same target then
  * scores this selection, runs its top-k on `stream` and prepares no next

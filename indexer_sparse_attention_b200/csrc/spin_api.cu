@@ -13,7 +13,7 @@
 using namespace spin;
 
 // Streams spin_prepare_selections spreads the layers over (created on first use).
-constexpr int kPrepStreams = 4;
+constexpr int kPrepStreams = 8;
 
 struct spin_state_s {
   spin_config cfg;

@@ -177,13 +177,12 @@ def test_lookahead_reports_a_broken_ctx_contract():
 @pytest.mark.parametrize("device_step", [False, True])
 def test_prepared_selections_match_sequential_steps(device_step):
     """spin_prepare_selections makes every layer's selection of a step up
-    front, over up to four streams (five layers: one stream takes two), and
-    each layer's step then scores it.  Masks, top-k and EMA state equal the
+    front, over up to eight streams, and each layer's step then scores it.  Masks, top-k and EMA state equal the
     sequential steps', also on steps without a preparation (the pipelined
     path runs instead), after a target change that drops a prepared
     selection, and on all-keep steps."""
     wl = _wl(steps=7)
-    Ly = 5
+    Ly = 9                                # one stream takes two layers
     caches = [workloads.make_key_cache(wl, l, "cuda") for l in range(Ly)]
     qw = [workloads.make_queries(wl, l, wl.steps, "cuda") for l in range(Ly)]
     ctx0 = torch.tensor(wl.ctx0, dtype=torch.int64, device="cuda")
@@ -198,7 +197,7 @@ def test_prepared_selections_match_sequential_steps(device_step):
         isa.spin_set_step(st, 0)
         sts.append(st)
     seq, pre = sts
-    base = [0.5, 0.4, 0.6, 0.5, 0.3]
+    base = [0.5, 0.4, 0.6, 0.5, 0.3, 0.5, 0.45, 0.5, 0.55]
     sched = [[0.0] * Ly, base, base, [0.0] + base[1:], base, base, base]
     prepared = {1, 2, 3, 5, 6}            # step 4 takes the pipelined path
     for t in range(wl.steps):
