@@ -127,9 +127,10 @@ typedef struct spin_state_s* spin_state;
  * and request (with max pooling and block_size >= 32 also V's maximum over
  * each aligned 32-slot group, which the prediction reads in place of V for
  * the blocks below the newest one), block-score / work-list / quantised-query / score scratch, the
- * per-layer selection a pipelined step prepares (spin_set_lookahead), one
- * row of block scores for each of min(num_layers, 8) streams of
- * spin_prepare_selections, and the device error word.  Returns 0 for an
+ * per-layer selection a pipelined step prepares (spin_set_lookahead), a
+ * block-score scratch (as large as the one above) for each of
+ * min(num_layers, 8) streams of spin_prepare_selections, and the device
+ * error word.  Returns 0 for an
  * invalid config. */
 SPIN_API size_t spin_state_bytes(const spin_config* cfg);
 

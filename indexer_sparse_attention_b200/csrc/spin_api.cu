@@ -67,7 +67,7 @@ struct spin_state_s {
   // spin_prepare_selections: every layer's predict + select on prep_k
   // streams at once, each stream with its own block-score scratch
   int prep_k;
-  float* prep_S;                     // [prep_k][Q][blk_stride]
+  float* prep_S;                     // [prep_k][Q][max_rows][blk_stride] (the block-score layout)
   cudaStream_t pstream[kPrepStreams];
   cudaEvent_t pev[kPrepStreams + 1]; // [0]: the fork; [1 + i]: stream i done
   uint32_t magic;
@@ -160,7 +160,7 @@ Carve carve(const Layout& L) {
   k.tk_work = take((size_t)L.Q * L.blk_stride * 4);
   k.tk_kept = take((size_t)L.Q * 4);
   k.tk_ctx = take((size_t)L.Q * 4);
-  k.prep_S = take((size_t)prep_streams(L) * L.Q * L.blk_stride * 4);
+  k.prep_S = take((size_t)prep_streams(L) * L.Q * L.R * L.blk_stride * 4);
   k.total = off;
   return k;
 }
@@ -566,7 +566,7 @@ spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* 
     spin_state_s::Prepared& P = st->prep[layer];
     P.ready = false;
     StepArgs a = step_args(st, layer, 1, step, ctx_len_dev, st->la_mask + (size_t)layer * L.Q * L.max_blocks);
-    a.S = st->prep_S + (size_t)i * L.Q * L.blk_stride;
+    a.S = st->prep_S + (size_t)i * L.Q * L.R * L.blk_stride;
     a.work = st->la_work + (size_t)layer * L.Q * L.blk_stride;
     a.kept = st->la_kept + (size_t)layer * L.Q;
     a.ctx_sel = st->la_ctx + (size_t)layer * L.Q;

@@ -59,7 +59,7 @@ def _expected_bytes(L, Q, R, H, d, b, max_slots, pooling=0):
              # the selection a pipelined step prepares for the next one, per layer, and ctx_len + 1
              L * Q * blk * 4, L * Q * 4, L * Q * mb, L * Q * 4, Q * 4,
              Q * blk * 4, Q * 4, Q * 4,  # and the top-k's copy of the kept lists
-             min(L, 8) * Q * blk * 4]    # block scores of the streams of spin_prepare_selections
+             min(L, 8) * Q * R * blk * 4]  # block scores of the streams of spin_prepare_selections
     return sum(a(p) for p in parts)
 
 

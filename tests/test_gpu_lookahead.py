@@ -174,13 +174,14 @@ def test_lookahead_reports_a_broken_ctx_contract():
     assert isa.spin_get_error(seq)[0] == 0
 
 
-@pytest.mark.parametrize("device_step", [False, True])
-def test_prepared_selections_match_sequential_steps(device_step):
+@pytest.mark.parametrize("device_step,max_rows", [(False, 1), (True, 1), (False, 4)])
+def test_prepared_selections_match_sequential_steps(device_step, max_rows):
     """spin_prepare_selections makes every layer's selection of a step up
     front, over up to eight streams, and each layer's step then scores it.  Masks, top-k and EMA state equal the
     sequential steps', also on steps without a preparation (the pipelined
     path runs instead), after a target change that drops a prepared
-    selection, and on all-keep steps."""
+    selection, and on all-keep steps; also in a state made for four MTP rows,
+    whose block-score layout is four rows wide."""
     wl = _wl(steps=7)
     Ly = 9                                # one stream takes two layers
     caches = [workloads.make_key_cache(wl, l, "cuda") for l in range(Ly)]
@@ -190,7 +191,7 @@ def test_prepared_selections_match_sequential_steps(device_step):
     sts = []
     for prep in (False, True):
         cfg = isa.make_config(num_layers=Ly, num_requests=wl.requests, max_slots=wl.max_slots, topk=wl.topk,
-                              target_sparsity=wl.sparsity, gamma=wl.gamma, seed=wl.seed)
+                              target_sparsity=wl.sparsity, gamma=wl.gamma, seed=wl.seed, max_rows=max_rows)
         st = isa.SpinState(cfg)
         if prep:
             isa.spin_set_lookahead(st, True)
