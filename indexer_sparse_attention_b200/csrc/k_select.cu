@@ -193,9 +193,11 @@ __global__ void __launch_bounds__(256, 4) k_predict_pool(StepArgs a) {
 // block's groups reduce with shuffles.  Lanes 0 .. NB-1 store the chunk's
 // block scores, one coalesced store.
 // ---------------------------------------------------------------------------
-template <int B>
-__global__ void __launch_bounds__(256, 4) k_predict_max_r1(StepArgs a) {
+template <int B, bool ML = false>
+__global__ void __launch_bounds__(256, 4) k_predict_max_r1(StepArgs a_in) {
   pdl_enter();
+  StepArgs a = a_in;
+  if constexpr (ML) layer_of_block(a);  // ML: one launch over several layers
   constexpr int NB = 1024 / B;                 // blocks per chunk
   constexpr int LPS = B / 4 < 32 ? B / 4 : 32;  // lanes of a block's run in one load instruction
   constexpr int IPB = B / 4 > 32 ? B / 128 : 1;  // load instructions per block (B = 256: 2)
@@ -408,6 +410,19 @@ cudaError_t launch_predict_pool(const StepArgs& a, cudaStream_t s) {
   PdlLaunch l(dim3((unsigned)a.lay.Q, (unsigned)gx), dim3(256), 0, s);
   l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
   void (*k)(StepArgs) = nullptr;
+  if (a.nl > 1) {  // several layers: one row, max pooling with V's group maxima only
+    if (a.nl > kMaxLayerBatch || a.rows != 1 || a.mtp_row0 || a.pooling != SPIN_POOL_MAX || !a.vmax)
+      return cudaErrorInvalidValue;
+    // a few blocks per (layer, request) and SM, each warp looping over its chunks: a grid
+    // sized by the longest context would be mostly blocks with nothing to do
+    int64_t cy = (a.lay.slot_stride + 8 * 1024 - 1) / (8 * 1024);
+    cy = std::max<int64_t>(1, std::min<int64_t>(cy, (148 * 8 + a.lay.Q * a.nl - 1) / (a.lay.Q * a.nl)));
+    PdlLaunch m(dim3((unsigned)a.lay.Q, (unsigned)std::min<int64_t>(cy, 65535), (unsigned)a.nl), dim3(256), 0, s);
+    m.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
+    k = a.lay.b == 32 ? k_predict_max_r1<32, true> : a.lay.b == 64 ? k_predict_max_r1<64, true>
+      : a.lay.b == 128 ? k_predict_max_r1<128, true> : k_predict_max_r1<256, true>;
+    return cudaLaunchKernelEx(&m.cfg, k, a);
+  }
   if (a.pooling == SPIN_POOL_MAX && a.vmax && (a.mtp_row0 || a.rows == 1)) {
     // one 1,024-slot chunk per warp, many short blocks: the hardware hands
     // them to SMs as they free up, so the kernel also fills the SMs another
@@ -688,10 +703,11 @@ __device__ void compact_row(const uint8_t* m, int n_last, int32_t* work, int32_t
 
 // RC: the number of query rows when fixed at compile time (0: a.rows); the
 // decode step's one row and the MTP step's four have their own instances.
-template <int RC>
+template <int RC, bool ML = false>
 __global__ void __launch_bounds__(kSelThreads) k_select(StepArgs a_in) {
   pdl_enter();
   StepArgs a = a_in;
+  if constexpr (ML) layer_of_block(a);  // ML: one launch over several layers
   if (a.step_dev) a.step = *a.step_dev + a.step_add;  // the state's counter (read after the predecessors finished)
   const Layout L = a.lay;
   const int rows = RC ? RC : a.rows;
@@ -1149,8 +1165,16 @@ cudaError_t launch_select(const StepArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k_select<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_select<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if (a.nl > 1) {  // several layers of one-row steps: one CTA per (layer, request)
+    if (a.nl > kMaxLayerBatch || a.rows != 1 || a.mtp_row0) return cudaErrorInvalidValue;
+    PdlLaunch l(dim3(a.lay.Q, 1, a.nl), dim3(kSelThreads), smem, s);
+    l.attr[0].val.programmaticStreamSerializationAllowed = a.no_pdl ? 0 : 1;
+    return cudaLaunchKernelEx(&l.cfg, k_select<1, true>, a);
+  }
   // Few requests with long contexts leave most SMs idle: a cluster of up to 8
   // CTAs per request, each keeping >= 2048 blocks (below that the cluster
   // barriers cost more than the split saves).  A cluster shape the device

@@ -210,6 +210,9 @@ StepArgs step_args(spin_state st, int layer, int rows, int64_t step, const int32
   a.w = nullptr;
   a.q_bf16 = st->cfg.q_dtype == SPIN_BF16;
   a.q8 = nullptr;
+  a.nl = 1;
+  a.state_stride = a.vg_layer_stride = a.s_stride = a.mask_stride = a.work_stride = a.req_stride = 0;
+  for (int i = 0; i < kMaxLayerBatch; ++i) a.sp[i] = 0.0f;
   a.wq = nullptr;
   return a;
 }
@@ -559,7 +562,52 @@ spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* 
   if (e == cudaSuccess) e = cudaEventRecord(st->pev[0], s);  // fork: after everything before on `stream`
   for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(st->pstream[i], st->pev[0], 0);
   if (e != cudaSuccess) return cuda_status(e);
-  // layer l on stream l mod prep_k, whose block scores only its own layers use
+  if (st->cfg.pooling == SPIN_POOL_MAX && vmax_of(st, 0)) {
+    // one predict and one select launch over up to eight layers at a time
+    // (a layer's place in the launch picks its state, scratch and target)
+    spin_status r = SPIN_OK;
+    for (int l0 = 0; l0 < L.L && r == SPIN_OK; l0 += kMaxLayerBatch) {
+      const int nl = std::min(kMaxLayerBatch, L.L - l0);
+      StepArgs a = step_args(st, l0, 1, step, ctx_len_dev, st->la_mask + (size_t)l0 * L.Q * L.max_blocks);
+      a.nl = nl;
+      a.S = st->prep_S;
+      a.work = st->la_work + (size_t)l0 * L.Q * L.blk_stride;
+      a.kept = st->la_kept + (size_t)l0 * L.Q;
+      a.ctx_sel = st->la_ctx + (size_t)l0 * L.Q;
+      a.state_stride = (int64_t)L.Q * L.slot_stride;
+      a.vg_layer_stride = (int64_t)L.Q * L.vg_stride;
+      a.s_stride = (int64_t)L.Q * L.R * L.blk_stride;
+      a.mask_stride = (int64_t)L.Q * L.max_blocks;
+      a.work_stride = (int64_t)L.Q * L.blk_stride;
+      a.req_stride = L.Q;
+      bool any = false;
+      for (int i = 0; i < nl; ++i) {
+        a.sp[i] = st->sparsity[l0 + i];
+        any = any || a.sp[i] > 0.0f;
+        st->prep[l0 + i].ready = false;
+      }
+      a.no_pdl = 1;  // follows the fork's wait
+      if (any) {
+        r = cuda_status(staged(st, kPredict, st->pstream[0], [&] { return launch_predict_pool(a, st->pstream[0]); }));
+        a.no_pdl = 0;
+      }
+      if (r == SPIN_OK)
+        r = cuda_status(staged(st, kSelect, st->pstream[0], [&] { return launch_select(a, st->pstream[0]); }));
+      for (int i = 0; i < nl && r == SPIN_OK; ++i) {
+        spin_state_s::Prepared& P = st->prep[l0 + i];
+        P.ready = true;
+        P.batch = true;
+        P.step = step;
+        P.sparsity = st->sparsity[l0 + i];
+      }
+    }
+    for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) {  // join
+      e = cudaEventRecord(st->pev[1 + i], st->pstream[i]);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->pev[1 + i], 0);
+    }
+    return r != SPIN_OK ? r : cuda_status(e);
+  }
+  // other poolings: layer l on stream l mod prep_k, whose block scores only its own layers use
   for (int layer = 0; layer < L.L; ++layer) {
     const int i = layer % st->prep_k;
     cudaStream_t ps = st->pstream[i];

@@ -226,6 +226,8 @@ struct PdlLaunch {
 // ---------------------------------------------------------------------------
 // Kernel launchers (one per .cu file).  All return cudaGetLastError().
 // ---------------------------------------------------------------------------
+constexpr int kMaxLayerBatch = 8;  // layers in one launch of the prepared selections
+
 struct StepArgs {
   Layout lay;
   int layer, rows;
@@ -256,7 +258,30 @@ struct StepArgs {
   int q_bf16;
   uint8_t* q8;
   float* wq;
+  // Several layers in one launch (prepared selections; one-row max-pooled
+  // predict and the one-CTA select): blockIdx.z is the layer's place in the
+  // batch, every per-layer pointer above advances by its stride per place,
+  // and the layer's target is sp[place].  nl = 1: the fields above are the
+  // one layer's.
+  int nl;
+  int64_t state_stride, vg_layer_stride, s_stride, mask_stride, work_stride, req_stride;
+  float sp[kMaxLayerBatch];
 };
+
+// The layer of this block in a launch over several layers (StepArgs::nl).
+__device__ __forceinline__ void layer_of_block(StepArgs& a) {
+  const int l = (int)blockIdx.z;
+  a.layer += l;
+  a.sparsity = a.sp[l];
+  a.V += l * a.state_stride;
+  a.D += l * a.state_stride;
+  if (a.vmax) a.vmax += l * a.vg_layer_stride;
+  a.S += l * a.s_stride;
+  a.mask += l * a.mask_stride;
+  a.work += l * a.work_stride;
+  a.kept += l * a.req_stride;
+  if (a.ctx_sel) a.ctx_sel += l * a.req_stride;
+}
 
 // V = +inf, D = -inf over n slots, and vmax (nv groups, or null) = +inf.
 cudaError_t launch_init_state(float* V, float* D, int64_t n, float* vmax, int64_t nv, cudaStream_t s);
