@@ -295,12 +295,12 @@ SPIN_API spin_status spin_set_lookahead(spin_state st, int enable);
  * its current target, the predict and select kernels of rows = 1 run for
  * `step` (>= 0, or SPIN_STEP_DEVICE: the counter's current value) at
  * ctx_len_dev [Q] (device, slots visible to row 0), into the per-layer slots
- * the pipelined step uses: with max pooling one predict and one select
- * launch cover up to eight layers at a time, with the other poolings the
- * layers are spread over up to eight streams; the work runs on streams of
- * the state forked from and joined back into `stream` (the first call
- * creates the streams and nine events, no device memory; make it outside
- * stream capture).  A layer's next spin_decode_step with rows = 1, no
+ * the pipelined step uses.  With max pooling (and block_size >= 32) one
+ * predict and one select launch on `stream` cover up to eight layers at a
+ * time; with the other poolings the layers' kernels are spread over up to
+ * eight streams of the state, forked from and joined back into `stream` (the
+ * first such call creates the streams and nine events, no device memory;
+ * make it outside stream capture).  A layer's next spin_decode_step with rows = 1, no
  * deferred update, that step, the same ctx_len and the same target then
  * scores this selection, runs its top-k on `stream` and prepares no next
  * selection; results are bit-identical to the sequential step's.  A request

@@ -554,19 +554,17 @@ spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* 
   if (!st->lookahead || !ctx_len_dev || (step < 0 && step != SPIN_STEP_DEVICE)) return SPIN_EINVAL;
   const Layout& L = st->lay;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaSuccess;
-  for (int i = 0; i <= st->prep_k && e == cudaSuccess; ++i)
-    if (!st->pev[i]) e = cudaEventCreateWithFlags(&st->pev[i], cudaEventDisableTiming);
-  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i)
-    if (!st->pstream[i]) e = cudaStreamCreateWithFlags(&st->pstream[i], cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaEventRecord(st->pev[0], s);  // fork: after everything before on `stream`
-  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(st->pstream[i], st->pev[0], 0);
-  if (e != cudaSuccess) return cuda_status(e);
+  auto mark = [&](int layer) {
+    spin_state_s::Prepared& P = st->prep[layer];
+    P.ready = true;
+    P.batch = true;
+    P.step = step;
+    P.sparsity = st->sparsity[layer];
+  };
   if (st->cfg.pooling == SPIN_POOL_MAX && vmax_of(st, 0)) {
-    // one predict and one select launch over up to eight layers at a time
-    // (a layer's place in the launch picks its state, scratch and target)
-    spin_status r = SPIN_OK;
-    for (int l0 = 0; l0 < L.L && r == SPIN_OK; l0 += kMaxLayerBatch) {
+    // one predict and one select launch over up to eight layers at a time, on
+    // `stream` (a layer's place in the launch picks its state, scratch and target)
+    for (int l0 = 0; l0 < L.L; l0 += kMaxLayerBatch) {
       const int nl = std::min(kMaxLayerBatch, L.L - l0);
       StepArgs a = step_args(st, l0, 1, step, ctx_len_dev, st->la_mask + (size_t)l0 * L.Q * L.max_blocks);
       a.nl = nl;
@@ -586,33 +584,28 @@ spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* 
         any = any || a.sp[i] > 0.0f;
         st->prep[l0 + i].ready = false;
       }
-      a.no_pdl = 1;  // follows the fork's wait
-      if (any) {
-        r = cuda_status(staged(st, kPredict, st->pstream[0], [&] { return launch_predict_pool(a, st->pstream[0]); }));
-        a.no_pdl = 0;
-      }
-      if (r == SPIN_OK)
-        r = cuda_status(staged(st, kSelect, st->pstream[0], [&] { return launch_select(a, st->pstream[0]); }));
-      for (int i = 0; i < nl && r == SPIN_OK; ++i) {
-        spin_state_s::Prepared& P = st->prep[l0 + i];
-        P.ready = true;
-        P.batch = true;
-        P.step = step;
-        P.sparsity = st->sparsity[l0 + i];
-      }
+      spin_status r = SPIN_OK;
+      if (any) r = cuda_status(staged(st, kPredict, s, [&] { return launch_predict_pool(a, s); }));
+      if (r == SPIN_OK) r = cuda_status(staged(st, kSelect, s, [&] { return launch_select(a, s); }));
+      if (r != SPIN_OK) return r;
+      for (int i = 0; i < nl; ++i) mark(l0 + i);
     }
-    for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) {  // join
-      e = cudaEventRecord(st->pev[1 + i], st->pstream[i]);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->pev[1 + i], 0);
-    }
-    return r != SPIN_OK ? r : cuda_status(e);
+    return SPIN_OK;
   }
-  // other poolings: layer l on stream l mod prep_k, whose block scores only its own layers use
+  // other poolings: the per-layer kernels, layer l on stream l mod prep_k of
+  // the state, whose block-score scratch only its own layers use
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i <= st->prep_k && e == cudaSuccess; ++i)
+    if (!st->pev[i]) e = cudaEventCreateWithFlags(&st->pev[i], cudaEventDisableTiming);
+  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i)
+    if (!st->pstream[i]) e = cudaStreamCreateWithFlags(&st->pstream[i], cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventRecord(st->pev[0], s);  // fork: after everything before on `stream`
+  for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(st->pstream[i], st->pev[0], 0);
+  if (e != cudaSuccess) return cuda_status(e);
   for (int layer = 0; layer < L.L; ++layer) {
     const int i = layer % st->prep_k;
     cudaStream_t ps = st->pstream[i];
-    spin_state_s::Prepared& P = st->prep[layer];
-    P.ready = false;
+    st->prep[layer].ready = false;
     StepArgs a = step_args(st, layer, 1, step, ctx_len_dev, st->la_mask + (size_t)layer * L.Q * L.max_blocks);
     a.S = st->prep_S + (size_t)i * L.Q * L.R * L.blk_stride;
     a.work = st->la_work + (size_t)layer * L.Q * L.blk_stride;
@@ -626,10 +619,7 @@ spin_status spin_prepare_selections(spin_state st, int64_t step, const int32_t* 
     }
     if (r == SPIN_OK) r = cuda_status(staged(st, kSelect, ps, [&] { return launch_select(a, ps); }));
     if (r != SPIN_OK) return r;
-    P.ready = true;
-    P.batch = true;
-    P.step = step;
-    P.sparsity = st->sparsity[layer];
+    mark(layer);
   }
   for (int i = 0; i < st->prep_k && e == cudaSuccess; ++i) {  // join
     e = cudaEventRecord(st->pev[1 + i], st->pstream[i]);

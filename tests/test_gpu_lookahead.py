@@ -174,14 +174,18 @@ def test_lookahead_reports_a_broken_ctx_contract():
     assert isa.spin_get_error(seq)[0] == 0
 
 
-@pytest.mark.parametrize("device_step,max_rows", [(False, 1), (True, 1), (False, 4)])
-def test_prepared_selections_match_sequential_steps(device_step, max_rows):
+@pytest.mark.parametrize("device_step,max_rows,pooling", [(False, 1, isa.SPIN_POOL_MAX), (True, 1, isa.SPIN_POOL_MAX),
+                                                          (False, 4, isa.SPIN_POOL_MAX),
+                                                          (False, 1, isa.SPIN_POOL_MEAN)])
+def test_prepared_selections_match_sequential_steps(device_step, max_rows, pooling):
     """spin_prepare_selections makes every layer's selection of a step up
-    front, over up to eight streams, and each layer's step then scores it.  Masks, top-k and EMA state equal the
+    front, and each layer's step then scores it.  Masks, top-k and EMA state equal the
     sequential steps', also on steps without a preparation (the pipelined
     path runs instead), after a target change that drops a prepared
     selection, and on all-keep steps; also in a state made for four MTP rows,
-    whose block-score layout is four rows wide."""
+    whose block-score layout is four rows wide.  Max pooling takes one launch
+    over up to eight layers (nine layers: a launch of eight and one of one);
+    mean pooling takes the per-layer kernels over the state's streams."""
     wl = _wl(steps=7)
     Ly = 9                                # one stream takes two layers
     caches = [workloads.make_key_cache(wl, l, "cuda") for l in range(Ly)]
@@ -191,7 +195,8 @@ def test_prepared_selections_match_sequential_steps(device_step, max_rows):
     sts = []
     for prep in (False, True):
         cfg = isa.make_config(num_layers=Ly, num_requests=wl.requests, max_slots=wl.max_slots, topk=wl.topk,
-                              target_sparsity=wl.sparsity, gamma=wl.gamma, seed=wl.seed, max_rows=max_rows)
+                              target_sparsity=wl.sparsity, gamma=wl.gamma, seed=wl.seed, max_rows=max_rows,
+                              pooling=pooling)
         st = isa.SpinState(cfg)
         if prep:
             isa.spin_set_lookahead(st, True)
