@@ -50,8 +50,8 @@ SCORE_BYTES_PER_SLOT = 128 + 4 + 4 + 16  # + score write + fused EMA read/write 
 # each is read once), valid for the kernel source with this hash prefix:
 #   "fused-r1": 16 requests at 512K, 50% sparsity, one row, fused EMA;
 #   "deferred-r4": 32 requests at 128K, 40% sparsity, four MTP rows, no EMA in the launch
-SCORE_TRAFFIC = {"src_sha256_16": "ba95974e639feb1a",
-                 "bytes_per_kept_slot": {"fused-r1": 151.43, "deferred-r4": 146.40},
+SCORE_TRAFFIC = {"src_sha256_16": "8ea7182b712ae393",
+                 "bytes_per_kept_slot": {"fused-r1": 151.33, "deferred-r4": 146.20},
                  "sources": ("indexer_sparse_attention_b200/csrc/k_score_tc.cu",
                              "indexer_sparse_attention_b200/csrc/spin_internal.cuh")}
 

@@ -601,6 +601,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
       int q, s, pres, valid, upd, t;
       int p0;  // ctx_len - 1 < 2^31 (max_slots is an int32)
       float sigma, v, d;
+      int kq;  // four rows: the request's kept blocks (whether the top-k can use the group maxima)
     };
     struct SideData {
       float sigma, v, d;
@@ -641,6 +642,7 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
         r.sigma = __ldg(a.kscale + (int64_t)(m.valid ? pg : 0) * kPage + tok);
         r.v = fused ? a.V[(int64_t)m.q * L.slot_stride + m.s] : 0.f;
         r.d = fused ? a.D[(int64_t)m.q * L.slot_stride + (m.upd ? m.p0 - m.s : 0)] : 0.f;
+        if constexpr (RC == 4) r.kq = __ldg(a.kept + m.q);
       } else {
         r.sigma = m.valid ? __ldg(a.kscale + (int64_t)pg * kPage + tok) : 0.f;
         // V of the page's slots past the context too, for its group maxima
@@ -750,7 +752,9 @@ __global__ void __launch_bounds__(threads_for(G), G == 2 ? 2 : 1)
         }
         const float sum = (part[0] + part[1]) + (part[2] + part[3]);
         const bool scored = cur.valid && cur.s <= cur.p0 + r;
-        if (a.gmax) {
+        // (four MTP rows of a request whose kept blocks are too few for the
+        // top-k's group path skip the maxima: nothing would read them)
+        if (a.gmax && (RC != 4 || topk_group_path_possible(cur.kq, L.b, L.k))) {
           // max over this warp's 32 slots = group 4t + quarter of the kept-slot order
           const float g = warp_max(scored ? sum * cur.sigma : __int_as_float(0xff800000));
           if (lane == 0) a.gmax[((int64_t)cur.q * L.R + r) * a.gstride + 4 * cur.t + quarter] = g;

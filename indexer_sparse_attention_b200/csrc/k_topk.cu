@@ -41,7 +41,7 @@ namespace spin {
 constexpr int kTopkThreads = 1024;
 constexpr int kBins = 8192;           // 13-bit first digit
 constexpr int kFirstShift = 19;
-constexpr int kCandCap = 8192;        // candidates kept on chip
+constexpr int kCandCap = kTopkCandCap;  // candidates kept on chip
 constexpr uint32_t kEmptyGroup = 0x007FFFFFu;  // key of -inf: a group with no scored slot
 
 // Dynamic shared memory: the slot bitmap, the histogram / candidate area and,

@@ -228,6 +228,19 @@ struct PdlLaunch {
 // ---------------------------------------------------------------------------
 constexpr int kMaxLayerBatch = 8;  // layers in one launch of the prepared selections
 
+// Candidates the top-k keeps on chip (k_topk.cu).
+constexpr int kTopkCandCap = 8192;
+
+// Whether the top-k can take its group-maxima path for a row whose request
+// kept `kept_blocks` blocks of b slots: the path is tried only when the scored
+// slots overflow the on-chip candidates (so it wants min(k, kTopkCandCap + 1)
+// scores at the least) and needs at least two 32-slot groups per wanted
+// score.  Where it cannot, the score kernel need not write the group maxima.
+__host__ __device__ inline bool topk_group_path_possible(int64_t kept_blocks, int b, int k) {
+  const int64_t want_min = k < kTopkCandCap + 1 ? k : kTopkCandCap + 1;
+  return kept_blocks * b + 31 >= 64 * want_min;
+}
+
 struct StepArgs {
   Layout lay;
   int layer, rows;
