@@ -79,6 +79,19 @@ def test_mtp_rows_union_and_prefix_valid_replay():
     assert max(realized) <= 0.4 + 1e-9                      # union only adds blocks
 
 
+def test_mtp_rows_small_topk_takes_the_group_path():
+    """Four MTP rows with a top-k small enough (k = 64) that rows of the longer
+    requests take the top-k's group-maxima path, which reads the score
+    maxima of each 32 slots, while the short request's rows fit on chip and
+    its maxima are skipped: every row's top-k equals the oracle's."""
+    wl = workloads.config(3, requests=4, ctx0=(30_000, 20_000, 64 * 40 + 5, 1500), steps=5, topk=64)
+    h = Harness(wl)
+    bootstrap(h)
+    acc = workloads.accepted_lengths(wl, wl.steps).numpy()
+    for t in range(1, wl.steps):
+        h.run_step(0, accepted=acc[t], check=range(4))
+
+
 @pytest.mark.parametrize("defer", [True, False])
 def test_mtp_row0_sharing_and_row0_update(defer):
     """The baseline MTP policy in lock step: row 0's mask for every row and
